@@ -1,0 +1,210 @@
+/*
+ * moe.h -- C ABI of a single-GPU Mixture-of-Experts layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (one MoE FFN block, all experts resident on one GPU):
+ *
+ *   1. router          logits[T,E]   = x[T,d] . Wr[d,E] (+ logit_bias[E])      fp32
+ *   2. gating          per token t, k_t experts and weights (three modes below)
+ *   3. capacity        per-expert histogram, capacity C, drops, prefix sum
+ *   4. dispatch        x_perm[r,:] = x[t(r),:], rows grouped by expert
+ *   5. expert FFN      y_perm[r,:] = (silu(x_perm[r].W1[e]) * (x_perm[r].W3[e])) . W2[e]
+ *   6. combine         out[t,:] = sum_j w[t,j] * y_perm[slot_row[t,j],:] (+ shared[t,:])
+ *
+ * Sources for what each step computes:
+ *   - router and top-k: "Paralelismo experto para el servicio MoE"
+ *     (aiunderstanding.org), section "Buceo profundo", and the FAQ entry on
+ *     per-token compute; "Expert Parallelism: MoE 模型的并行切分" (SGLang
+ *     learning notes), section 1;
+ *   - the four steps route / send to the expert / local expert compute / send
+ *     back and combine: "LLM MoE Expert Parallel 生产实战" (oh-bug.com), section
+ *     "为什么 MoE 推理会慢在'最热专家'";
+ *   - capacity factor, token dropping: "Paralelismo experto ...", section
+ *     "Información técnica" and the FAQ entry on uniform expert GEMMs;
+ *   - dispatch = one copy of the token per selected expert, combine = weighted
+ *     sum by the router weight: "Expert Parallelism: MoE 模型的并行切分",
+ *     section 12 question 2; grouping tokens by destination: same page,
+ *     section 4 ("Token sorting"), and question 4 (no padding);
+ *   - per-token routing budget k_t and sub-experts: "MoE-Prism" (gist.science
+ *     summary of arXiv 2510.19366), section 2.A and 2.B;
+ *   - shared expert: "LLM MoE Expert Parallel 生产实战", launch checklist;
+ *   - sigmoid scores + selection bias + group-limited routing + routed scale:
+ *     the DeepSeek-V3-shaped workload specification (the pages only name
+ *     DeepSeek-V3's node-limited routing, "Paralelismo experto ...",
+ *     "Implementación en el mundo real").
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers, row-major, owned by the caller.
+ *     The library never allocates, frees or synchronises in these calls;
+ *     scratch memory comes from a caller workspace sized by moe_workspace_size.
+ *   - Floating tensors x, Wr, W1, W3, W2, Ws1, Ws3, Ws2, x_perm, y_perm, out
+ *     are stored in cfg->dtype (fp32 or bf16).  logits, topk_w, logit_bias and
+ *     sel_bias are always fp32.  Indices and counts are int32.
+ *   - Alignment: every tensor pointer and the workspace must be 16-byte aligned,
+ *     and d and f (and f_shared) must make rows a multiple of 16 bytes:
+ *     d % 8 == 0 and f % 8 == 0 for bf16, d % 4 == 0 and f % 4 == 0 for fp32.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously; results are valid once the stream reaches them.
+ *   - Host-side validation happens before any launch and returns an error code
+ *     with nothing enqueued.  A failed launch returns MOE_ERR_CUDA.  Device-side
+ *     checks (index bounds, pipeline wait limits) set a device error word that
+ *     moe_check_errors reports.
+ *   - Rows: x_perm and y_perm hold at most T*k_max rows (an upper bound known on
+ *     the host); the number actually kept, R = offsets[E], stays on the device
+ *     and the kernels read it there, so no call needs a device-to-host copy.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,  /* a null pointer, a size out of range, k_max > E, ... */
+  MOE_ERR_UNSUPPORTED = -2,  /* a valid but unsupported combination (dtype, shape) */
+  MOE_ERR_WORKSPACE = -3,    /* workspace missing or smaller than moe_workspace_size */
+  MOE_ERR_ALIGNMENT = -4,    /* a pointer or a row size breaks the 16-byte rule */
+  MOE_ERR_CUDA = -5,         /* a CUDA runtime call or a launch failed */
+  MOE_ERR_DEVICE_CHECK = -6  /* moe_check_errors: a device-side check fired */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Gating modes.
+ *  MOE_TOPK_SOFTMAX:        select the k_t largest logits; weights are the
+ *                           softmax over the selected logits.
+ *  MOE_SOFTMAX_TOPK_RENORM: p = softmax over all E logits; select the k_t
+ *                           largest p; weights p_j / sum of the selected p.
+ *                           (Selection is taken on the logits: softmax is
+ *                           monotone, so the selected set is the same.)
+ *  MOE_SIGMOID_GROUPED:     s_e = sigmoid(logit_e), u_e = s_e + sel_bias_e;
+ *                           experts form n_groups contiguous groups; a group's
+ *                           score is the sum of its group_score_topk largest u;
+ *                           keep the topk_groups best groups; select the k_t
+ *                           largest u inside kept groups; weights
+ *                           routed_scale * s_j / sum of the selected s.
+ * Every ranking breaks ties toward the lower expert (or group) index.  The
+ * sigmoid is a fully specified fp32 function (Cody-Waite reduction, degree-7
+ * Taylor polynomial, Horner with fused multiply-adds) so that selection is
+ * reproducible bit for bit on any IEEE machine. */
+typedef enum {
+  MOE_TOPK_SOFTMAX = 0,
+  MOE_SOFTMAX_TOPK_RENORM = 1,
+  MOE_SIGMOID_GROUPED = 2
+} moe_gating;
+
+typedef struct {
+  int32_t T;                /* tokens, >= 0 */
+  int32_t d;                /* hidden size */
+  int32_t E;                /* routed experts, 1..1024 */
+  int32_t k_max;            /* slots per token, 1..min(E, 32) */
+  int32_t f;                /* routed expert intermediate size */
+  int32_t f_shared;         /* shared expert intermediate size; 0 = no shared expert */
+  int32_t dtype;            /* moe_dtype: storage type of x, weights and outputs */
+  int32_t gating;           /* moe_gating */
+  float capacity_factor;    /* > 0: C = ceil(cf * sum_t k_t / E) in double; <= 0: no limit */
+  int32_t n_groups;         /* MOE_SIGMOID_GROUPED only: E % n_groups == 0 */
+  int32_t topk_groups;      /* MOE_SIGMOID_GROUPED only: 1..n_groups */
+  int32_t group_score_topk; /* MOE_SIGMOID_GROUPED only: 1..E/n_groups */
+  float routed_scale;       /* MOE_SIGMOID_GROUPED only: multiplies the weights */
+} moe_config;
+
+/* Routing results (all DEVICE pointers, caller-owned; sizes in elements).
+ * Slots are (t, j) with 0 <= j < k_max; slot a = t*k_max + j.
+ *   logits   [T*E]      fp32 router logits
+ *   topk_idx [T*k_max]  j-th best expert of token t; -1 for j >= k_t
+ *   topk_w   [T*k_max]  combine weight of the slot (0 for j >= k_t); weights
+ *                       of dropped slots are kept as computed (the slot is
+ *                       skipped by combine, not renormalised away)
+ *   counts   [E]        assignments per expert before capacity
+ *   kept     [E]        min(counts[e], C)
+ *   offsets  [E+1]      exclusive prefix sum of kept; R = offsets[E]
+ *   slot_row [T*k_max]  row of a kept slot in x_perm/y_perm, -1 when dropped or padding
+ *   row_src  [T*k_max]  first R entries: slot a = t*k_max+j of each row; rows of
+ *                       expert e are offsets[e]..offsets[e+1]-1, in (t, j) order;
+ *                       slots are admitted per expert in (t, j) order, first C kept
+ *   n_dropped [1]       sum over e of counts[e] - kept[e] */
+typedef struct {
+  float *logits;
+  int32_t *topk_idx;
+  float *topk_w;
+  int32_t *counts;
+  int32_t *kept;
+  int32_t *offsets;
+  int32_t *slot_row;
+  int32_t *row_src;
+  int32_t *n_dropped;
+} moe_route_out;
+
+/* Which call a workspace is sized for. */
+typedef enum {
+  MOE_WS_ROUTE = 0,       /* moe_route */
+  MOE_WS_EXPERT_FFN = 1,  /* moe_expert_ffn */
+  MOE_WS_LAYER = 2        /* moe_layer (covers the other two as well) */
+} moe_ws_kind;
+
+/* Host-only: bytes of workspace `kind` needs for cfg.  Touches no device. */
+moe_status moe_workspace_size(const moe_config *cfg, int32_t kind, size_t *bytes);
+
+/* Steps 1-3.  x [T,d], Wr [d,E] in cfg->dtype; logit_bias [E] fp32 or NULL;
+ * sel_bias [E] fp32 or NULL (MOE_SIGMOID_GROUPED); k_per_token [T] int32 in
+ * [1, k_max] or NULL (k_t = k_max).  Every field of `out` must be set.
+ * ws: at least moe_workspace_size(cfg, MOE_WS_ROUTE) bytes. */
+moe_status moe_route(const moe_config *cfg, const void *x, const void *Wr,
+                     const float *logit_bias, const float *sel_bias,
+                     const int32_t *k_per_token, const moe_route_out *out, void *ws,
+                     size_t ws_bytes, void *stream);
+
+/* Step 4.  x [T,d] -> x_perm [T*k_max, d]: x_perm[r] = x[row_src[r] / k_max]
+ * for r < offsets[E]; rows past R are left untouched. */
+moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *offsets,
+                        const int32_t *row_src, void *x_perm, void *stream);
+
+/* Step 5.  Grouped SwiGLU over expert-contiguous rows: rows offsets[e] ..
+ * offsets[e+1]-1 of x_perm [>= R, d] use expert e.  W1, W3 [E,d,f] and
+ * W2 [E,f,d] in cfg->dtype; y_perm [T*k_max, d].  The intermediate
+ * silu(x.W1)*(x.W3) is stored in the workspace (bf16 for bf16 layers, fp32 for
+ * fp32 layers); accumulation is fp32.  ws: moe_workspace_size(cfg,
+ * MOE_WS_EXPERT_FFN). */
+moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                          const void *W1, const void *W3, const void *W2, void *y_perm,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/* Step 6.  out [T,d] = sum over j < k_max with slot_row >= 0 of
+ * topk_w[t,j] * y_perm[slot_row[t,j]] (+ shared_y[t] when shared_y is not NULL),
+ * accumulated in fp32 and rounded once to cfg->dtype.  A token whose slots are
+ * all dropped gets 0 (+ shared_y[t]). */
+moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *slot_row,
+                       const float *topk_w, const void *shared_y, void *out, void *stream);
+
+/* The whole layer, steps 1-6, plus the always-on shared expert when
+ * cfg->f_shared > 0 (Ws1, Ws3 [d,f_shared], Ws2 [f_shared,d]; NULL otherwise),
+ * whose output is added with weight 1.  route_out may be NULL (routing then
+ * lives in the workspace) or name caller buffers to receive the routing.
+ * ws: at least moe_workspace_size(cfg, MOE_WS_LAYER) bytes. */
+moe_status moe_layer(const moe_config *cfg, const void *x, const void *Wr,
+                     const float *logit_bias, const float *sel_bias,
+                     const int32_t *k_per_token, const void *W1, const void *W3,
+                     const void *W2, const void *Ws1, const void *Ws3, const void *Ws2,
+                     void *out, const moe_route_out *route_out, void *ws, size_t ws_bytes,
+                     void *stream);
+
+/* Synchronises `stream`, then reads and clears the device error flags of the
+ * current device.  *flags (may be NULL) receives them: bit 0 an index out of
+ * range in a gather/scatter, bit 1 a pipeline wait that hit its iteration
+ * limit, bit 2 an expert index or k_t out of range.  Returns
+ * MOE_ERR_DEVICE_CHECK when any flag was set. */
+moe_status moe_check_errors(void *stream, uint32_t *flags);
+
+/* Static description of a status code. */
+const char *moe_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */
