@@ -44,6 +44,8 @@
  *     d % 8 == 0 and f % 8 == 0 for bf16, d % 4 == 0 and f % 4 == 0 for fp32.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
  *     enqueued asynchronously; results are valid once the stream reaches them.
+ *   - T == 0 is an empty batch: a call with a valid config returns MOE_OK and
+ *     touches none of its pointers.
  *   - Host-side validation happens before any launch and returns an error code
  *     with nothing enqueued.  A failed launch returns MOE_ERR_CUDA.  Device-side
  *     checks (index bounds, pipeline wait limits) set a device error word that
@@ -57,6 +59,12 @@
 
 #include <stddef.h>
 #include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
 
 #ifdef __cplusplus
 extern "C" {
@@ -148,20 +156,20 @@ typedef enum {
 } moe_ws_kind;
 
 /* Host-only: bytes of workspace `kind` needs for cfg.  Touches no device. */
-moe_status moe_workspace_size(const moe_config *cfg, int32_t kind, size_t *bytes);
+MOE_API moe_status moe_workspace_size(const moe_config *cfg, int32_t kind, size_t *bytes);
 
 /* Steps 1-3.  x [T,d], Wr [d,E] in cfg->dtype; logit_bias [E] fp32 or NULL;
  * sel_bias [E] fp32 or NULL (MOE_SIGMOID_GROUPED); k_per_token [T] int32 in
  * [1, k_max] or NULL (k_t = k_max).  Every field of `out` must be set.
  * ws: at least moe_workspace_size(cfg, MOE_WS_ROUTE) bytes. */
-moe_status moe_route(const moe_config *cfg, const void *x, const void *Wr,
+MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *Wr,
                      const float *logit_bias, const float *sel_bias,
                      const int32_t *k_per_token, const moe_route_out *out, void *ws,
                      size_t ws_bytes, void *stream);
 
 /* Step 4.  x [T,d] -> x_perm [T*k_max, d]: x_perm[r] = x[row_src[r] / k_max]
  * for r < offsets[E]; rows past R are left untouched. */
-moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *offsets,
+MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *offsets,
                         const int32_t *row_src, void *x_perm, void *stream);
 
 /* Step 5.  Grouped SwiGLU over expert-contiguous rows: rows offsets[e] ..
@@ -170,7 +178,7 @@ moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *off
  * silu(x.W1)*(x.W3) is stored in the workspace (bf16 for bf16 layers, fp32 for
  * fp32 layers); accumulation is fp32.  ws: moe_workspace_size(cfg,
  * MOE_WS_EXPERT_FFN). */
-moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
                           const void *W1, const void *W3, const void *W2, void *y_perm,
                           void *ws, size_t ws_bytes, void *stream);
 
@@ -178,7 +186,7 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32
  * topk_w[t,j] * y_perm[slot_row[t,j]] (+ shared_y[t] when shared_y is not NULL),
  * accumulated in fp32 and rounded once to cfg->dtype.  A token whose slots are
  * all dropped gets 0 (+ shared_y[t]). */
-moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *slot_row,
+MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *slot_row,
                        const float *topk_w, const void *shared_y, void *out, void *stream);
 
 /* The whole layer, steps 1-6, plus the always-on shared expert when
@@ -186,7 +194,7 @@ moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t 
  * whose output is added with weight 1.  route_out may be NULL (routing then
  * lives in the workspace) or name caller buffers to receive the routing.
  * ws: at least moe_workspace_size(cfg, MOE_WS_LAYER) bytes. */
-moe_status moe_layer(const moe_config *cfg, const void *x, const void *Wr,
+MOE_API moe_status moe_layer(const moe_config *cfg, const void *x, const void *Wr,
                      const float *logit_bias, const float *sel_bias,
                      const int32_t *k_per_token, const void *W1, const void *W3,
                      const void *W2, const void *Ws1, const void *Ws3, const void *Ws2,
@@ -198,10 +206,10 @@ moe_status moe_layer(const moe_config *cfg, const void *x, const void *Wr,
  * range in a gather/scatter, bit 1 a pipeline wait that hit its iteration
  * limit, bit 2 an expert index or k_t out of range.  Returns
  * MOE_ERR_DEVICE_CHECK when any flag was set. */
-moe_status moe_check_errors(void *stream, uint32_t *flags);
+MOE_API moe_status moe_check_errors(void *stream, uint32_t *flags);
 
 /* Static description of a status code. */
-const char *moe_status_string(int32_t status);
+MOE_API const char *moe_status_string(int32_t status);
 
 #ifdef __cplusplus
 }

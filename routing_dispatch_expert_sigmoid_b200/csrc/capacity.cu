@@ -1,0 +1,192 @@
+// K3 -- per-expert histogram, capacity, prefix sum and stable dispatch ranks.
+//
+// "Paralelismo experto para el servicio MoE", section "Información técnica"
+// and FAQ: a per-expert capacity bounds the tokens an expert takes; the rest
+// are dropped.  "Expert Parallelism: MoE 模型的并行切分", section 4 ("Token
+// sorting") and question 4 (no padding): tokens bound for the same expert are
+// grouped together, in a ragged (unpadded) layout.
+//
+// Slots a = t*k_max + j are admitted per expert in (t, j) order; the first C
+// of each expert are kept.  Positions are decided without atomics, so the
+// layout is deterministic and equals a stable sort of the kept slots by
+// expert:
+//   K3a  one CTA per chunk of kChunk slots: per-chunk expert histogram
+//        (shared-memory atomics; counts do not depend on order);
+//   K3b  one CTA: per expert, exclusive scan of the chunk histograms (the
+//        chunk's first rank), totals, C = ceil(cf * sum k_t / E) in double,
+//        kept = min(count, C), offsets = exclusive scan of kept, drops;
+//   K3c  one warp per chunk walks its slots 32 at a time in order; lanes
+//        with the same expert find each other with __match_any_sync and rank
+//        themselves by lane order on top of the chunk's running count.
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kChunk = 1024;
+
+int num_chunks(const moe_config &c) {
+  const long long slots = (long long)c.T * c.k_max;
+  return (int)((slots + kChunk - 1) / kChunk);
+}
+
+__global__ void __launch_bounds__(256) k_hist(const int32_t *__restrict__ idx, long long n_slots,
+                                              int E, int32_t *__restrict__ chunk_counts,
+                                              uint32_t *err) {
+  extern __shared__ int32_t cnt[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const long long a0 = (long long)blockIdx.x * kChunk;
+  const long long a1 = min(a0 + kChunk, n_slots);
+  bool bad = false;
+  for (long long a = a0 + threadIdx.x; a < a1; a += blockDim.x) {
+    const int e = idx[a];
+    if (e >= 0 && e < E)
+      atomicAdd(&cnt[e], 1);
+    else if (e != -1)
+      bad = true;
+  }
+  if (bad) raise_error(err, kErrRouting);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    chunk_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads)
+    k_scan(const int32_t *__restrict__ chunk_counts, int n_chunks, int E, double cf,
+           int32_t *__restrict__ chunk_base, int32_t *__restrict__ counts,
+           int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
+           int32_t *__restrict__ n_dropped, int32_t *__restrict__ cap_out) {
+  __shared__ long long s_part[kScanThreads / 32];
+  __shared__ long long s_total;
+  __shared__ int32_t s_cnt[1024];
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  // E <= 1024 = blockDim: thread e owns expert e.
+  long long my = 0;
+  if (tid < E) {
+    int run = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+      chunk_base[(size_t)c * E + tid] = run;
+      run += chunk_counts[(size_t)c * E + tid];
+    }
+    counts[tid] = run;
+    s_cnt[tid] = run;
+    my = run;
+  }
+  // block sum of counts = sum over tokens of k_t
+  long long v = my;
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  if (lane == 0) s_part[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = s_part[lane];
+    for (int off = 16; off > 0; off >>= 1) w += __shfl_xor_sync(0xffffffffu, w, off);
+    if (lane == 0) s_total = w;
+  }
+  __syncthreads();
+  const long long sum_k = s_total;
+  long long C = -1;
+  if (cf > 0.0) C = (long long)ceil(cf * (double)sum_k / (double)E);
+  int k = 0;
+  if (tid < E) {
+    k = s_cnt[tid];
+    if (C >= 0 && k > C) k = (int)C;
+    kept[tid] = k;
+  }
+  // exclusive scan of kept over experts
+  int incl = k;
+  for (int off = 1; off < 32; off <<= 1) {
+    int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  __syncthreads();
+  if (lane == 31) s_part[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = s_part[lane];
+    long long winc = w;
+    for (int off = 1; off < 32; off <<= 1) {
+      long long o = __shfl_up_sync(0xffffffffu, winc, off);
+      if (lane >= off) winc += o;
+    }
+    s_part[lane] = winc - w;  // exclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = (int)s_part[warp] + incl - k;
+  if (tid < E) offsets[tid] = excl;
+  if (tid == E - 1) {
+    offsets[E] = excl + k;
+    n_dropped[0] = (int32_t)(sum_k - (excl + k));
+    cap_out[0] = C < 0 ? -1 : (C > 0x7fffffffLL ? 0x7fffffff : (int32_t)C);
+  }
+}
+
+__global__ void __launch_bounds__(32)
+    k_rank(const int32_t *__restrict__ idx, long long n_slots, int E,
+           const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ offsets,
+           const int32_t *__restrict__ cap, int32_t *__restrict__ slot_row,
+           int32_t *__restrict__ row_src) {
+  extern __shared__ int32_t run[];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) run[e] = chunk_base[(size_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int C = cap[0];
+  const long long a0 = (long long)blockIdx.x * kChunk;
+  const long long a1 = min(a0 + kChunk, n_slots);
+  for (long long base = a0; base < a1; base += 32) {
+    const long long a = base + lane;
+    const bool valid = a < a1;
+    const int e = valid ? idx[a] : -1;
+    const bool real = valid && e >= 0 && e < E;
+    const unsigned peers = __match_any_sync(0xffffffffu, real ? e : E + lane);
+    const int before = __popc(peers & ((1u << lane) - 1u));
+    const int start = real ? run[e] : 0;
+    __syncwarp();
+    if (real) {
+      const int rho = start + before;
+      if (lane == 31 - __clz(peers)) run[e] = start + __popc(peers);
+      if (C >= 0 && rho >= C) {
+        slot_row[a] = -1;
+      } else {
+        const int row = offsets[e] + rho;
+        slot_row[a] = row;
+        row_src[row] = (int32_t)a;
+      }
+    } else if (valid) {
+      slot_row[a] = -1;
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+size_t capacity_scratch_bytes(const moe_config &c) {
+  // chunk_counts + chunk_base (n_chunks x E each) + capacity word, 256-byte aligned
+  const size_t n = (size_t)num_chunks(c) * c.E;
+  return ((2 * n * sizeof(int32_t) + 255) / 256) * 256 + 256;
+}
+
+cudaError_t launch_capacity(const moe_config &c, const int32_t *topk_idx, int32_t *counts,
+                            int32_t *kept, int32_t *offsets, int32_t *slot_row,
+                            int32_t *row_src, int32_t *n_dropped, void *scratch, uint32_t *err,
+                            cudaStream_t s) {
+  const int nch = num_chunks(c);
+  const long long slots = (long long)c.T * c.k_max;
+  const size_t n = (size_t)nch * c.E;
+  int32_t *chunk_counts = static_cast<int32_t *>(scratch);
+  int32_t *chunk_base = chunk_counts + n;
+  int32_t *cap = reinterpret_cast<int32_t *>(static_cast<char *>(scratch) +
+                                             ((2 * n * sizeof(int32_t) + 255) / 256) * 256);
+  const size_t eb = sizeof(int32_t) * (size_t)c.E;
+  if (nch > 0) k_hist<<<nch, 256, eb, s>>>(topk_idx, slots, c.E, chunk_counts, err);
+  k_scan<<<1, kScanThreads, 0, s>>>(chunk_counts, nch, c.E, (double)c.capacity_factor, chunk_base,
+                                    counts, kept, offsets, n_dropped, cap);
+  if (nch > 0)
+    k_rank<<<nch, 32, eb, s>>>(topk_idx, slots, c.E, chunk_base, offsets, cap, slot_row, row_src);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

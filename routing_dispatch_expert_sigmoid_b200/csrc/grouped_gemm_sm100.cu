@@ -1,0 +1,587 @@
+// K5/K6 -- grouped GEMM for the expert FFN on the 5th-generation tensor cores.
+//
+// "LLM MoE Expert Parallel 生产实战", section "为什么 MoE 推理会慢在'最热专家'",
+// step 3 (each expert computes on the rows routed to it) and "Paralelismo
+// experto para el servicio MoE", "Información técnica" (the expert GEMMs see
+// data-dependent row counts).  Rows of group g are offsets[g]..offsets[g+1]-1
+// of A; the counts stay on the device and each CTA derives its tile list from
+// them, so no host synchronisation is needed between routing and the FFN.
+//
+//   SWIGLU: out[r, n] = silu(A[r].B1[g][:, n]) * (A[r].B3[g][:, n])   (K5, x_perm -> h)
+//   PLAIN:  out[r, n] = A[r].B1[g][:, n]                              (K6, h -> y_perm)
+//
+// A [rows_cap, K] bf16 row-major (K-major); B [G, K, N] bf16 row-major, i.e.
+// N-major for the MMA ("MN-major" operand); fp32 accumulation in tensor
+// memory; bf16 output.
+//
+// Design (one CTA per SM, persistent, warp-specialised, 192 threads):
+//   warp 0      TMA producer: A tile 128 x 64 and B tiles 64 x 64 (one 128-byte
+//               swizzle span of N each) into a STAGES-deep shared-memory ring;
+//   warp 1      allocates tensor memory and issues tcgen05.mma (M=128, N=256,
+//               K=16) from one thread; tcgen05.commit releases ring slots and
+//               hands finished accumulators to the epilogue;
+//   warps 2-5   epilogue: tcgen05.ld of the 128 x 256 fp32 accumulator (warp w
+//               reads TMEM lanes 32*(w%4)...), SiLU-gate multiply for K5,
+//               bf16 conversion, masked 16-byte stores of the group's rows.
+// The accumulator is double-buffered in tensor memory (2 x 256 columns) so
+// the epilogue of one tile overlaps the main loop of the next.
+// For SWIGLU the W1 and W3 tiles of the same 128 output columns sit next to
+// each other in shared memory, so one N=256 MMA produces gate (columns
+// 0..127) and up (columns 128..255) of the same rows.
+//
+// Tiles are enumerated (group, n-tile, m-tile) with m fastest and dealt
+// round-robin to the CTAs: CTAs running at the same time share the weight
+// tile of one expert and its rows of A, so weights are read from HBM about
+// once and A stays in L2.  All tiles of a launch have the same K, so the
+// deal is balanced to within one tile.
+//
+// Every wait on an mbarrier is bounded (by %globaltimer): on expiry the CTA
+// records kErrWait in the device error word, tells its other roles to stop,
+// waits (again bounded) for its own copies and MMAs in flight, frees its
+// tensor memory and returns.  No TMA multicast is used.
+#include <cuda.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;          // rows per tile (UMMA M, one TMEM lane per row)
+constexpr int BK = 64;           // K per stage: one 128-byte swizzle span of bf16
+constexpr int kThreads = 192;    // 6 warps
+constexpr int kMaxGroups = 1024;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+struct Ctl {
+  volatile int *abort;
+  uint32_t *err;
+};
+
+// Wait until the phase of parity `parity` of barrier `bar` has completed.
+// Returns false (and stops the CTA) on time-out or when another role stopped.
+__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const Ctl &c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*c.abort) return false;
+    if (global_timer() - t0 > kWaitLimitNs) {
+      *c.abort = 1;
+      raise_error(c.err, kErrWait);
+      return false;
+    }
+  }
+}
+
+// Wait without honouring the stop flag (used to drain work in flight).
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint32_t *err) {
+  const uint64_t t0 = global_timer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer() - t0 > kWaitLimitNs) {
+      raise_error(err, kErrWait);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   slot_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 inputs, fp32 accumulate).
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                     uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on `bar` when every tcgen05 operation issued so far by this
+// thread has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+// Load 32 consecutive fp32 columns of this thread's TMEM lane (and wait).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor (sm_100 format): start address, leading and
+// stride byte offsets (all >> 4), descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // version
+  d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A
+// K-major, B MN-major, N >> 3 at bit 17, M >> 4 at bit 24.
+constexpr uint32_t instr_desc(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel
+// ---------------------------------------------------------------------------
+struct Params {
+  const int32_t *offsets;  // [G+1] or nullptr
+  int G;
+  int fixed_rows;  // rows of the single group when offsets == nullptr
+  int rows_cap;    // rows of A and out
+  int K, N;
+  __nv_bfloat16 *out;  // [rows_cap, N]
+  uint32_t *err;
+};
+
+template <bool SWIGLU>
+struct Shape {
+  static constexpr int BN = SWIGLU ? 128 : 256;       // output columns per tile
+  static constexpr int kSpans = BN / 64;              // 64-column spans per B operand
+  static constexpr int kBOps = SWIGLU ? 2 : 1;
+  static constexpr uint32_t kABytes = BM * BK * 2;    // 16 KB
+  static constexpr uint32_t kSpanBytes = BK * 128;    // 8 KB: 64 K-rows x 128 B
+  static constexpr uint32_t kBBytes = kBOps * kSpans * kSpanBytes;  // 32 KB
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;        // 48 KB
+  static constexpr int kStages = 4;
+  static constexpr int kMmaN = kBOps * BN;            // 256
+  static constexpr uint32_t kAccCols = kMmaN;         // fp32 columns per accumulator
+  static constexpr uint32_t kTmemCols = 2 * kAccCols; // 512
+  static constexpr uint32_t kIdesc = instr_desc(BM, kMmaN);
+  static constexpr size_t kSmemFixed = 1024 /*align slack*/ + kStages * kStageBytes + 256;
+  static_assert(kMmaN % 16 == 0 && kMmaN <= 256, "UMMA N");
+  static_assert(kTmemCols <= 512, "TMEM");
+};
+
+__device__ __forceinline__ void tile_of(int tile, const int32_t *s_tstart, const int32_t *s_off,
+                                        int G, int &g, int &m, int &n) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {  // largest g with s_tstart[g] <= tile
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_tstart[mid] <= tile)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  g = lo;
+  const int rows = s_off[g + 1] - s_off[g];
+  const int mt = (rows + BM - 1) / BM;
+  const int local = tile - s_tstart[g];
+  n = local / mt;
+  m = local - n * mt;
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ CUtensorMap tmB3, const Params p) {
+  using S = Shape<SWIGLU>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *ring = smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + S::kStages * S::kStageBytes);
+  // bars: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain[1]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S::kStages + 5);
+  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kStages * S::kStageBytes + 256);
+  int32_t *s_tstart = s_off + (p.G + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + S::kStages);
+  const uint32_t accf0 = smem_addr(bars + 2 * S::kStages);
+  const uint32_t acce0 = smem_addr(bars + 2 * S::kStages + 2);
+  const uint32_t drain = smem_addr(bars + 2 * S::kStages + 4);
+  const Ctl ctl{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf0 + 8 * b, 1);
+      mbar_init(acce0 + 8 * b, 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB1);
+    if (SWIGLU) prefetch_tmap(&tmB3);
+  }
+  // Group table: row offsets, then tile starts (exclusive scan of the
+  // per-group tile counts), checked against the buffer size.
+  bool bad = false;
+  for (int g = threadIdx.x; g <= p.G; g += kThreads) {
+    const int v = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.fixed_rows);
+    s_off[g] = v;
+    if (v < 0 || v > p.rows_cap) bad = true;
+  }
+  if (warp == 1) tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
+  __syncthreads();
+  const int n_tiles = (p.N + S::BN - 1) / S::BN;
+  for (int g = threadIdx.x; g < p.G; g += kThreads) {
+    const int rows = s_off[g + 1] - s_off[g];
+    if (rows < 0) bad = true;
+    s_tstart[g] = rows > 0 ? ((rows + BM - 1) / BM) * n_tiles : 0;
+  }
+  if (bad) {
+    *abort_flag = 1;
+    raise_error(p.err, kErrIndex);
+  }
+  __syncthreads();
+  if (warp == 0) {  // in-place exclusive scan, 32 groups per step
+    int carry = 0;
+    for (int base = 0; base < p.G; base += 32) {
+      const int g = base + lane;
+      const int v = g < p.G ? s_tstart[g] : 0;
+      int incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (g < p.G) s_tstart[g] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_tstart[p.G] = carry;
+  }
+  if (warp == 1) tmem_relinquish();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = *abort_flag ? 0 : s_tstart[p.G];
+  const int num_kb = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int g, m, n;
+        tile_of(tile, s_tstart, s_off, p.G, g, m, n);
+        const int row = s_off[g] + m * BM;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+          const uint32_t fb = full0 + 8 * s;
+          mbar_expect_tx(fb, S::kStageBytes);
+          tma_load_2d(st, &tmA, fb, kb * BK, row);
+#pragma unroll
+          for (int j = 0; j < S::kSpans; ++j)
+            tma_load_3d(st + S::kABytes + j * S::kSpanBytes, &tmB1, fb, n * S::BN + j * 64,
+                        kb * BK, g);
+          if (SWIGLU) {
+#pragma unroll
+            for (int j = 0; j < S::kSpans; ++j)
+              tma_load_3d(st + S::kABytes + (S::kSpans + j) * S::kSpanBytes, &tmB3, fb,
+                          n * S::BN + j * 64, kb * BK, g);
+          }
+          issued_mask |= 1u << s;
+          issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
+          if (++s == S::kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {  // stopped early: let the copies already issued land first
+        for (int q = 0; q < S::kStages; ++q)
+          if ((issued_mask >> q) & 1u) wait_drain(full0 + 8 * q, (issued_parity >> q) & 1u, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0, buf = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool ok = true, any = false;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        if (!wait(acce0 + 8 * buf, acc_ph ^ 1, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * S::kAccCols;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait(full0 + 8 * s, ph, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // A: K-major, 128-byte rows, 8-row groups 1024 B apart; step K by 32 B.
+            const uint64_t ad = smem_desc(st + kk * 32, 16, 1024);
+            // B: MN-major, 64-column spans kSpanBytes apart (LBO), 8-row K
+            // groups 1024 B apart (SBO); step K by 16 rows = 2048 B.
+            const uint64_t bd = smem_desc(st + S::kABytes + kk * 2048, S::kSpanBytes, 1024);
+            umma(d_tmem, ad, bd, S::kIdesc, (kb | kk) != 0);
+          }
+          any = true;
+          umma_commit(empty0 + 8 * s);
+          if (++s == S::kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(accf0 + 8 * buf);
+        buf ^= 1;
+        if (buf == 0) acc_ph ^= 1;
+      }
+      if (!ok && any) {  // stopped early: wait for the MMAs in flight
+        umma_commit(drain);
+        wait_drain(drain, 0, p.err);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    int buf = 0;
+    uint32_t acc_ph = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int g, m, n;
+      tile_of(tile, s_tstart, s_off, p.G, g, m, n);
+      // One lane waits, the warp follows: tcgen05.ld needs a converged warp.
+      int ready = 0;
+      if (lane == 0) ready = wait(accf0 + 8 * buf, acc_ph, ctl) ? 1 : 0;
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (!ready) break;
+      tc_fence_after();
+      const int row = s_off[g] + m * BM + quarter * 32 + lane;
+      const bool row_ok = row < s_off[g + 1];
+      const uint32_t tb = tmem_base + buf * S::kAccCols + ((uint32_t)(quarter * 32) << 16);
+      __nv_bfloat16 *orow = p.out + (size_t)row * p.N;
+#pragma unroll 1
+      for (int c = 0; c < S::BN; c += 32) {
+        float v[32];
+        tmem_ld32(tb + c, v);
+        if (SWIGLU) {
+          float u[32];
+          tmem_ld32(tb + S::BN + c, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
+        }
+        const int col = n * S::BN + c;
+        if (row_ok) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (col + q * 8 < p.N) {
+              uint32_t w[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+                w[i] = *reinterpret_cast<uint32_t *>(&b2);
+              }
+              *reinterpret_cast<uint4 *>(orow + col + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce0 + 8 * buf);
+      buf ^= 1;
+      if (buf == 0) acc_ph ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over A [rows, K] (K contiguous), box 64 x 128, 128-byte swizzle.
+bool make_map_a(CUtensorMap *m, const void *A, int rows, int K) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)BM};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over B [G, K, N] (N contiguous), box 64 (N) x 64 (K) x 1, 128-byte swizzle.
+bool make_map_b(CUtensorMap *m, const void *B, int G, int K, int N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)G};
+  cuuint64_t strides[2] = {(cuuint64_t)N * 2, (cuuint64_t)K * N * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)BK, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(B), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool SWIGLU>
+cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, int fixed_rows,
+                   const void *A, const void *B1, const void *B3, void *out, uint32_t *err,
+                   cudaStream_t s) {
+  using S = Shape<SWIGLU>;
+  CUtensorMap ma, mb1, mb3;
+  if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
+      !make_map_b(&mb3, SWIGLU ? B3 : B1, G, K, N))
+    return cudaErrorInvalidValue;
+  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  static bool attr_set[64] = {};  // per device
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(
+        k_grouped_gemm<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, static_cast<__nv_bfloat16 *>(out), err};
+  k_grouped_gemm<SWIGLU><<<sms, kThreads, smem, s>>>(ma, mb1, mb3, p);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
+                                     const int32_t *offsets, int fixed_rows, const void *A,
+                                     const void *B1, const void *B3, void *out, uint32_t *err,
+                                     cudaStream_t s) {
+  if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
+  if (rows_cap == 0) return cudaSuccess;
+  return swiglu ? tc::launch<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out, err, s)
+                : tc::launch<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out, err,
+                                    s);
+}
+
+}  // namespace moe

@@ -1,0 +1,345 @@
+// The C ABI of include/moe.h: host-side validation, workspace layout and the
+// order of launches.  Every call validates its arguments on the host before
+// anything is enqueued; no call allocates, frees or synchronises (except
+// moe_check_errors, whose job is to synchronise).
+#include <stdint.h>
+#include <string.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+__device__ uint32_t g_moe_error_word;
+
+uint32_t *device_error_word() {
+  static uint32_t *addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_error_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint32_t *>(p);
+  }
+  return addr[dev];
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+size_t esize(const moe_config &c) { return c.dtype == MOE_F32 ? 4 : 2; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_config(const moe_config *c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d <= 0 || c->f <= 0 || c->f_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (c->E < 1 || c->E > 1024) return MOE_ERR_INVALID_ARG;
+  if (c->k_max < 1 || c->k_max > c->E || c->k_max > 32) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (c->gating < MOE_TOPK_SOFTMAX || c->gating > MOE_SIGMOID_GROUPED) return MOE_ERR_UNSUPPORTED;
+  if ((long long)c->T * c->k_max > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  const int q = c->dtype == MOE_F32 ? 4 : 8;  // elements per 16 bytes
+  if (c->d % q || c->f % q || c->f_shared % q) return MOE_ERR_ALIGNMENT;
+  if (c->gating == MOE_SIGMOID_GROUPED) {
+    if (c->n_groups < 1 || c->n_groups > 32 || c->E % c->n_groups) return MOE_ERR_INVALID_ARG;
+    const int gsz = c->E / c->n_groups;
+    if (c->topk_groups < 1 || c->topk_groups > c->n_groups) return MOE_ERR_INVALID_ARG;
+    if (c->group_score_topk < 1 || c->group_score_topk > gsz) return MOE_ERR_INVALID_ARG;
+    if (c->group_score_topk > 8) return MOE_ERR_UNSUPPORTED;
+    if (c->k_max > c->topk_groups * gsz) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+// Workspace regions, each 256-byte aligned.
+struct Layout {
+  size_t logits, topk_idx, topk_w, counts, kept, offsets, slot_row, row_src, n_dropped;
+  size_t cap_scratch, x_perm, h, y_perm, h_sh, y_sh, total;
+};
+
+Layout layout(const moe_config &c, int kind) {
+  Layout L{};
+  size_t o = 0;
+  const size_t slots = (size_t)c.T * c.k_max, s = esize(c);
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += up(bytes);
+    return at;
+  };
+  if (kind == MOE_WS_LAYER) {
+    L.logits = take(sizeof(float) * (size_t)c.T * c.E);
+    L.topk_idx = take(sizeof(int32_t) * slots);
+    L.topk_w = take(sizeof(float) * slots);
+    L.counts = take(sizeof(int32_t) * c.E);
+    L.kept = take(sizeof(int32_t) * c.E);
+    L.offsets = take(sizeof(int32_t) * (c.E + 1));
+    L.slot_row = take(sizeof(int32_t) * slots);
+    L.row_src = take(sizeof(int32_t) * slots);
+    L.n_dropped = take(sizeof(int32_t));
+  }
+  if (kind == MOE_WS_LAYER || kind == MOE_WS_ROUTE) L.cap_scratch = take(capacity_scratch_bytes(c));
+  if (kind == MOE_WS_LAYER) L.x_perm = take(slots * c.d * s);
+  if (kind == MOE_WS_LAYER || kind == MOE_WS_EXPERT_FFN) L.h = take(slots * c.f * s);
+  if (kind == MOE_WS_LAYER) {
+    L.y_perm = take(slots * c.d * s);
+    if (c.f_shared > 0) {
+      L.h_sh = take((size_t)c.T * c.f_shared * s);
+      L.y_sh = take((size_t)c.T * c.d * s);
+    }
+  }
+  L.total = o;
+  return L;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                  \
+  do {                                 \
+    moe_status _st = (expr);           \
+    if (_st != MOE_OK) return _st;     \
+  } while (0)
+
+#define MOE_TRY_CUDA(expr)                                  \
+  do {                                                      \
+    if ((expr) != cudaSuccess) return MOE_ERR_CUDA;         \
+  } while (0)
+
+moe_status need(const void *p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  return aligned16(p) ? MOE_OK : MOE_ERR_ALIGNMENT;
+}
+moe_status need_opt(const void *p) { return (!p || aligned16(p)) ? MOE_OK : MOE_ERR_ALIGNMENT; }
+// Index / small fp32 arrays: 4-byte alignment is enough.
+moe_status need4(const void *p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  return (reinterpret_cast<uintptr_t>(p) & 3u) ? MOE_ERR_ALIGNMENT : MOE_OK;
+}
+moe_status need4_opt(const void *p) { return p ? need4(p) : MOE_OK; }
+
+moe_status check_route_out(const moe_route_out *o) {
+  if (!o) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(need4(o->logits));
+  MOE_TRY(need4(o->topk_idx));
+  MOE_TRY(need4(o->topk_w));
+  MOE_TRY(need4(o->counts));
+  MOE_TRY(need4(o->kept));
+  MOE_TRY(need4(o->offsets));
+  MOE_TRY(need4(o->slot_row));
+  MOE_TRY(need4(o->row_src));
+  MOE_TRY(need4(o->n_dropped));
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_config &c, int kind, void *ws, size_t ws_bytes) {
+  const size_t need_bytes = layout(c, kind).total;
+  if (need_bytes == 0) return MOE_OK;
+  if (!ws || ws_bytes < need_bytes) return MOE_ERR_WORKSPACE;
+  return aligned16(ws) ? MOE_OK : MOE_ERR_ALIGNMENT;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+moe_status route_impl(const moe_config &c, const void *x, const void *Wr, const float *logit_bias,
+                      const float *sel_bias, const int32_t *k_per_token, const moe_route_out &o,
+                      void *cap_scratch, uint32_t *err, cudaStream_t s) {
+  MOE_TRY_CUDA(launch_router(c, x, Wr, logit_bias, o.logits, s));
+  MOE_TRY_CUDA(launch_gating(c, o.logits, sel_bias, k_per_token, o.topk_idx, o.topk_w, err, s));
+  MOE_TRY_CUDA(launch_capacity(c, o.topk_idx, o.counts, o.kept, o.offsets, o.slot_row, o.row_src,
+                               o.n_dropped, cap_scratch, err, s));
+  return MOE_OK;
+}
+
+// Routed experts (G = E groups over rows_cap rows) or the shared expert
+// (offsets == nullptr: one group of T rows).
+moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixed_rows,
+                    int rows_cap, int f, const void *A, const void *W1, const void *W3,
+                    const void *W2, void *h, void *y, uint32_t *err, cudaStream_t s) {
+  if (c.dtype == MOE_F32) {
+    MOE_TRY_CUDA(launch_ffn_simt_f32(rows_cap, c.d, f, G, offsets, fixed_rows,
+                                     static_cast<const float *>(A), static_cast<const float *>(W1),
+                                     static_cast<const float *>(W3),
+                                     static_cast<const float *>(W2), static_cast<float *>(h),
+                                     static_cast<float *>(y), s));
+    return MOE_OK;
+  }
+  MOE_TRY_CUDA(launch_grouped_gemm_bf16(true, rows_cap, c.d, f, G, offsets, fixed_rows, A, W1, W3,
+                                        h, err, s));
+  MOE_TRY_CUDA(launch_grouped_gemm_bf16(false, rows_cap, f, c.d, G, offsets, fixed_rows, h, W2,
+                                        nullptr, y, err, s));
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_workspace_size(const moe_config *cfg, int32_t kind, size_t *bytes) {
+  MOE_TRY(check_config(cfg));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  if (kind < MOE_WS_ROUTE || kind > MOE_WS_LAYER) return MOE_ERR_INVALID_ARG;
+  *bytes = layout(*cfg, kind).total;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_config *cfg, const void *x, const void *Wr,
+                     const float *logit_bias, const float *sel_bias, const int32_t *k_per_token,
+                     const moe_route_out *out, void *ws, size_t ws_bytes, void *stream) {
+  MOE_TRY(check_config(cfg));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
+  const moe_config &c = *cfg;
+  MOE_TRY(need(x));
+  MOE_TRY(need(Wr));
+  MOE_TRY(need4_opt(logit_bias));
+  MOE_TRY(need4_opt(sel_bias));
+  MOE_TRY(need4_opt(k_per_token));
+  MOE_TRY(check_route_out(out));
+  MOE_TRY(check_ws(c, MOE_WS_ROUTE, ws, ws_bytes));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  const Layout L = layout(c, MOE_WS_ROUTE);
+  return route_impl(c, x, Wr, logit_bias, sel_bias, k_per_token, *out, at<void>(ws, L.cap_scratch),
+                    err, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *offsets,
+                        const int32_t *row_src, void *x_perm, void *stream) {
+  MOE_TRY(check_config(cfg));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
+  MOE_TRY(need(x));
+  MOE_TRY(need4(offsets));
+  MOE_TRY(need4(row_src));
+  MOE_TRY(need(x_perm));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  return cuda_status(
+      launch_dispatch(*cfg, x, offsets, row_src, x_perm, err, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                          const void *W1, const void *W3, const void *W2, void *y_perm, void *ws,
+                          size_t ws_bytes, void *stream) {
+  MOE_TRY(check_config(cfg));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
+  const moe_config &c = *cfg;
+  MOE_TRY(need(x_perm));
+  MOE_TRY(need4(offsets));
+  MOE_TRY(need(W1));
+  MOE_TRY(need(W3));
+  MOE_TRY(need(W2));
+  MOE_TRY(need(y_perm));
+  MOE_TRY(check_ws(c, MOE_WS_EXPERT_FFN, ws, ws_bytes));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  const Layout L = layout(c, MOE_WS_EXPERT_FFN);
+  const int rows_cap = c.T * c.k_max;
+  return ffn_impl(c, c.E, offsets, 0, rows_cap, c.f, x_perm, W1, W3, W2, at<void>(ws, L.h), y_perm,
+                  err, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *slot_row,
+                       const float *topk_w, const void *shared_y, void *out, void *stream) {
+  MOE_TRY(check_config(cfg));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
+  MOE_TRY(need(y_perm));
+  MOE_TRY(need4(slot_row));
+  MOE_TRY(need4(topk_w));
+  MOE_TRY(need_opt(shared_y));
+  MOE_TRY(need(out));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  return cuda_status(launch_combine(*cfg, y_perm, slot_row, topk_w, shared_y, out, err,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_layer(const moe_config *cfg, const void *x, const void *Wr,
+                     const float *logit_bias, const float *sel_bias, const int32_t *k_per_token,
+                     const void *W1, const void *W3, const void *W2, const void *Ws1,
+                     const void *Ws3, const void *Ws2, void *out, const moe_route_out *route_out,
+                     void *ws, size_t ws_bytes, void *stream) {
+  MOE_TRY(check_config(cfg));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
+  const moe_config &c = *cfg;
+  MOE_TRY(need(x));
+  MOE_TRY(need(Wr));
+  MOE_TRY(need4_opt(logit_bias));
+  MOE_TRY(need4_opt(sel_bias));
+  MOE_TRY(need4_opt(k_per_token));
+  MOE_TRY(need(W1));
+  MOE_TRY(need(W3));
+  MOE_TRY(need(W2));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(Ws1));
+    MOE_TRY(need(Ws3));
+    MOE_TRY(need(Ws2));
+  }
+  MOE_TRY(need(out));
+  if (route_out) MOE_TRY(check_route_out(route_out));
+  MOE_TRY(check_ws(c, MOE_WS_LAYER, ws, ws_bytes));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(c, MOE_WS_LAYER);
+  moe_route_out r;
+  if (route_out) {
+    r = *route_out;
+  } else {
+    r.logits = at<float>(ws, L.logits);
+    r.topk_idx = at<int32_t>(ws, L.topk_idx);
+    r.topk_w = at<float>(ws, L.topk_w);
+    r.counts = at<int32_t>(ws, L.counts);
+    r.kept = at<int32_t>(ws, L.kept);
+    r.offsets = at<int32_t>(ws, L.offsets);
+    r.slot_row = at<int32_t>(ws, L.slot_row);
+    r.row_src = at<int32_t>(ws, L.row_src);
+    r.n_dropped = at<int32_t>(ws, L.n_dropped);
+  }
+  MOE_TRY(route_impl(c, x, Wr, logit_bias, sel_bias, k_per_token, r, at<void>(ws, L.cap_scratch),
+                     err, s));
+  const int rows_cap = c.T * c.k_max;
+  void *x_perm = at<void>(ws, L.x_perm), *y_perm = at<void>(ws, L.y_perm);
+  MOE_TRY_CUDA(launch_dispatch(c, x, r.offsets, r.row_src, x_perm, err, s));
+  MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x_perm, W1, W3, W2, at<void>(ws, L.h),
+                   y_perm, err, s));
+  const void *shared_y = nullptr;
+  if (c.f_shared > 0) {
+    MOE_TRY(ffn_impl(c, 1, nullptr, c.T, c.T, c.f_shared, x, Ws1, Ws3, Ws2, at<void>(ws, L.h_sh),
+                     at<void>(ws, L.y_sh), err, s));
+    shared_y = at<void>(ws, L.y_sh);
+  }
+  MOE_TRY_CUDA(launch_combine(c, y_perm, r.slot_row, r.topk_w, shared_y, out, err, s));
+  return MOE_OK;
+}
+
+moe_status moe_check_errors(void *stream, uint32_t *flags) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v && cudaMemset(err, 0, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;
+  if (flags) *flags = v;
+  return v ? MOE_ERR_DEVICE_CHECK : MOE_OK;
+}
+
+const char *moe_status_string(int32_t status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null pointer or size out of range";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: valid but unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT: pointer or row size not 16-byte aligned";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or launch failed";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: a device-side check fired";
+    default: return "unknown moe_status";
+  }
+}
+
+}  // extern "C"

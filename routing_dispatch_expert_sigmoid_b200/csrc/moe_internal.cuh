@@ -1,0 +1,88 @@
+// Internal declarations shared by the CUDA translation units of libmoe.so.
+// Nothing here is part of the public ABI (include/moe.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Device error flags (bit positions documented with moe_check_errors).
+enum : uint32_t {
+  kErrIndex = 1u,    // a gather/scatter index out of range
+  kErrWait = 2u,     // a pipeline wait hit its time limit
+  kErrRouting = 4u,  // an expert index or k_t out of range
+};
+
+// Address of this device's error word (a file-scope __device__ variable of
+// moe_api.cu), looked up once per device.
+uint32_t *device_error_word();
+
+__device__ __forceinline__ void raise_error(uint32_t *err, uint32_t bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// ---- element access -------------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) {
+  return v;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// ---- launchers (host) -----------------------------------------------------
+// Every launcher enqueues on `stream` and returns the cudaGetLastError() of its
+// launches.  Shapes have been validated by the ABI layer before the call.
+
+// K1: logits[T,E] = x[T,d] . Wr[d,E] (+ bias) in fp32 (SIMT, full fp32 FMA).
+cudaError_t launch_router(const moe_config &c, const void *x, const void *Wr,
+                          const float *logit_bias, float *logits, cudaStream_t s);
+
+// K2: gating, one warp per token.
+cudaError_t launch_gating(const moe_config &c, const float *logits, const float *sel_bias,
+                          const int32_t *k_per_token, int32_t *topk_idx, float *topk_w,
+                          uint32_t *err, cudaStream_t s);
+
+// K3: histogram, capacity, prefix sum, stable ranks.  `scratch` holds
+// capacity_scratch_bytes(c) bytes.
+size_t capacity_scratch_bytes(const moe_config &c);
+cudaError_t launch_capacity(const moe_config &c, const int32_t *topk_idx, int32_t *counts,
+                            int32_t *kept, int32_t *offsets, int32_t *slot_row,
+                            int32_t *row_src, int32_t *n_dropped, void *scratch, uint32_t *err,
+                            cudaStream_t s);
+
+// K4: x_perm[r] = x[row_src[r] / k_max] for r < offsets[E].
+cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *offsets,
+                            const int32_t *row_src, void *x_perm, uint32_t *err, cudaStream_t s);
+
+// K7: out[t] = sum_j w[t,j] y_perm[slot_row[t,j]] (+ shared[t]).
+cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
+                           const float *topk_w, const void *shared_y, void *out, uint32_t *err,
+                           cudaStream_t s);
+
+// K9: fp32 SIMT grouped SwiGLU FFN (fp32 layers).  h: [rows_cap, f] fp32.
+cudaError_t launch_ffn_simt_f32(int rows_cap, int d, int f, int G, const int32_t *offsets,
+                                int fixed_rows, const float *x_perm, const float *W1,
+                                const float *W3, const float *W2, float *h, float *y,
+                                cudaStream_t s);
+
+// K5/K6: tcgen05 grouped GEMMs (bf16 in, fp32 accumulate, bf16 out).
+//   swiglu: out[r, :] = silu(A[r].B1[g]) * (A[r].B3[g])     (B*: [G, K, N])
+//   plain:  out[r, :] = A[r].B1[g]
+// Rows of group g are offsets[g]..offsets[g+1]-1 of A (rows_cap rows, K
+// columns); offsets == nullptr means one group of fixed_rows rows.
+cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
+                                     const int32_t *offsets, int fixed_rows, const void *A,
+                                     const void *B1, const void *B3, void *out, uint32_t *err,
+                                     cudaStream_t s);
+
+}  // namespace moe

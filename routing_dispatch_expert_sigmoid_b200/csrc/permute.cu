@@ -1,0 +1,207 @@
+// K4 dispatch and K7 combine: the local (single-GPU) form of the two exchange
+// steps of an MoE layer.
+//
+// "Expert Parallelism: MoE 模型的并行切分", section 12 question 2: dispatch
+// copies each token's hidden state once per selected expert; combine returns
+// the k outputs to the token's position and sums them weighted by the router
+// weight.  Section 3 and "LLM MoE Expert Parallel 生产实战" (steps 2 and 4)
+// describe the same two steps as all-to-alls across GPUs; here both sides are
+// on one GPU, so they are a gather into expert-contiguous rows and a weighted
+// gather back.
+//
+// Both kernels are HBM-bound row copies: one warp per row (dispatch) or per
+// token (combine), 16-byte vector loads and stores, rows of d*s bytes with
+// d*s a multiple of 16.  The number of rows R lives on the device
+// (offsets[E]); a fixed grid strides over the row space and stops at R.
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ uint4 ldg_nc(const uint4 *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__global__ void __launch_bounds__(256)
+    k_dispatch(const uint4 *__restrict__ x, const int32_t *__restrict__ offsets,
+               const int32_t *__restrict__ row_src, uint4 *__restrict__ x_perm, int E,
+               int k_max, int T, int rows_cap, int row_vecs, uint32_t *err) {
+  int R = offsets[E];
+  if (R > rows_cap || R < 0) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(err, kErrIndex);
+    R = R < 0 ? 0 : rows_cap;
+  }
+  const int lane = threadIdx.x % 32;
+  const int warps = gridDim.x * (blockDim.x / 32);
+  for (int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; row < R; row += warps) {
+    const int a = row_src[row];
+    const int t = a / k_max;
+    if (a < 0 || t >= T) {
+      if (lane == 0) raise_error(err, kErrIndex);
+      continue;
+    }
+    const uint4 *src = x + (size_t)t * row_vecs;
+    uint4 *dst = x_perm + (size_t)row * row_vecs;
+    int v = lane;
+    for (; v + 96 < row_vecs; v += 128) {
+      const uint4 a0 = ldg_nc(src + v), a1 = ldg_nc(src + v + 32);
+      const uint4 a2 = ldg_nc(src + v + 64), a3 = ldg_nc(src + v + 96);
+      dst[v] = a0;
+      dst[v + 32] = a1;
+      dst[v + 64] = a2;
+      dst[v + 96] = a3;
+    }
+    for (; v < row_vecs; v += 32) dst[v] = ldg_nc(src + v);
+  }
+}
+
+// 16 bytes of T as fp32 values.
+template <typename T>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const uint4 &u, float *f) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
+  }
+  __device__ static uint4 store(const float *f) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const uint4 &u, float *f) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ static uint4 store(const float *f) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 p = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t *>(&p);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    k_combine(const uint4 *__restrict__ y, const int32_t *__restrict__ slot_row,
+              const float *__restrict__ topk_w, const uint4 *__restrict__ shared_y,
+              uint4 *__restrict__ out, int Tn, int k_max, int rows_cap, int row_vecs,
+              uint32_t *err) {
+  constexpr int N = Vec<T>::N;
+  // Per warp: the token's kept slots, compacted in slot order.
+  __shared__ int32_t s_row[8][32];
+  __shared__ float s_w[8][32];
+  const int lane = threadIdx.x % 32, wib = threadIdx.x / 32;
+  const int warps = gridDim.x * (blockDim.x / 32);
+  for (int t = blockIdx.x * (blockDim.x / 32) + wib; t < Tn; t += warps) {
+    int my_row = -1;
+    float my_w = 0.f;
+    if (lane < k_max) {
+      my_row = slot_row[(size_t)t * k_max + lane];
+      my_w = topk_w[(size_t)t * k_max + lane];
+      if (my_row >= rows_cap) {
+        raise_error(err, kErrIndex);
+        my_row = -1;
+      }
+    }
+    const unsigned live = __ballot_sync(0xffffffffu, my_row >= 0);
+    const int n_live = __popc(live);
+    if (my_row >= 0) {
+      const int pos = __popc(live & ((1u << lane) - 1u));
+      s_row[wib][pos] = my_row;
+      s_w[wib][pos] = my_w;
+    }
+    __syncwarp();
+    for (int v = lane; v < row_vecs; v += 32) {
+      float acc[N];
+      if (shared_y) {
+        Vec<T>::load(ldg_nc(shared_y + (size_t)t * row_vecs + v), acc);
+      } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) acc[i] = 0.f;
+      }
+      for (int j0 = 0; j0 < n_live; j0 += 4) {
+        uint4 u[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)  // issue the loads before the FMAs
+          if (j0 + q < n_live) u[q] = ldg_nc(y + (size_t)s_row[wib][j0 + q] * row_vecs + v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (j0 + q < n_live) {
+            const float wj = s_w[wib][j0 + q];
+            float f[N];
+            Vec<T>::load(u[q], f);
+#pragma unroll
+            for (int i = 0; i < N; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+          }
+        }
+      }
+      out[(size_t)t * row_vecs + v] = Vec<T>::store(acc);
+    }
+    __syncwarp();
+  }
+}
+
+int grid_for(long long warps_needed) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long blocks = (warps_needed + 7) / 8;
+  const long long cap = (long long)sms * 8;
+  return (int)(blocks < 1 ? 1 : (blocks > cap ? cap : blocks));
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *offsets,
+                            const int32_t *row_src, void *x_perm, uint32_t *err,
+                            cudaStream_t s) {
+  const int esz = c.dtype == MOE_F32 ? 4 : 2;
+  const int rows_cap = c.T * c.k_max;
+  if (rows_cap == 0) return cudaSuccess;
+  const int row_vecs = c.d * esz / 16;
+  k_dispatch<<<grid_for(rows_cap), 256, 0, s>>>(
+      static_cast<const uint4 *>(x), offsets, row_src, static_cast<uint4 *>(x_perm), c.E,
+      c.k_max, c.T, rows_cap, row_vecs, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
+                           const float *topk_w, const void *shared_y, void *out, uint32_t *err,
+                           cudaStream_t s) {
+  if (c.T == 0) return cudaSuccess;
+  const int esz = c.dtype == MOE_F32 ? 4 : 2;
+  const int row_vecs = c.d * esz / 16;
+  const int rows_cap = c.T * c.k_max;
+  const int grid = grid_for(c.T);
+  if (c.dtype == MOE_F32)
+    k_combine<float><<<grid, 256, 0, s>>>(
+        static_cast<const uint4 *>(y_perm), slot_row, topk_w,
+        static_cast<const uint4 *>(shared_y), static_cast<uint4 *>(out), c.T, c.k_max, rows_cap,
+        row_vecs, err);
+  else
+    k_combine<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        static_cast<const uint4 *>(y_perm), slot_row, topk_w,
+        static_cast<const uint4 *>(shared_y), static_cast<uint4 *>(out), c.T, c.k_max, rows_cap,
+        row_vecs, err);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,171 @@
+"""Thin ctypes binding of libmoe.so (include/moe.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: torch tensors supply device pointers and the current
+CUDA stream, the library does the work.  There is no fallback: if libmoe.so
+is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .workloads import Workload
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+GATING = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_grouped": 2}
+WS_ROUTE, WS_EXPERT_FFN, WS_LAYER = 0, 1, 2
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {moe_status_string(status)} ({status})")
+        self.status = status
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k_max", ctypes.c_int32), ("f", ctypes.c_int32), ("f_shared", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("gating", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_float), ("n_groups", ctypes.c_int32),
+                ("topk_groups", ctypes.c_int32), ("group_score_topk", ctypes.c_int32),
+                ("routed_scale", ctypes.c_float)]
+
+
+class MoeRouteOut(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("logits", "topk_idx", "topk_w", "counts", "kept", "offsets", "slot_row",
+                 "row_src", "n_dropped")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (built by routing_dispatch_expert_sigmoid_b200/build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so not built ({LIB_PATH}); run __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        cfgp = ctypes.POINTER(MoeConfig)
+        outp = ctypes.POINTER(MoeRouteOut)
+        L.moe_workspace_size.argtypes = [cfgp, I, ctypes.POINTER(S)]
+        L.moe_route.argtypes = [cfgp, P, P, P, P, P, outp, P, S, P]
+        L.moe_dispatch.argtypes = [cfgp, P, P, P, P, P]
+        L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, S, P]
+        L.moe_combine.argtypes = [cfgp, P, P, P, P, P, P]
+        L.moe_layer.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, outp, P, S, P]
+        L.moe_check_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+        L.moe_status_string.argtypes = [I]
+        L.moe_status_string.restype = ctypes.c_char_p
+        for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn",
+                   "moe_combine", "moe_layer", "moe_check_errors"):
+            getattr(L, fn).restype = I
+        _lib = L
+    return _lib
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise MoeError(status, what)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def config(w: Workload, T: int | None = None) -> MoeConfig:
+    """The moe_config of a workload (optionally with another token count)."""
+    return MoeConfig(T=w.T if T is None else T, d=w.d, E=w.E, k_max=w.k_max, f=w.f,
+                     f_shared=w.f_shared, dtype=MOE_F32 if w.dtype == "f32" else MOE_BF16,
+                     gating=GATING[w.gating], capacity_factor=w.capacity_factor,
+                     n_groups=w.n_groups, topk_groups=w.topk_groups,
+                     group_score_topk=w.group_score_topk, routed_scale=w.routed_scale)
+
+
+def moe_workspace_size(cfg: MoeConfig, kind: int = WS_LAYER) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_workspace_size(ctypes.byref(cfg), kind, ctypes.byref(n)),
+           "moe_workspace_size")
+    return int(n.value)
+
+
+def workspace(cfg: MoeConfig, kind: int = WS_LAYER, device="cuda") -> torch.Tensor:
+    """A caller-owned workspace of the size moe_workspace_size asks for."""
+    return torch.empty(max(moe_workspace_size(cfg, kind), 1), dtype=torch.uint8, device=device)
+
+
+def route_buffers(cfg: MoeConfig, device="cuda") -> dict:
+    """Caller-owned routing output tensors for moe_route / moe_layer."""
+    T, E, k = cfg.T, cfg.E, cfg.k_max
+    i32 = dict(dtype=torch.int32, device=device)
+    return dict(logits=torch.empty((T, E), dtype=torch.float32, device=device),
+                topk_idx=torch.empty((T, k), **i32), topk_w=torch.empty((T, k), dtype=torch.float32,
+                                                                        device=device),
+                counts=torch.empty(E, **i32), kept=torch.empty(E, **i32),
+                offsets=torch.empty(E + 1, **i32), slot_row=torch.empty((T, k), **i32),
+                row_src=torch.empty(max(T * k, 1), **i32), n_dropped=torch.empty(1, **i32))
+
+
+def _route_struct(b: dict) -> MoeRouteOut:
+    return MoeRouteOut(*[b[name].data_ptr() for name, _ in MoeRouteOut._fields_])
+
+
+def moe_route(cfg, x, Wr, logit_bias, sel_bias, k_per_token, out: dict, ws, stream=None):
+    r = _route_struct(out)
+    _check(lib().moe_route(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias),
+                           _p(k_per_token), ctypes.byref(r), _p(ws),
+                           0 if ws is None else ws.numel(), _stream(stream)), "moe_route")
+
+
+def moe_dispatch(cfg, x, offsets, row_src, x_perm, stream=None):
+    _check(lib().moe_dispatch(ctypes.byref(cfg), _p(x), _p(offsets), _p(row_src), _p(x_perm),
+                              _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_ffn(cfg, x_perm, offsets, W1, W3, W2, y_perm, ws, stream=None):
+    _check(lib().moe_expert_ffn(ctypes.byref(cfg), _p(x_perm), _p(offsets), _p(W1), _p(W3),
+                                _p(W2), _p(y_perm), _p(ws), 0 if ws is None else ws.numel(),
+                                _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(cfg, y_perm, slot_row, topk_w, shared_y, out, stream=None):
+    _check(lib().moe_combine(ctypes.byref(cfg), _p(y_perm), _p(slot_row), _p(topk_w),
+                             _p(shared_y), _p(out), _stream(stream)), "moe_combine")
+
+
+def moe_layer(cfg, x, Wr, logit_bias, sel_bias, k_per_token, W1, W3, W2, Ws1, Ws3, Ws2, out,
+              route_out: dict | None, ws, stream=None):
+    r = None if route_out is None else ctypes.byref(_route_struct(route_out))
+    _check(lib().moe_layer(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias),
+                           _p(k_per_token), _p(W1), _p(W3), _p(W2), _p(Ws1), _p(Ws3), _p(Ws2),
+                           _p(out), r, _p(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+           "moe_layer")
+
+
+def moe_check_errors(stream=None) -> int:
+    """Synchronise the stream and return the device error flags (raises if any)."""
+    flags = ctypes.c_uint32(0)
+    st = lib().moe_check_errors(_stream(stream), ctypes.byref(flags))
+    if st not in (0, -6):
+        _check(st, "moe_check_errors")
+    if flags.value:
+        raise MoeError(st, f"moe_check_errors: device flags {flags.value:#x}")
+    return 0

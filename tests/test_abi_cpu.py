@@ -1,0 +1,173 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/moe.h declares, sizes workspaces, and rejects bad arguments on the
+host before touching the device.  Nothing here launches a kernel.
+"""
+import ctypes
+import math
+import os
+import re
+import struct
+from fractions import Fraction
+
+import pytest
+
+from routing_dispatch_expert_sigmoid_b200 import ops
+from routing_dispatch_expert_sigmoid_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 8, names
+    L = ops.lib()
+    for n in names:
+        assert hasattr(L, n), f"libmoe.so does not export {n}"
+    assert {"moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer"} <= set(names)
+
+
+def test_status_strings():
+    for st in range(-6, 1):
+        s = ops.moe_status_string(st)
+        assert s.startswith("MOE_")
+    assert "unknown" in ops.moe_status_string(42)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workspace_sizes(name):
+    w = WORKLOADS[name]
+    cfg = ops.config(w)
+    s = w.elem_bytes
+    slots = w.T * w.k_max
+    layer = ops.moe_workspace_size(cfg, ops.WS_LAYER)
+    # x_perm, h and y_perm are the dominant regions
+    assert layer >= slots * (2 * w.d + w.f) * s
+    assert ops.moe_workspace_size(cfg, ops.WS_EXPERT_FFN) >= slots * w.f * s
+    assert 0 < ops.moe_workspace_size(cfg, ops.WS_ROUTE) < layer
+    for kind in (ops.WS_ROUTE, ops.WS_EXPERT_FFN, ops.WS_LAYER):
+        assert ops.moe_workspace_size(cfg, kind) % 256 == 0
+
+
+def _status(fn, *args):
+    return getattr(ops.lib(), fn)(*args)
+
+
+def _cfg(**kw):
+    c = ops.config(WORKLOADS["dsv3_decode"])
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(k_max=300), -1), (dict(k_max=0), -1), (dict(E=0), -1), (dict(E=2048), -1),
+    (dict(T=-1), -1), (dict(d=0), -1), (dict(dtype=7), -2), (dict(gating=9), -2),
+    (dict(d=7164), -4), (dict(f=2044), -4), (dict(n_groups=7), -1), (dict(n_groups=64), -1),
+    (dict(topk_groups=9), -1), (dict(group_score_topk=33), -1), (dict(group_score_topk=9), -2),
+    (dict(topk_groups=1, k_max=33), -1),
+])
+def test_config_validation(kw, expect):
+    c = _cfg(**kw)
+    n = ctypes.c_size_t(0)
+    assert ops.lib().moe_workspace_size(ctypes.byref(c), ops.WS_LAYER, ctypes.byref(n)) == expect
+
+
+FAKE = 0x7f0000000000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _route_out(ptr=FAKE):
+    return ops.MoeRouteOut(*([ptr] * 9))
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch():
+    c = _cfg()
+    L = ops.lib()
+    r = _route_out()
+    P = ctypes.c_void_p
+    ws = ctypes.c_size_t(1 << 40)
+    # null x
+    assert L.moe_route(ctypes.byref(c), None, P(FAKE), None, None, None, ctypes.byref(r), P(FAKE),
+                       ws, None) == -1
+    # misaligned x
+    assert L.moe_route(ctypes.byref(c), P(FAKE + 8), P(FAKE), None, None, None, ctypes.byref(r),
+                       P(FAKE), ws, None) == -4
+    # misaligned k_per_token (int32 array: 4-byte rule)
+    assert L.moe_route(ctypes.byref(c), P(FAKE), P(FAKE), None, None, P(FAKE + 2),
+                       ctypes.byref(r), P(FAKE), ws, None) == -4
+    # a null routing output
+    bad = _route_out()
+    bad.offsets = None
+    assert L.moe_route(ctypes.byref(c), P(FAKE), P(FAKE), None, None, None, ctypes.byref(bad),
+                       P(FAKE), ws, None) == -1
+    assert L.moe_dispatch(ctypes.byref(c), P(FAKE), None, P(FAKE), P(FAKE), None) == -1
+    assert L.moe_combine(ctypes.byref(c), P(FAKE), P(FAKE), P(FAKE), P(FAKE + 4), P(FAKE),
+                         None) == -4
+    # shared expert weights are required when f_shared > 0
+    args = [P(FAKE)] * 5 + [P(FAKE)] * 3 + [None, P(FAKE), P(FAKE), P(FAKE)]
+    assert L.moe_layer(ctypes.byref(c), P(FAKE), P(FAKE), None, None, None, P(FAKE), P(FAKE),
+                       P(FAKE), None, P(FAKE), P(FAKE), P(FAKE), None, P(FAKE), ws, None) == -1
+    del args
+
+
+def test_workspace_too_small_rejected():
+    c = _cfg()
+    L = ops.lib()
+    P = ctypes.c_void_p
+    need = ops.moe_workspace_size(c, ops.WS_LAYER)
+    small = ctypes.c_size_t(need - 1)
+    assert L.moe_layer(ctypes.byref(c), P(FAKE), P(FAKE), None, None, None, P(FAKE), P(FAKE),
+                       P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, P(FAKE), small,
+                       None) == -3
+    assert L.moe_layer(ctypes.byref(c), P(FAKE), P(FAKE), None, None, None, P(FAKE), P(FAKE),
+                       P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, None,
+                       ctypes.c_size_t(need), None) == -3
+    r = _route_out()
+    need_r = ops.moe_workspace_size(c, ops.WS_ROUTE)
+    assert L.moe_route(ctypes.byref(c), P(FAKE), P(FAKE), None, None, None, ctypes.byref(r),
+                       P(FAKE), ctypes.c_size_t(need_r - 256), None) == -3
+
+
+def test_empty_batch_is_a_noop_without_pointers():
+    c = _cfg(T=0)
+    L = ops.lib()
+    assert L.moe_layer(ctypes.byref(c), None, None, None, None, None, None, None, None, None,
+                       None, None, None, None, None, ctypes.c_size_t(0), None) == 0
+
+
+def _exact_f32(fr: Fraction) -> int:
+    """binary32 bits of a positive rational, rounded to nearest even."""
+    e = math.floor(math.log2(fr.numerator) - math.log2(fr.denominator))
+    while Fraction(2) ** e > fr:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= fr:
+        e += 1
+    m = fr * Fraction(2) ** (23 - e)
+    lo = m.numerator // m.denominator
+    rem = m - lo
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2):
+        lo += 1
+    return struct.unpack("<I", struct.pack("<f", float(Fraction(lo) * Fraction(2) ** (e - 23))))[0]
+
+
+def test_gpu_sigmoid_constants_are_the_rounded_definitions():
+    """The GPU's specified exp takes its constants from their definitions."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 60
+    ln2 = Fraction(Decimal(2).ln())
+    src = open(os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc", "gating.cu")).read()
+    lits = dict(re.findall(r"const float (k\w+) = ([0-9.e+-]+)f;", src))
+
+    def bits(name):
+        return struct.unpack("<I", struct.pack("<f", float(lits[name])))[0]
+
+    assert bits("kLog2e") == _exact_f32(1 / ln2)
+    assert Fraction(float(lits["kLn2Hi"])) == Fraction(2839, 4096)
+    assert bits("kLn2Lo") == _exact_f32(ln2 - Fraction(2839, 4096))
+    for k in range(3, 8):
+        assert bits(f"kC{k}") == _exact_f32(Fraction(1, math.factorial(k))), k

@@ -1,0 +1,228 @@
+"""CUDA path vs the CPU oracle, element by element, on seeded inputs.
+
+Small cases: every gating mode, both dtypes, several tiles of every kernel,
+ragged tails in T, d, f and the expert groups, variable k, capacity drops,
+shared expert.  Each step is checked on its own through its C-ABI entry point
+(moe_route, moe_dispatch, moe_expert_ffn, moe_combine) and then as a whole
+(moe_layer).  Tolerances are those of tests/parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import (assert_logits_close, assert_out_close, check_routing_bit_exact, f64,
+                    gpu_inputs, oracle_gating_kw, oracle_layer_on_tokens, run_layer, run_route)
+from routing_dispatch_expert_sigmoid_b200 import ops
+from routing_dispatch_expert_sigmoid_b200.workloads import WORKLOADS, make_inputs, to_numpy
+
+pytestmark = pytest.mark.gpu
+
+# Scaled-down layers of every workload family: same gating, k, groups, dtype;
+# dimensions cross tile edges (128-row M tiles, 128/256-column N tiles, 64-deep
+# K steps) with ragged tails.
+SMALL = {
+    "tiny_f32": WORKLOADS["tiny_f32"],
+    "mixtral_small": WORKLOADS["mixtral_prefill"].scaled(T=300, d=256, f=384),
+    "qwen3_small": WORKLOADS["qwen3_prefill"].scaled(T=257, d=192, E=16, k_max=4, f=200),
+    "dsv3_small": WORKLOADS["dsv3_prefill"].scaled(T=130, d=256, E=64, f=136, f_shared=72),
+    "gptoss_small": WORKLOADS["gptoss_sub"].scaled(T=211, d=200, E=32, k_max=6, k_min=2, f=72),
+    "mixtral_decode_small": WORKLOADS["mixtral_decode"].scaled(T=5, d=512, f=1024),
+}
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ops.lib()
+    return torch.device("cuda:0")
+
+
+def _host_inputs(w, seed=0):
+    return make_inputs(w, seed, device="cpu")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_route_bit_exact_and_logits(name, dev):
+    w = SMALL[name]
+    hin = _host_inputs(w)
+    inp = gpu_inputs(w, 0, dev, hin)
+    cfg, out = run_route(w, inp)
+    ref = oracle.router_logits(to_numpy(hin["x"]), to_numpy(hin["Wr"]),
+                               to_numpy(hin["logit_bias"]))
+    assert_logits_close(out["logits"], ref)
+    check_routing_bit_exact(w, hin, out)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_dispatch_bit_exact(name, dev):
+    w = SMALL[name]
+    hin = _host_inputs(w)
+    inp = gpu_inputs(w, 0, dev, hin)
+    cfg, out = run_route(w, inp)
+    lay = check_routing_bit_exact(w, hin, out)
+    R = int(lay["offsets"][-1])
+    x_perm = torch.full((w.T * w.k_max, w.d), float("nan"), dtype=inp["x"].dtype, device=dev)
+    ops.moe_dispatch(cfg, inp["x"], out["offsets"], out["row_src"], x_perm)
+    ops.moe_check_errors()
+    ref = oracle.dispatch(to_numpy(hin["x"]), lay["row_src"], w.k_max)
+    assert (to_numpy(x_perm[:R]) == ref).all()
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_expert_ffn_matches_oracle(name, dev):
+    """Grouped FFN alone, on the oracle's dispatched rows and layout."""
+    w = SMALL[name]
+    hin = _host_inputs(w)
+    inp = gpu_inputs(w, 0, dev, hin)
+    cfg, out = run_route(w, inp)
+    lay = check_routing_bit_exact(w, hin, out)
+    R = int(lay["offsets"][-1])
+    xp = oracle.dispatch(to_numpy(hin["x"]), lay["row_src"], w.k_max)
+    x_perm = torch.zeros((w.T * w.k_max, w.d), dtype=inp["x"].dtype)
+    x_perm[:R] = hin["x"][torch.from_numpy(lay["row_src"] // w.k_max).long()]
+    assert (to_numpy(x_perm[:R]) == xp).all()
+    x_perm = x_perm.to(dev)
+    y_perm = torch.zeros_like(x_perm)
+    ws = ops.workspace(cfg, ops.WS_EXPERT_FFN)
+    offs = torch.from_numpy(lay["offsets"]).to(dev)
+    ops.moe_expert_ffn(cfg, x_perm, offs, inp["W1"], inp["W3"], inp["W2"], y_perm, ws)
+    ops.moe_check_errors()
+    ref = oracle.grouped_ffn(xp, lay["offsets"], to_numpy(hin["W1"]), to_numpy(hin["W3"]),
+                             to_numpy(hin["W2"]))
+    assert_out_close(f64(y_perm[:R]), ref, "y_perm")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_combine_matches_oracle(name, dev):
+    """Combine alone, on seeded synthetic expert outputs and the oracle's layout."""
+    w = SMALL[name]
+    hin = _host_inputs(w)
+    cfg = ops.config(w)
+    l32 = oracle.router_logits(to_numpy(hin["x"]), to_numpy(hin["Wr"]),
+                               to_numpy(hin["logit_bias"])).astype(np.float32)
+    idx, wts = oracle.gating(l32, w.k_max, w.gating, **oracle_gating_kw(w, hin))
+    lay = oracle.capacity_dispatch(idx, w.E, float(np.float32(w.capacity_factor)))
+    dt = hin["x"].dtype
+    g = torch.Generator().manual_seed(1)
+    y_perm = torch.randn((w.T * w.k_max, w.d), generator=g).to(dt)
+    shared = torch.randn((w.T, w.d), generator=g).to(dt) if w.f_shared else None
+    out = torch.empty((w.T, w.d), dtype=dt, device=dev)
+    ops.moe_combine(cfg, y_perm.to(dev), torch.from_numpy(lay["slot_row"]).to(dev),
+                    torch.from_numpy(wts.astype(np.float32)).to(dev),
+                    None if shared is None else shared.to(dev), out)
+    ops.moe_check_errors()
+    ref = oracle.combine_rows(wts.astype(np.float32).astype(np.float64), lay["slot_row"],
+                              to_numpy(y_perm), to_numpy(shared))
+    assert_out_close(f64(out), ref, "combine")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_matches_oracle(name, dev):
+    w = SMALL[name]
+    hin = _host_inputs(w)
+    inp = gpu_inputs(w, 0, dev, hin)
+    out, rb = run_layer(w, inp)
+    routing = check_routing_bit_exact(w, hin, rb)
+    ref = oracle_layer_on_tokens(hin, routing, list(range(w.T)))
+    assert_out_close(f64(out), ref, "layer out")
+    # the layer without caller routing buffers gives the same output
+    out2, _ = run_layer(w, inp, route_out=False)
+    assert torch.equal(out, out2)
+
+
+# ---------------------------------------------------------------------------
+# Edge cases
+# ---------------------------------------------------------------------------
+def _layer_vs_oracle(w, hin, dev):
+    inp = gpu_inputs(w, 0, dev, hin)
+    out, rb = run_layer(w, inp)
+    routing = check_routing_bit_exact(w, hin, rb)
+    ref = oracle_layer_on_tokens(hin, routing, list(range(w.T)))
+    assert_out_close(f64(out), ref, "layer out")
+    return rb
+
+
+@pytest.mark.parametrize("T", [1, 2, 127, 129])
+def test_token_counts_across_tile_edges(T, dev):
+    w = SMALL["mixtral_small"].scaled(T=T)
+    _layer_vs_oracle(w, _host_inputs(w, seed=T), dev)
+
+
+def test_all_equal_logits_tie_to_lower_index(dev):
+    w = SMALL["qwen3_small"].scaled(zipf_s=0.0, capacity_factor=0.0)
+    hin = _host_inputs(w)
+    hin["Wr"] = torch.zeros_like(hin["Wr"])
+    rb = _layer_vs_oracle(w, hin, dev)
+    assert (rb["topk_idx"].cpu() == torch.arange(w.k_max, dtype=torch.int32)).all()
+
+
+def test_one_expert_takes_every_token_and_others_idle(dev):
+    w = SMALL["mixtral_small"].scaled(T=260, k_max=1, zipf_s=0.0)
+    hin = _host_inputs(w)
+    hin["logit_bias"] = torch.tensor([0, 0, 0, 50.0, 0, 0, 0, 0])
+    rb = _layer_vs_oracle(w, hin, dev)
+    counts = rb["counts"].cpu().numpy()
+    assert counts[3] == w.T and counts.sum() == w.T
+
+
+def test_heavy_drops_small_capacity(dev):
+    w = SMALL["qwen3_small"].scaled(capacity_factor=0.3)
+    rb = _layer_vs_oracle(w, _host_inputs(w), dev)
+    assert int(rb["n_dropped"].item()) > 0
+
+
+def test_single_expert_dense(dev):
+    w = SMALL["mixtral_small"].scaled(E=1, k_max=1, T=77)
+    _layer_vs_oracle(w, _host_inputs(w), dev)
+
+
+def test_k_equals_E_uniform(dev):
+    w = SMALL["mixtral_small"].scaled(E=8, k_max=8, T=40, zipf_s=0.0)
+    hin = _host_inputs(w)
+    hin["Wr"] = torch.zeros_like(hin["Wr"])
+    _layer_vs_oracle(w, hin, dev)
+
+
+def test_empty_batch(dev):
+    w = SMALL["dsv3_small"].scaled(T=0)
+    cfg = ops.config(w)
+    inp = make_inputs(w.scaled(T=1), 0, device=dev)
+    x = inp["x"][:0]
+    ws = ops.workspace(cfg, ops.WS_LAYER)
+    out = torch.empty((0, w.d), dtype=x.dtype, device=dev)
+    ops.moe_layer(cfg, inp["x"], inp["Wr"], None, inp["sel_bias"], None, inp["W1"], inp["W3"],
+                  inp["W2"], inp["Ws1"], inp["Ws3"], inp["Ws2"], out, None, ws)
+    ops.moe_check_errors()
+
+
+def test_sigmoid_grouped_near_ties_bit_exact(dev):
+    """Logits on a fine grid with many exact and one-ulp ties in the biased
+    scores: selection must follow the specified sigmoid bit for bit."""
+    w = SMALL["dsv3_small"].scaled(T=512)
+    hin = _host_inputs(w)
+    cfg = ops.config(w)
+    g = torch.Generator().manual_seed(5)
+    # logits from a coarse grid -> many equal sigmoid values; bias on a grid too
+    logits = (torch.randint(-8, 9, (w.T, w.E), generator=g).float() / 8.0)
+    sel_bias = (torch.randint(-4, 5, (w.E,), generator=g).float() / 64.0)
+    l_dev = logits.to(dev)
+    out = ops.route_buffers(cfg)
+    # route with Wr = 0 and the grid as logit bias would tie every token; instead
+    # drive the gating through a router whose logits are exactly the grid:
+    # x = identity rows (T <= d is not required: use d >= E and one-hot x).
+    assert w.d >= w.E
+    x = torch.zeros((w.T, w.d))
+    Wr = torch.zeros((w.d, w.E))
+    Wr[: w.E, :] = torch.eye(w.E)
+    # x[t, :E] = logits[t] makes x.Wr = logits exactly (values are bf16-exact)
+    x[:, : w.E] = logits
+    hin2 = dict(hin, x=x.to(torch.bfloat16), Wr=Wr.to(torch.bfloat16), sel_bias=sel_bias,
+                logit_bias=None)
+    inp = gpu_inputs(w, 0, dev, hin2)
+    ws = ops.workspace(cfg, ops.WS_ROUTE)
+    ops.moe_route(cfg, inp["x"], inp["Wr"], None, inp["sel_bias"], None, out, ws)
+    ops.moe_check_errors()
+    assert torch.equal(out["logits"], l_dev)
+    check_routing_bit_exact(w, hin2, out)
