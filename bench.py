@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""MoE-layer tokens/s on B200: prefill and decode regimes of the Mixtral-8x7B
+shaped layer (d=4096, E=8, top-2, f=14336, bf16, Zipf(0.5) router bias).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one moe_layer call over one batch (router, gating, capacity,
+dispatch, grouped SwiGLU expert FFN, combine), inputs resident in HBM.  Time
+is taken on the device with CUDA events around K back-to-back steps, between
+a barrier and a synchronize on both sides; with N GPUs (torchrun, one process
+per GPU) every rank runs its own replica of the layer on its own batch and
+the time is the max over ranks (weak scaling, no collective on the data path).
+
+Extra keys of the JSON line:
+  roofline     the up-projection + SwiGLU grouped GEMM (the dominant kernel):
+               algorithmic FLOPs (prefill) or bytes (decode) per launch over its
+               mean launch time, from CUDA events recorded on the launching
+               stream at its boundaries inside the timed steps;
+  e2e          the same metric through the C ABI with host buffers: per step a
+               pinned-host -> device copy of x and a device -> pinned-host copy
+               of the layer output are inside the timed region;
+  cpu_baseline the CPU oracle as it stands, on a bounded sample of the same
+               workload, on the host cores (rank 0, N=1 only);
+  clocks       nvidia-smi samples taken during the timed region.
+`--impl reference` times the CPU oracle alone on the same workload (the
+reference arm: there is no other implementation of this layer to run).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from routing_dispatch_expert_sigmoid_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILES = os.path.join(ROOT, "profiles")
+GEMM_SRC = os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc",
+                        "grouped_gemm_sm100.cu")
+METRIC = "MoE-layer tokens/sec on 1 B200 (decode & prefill); % of roofline"
+PREFILL, DECODE = "mixtral_prefill", "mixtral_decode"
+L2_BYTES = 126 * 2 ** 20
+
+
+# ---------------------------------------------------------------------------
+# process group / ranks
+# ---------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(value: float, dist) -> float:
+    """Max over ranks (control plane only)."""
+    if dist is None:
+        return value
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(local_ms: float, local_units: int, dist) -> tuple[float, int]:
+    """(max elapsed ms over ranks, total units over ranks) -- whole-job numbers."""
+    ms = reduce_max(local_ms, dist)
+    if dist is None:
+        return ms, local_units
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([local_units], dtype=torch.int64, device=dev)
+    dist.all_reduce(t)
+    return ms, int(t.item())
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.file,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self) -> dict:
+        if self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.file.flush()
+        with open(self.file.name) as fh:
+            rows = [r for r in csv.reader(io.StringIO(fh.read())) if len(r) >= 9]
+        os.unlink(self.file.name)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, pw, reasons = [], [], [], set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                pw.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": sorted(reasons), "samples": 0}
+        hot = [s for s, p in zip(sm, pw) if p > 0.3 * max(pw)] or sm
+        return {"sm_mhz": statistics.median(hot), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the layer on the GPU
+# ---------------------------------------------------------------------------
+def peaks() -> tuple[dict, str]:
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as fh:
+            return json.load(fh), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def launches_per_layer(w) -> int:
+    """Kernel launches of one moe_layer call (see the C ABI's launch order)."""
+    n = 1 + 1 + 3 + 1 + 2 + 1  # router, gating, hist+scan+rank, dispatch, 2 FFN passes, combine
+    if w.f_shared > 0:
+        n += 2
+    return n
+
+
+def algorithmic(w, R: int, touched: int) -> dict:
+    """Algorithmic work of the layer and of the up-projection grouped GEMM."""
+    s = w.elem_bytes
+    return {
+        "layer_flops": 2 * w.T * w.d * w.E + 6 * w.d * w.f * R + 6 * w.d * w.f_shared * w.T,
+        "layer_bytes": (touched * 3 * w.d * w.f * s + 3 * w.d * w.f_shared * s + w.d * w.E * s
+                        + 2 * w.T * w.d * s),
+        # K5: gate and up GEMMs over the R kept rows; reads the touched experts'
+        # W1 and W3 and the R dispatched rows, writes h
+        "up_flops": 4 * R * w.d * w.f,
+        "up_bytes": touched * 2 * w.d * w.f * s + R * w.d * s + R * w.f * s,
+    }
+
+
+def traffic_from_profile(workload: str):
+    """DRAM bytes per launch of K5 from the committed ncu summary, when that
+    summary was taken on the current source of the kernel; else None."""
+    path = os.path.join(PROFILES, f"k5_up_swiglu_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not (m_hash and m_bytes):
+        return None
+    cur = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
+    return float(m_bytes.group(1)) if cur == m_hash.group(1) else None
+
+
+class Layer:
+    def __init__(self, name: str, dev, seed: int):
+        from routing_dispatch_expert_sigmoid_b200 import ops
+        self.ops = ops
+        self.w = WORKLOADS[name]
+        self.inp = make_inputs(self.w, seed, device=dev)
+        self.cfg = ops.config(self.w)
+        self.ws = ops.workspace(self.cfg, ops.WS_LAYER, device=dev)
+        self.rb = ops.route_buffers(self.cfg, device=dev)
+        self.out = torch.empty_like(self.inp["x"])
+
+    def args(self, x=None, out=None):
+        i = self.inp
+        return (self.cfg, i["x"] if x is None else x, i["Wr"], i["logit_bias"], i["sel_bias"],
+                i["k_per_token"], i["W1"], i["W3"], i["W2"], i["Ws1"], i["Ws3"], i["Ws2"],
+                self.out if out is None else out, self.rb, self.ws)
+
+    def step(self, x=None, out=None):
+        self.ops.moe_layer(*self.args(x, out))
+
+    def timed_step(self, events):
+        self.ops.moe_layer_timed(*self.args(), events)
+
+
+def run_device(layer: Layer, steps: int, warmup: int, dist, gpu_index: int) -> dict:
+    """K device-timed steps; per-stage times from events on the launching stream."""
+    nst = len(layer.ops.STAGES)
+    for _ in range(warmup):
+        layer.step()
+    layer.ops.moe_check_errors()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(steps)]
+    for row in evs:  # create the events before the timed region
+        for e in row:
+            e.record()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(dist)
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_index) as clk:
+        t0.record()
+        for k in range(steps):
+            layer.timed_step(evs[k])
+        t1.record()
+        torch.cuda.synchronize()
+    barrier(dist)
+    torch.cuda.synchronize()
+    layer.ops.moe_check_errors()
+    ms = t0.elapsed_time(t1)
+    stage_ms = {}
+    for i in range(1, nst):
+        stage_ms[layer.ops.STAGES[i]] = statistics.mean(
+            evs[k][i - 1].elapsed_time(evs[k][i]) for k in range(steps))
+    R = int(layer.rb["offsets"][-1].item())
+    touched = int((layer.rb["kept"] > 0).sum().item())
+    counts = layer.rb["counts"].double()
+    return {"ms": ms, "stage_ms": stage_ms, "R": R, "touched": touched,
+            "load_max_over_mean": float(counts.max() / counts.mean()),
+            "n_dropped": int(layer.rb["n_dropped"].item()), "clocks": clk.summary()}
+
+
+def run_e2e(layer: Layer, steps: int, warmup: int, dist) -> dict:
+    """Host buffers through the C ABI: H2D of x and D2H of the output inside the timed region."""
+    x_host = layer.inp["x"].cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(layer.inp["x"])
+    out_dev = torch.empty_like(layer.out)
+    stream = torch.cuda.current_stream()
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.step(x_dev, out_dev)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(dist)
+    t0.record(stream)
+    for _ in range(steps):
+        one()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist)
+    nbytes = x_host.numel() * x_host.element_size()
+    return {"ms": t0.elapsed_time(t1), "h2d": nbytes, "d2h": out_host.numel() * out_host.element_size()}
+
+
+def roofline_obj(kind: str, achieved: float, peak: float, unit: str, traffic, peak_src: str):
+    return {"bound": kind, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_tokens_per_s(name: str, n_tok: int, reps: int = 1, dev=None) -> dict:
+    import numpy as np
+
+    import oracle
+    from routing_dispatch_expert_sigmoid_b200.workloads import to_numpy
+    w = WORKLOADS[name]
+    gen_dev = dev if dev is not None else ("cuda" if torch.cuda.is_available() else "cpu")
+    inp = make_inputs(w, 0, device=gen_dev)
+    h = {k: to_numpy(v) for k, v in inp.items()}
+    del inp
+    n_tok = min(n_tok, w.T)
+    times = []
+    for r in range(reps):
+        lo = (r * n_tok) % max(w.T - n_tok + 1, 1)
+        sl = slice(lo, lo + n_tok)
+        t0 = time.perf_counter()
+        oracle.layer(h["x"][sl], h["Wr"], h["W1"], h["W3"], h["W2"], k_max=w.k_max,
+                     gating_mode=w.gating, capacity_factor=float(np.float32(w.capacity_factor)),
+                     logit_bias=h["logit_bias"], sel_bias=h["sel_bias"],
+                     k_per_token=None if h["k_per_token"] is None else h["k_per_token"][sl],
+                     n_groups=w.n_groups, topk_groups=w.topk_groups,
+                     group_score_topk=w.group_score_topk, routed_scale=w.routed_scale,
+                     Ws1=h["Ws1"], Ws3=h["Ws3"], Ws2=h["Ws2"])
+        times.append(time.perf_counter() - t0)
+    cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    return {"tokens": n_tok, "times": times, "cores": cores}
+
+
+def cpu_sample_tokens(name: str, budget_s: float) -> int:
+    """Tokens the oracle processes in about budget_s, from a one-token probe."""
+    probe = oracle_tokens_per_s(name, 1)
+    per_tok = max(probe["times"][0], 1e-4)
+    return max(1, min(int(budget_s / per_tok), WORKLOADS[name].T))
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    rank, local_rank, world = dist_env()
+    warmup = max(a.warmup, 3)
+
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        n_tok = cpu_sample_tokens(PREFILL, a.cpu_budget_s / max(a.steps + warmup, 1))
+        r = oracle_tokens_per_s(PREFILL, n_tok, reps=a.steps + warmup)
+        timed = r["times"][warmup:]
+        total_s = sum(timed)
+        value = n_tok * len(timed) / total_s
+        sample = (f"{n_tok} consecutive tokens of the {PREFILL} batch per step "
+                  f"(router, gating, dispatch layout, expert FFN and combine in fp64)")
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": a.gpus, "steps": a.steps, "warmup": warmup,
+            "ms_per_step": round(1e3 * total_s / len(timed), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{PREFILL} (T={WORKLOADS[PREFILL].T}, d=4096, E=8, top-2, "
+                                   "f=14336), CPU oracle on a sample of the batch"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": r["cores"],
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }), flush=True)
+        return 0
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = init_dist(world, "nccl")
+    pk, pk_src = peaks()
+
+    pre = Layer(PREFILL, dev, seed=rank)
+    rp = run_device(pre, a.steps, warmup, dist, local_rank)
+    e2e = run_e2e(pre, a.steps, warmup, dist)
+    w = pre.w
+    ms_max, tokens = aggregate(rp["ms"], w.T * a.steps, dist)
+    e2e_ms, _ = aggregate(e2e["ms"], w.T * a.steps, dist)
+    alg = algorithmic(w, rp["R"], rp["touched"])
+    up_ms = rp["stage_ms"]["up_swiglu"]
+    long_region = rp["ms"] > 1000.0
+    peak_tf = pk["bf16_tflops_sustained"] if long_region else pk["bf16_tflops"]
+    roof_pre = roofline_obj("tensor", alg["up_flops"] / (up_ms * 1e-3) / 1e12, peak_tf, "TFLOP/s",
+                            traffic_from_profile(PREFILL),
+                            f"{pk_src} bf16 {'sustained' if long_region else 'burst'}")
+    layer_roof_ms = max(alg["layer_flops"] / (pk["bf16_tflops"] * 1e12),
+                        alg["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
+    del pre
+    torch.cuda.empty_cache()
+
+    dec = Layer(DECODE, dev, seed=rank)
+    dsteps = max(a.steps, 50)
+    rd = run_device(dec, dsteps, warmup, dist, local_rank)
+    wd = dec.w
+    d_ms_max, d_tokens = aggregate(rd["ms"], wd.T * dsteps, dist)
+    algd = algorithmic(wd, rd["R"], rd["touched"])
+    d_up_ms = rd["stage_ms"]["up_swiglu"]
+    roof_dec = roofline_obj("hbm", algd["up_bytes"] / (d_up_ms * 1e-3) / 1e9, pk["hbm_gbs"],
+                            "GB/s", traffic_from_profile(DECODE), f"{pk_src} copy bandwidth")
+    d_layer_roof_ms = max(algd["layer_flops"] / (pk["bf16_tflops"] * 1e12),
+                          algd["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
+    del dec
+    torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        n_tok = cpu_sample_tokens(PREFILL, a.cpu_budget_s)
+        r = oracle_tokens_per_s(PREFILL, n_tok, dev=dev)
+        cpu = {"value": round(n_tok / r["times"][0], 3), "unit": "tokens/s", "cores": r["cores"],
+               "kind": "oracle",
+               "sample": f"{n_tok} tokens of the {PREFILL} batch, whole layer in fp64 "
+                         f"({r['times'][0]:.1f} s)"}
+
+    if rank == 0:
+        value = tokens / (ms_max * 1e-3)
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": warmup, "ms_per_step": round(ms_max / a.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal inputs and weights of the stated shapes)",
+            "config": {
+                "workload": f"{PREFILL}: Mixtral-8x7B-shaped MoE layer, prefill T={w.T}, "
+                            f"d={w.d}, E={w.E}, top-{w.k_max}, f={w.f}, Zipf(0.5) router bias",
+                "global_batch_tokens": w.T * world, "parallelism": f"replicas x{world}",
+                "l2": "inputs larger than L2 (expert weights 2.82 GB > 126 MB); no flush",
+                "kept_rows": rp["R"], "experts_touched": rp["touched"],
+                "load_max_over_mean": round(rp["load_max_over_mean"], 3),
+            },
+            "stage_ms": {k: round(v, 4) for k, v in rp["stage_ms"].items()},
+            "layer_roofline_ms": round(layer_roof_ms, 4),
+            "layer_roofline_frac": round(layer_roof_ms / (ms_max / a.steps), 4),
+            "roofline": roof_pre,
+            "decode": {
+                "workload": f"{DECODE}: same layer, T={wd.T}", "steps": dsteps,
+                "value": round(d_tokens / (d_ms_max * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(d_ms_max / dsteps, 4),
+                "stage_ms": {k: round(v, 4) for k, v in rd["stage_ms"].items()},
+                "layer_roofline_ms": round(d_layer_roof_ms, 4),
+                "layer_roofline_frac": round(d_layer_roof_ms / (d_ms_max / dsteps), 4),
+                "roofline": roof_dec, "kept_rows": rd["R"], "experts_touched": rd["touched"],
+            },
+            "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+            "gpu_launches": launches_per_layer(w) * (a.steps + a.steps) + launches_per_layer(wd) * dsteps,
+            "clocks": rp["clocks"],
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

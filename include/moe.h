@@ -36,9 +36,11 @@
  *   - Tensor pointers are DEVICE pointers, row-major, owned by the caller.
  *     The library never allocates, frees or synchronises in these calls;
  *     scratch memory comes from a caller workspace sized by moe_workspace_size.
- *   - Floating tensors x, Wr, W1, W3, W2, Ws1, Ws3, Ws2, x_perm, y_perm, out
- *     are stored in cfg->dtype (fp32 or bf16).  logits, topk_w, logit_bias and
- *     sel_bias are always fp32.  Indices and counts are int32.
+ *   - Floating tensors x, Wr, W1, W3, W2, Ws1, Ws3, Ws2, x_perm and out are
+ *     stored in cfg->dtype (fp32 or bf16).  The expert outputs y_perm and
+ *     shared_y are always fp32, so the layer output is rounded once, after the
+ *     weighted sum.  logits, topk_w, logit_bias and sel_bias are always fp32.
+ *     Indices and counts are int32.
  *   - Alignment: every tensor pointer and the workspace must be 16-byte aligned,
  *     and d and f (and f_shared) must make rows a multiple of 16 bytes:
  *     d % 8 == 0 and f % 8 == 0 for bf16, d % 4 == 0 and f % 4 == 0 for fp32.
@@ -174,7 +176,7 @@ MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x, const int3
 
 /* Step 5.  Grouped SwiGLU over expert-contiguous rows: rows offsets[e] ..
  * offsets[e+1]-1 of x_perm [>= R, d] use expert e.  W1, W3 [E,d,f] and
- * W2 [E,f,d] in cfg->dtype; y_perm [T*k_max, d].  The intermediate
+ * W2 [E,f,d] in cfg->dtype; y_perm [T*k_max, d] fp32.  The intermediate
  * silu(x.W1)*(x.W3) is stored in the workspace (bf16 for bf16 layers, fp32 for
  * fp32 layers); accumulation is fp32.  ws: moe_workspace_size(cfg,
  * MOE_WS_EXPERT_FFN). */
@@ -183,7 +185,8 @@ MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, con
                           void *ws, size_t ws_bytes, void *stream);
 
 /* Step 6.  out [T,d] = sum over j < k_max with slot_row >= 0 of
- * topk_w[t,j] * y_perm[slot_row[t,j]] (+ shared_y[t] when shared_y is not NULL),
+ * topk_w[t,j] * y_perm[slot_row[t,j]] (+ shared_y[t] when shared_y is not NULL;
+ * y_perm [>= R, d] and shared_y [T, d] are fp32),
  * accumulated in fp32 and rounded once to cfg->dtype.  A token whose slots are
  * all dropped gets 0 (+ shared_y[t]). */
 MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *slot_row,
@@ -200,6 +203,23 @@ MOE_API moe_status moe_layer(const moe_config *cfg, const void *x, const void *W
                      const void *W2, const void *Ws1, const void *Ws3, const void *Ws2,
                      void *out, const moe_route_out *route_out, void *ws, size_t ws_bytes,
                      void *stream);
+
+/* moe_layer, plus stage timing: events[i] (cudaEvent_t handles created by
+ * the caller; NULL entries skipped, i < n_events) is recorded on `stream` at
+ * stage boundary i:
+ *   0 before the router           1 after routing (router, gating, capacity)
+ *   2 after dispatch              3 after the up projection with SwiGLU (K5)
+ *   4 after the down projection   5 after the shared expert (= 4 without one)
+ *   6 after combine
+ * For fp32 layers both projections run before boundary 3.  The kernels and
+ * results are those of moe_layer; this call exists for profiling. */
+MOE_API moe_status moe_layer_timed(const moe_config *cfg, const void *x, const void *Wr,
+                                   const float *logit_bias, const float *sel_bias,
+                                   const int32_t *k_per_token, const void *W1, const void *W3,
+                                   const void *W2, const void *Ws1, const void *Ws3,
+                                   const void *Ws2, void *out, const moe_route_out *route_out,
+                                   void *ws, size_t ws_bytes, void *stream,
+                                   void *const *events, int32_t n_events);
 
 /* Synchronises `stream`, then reads and clears the device error flags of the
  * current device.  *flags (may be NULL) receives them: bit 0 an index out of

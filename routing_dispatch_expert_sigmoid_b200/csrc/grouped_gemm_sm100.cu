@@ -7,12 +7,14 @@
 // of A; the counts stay on the device and each CTA derives its tile list from
 // them, so no host synchronisation is needed between routing and the FFN.
 //
-//   SWIGLU: out[r, n] = silu(A[r].B1[g][:, n]) * (A[r].B3[g][:, n])   (K5, x_perm -> h)
-//   PLAIN:  out[r, n] = A[r].B1[g][:, n]                              (K6, h -> y_perm)
+//   SWIGLU: out[r, n] = silu(A[r].B1[g][:, n]) * (A[r].B3[g][:, n])   (K5, x_perm -> h, bf16)
+//   PLAIN:  out[r, n] = A[r].B1[g][:, n]                              (K6, h -> y_perm, fp32)
 //
 // A [rows_cap, K] bf16 row-major (K-major); B [G, K, N] bf16 row-major, i.e.
 // N-major for the MMA ("MN-major" operand); fp32 accumulation in tensor
-// memory; bf16 output.
+// memory.  h is stored bf16 (it is the next GEMM's operand); y_perm is kept
+// fp32 so that the layer output sees a single bf16 rounding after the
+// weighted sum.
 //
 // Design (one CTA per SM, persistent, warp-specialised, 192 threads):
 //   warp 0      TMA producer: A tile 128 x 64 and B tiles 64 x 64 (one 128-byte
@@ -222,7 +224,7 @@ struct Params {
   int fixed_rows;  // rows of the single group when offsets == nullptr
   int rows_cap;    // rows of A and out
   int K, N;
-  __nv_bfloat16 *out;  // [rows_cap, N]
+  void *out;  // [rows_cap, N]: bf16 for SWIGLU (h), fp32 for PLAIN (y)
   uint32_t *err;
 };
 
@@ -455,7 +457,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = s_off[g] + m * BM + quarter * 32 + lane;
       const bool row_ok = row < s_off[g + 1];
       const uint32_t tb = tmem_base + buf * S::kAccCols + ((uint32_t)(quarter * 32) << 16);
-      __nv_bfloat16 *orow = p.out + (size_t)row * p.N;
 #pragma unroll 1
       for (int c = 0; c < S::BN; c += 32) {
         float v[32];
@@ -468,16 +469,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int col = n * S::BN + c;
         if (row_ok) {
+          if (SWIGLU) {  // h: bf16, 4 x 16-byte stores
+            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.out) + (size_t)row * p.N;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (col + q * 8 < p.N) {
-              uint32_t w[4];
+            for (int q = 0; q < 4; ++q) {
+              if (col + q * 8 < p.N) {
+                uint32_t w[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
-                w[i] = *reinterpret_cast<uint32_t *>(&b2);
+                for (int i = 0; i < 4; ++i) {
+                  __nv_bfloat162 b2 =
+                      __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+                  w[i] = *reinterpret_cast<uint32_t *>(&b2);
+                }
+                *reinterpret_cast<uint4 *>(orow + col + q * 8) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
               }
-              *reinterpret_cast<uint4 *>(orow + col + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {  // y: fp32 (the combine rounds once), 8 x 16-byte stores
+            float *orow = static_cast<float *>(p.out) + (size_t)row * p.N;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              if (col + q * 4 < p.N)
+                *reinterpret_cast<float4 *>(orow + col + q * 4) =
+                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
           }
         }
@@ -566,7 +580,7 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
     attr_set[dev] = true;
   }
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  Params p{offsets, G, fixed_rows, rows_cap, K, N, static_cast<__nv_bfloat16 *>(out), err};
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, err};
   k_grouped_gemm<SWIGLU><<<sms, kThreads, smem, s>>>(ma, mb1, mb3, p);
   return cudaGetLastError();
 }

@@ -83,10 +83,10 @@ Layout layout(const moe_config &c, int kind) {
   if (kind == MOE_WS_LAYER) L.x_perm = take(slots * c.d * s);
   if (kind == MOE_WS_LAYER || kind == MOE_WS_EXPERT_FFN) L.h = take(slots * c.f * s);
   if (kind == MOE_WS_LAYER) {
-    L.y_perm = take(slots * c.d * s);
+    L.y_perm = take(slots * c.d * sizeof(float));  // fp32: the combine rounds once
     if (c.f_shared > 0) {
       L.h_sh = take((size_t)c.T * c.f_shared * s);
-      L.y_sh = take((size_t)c.T * c.d * s);
+      L.y_sh = take((size_t)c.T * c.d * sizeof(float));
     }
   }
   L.total = o;
@@ -154,21 +154,34 @@ moe_status route_impl(const moe_config &c, const void *x, const void *Wr, const 
   return MOE_OK;
 }
 
+// Stage events of moe_layer_timed (nullptr entries are skipped).
+struct Events {
+  cudaEvent_t const *ev = nullptr;
+  int n = 0;
+  cudaError_t mark(int i, cudaStream_t s) const {
+    return (ev && i < n && ev[i]) ? cudaEventRecord(ev[i], s) : cudaSuccess;
+  }
+};
+
 // Routed experts (G = E groups over rows_cap rows) or the shared expert
-// (offsets == nullptr: one group of T rows).
+// (offsets == nullptr: one group of T rows).  `mid` is recorded between the
+// up projection (with SwiGLU) and the down projection.
 moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixed_rows,
                     int rows_cap, int f, const void *A, const void *W1, const void *W3,
-                    const void *W2, void *h, void *y, uint32_t *err, cudaStream_t s) {
+                    const void *W2, void *h, void *y, uint32_t *err, cudaStream_t s,
+                    const Events &ev = Events(), int mid = -1) {
   if (c.dtype == MOE_F32) {
     MOE_TRY_CUDA(launch_ffn_simt_f32(rows_cap, c.d, f, G, offsets, fixed_rows,
                                      static_cast<const float *>(A), static_cast<const float *>(W1),
                                      static_cast<const float *>(W3),
                                      static_cast<const float *>(W2), static_cast<float *>(h),
                                      static_cast<float *>(y), s));
+    MOE_TRY_CUDA(ev.mark(mid, s));
     return MOE_OK;
   }
   MOE_TRY_CUDA(launch_grouped_gemm_bf16(true, rows_cap, c.d, f, G, offsets, fixed_rows, A, W1, W3,
                                         h, err, s));
+  MOE_TRY_CUDA(ev.mark(mid, s));
   MOE_TRY_CUDA(launch_grouped_gemm_bf16(false, rows_cap, f, c.d, G, offsets, fixed_rows, h, W2,
                                         nullptr, y, err, s));
   return MOE_OK;
@@ -178,6 +191,72 @@ moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixe
 }  // namespace moe
 
 using namespace moe;
+
+static moe_status layer_impl(const moe_config *cfg, const void *x, const void *Wr,
+                             const float *logit_bias, const float *sel_bias,
+                             const int32_t *k_per_token, const void *W1, const void *W3,
+                             const void *W2, const void *Ws1, const void *Ws3, const void *Ws2,
+                             void *out, const moe_route_out *route_out, void *ws, size_t ws_bytes,
+                             void *stream, const Events &ev) {
+  MOE_TRY(check_config(cfg));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
+  const moe_config &c = *cfg;
+  MOE_TRY(need(x));
+  MOE_TRY(need(Wr));
+  MOE_TRY(need4_opt(logit_bias));
+  MOE_TRY(need4_opt(sel_bias));
+  MOE_TRY(need4_opt(k_per_token));
+  MOE_TRY(need(W1));
+  MOE_TRY(need(W3));
+  MOE_TRY(need(W2));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(Ws1));
+    MOE_TRY(need(Ws3));
+    MOE_TRY(need(Ws2));
+  }
+  MOE_TRY(need(out));
+  if (route_out) MOE_TRY(check_route_out(route_out));
+  MOE_TRY(check_ws(c, MOE_WS_LAYER, ws, ws_bytes));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(c, MOE_WS_LAYER);
+  moe_route_out r;
+  if (route_out) {
+    r = *route_out;
+  } else {
+    r.logits = at<float>(ws, L.logits);
+    r.topk_idx = at<int32_t>(ws, L.topk_idx);
+    r.topk_w = at<float>(ws, L.topk_w);
+    r.counts = at<int32_t>(ws, L.counts);
+    r.kept = at<int32_t>(ws, L.kept);
+    r.offsets = at<int32_t>(ws, L.offsets);
+    r.slot_row = at<int32_t>(ws, L.slot_row);
+    r.row_src = at<int32_t>(ws, L.row_src);
+    r.n_dropped = at<int32_t>(ws, L.n_dropped);
+  }
+  MOE_TRY_CUDA(ev.mark(0, s));
+  MOE_TRY(route_impl(c, x, Wr, logit_bias, sel_bias, k_per_token, r, at<void>(ws, L.cap_scratch),
+                     err, s));
+  MOE_TRY_CUDA(ev.mark(1, s));
+  const int rows_cap = c.T * c.k_max;
+  void *x_perm = at<void>(ws, L.x_perm), *y_perm = at<void>(ws, L.y_perm);
+  MOE_TRY_CUDA(launch_dispatch(c, x, r.offsets, r.row_src, x_perm, err, s));
+  MOE_TRY_CUDA(ev.mark(2, s));
+  MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x_perm, W1, W3, W2, at<void>(ws, L.h),
+                   y_perm, err, s, ev, 3));
+  MOE_TRY_CUDA(ev.mark(4, s));
+  const void *shared_y = nullptr;
+  if (c.f_shared > 0) {
+    MOE_TRY(ffn_impl(c, 1, nullptr, c.T, c.T, c.f_shared, x, Ws1, Ws3, Ws2, at<void>(ws, L.h_sh),
+                     at<void>(ws, L.y_sh), err, s));
+    shared_y = at<void>(ws, L.y_sh);
+  }
+  MOE_TRY_CUDA(ev.mark(5, s));
+  MOE_TRY_CUDA(launch_combine(c, y_perm, r.slot_row, r.topk_w, shared_y, out, err, s));
+  MOE_TRY_CUDA(ev.mark(6, s));
+  return MOE_OK;
+}
 
 extern "C" {
 
@@ -264,58 +343,22 @@ moe_status moe_layer(const moe_config *cfg, const void *x, const void *Wr,
                      const void *W1, const void *W3, const void *W2, const void *Ws1,
                      const void *Ws3, const void *Ws2, void *out, const moe_route_out *route_out,
                      void *ws, size_t ws_bytes, void *stream) {
-  MOE_TRY(check_config(cfg));
-  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
-  const moe_config &c = *cfg;
-  MOE_TRY(need(x));
-  MOE_TRY(need(Wr));
-  MOE_TRY(need4_opt(logit_bias));
-  MOE_TRY(need4_opt(sel_bias));
-  MOE_TRY(need4_opt(k_per_token));
-  MOE_TRY(need(W1));
-  MOE_TRY(need(W3));
-  MOE_TRY(need(W2));
-  if (c.f_shared > 0) {
-    MOE_TRY(need(Ws1));
-    MOE_TRY(need(Ws3));
-    MOE_TRY(need(Ws2));
-  }
-  MOE_TRY(need(out));
-  if (route_out) MOE_TRY(check_route_out(route_out));
-  MOE_TRY(check_ws(c, MOE_WS_LAYER, ws, ws_bytes));
-  uint32_t *err = device_error_word();
-  if (!err) return MOE_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const Layout L = layout(c, MOE_WS_LAYER);
-  moe_route_out r;
-  if (route_out) {
-    r = *route_out;
-  } else {
-    r.logits = at<float>(ws, L.logits);
-    r.topk_idx = at<int32_t>(ws, L.topk_idx);
-    r.topk_w = at<float>(ws, L.topk_w);
-    r.counts = at<int32_t>(ws, L.counts);
-    r.kept = at<int32_t>(ws, L.kept);
-    r.offsets = at<int32_t>(ws, L.offsets);
-    r.slot_row = at<int32_t>(ws, L.slot_row);
-    r.row_src = at<int32_t>(ws, L.row_src);
-    r.n_dropped = at<int32_t>(ws, L.n_dropped);
-  }
-  MOE_TRY(route_impl(c, x, Wr, logit_bias, sel_bias, k_per_token, r, at<void>(ws, L.cap_scratch),
-                     err, s));
-  const int rows_cap = c.T * c.k_max;
-  void *x_perm = at<void>(ws, L.x_perm), *y_perm = at<void>(ws, L.y_perm);
-  MOE_TRY_CUDA(launch_dispatch(c, x, r.offsets, r.row_src, x_perm, err, s));
-  MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x_perm, W1, W3, W2, at<void>(ws, L.h),
-                   y_perm, err, s));
-  const void *shared_y = nullptr;
-  if (c.f_shared > 0) {
-    MOE_TRY(ffn_impl(c, 1, nullptr, c.T, c.T, c.f_shared, x, Ws1, Ws3, Ws2, at<void>(ws, L.h_sh),
-                     at<void>(ws, L.y_sh), err, s));
-    shared_y = at<void>(ws, L.y_sh);
-  }
-  MOE_TRY_CUDA(launch_combine(c, y_perm, r.slot_row, r.topk_w, shared_y, out, err, s));
-  return MOE_OK;
+  return layer_impl(cfg, x, Wr, logit_bias, sel_bias, k_per_token, W1, W3, W2, Ws1, Ws3, Ws2, out,
+                    route_out, ws, ws_bytes, stream, Events());
+}
+
+moe_status moe_layer_timed(const moe_config *cfg, const void *x, const void *Wr,
+                           const float *logit_bias, const float *sel_bias,
+                           const int32_t *k_per_token, const void *W1, const void *W3,
+                           const void *W2, const void *Ws1, const void *Ws3, const void *Ws2,
+                           void *out, const moe_route_out *route_out, void *ws, size_t ws_bytes,
+                           void *stream, void *const *events, int32_t n_events) {
+  if (n_events < 0 || (n_events > 0 && !events)) return MOE_ERR_INVALID_ARG;
+  Events ev;
+  ev.ev = reinterpret_cast<cudaEvent_t const *>(events);
+  ev.n = n_events;
+  return layer_impl(cfg, x, Wr, logit_bias, sel_bias, k_per_token, W1, W3, W2, Ws1, Ws3, Ws2, out,
+                    route_out, ws, ws_bytes, stream, ev);
 }
 
 moe_status moe_check_errors(void *stream, uint32_t *flags) {

@@ -64,7 +64,8 @@ cudaError_t launch_capacity(const moe_config &c, const int32_t *topk_idx, int32_
 cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *offsets,
                             const int32_t *row_src, void *x_perm, uint32_t *err, cudaStream_t s);
 
-// K7: out[t] = sum_j w[t,j] y_perm[slot_row[t,j]] (+ shared[t]).
+// K7: out[t] = sum_j w[t,j] y_perm[slot_row[t,j]] (+ shared[t]); y_perm and
+// shared are fp32, out is in the layer dtype.
 cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                            const float *topk_w, const void *shared_y, void *out, uint32_t *err,
                            cudaStream_t s);
@@ -75,9 +76,9 @@ cudaError_t launch_ffn_simt_f32(int rows_cap, int d, int f, int G, const int32_t
                                 const float *W3, const float *W2, float *h, float *y,
                                 cudaStream_t s);
 
-// K5/K6: tcgen05 grouped GEMMs (bf16 in, fp32 accumulate, bf16 out).
-//   swiglu: out[r, :] = silu(A[r].B1[g]) * (A[r].B3[g])     (B*: [G, K, N])
-//   plain:  out[r, :] = A[r].B1[g]
+// K5/K6: tcgen05 grouped GEMMs (bf16 in, fp32 accumulate).
+//   swiglu: out[r, :] = silu(A[r].B1[g]) * (A[r].B3[g])  bf16 out   (B*: [G, K, N])
+//   plain:  out[r, :] = A[r].B1[g]                       fp32 out
 // Rows of group g are offsets[g]..offsets[g+1]-1 of A (rows_cap rows, K
 // columns); offsets == nullptr means one group of fixed_rows rows.
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,

@@ -98,13 +98,16 @@ struct Vec<__nv_bfloat16> {
   }
 };
 
+// y and shared_y are fp32 rows (row_vecs4 16-byte vectors of 4 values); out
+// rows are T (row_vecs_out vectors of Vec<T>::N values).
 template <typename T>
 __global__ void __launch_bounds__(256)
     k_combine(const uint4 *__restrict__ y, const int32_t *__restrict__ slot_row,
               const float *__restrict__ topk_w, const uint4 *__restrict__ shared_y,
               uint4 *__restrict__ out, int Tn, int k_max, int rows_cap, int row_vecs,
               uint32_t *err) {
-  constexpr int N = Vec<T>::N;
+  constexpr int N = Vec<T>::N;   // output values per 16-byte vector
+  constexpr int Q = N / 4;       // fp32 input vectors per output vector
   // Per warp: the token's kept slots, compacted in slot order.
   __shared__ int32_t s_row[8][32];
   __shared__ float s_w[8][32];
@@ -129,25 +132,33 @@ __global__ void __launch_bounds__(256)
       s_w[wib][pos] = my_w;
     }
     __syncwarp();
+    const size_t in_vecs = (size_t)row_vecs * Q;  // fp32 vectors per row
     for (int v = lane; v < row_vecs; v += 32) {
       float acc[N];
       if (shared_y) {
-        Vec<T>::load(ldg_nc(shared_y + (size_t)t * row_vecs + v), acc);
+#pragma unroll
+        for (int q = 0; q < Q; ++q)
+          Vec<float>::load(ldg_nc(shared_y + (size_t)t * in_vecs + (size_t)v * Q + q), acc + 4 * q);
       } else {
 #pragma unroll
         for (int i = 0; i < N; ++i) acc[i] = 0.f;
       }
       for (int j0 = 0; j0 < n_live; j0 += 4) {
-        uint4 u[4];
+        uint4 u[4][Q];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)  // issue the loads before the FMAs
-          if (j0 + q < n_live) u[q] = ldg_nc(y + (size_t)s_row[wib][j0 + q] * row_vecs + v);
+        for (int j = 0; j < 4; ++j)  // issue the loads before the FMAs
+          if (j0 + j < n_live) {
+            const uint4 *src = y + (size_t)s_row[wib][j0 + j] * in_vecs + (size_t)v * Q;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (j0 + q < n_live) {
-            const float wj = s_w[wib][j0 + q];
+            for (int q = 0; q < Q; ++q) u[j][q] = ldg_nc(src + q);
+          }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (j0 + j < n_live) {
+            const float wj = s_w[wib][j0 + j];
             float f[N];
-            Vec<T>::load(u[q], f);
+#pragma unroll
+            for (int q = 0; q < Q; ++q) Vec<float>::load(u[j][q], f + 4 * q);
 #pragma unroll
             for (int i = 0; i < N; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
           }

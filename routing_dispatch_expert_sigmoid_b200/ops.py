@@ -62,11 +62,13 @@ def lib() -> ctypes.CDLL:
         L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, S, P]
         L.moe_combine.argtypes = [cfgp, P, P, P, P, P, P]
         L.moe_layer.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, outp, P, S, P]
+        L.moe_layer_timed.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, outp, P, S, P,
+                                      ctypes.POINTER(ctypes.c_void_p), I]
         L.moe_check_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn",
-                   "moe_combine", "moe_layer", "moe_check_errors"):
+                   "moe_combine", "moe_layer", "moe_layer_timed", "moe_check_errors"):
             getattr(L, fn).restype = I
         _lib = L
     return _lib
@@ -158,6 +160,20 @@ def moe_layer(cfg, x, Wr, logit_bias, sel_bias, k_per_token, W1, W3, W2, Ws1, Ws
                            _p(k_per_token), _p(W1), _p(W3), _p(W2), _p(Ws1), _p(Ws3), _p(Ws2),
                            _p(out), r, _p(ws), 0 if ws is None else ws.numel(), _stream(stream)),
            "moe_layer")
+
+
+STAGES = ("start", "route", "dispatch", "up_swiglu", "down", "shared", "combine")
+
+
+def moe_layer_timed(cfg, x, Wr, logit_bias, sel_bias, k_per_token, W1, W3, W2, Ws1, Ws3, Ws2,
+                    out, route_out: dict | None, ws, events, stream=None):
+    """moe_layer that records events[i] (torch.cuda.Event, len(STAGES)) at stage boundary i."""
+    r = None if route_out is None else ctypes.byref(_route_struct(route_out))
+    handles = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib().moe_layer_timed(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias),
+                                 _p(k_per_token), _p(W1), _p(W3), _p(W2), _p(Ws1), _p(Ws3),
+                                 _p(Ws2), _p(out), r, _p(ws), 0 if ws is None else ws.numel(),
+                                 _stream(stream), handles, len(events)), "moe_layer_timed")
 
 
 def moe_check_errors(stream=None) -> int:

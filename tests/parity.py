@@ -7,7 +7,13 @@ Tolerances (written here once, used by every test):
   - router logits: max-abs error <= 1e-4 x RMS of the fp64 logits;
   - gate weights: |w_gpu - w_oracle| <= 1e-5 (fp32 softmax/sigmoid sums vs fp64);
   - layer / FFN outputs: max-abs error <= 2e-2 x RMS(reference) and relative
-    Frobenius error <= 5e-3 (bf16 storage, fp32 accumulation).
+    Frobenius error <= 5e-3 (bf16 storage, fp32 accumulation).  The max-abs
+    bound is on the error beyond the rounding of the result to its storage
+    type: elementwise |got - ref| <= 2e-2 x RMS(ref) + half an ulp of the
+    storage type at ref.  A correctly rounded bf16 copy of the exact output
+    is already off by up to 2^-8 of |ref| just above a power of two, which
+    exceeds 2e-2 x RMS on heavy-tailed outputs (2.1% measured on a case with
+    many dropped tokens); the Frobenius bound is applied as stated.
 """
 from __future__ import annotations
 
@@ -35,17 +41,31 @@ def assert_logits_close(gpu_logits, ref64):
     assert err <= LOGIT_TOL * rms, f"logits max-abs {err:.3e} > {LOGIT_TOL} x RMS {rms:.3e}"
 
 
-def assert_out_close(got, ref, what="output"):
+def half_ulp(ref, storage):
+    """Half an ulp of the storage type (bf16: 8 significant bits, fp32: 24) at |ref|."""
+    bits = {"bf16": 8, "f32": 24}[storage]
+    e = np.floor(np.log2(np.maximum(np.abs(ref), np.finfo(np.float64).tiny)))
+    return np.exp2(e - bits)
+
+
+def assert_out_close(got, ref, what="output", storage="bf16"):
     got = got if isinstance(got, np.ndarray) else f64(got)
     if ref.size == 0:
         return
     diff = got - ref
     rms = np.sqrt(np.mean(ref ** 2))
-    max_abs = np.abs(diff).max()
+    excess = (np.abs(diff) - half_ulp(ref, storage)).max()
     frob = np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300)
     assert np.isfinite(got).all(), f"{what}: non-finite values"
-    assert max_abs <= OUT_MAXABS * rms, f"{what}: max-abs {max_abs:.3e} > {OUT_MAXABS} x RMS {rms:.3e}"
-    assert frob <= OUT_FROB, f"{what}: relative Frobenius {frob:.3e} > {OUT_FROB}"
+    msg = (f"{what}: max-abs beyond {storage} rounding / RMS {excess / rms:.3e} (bound "
+           f"{OUT_MAXABS}; raw max-abs/RMS {np.abs(diff).max() / rms:.3e}), "
+           f"relative Frobenius {frob:.3e} (bound {OUT_FROB})")
+    assert excess <= OUT_MAXABS * rms and frob <= OUT_FROB, msg
+    return excess / rms, frob
+
+
+def storage(w: Workload) -> str:
+    return "f32" if w.dtype == "f32" else "bf16"
 
 
 def oracle_cf(w: Workload) -> float:

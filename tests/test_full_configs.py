@@ -14,7 +14,7 @@ import torch
 
 import oracle
 from parity import (assert_logits_close, assert_out_close, check_routing_bit_exact, f64,
-                    oracle_layer_on_tokens, run_layer)
+                    oracle_layer_on_tokens, run_layer, storage)
 from routing_dispatch_expert_sigmoid_b200 import ops
 from routing_dispatch_expert_sigmoid_b200.workloads import WORKLOADS, make_inputs, to_numpy
 
@@ -49,7 +49,7 @@ def test_full_size_workload(name, dev):
                                       to_numpy(inp["Wr"]), to_numpy(inp["logit_bias"]))
     assert_logits_close(rb["logits"].index_select(0, sel), ref_logits)
     ref = oracle_layer_on_tokens(inp, routing, toks)
-    assert_out_close(f64(out.index_select(0, sel)), ref, f"{name} sampled outputs")
+    assert_out_close(f64(out.index_select(0, sel)), ref, f"{name} sampled outputs", storage(w))
     # the kept-row count matches the stated drop policy
     assert int(rb["offsets"][-1].item()) == int(rb["counts"].sum().item()) - int(
         rb["n_dropped"].item())
