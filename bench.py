@@ -212,10 +212,10 @@ def traffic_from_profile(workload: str):
 
 
 class Layer:
-    def __init__(self, name: str, dev, seed: int):
+    def __init__(self, name: str, dev, seed: int, T: int = 0):
         from routing_dispatch_expert_sigmoid_b200 import ops
         self.ops = ops
-        self.w = WORKLOADS[name]
+        self.w = WORKLOADS[name] if T <= 0 else WORKLOADS[name].scaled(T=T)
         self.inp = make_inputs(self.w, seed, device=dev)
         self.cfg = ops.config(self.w)
         self.ws = ops.workspace(self.cfg, ops.WS_LAYER, device=dev)
@@ -331,14 +331,17 @@ def oracle_tokens_per_s(name: str, n_tok: int, reps: int = 1, dev=None) -> dict:
                      group_score_topk=w.group_score_topk, routed_scale=w.routed_scale,
                      Ws1=h["Ws1"], Ws3=h["Ws3"], Ws2=h["Ws2"])
         times.append(time.perf_counter() - t0)
-    cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
-    return {"tokens": n_tok, "times": times, "cores": cores}
+    threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    # the oracle parallelises the FFN over tokens: it keeps min(tokens, threads) cores busy
+    return {"tokens": n_tok, "times": times, "cores": min(threads, n_tok)}
 
 
 def cpu_sample_tokens(name: str, budget_s: float) -> int:
-    """Tokens the oracle processes in about budget_s, from a one-token probe."""
-    probe = oracle_tokens_per_s(name, 1)
-    per_tok = max(probe["times"][0], 1e-4)
+    """Tokens the oracle processes in about budget_s on all host cores, from a
+    probe of one token per core."""
+    cores = len(os.sched_getaffinity(0))
+    probe = oracle_tokens_per_s(name, cores)
+    per_tok = max(probe["times"][0] / cores, 1e-4)
     return max(1, min(int(budget_s / per_tok), WORKLOADS[name].T))
 
 
@@ -351,6 +354,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default=PREFILL, choices=sorted(WORKLOADS),
+                    help="workload of the main (prefill) leg")
+    ap.add_argument("--T", type=int, default=0, help="override the main leg's token count")
+    ap.add_argument("--decode-workload", default=DECODE,
+                    choices=sorted(WORKLOADS) + ["none"], help="workload of the decode leg")
     a = ap.parse_args()
     rank, local_rank, world = dist_env()
     warmup = max(a.warmup, 3)
@@ -358,7 +367,8 @@ def main():
     if a.impl == "reference":
         if rank != 0:
             return 0
-        n_tok = cpu_sample_tokens(PREFILL, a.cpu_budget_s / max(a.steps + warmup, 1))
+        cores = len(os.sched_getaffinity(0))
+        n_tok = max(cores, cpu_sample_tokens(PREFILL, a.cpu_budget_s / max(a.steps + warmup, 1)))
         r = oracle_tokens_per_s(PREFILL, n_tok, reps=a.steps + warmup)
         timed = r["times"][warmup:]
         total_s = sum(timed)
@@ -385,45 +395,59 @@ def main():
     dist = init_dist(world, "nccl")
     pk, pk_src = peaks()
 
-    pre = Layer(PREFILL, dev, seed=rank)
+    pre = Layer(a.workload, dev, seed=rank, T=a.T)
     rp = run_device(pre, a.steps, warmup, dist, local_rank)
-    e2e = run_e2e(pre, a.steps, warmup, dist)
+    e2e = None if a.no_e2e else run_e2e(pre, a.steps, warmup, dist)
     w = pre.w
     ms_max, tokens = aggregate(rp["ms"], w.T * a.steps, dist)
-    e2e_ms, _ = aggregate(e2e["ms"], w.T * a.steps, dist)
+    e2e_ms = None if e2e is None else aggregate(e2e["ms"], w.T * a.steps, dist)[0]
     alg = algorithmic(w, rp["R"], rp["touched"])
     up_ms = rp["stage_ms"]["up_swiglu"]
     long_region = rp["ms"] > 1000.0
     peak_tf = pk["bf16_tflops_sustained"] if long_region else pk["bf16_tflops"]
     roof_pre = roofline_obj("tensor", alg["up_flops"] / (up_ms * 1e-3) / 1e12, peak_tf, "TFLOP/s",
-                            traffic_from_profile(PREFILL),
+                            traffic_from_profile(a.workload) if a.T <= 0 else None,
                             f"{pk_src} bf16 {'sustained' if long_region else 'burst'}")
     layer_roof_ms = max(alg["layer_flops"] / (pk["bf16_tflops"] * 1e12),
                         alg["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
     del pre
     torch.cuda.empty_cache()
 
-    dec = Layer(DECODE, dev, seed=rank)
-    dsteps = max(a.steps, 50)
-    rd = run_device(dec, dsteps, warmup, dist, local_rank)
-    wd = dec.w
-    d_ms_max, d_tokens = aggregate(rd["ms"], wd.T * dsteps, dist)
-    algd = algorithmic(wd, rd["R"], rd["touched"])
-    d_up_ms = rd["stage_ms"]["up_swiglu"]
-    roof_dec = roofline_obj("hbm", algd["up_bytes"] / (d_up_ms * 1e-3) / 1e9, pk["hbm_gbs"],
-                            "GB/s", traffic_from_profile(DECODE), f"{pk_src} copy bandwidth")
-    d_layer_roof_ms = max(algd["layer_flops"] / (pk["bf16_tflops"] * 1e12),
-                          algd["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
-    del dec
-    torch.cuda.empty_cache()
+    dec_obj = None
+    if a.decode_workload != "none":
+        dec = Layer(a.decode_workload, dev, seed=rank)
+        dsteps = max(a.steps, 50)
+        rd = run_device(dec, dsteps, warmup, dist, local_rank)
+        wd = dec.w
+        d_ms_max, d_tokens = aggregate(rd["ms"], wd.T * dsteps, dist)
+        algd = algorithmic(wd, rd["R"], rd["touched"])
+        d_up_ms = rd["stage_ms"]["up_swiglu"]
+        roof_dec = roofline_obj("hbm", algd["up_bytes"] / (d_up_ms * 1e-3) / 1e9, pk["hbm_gbs"],
+                                "GB/s", traffic_from_profile(a.decode_workload),
+                                f"{pk_src} copy bandwidth")
+        d_layer_roof_ms = max(algd["layer_flops"] / (pk["bf16_tflops"] * 1e12),
+                              algd["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
+        dec_obj = {
+            "workload": f"{a.decode_workload}: T={wd.T}, d={wd.d}, E={wd.E}, top-{wd.k_max}, "
+                        f"f={wd.f}", "steps": dsteps,
+            "value": round(d_tokens / (d_ms_max * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(d_ms_max / dsteps, 4),
+            "stage_ms": {k: round(v, 4) for k, v in rd["stage_ms"].items()},
+            "layer_roofline_ms": round(d_layer_roof_ms, 4),
+            "layer_roofline_frac": round(d_layer_roof_ms / (d_ms_max / dsteps), 4),
+            "roofline": roof_dec, "kept_rows": rd["R"], "experts_touched": rd["touched"],
+            "gpu_launches": launches_per_layer(wd) * dsteps,
+        }
+        del dec
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        n_tok = cpu_sample_tokens(PREFILL, a.cpu_budget_s)
-        r = oracle_tokens_per_s(PREFILL, n_tok, dev=dev)
+        n_tok = cpu_sample_tokens(a.workload, a.cpu_budget_s)
+        r = oracle_tokens_per_s(a.workload, n_tok, dev=dev)
         cpu = {"value": round(n_tok / r["times"][0], 3), "unit": "tokens/s", "cores": r["cores"],
                "kind": "oracle",
-               "sample": f"{n_tok} tokens of the {PREFILL} batch, whole layer in fp64 "
+               "sample": f"{n_tok} tokens of the {a.workload} batch, whole layer in fp64 "
                          f"({r['times'][0]:.1f} s)"}
 
     if rank == 0:
@@ -434,29 +458,25 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded normal inputs and weights of the stated shapes)",
             "config": {
-                "workload": f"{PREFILL}: Mixtral-8x7B-shaped MoE layer, prefill T={w.T}, "
-                            f"d={w.d}, E={w.E}, top-{w.k_max}, f={w.f}, Zipf(0.5) router bias",
+                "workload": f"{a.workload}: T={w.T}, d={w.d}, E={w.E}, top-{w.k_max}, f={w.f}"
+                            + (f", shared f={w.f_shared}" if w.f_shared else "")
+                            + f", {w.gating}, capacity factor {w.capacity_factor or 'none'}",
                 "global_batch_tokens": w.T * world, "parallelism": f"replicas x{world}",
-                "l2": "inputs larger than L2 (expert weights 2.82 GB > 126 MB); no flush",
+                "l2": "inputs larger than L2 (expert weights > 126 MB L2); no flush",
                 "kept_rows": rp["R"], "experts_touched": rp["touched"],
                 "load_max_over_mean": round(rp["load_max_over_mean"], 3),
+                "n_dropped": rp["n_dropped"],
             },
             "stage_ms": {k: round(v, 4) for k, v in rp["stage_ms"].items()},
             "layer_roofline_ms": round(layer_roof_ms, 4),
             "layer_roofline_frac": round(layer_roof_ms / (ms_max / a.steps), 4),
             "roofline": roof_pre,
-            "decode": {
-                "workload": f"{DECODE}: same layer, T={wd.T}", "steps": dsteps,
-                "value": round(d_tokens / (d_ms_max * 1e-3), 1), "unit": "tokens/s",
-                "ms_per_step": round(d_ms_max / dsteps, 4),
-                "stage_ms": {k: round(v, 4) for k, v in rd["stage_ms"].items()},
-                "layer_roofline_ms": round(d_layer_roof_ms, 4),
-                "layer_roofline_frac": round(d_layer_roof_ms / (d_ms_max / dsteps), 4),
-                "roofline": roof_dec, "kept_rows": rd["R"], "experts_touched": rd["touched"],
-            },
-            "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
-                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
-            "gpu_launches": launches_per_layer(w) * (a.steps + a.steps) + launches_per_layer(wd) * dsteps,
+            "decode": dec_obj,
+            "e2e": None if e2e is None else {
+                "value": round(tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+            "gpu_launches": (launches_per_layer(w) * a.steps * (1 if e2e is None else 2)
+                             + (dec_obj["gpu_launches"] if dec_obj else 0)),
             "clocks": rp["clocks"],
             "cpu_baseline": cpu,
         }

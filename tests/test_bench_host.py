@@ -1,0 +1,92 @@
+"""Host-side logic of bench.py, on the CPU: the whole-job aggregation over
+ranks (world size 2, gloo), the roofline bookkeeping and the clock parser.
+The layer itself has no collective: ranks are independent replicas, and the
+only cross-rank traffic is the control-plane max/sum done here."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from routing_dispatch_expert_sigmoid_b200.workloads import WORKLOADS  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist = bench.init_dist(world, "gloo")
+    ms, units = bench.aggregate(10.0 + 5.0 * rank, 1000 * (rank + 1), dist)
+    bench.barrier(dist)
+    q.put((rank, ms, units))
+    dist.destroy_process_group()
+
+
+def test_aggregate_max_time_sum_units_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # every rank sees the slowest rank's time and the job's total units
+    assert [r[1] for r in res] == [15.0, 15.0]
+    assert [r[2] for r in res] == [3000, 3000]
+
+
+def test_aggregate_single_process():
+    assert bench.aggregate(7.5, 42, None) == (7.5, 42)
+
+
+def test_launch_count_and_algorithmic_work():
+    w = WORKLOADS["mixtral_prefill"]
+    assert bench.launches_per_layer(w) == 9
+    assert bench.launches_per_layer(WORKLOADS["dsv3_prefill"]) == 11
+    a = bench.algorithmic(w, R=16384, touched=8)
+    assert a["up_flops"] == 4 * 16384 * 4096 * 14336
+    assert a["layer_flops"] == 2 * 8192 * 4096 * 8 + 6 * 4096 * 14336 * 16384
+    assert a["layer_bytes"] == 8 * 3 * 4096 * 14336 * 2 + 4096 * 8 * 2 + 2 * 8192 * 4096 * 2
+
+
+def test_traffic_only_for_the_profiled_kernel_source(tmp_path, monkeypatch):
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    import hashlib
+    h = hashlib.sha256(b"kernel v1").hexdigest()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "k5_up_swiglu_demo.md").write_text(
+        f"dram_bytes_per_launch: 1.5e+09\nkernel_source_sha256: {h}\n")
+    monkeypatch.setattr(bench, "PROFILES", str(prof))
+    monkeypatch.setattr(bench, "GEMM_SRC", str(src))
+    assert bench.traffic_from_profile("demo") == 1.5e9
+    src.write_text("kernel v2")  # the kernel changed since the counters were taken
+    assert bench.traffic_from_profile("demo") is None
+    assert bench.traffic_from_profile("missing") is None
+
+
+def test_clock_summary_parses_reasons():
+    c = bench.ClockSampler(0)
+    import tempfile
+    c.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+    c.file.write("0, 1920, 1965, 900.1, 0x4, Not Active, Not Active, Not Active, Active\n"
+                 "0, 1900, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active\n"
+                 "0, 600, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    c.file.flush()
+    s = c.summary()
+    assert s["sm_mhz"] == pytest.approx(1910.0) and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
