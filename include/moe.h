@@ -169,6 +169,25 @@ MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *W
                      const int32_t *k_per_token, const moe_route_out *out, void *ws,
                      size_t ws_bytes, void *stream);
 
+/* moe_route without a workspace argument, for callers that cannot give this
+ * library scratch memory (a plugin interface that passes only inputs and
+ * outputs, a runtime whose device memory is fully planned in advance, a path
+ * that must not call an allocator).  The pages have no counterpart: this is
+ * an interface convenience, not a step of the method.  Results are those of
+ * moe_route.  The scratch of the capacity step lives in a fixed 1 MiB device
+ * array inside this library, held on every GPU that loads it until exit; a
+ * configuration that needs more (8 * ceil(T*k_max/1024) * E bytes rounded up
+ * to a multiple of 256, plus 256) is rejected with MOE_ERR_WORKSPACE before
+ * anything is enqueued.  No
+ * call allocates or frees memory.  The first call on a device looks up the
+ * array's device address with that device current.  All calls share the
+ * array, so calls whose work overlaps on the GPU (other streams or host
+ * threads on the same device) race; serialise them. */
+MOE_API moe_status moe_route_static_scratch(const moe_config *cfg, const void *x,
+                                            const void *Wr, const float *logit_bias,
+                                            const float *sel_bias, const int32_t *k_per_token,
+                                            const moe_route_out *out, void *stream);
+
 /* Step 4.  x [T,d] -> x_perm [T*k_max, d]: x_perm[r] = x[row_src[r] / k_max]
  * for r < offsets[E]; rows past R are left untouched. */
 MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *offsets,

@@ -288,6 +288,61 @@ moe_status moe_route(const moe_config *cfg, const void *x, const void *Wr,
                     err, static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------------------
+// Routing without a caller workspace.
+//
+// Some callers cannot hand this library device memory for scratch: a plugin
+// interface whose fixed signature carries only inputs and outputs, a runtime
+// with a static memory plan in which every byte of HBM is already assigned
+// (weights, caches) and a stray cudaMalloc would fail or fragment the pool, or
+// a latency-critical path that must not pay for an allocator call.  For them,
+// moe_route_static_scratch keeps the capacity step's scratch (per-chunk
+// expert histograms and their prefix sums) in the fixed device array below.
+//
+// The array is kStaticScratchBytes (1 MiB) on every GPU that loads this
+// library, held until the process exits.  In host code its name is only a
+// stand-in for the device symbol, so the device address is looked up with
+// cudaGetSymbolAddress, once per device, with that device current, on the
+// first call made on that device.  Every call shares the array: two calls
+// whose work overlaps on the GPU (different streams, or different host
+// threads on one device) race on it.  Nothing in it needs to start at zero:
+// each call writes every scratch element before reading it.
+static constexpr size_t kStaticScratchBytes = 1u << 20;
+static __device__ __align__(256) unsigned char g_route_scratch[kStaticScratchBytes];
+
+static void *route_scratch_address() {
+  static void *addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+moe_status moe_route_static_scratch(const moe_config *cfg, const void *x, const void *Wr,
+                                    const float *logit_bias, const float *sel_bias,
+                                    const int32_t *k_per_token, const moe_route_out *out,
+                                    void *stream) {
+  MOE_TRY(check_config(cfg));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
+  const moe_config &c = *cfg;
+  MOE_TRY(need(x));
+  MOE_TRY(need(Wr));
+  MOE_TRY(need4_opt(logit_bias));
+  MOE_TRY(need4_opt(sel_bias));
+  MOE_TRY(need4_opt(k_per_token));
+  MOE_TRY(check_route_out(out));
+  if (capacity_scratch_bytes(c) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
+  void *scratch = route_scratch_address();
+  uint32_t *err = device_error_word();
+  if (!scratch || !err) return MOE_ERR_CUDA;
+  return route_impl(c, x, Wr, logit_bias, sel_bias, k_per_token, *out, scratch, err,
+                    static_cast<cudaStream_t>(stream));
+}
+
 moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *offsets,
                         const int32_t *row_src, void *x_perm, void *stream) {
   MOE_TRY(check_config(cfg));

@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
         outp = ctypes.POINTER(MoeRouteOut)
         L.moe_workspace_size.argtypes = [cfgp, I, ctypes.POINTER(S)]
         L.moe_route.argtypes = [cfgp, P, P, P, P, P, outp, P, S, P]
+        L.moe_route_static_scratch.argtypes = [cfgp, P, P, P, P, P, outp, P]
         L.moe_dispatch.argtypes = [cfgp, P, P, P, P, P]
         L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, S, P]
         L.moe_combine.argtypes = [cfgp, P, P, P, P, P, P]
@@ -67,7 +68,8 @@ def lib() -> ctypes.CDLL:
         L.moe_check_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
-        for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn",
+        for fn in ("moe_workspace_size", "moe_route", "moe_route_static_scratch", "moe_dispatch",
+                   "moe_expert_ffn",
                    "moe_combine", "moe_layer", "moe_layer_timed", "moe_check_errors"):
             getattr(L, fn).restype = I
         _lib = L
@@ -135,6 +137,16 @@ def moe_route(cfg, x, Wr, logit_bias, sel_bias, k_per_token, out: dict, ws, stre
     _check(lib().moe_route(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias),
                            _p(k_per_token), ctypes.byref(r), _p(ws),
                            0 if ws is None else ws.numel(), _stream(stream)), "moe_route")
+
+
+def moe_route_static_scratch(cfg, x, Wr, logit_bias, sel_bias, k_per_token, out: dict,
+                             stream=None):
+    """moe_route for callers that cannot provide a workspace: the library's
+    fixed device scratch is used instead (see include/moe.h)."""
+    r = _route_struct(out)
+    _check(lib().moe_route_static_scratch(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias),
+                                          _p(sel_bias), _p(k_per_token), ctypes.byref(r),
+                                          _stream(stream)), "moe_route_static_scratch")
 
 
 def moe_dispatch(cfg, x, offsets, row_src, x_perm, stream=None):
