@@ -224,27 +224,30 @@ struct Params {
   int fixed_rows;  // rows of the single group when offsets == nullptr
   int rows_cap;    // rows of A and out
   int K, N;
-  void *out;  // [rows_cap, N]: bf16 for SWIGLU (h), fp32 for PLAIN (y)
+  void *out;  // [rows_cap, N]: bf16 for SWIGLU (h), fp32 for PLAIN (y, logits)
+  const float *bias;  // PLAIN only: [N] added to every row (router logit bias), or nullptr
   uint32_t *err;
 };
 
-template <bool SWIGLU>
+template <bool SWIGLU, int SPANS>
 struct Shape {
-  static constexpr int BN = SWIGLU ? 128 : 256;       // output columns per tile
-  static constexpr int kSpans = BN / 64;              // 64-column spans per B operand
+  static constexpr int kSpans = SPANS;                // 64-column spans per B operand
+  static constexpr int BN = 64 * SPANS;               // output columns per tile
   static constexpr int kBOps = SWIGLU ? 2 : 1;
   static constexpr uint32_t kABytes = BM * BK * 2;    // 16 KB
   static constexpr uint32_t kSpanBytes = BK * 128;    // 8 KB: 64 K-rows x 128 B
-  static constexpr uint32_t kBBytes = kBOps * kSpans * kSpanBytes;  // 32 KB
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes;        // 48 KB
-  static constexpr int kStages = 4;
+  static constexpr uint32_t kBBytes = kBOps * kSpans * kSpanBytes;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  // as many stages as fit in ~192 KB of the ring, at most 8
+  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
   static constexpr int kMmaN = kBOps * BN;            // 256
   static constexpr uint32_t kAccCols = kMmaN;         // fp32 columns per accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccCols; // 512
   static constexpr uint32_t kIdesc = instr_desc(BM, kMmaN);
   static constexpr size_t kSmemFixed = 1024 /*align slack*/ + kStages * kStageBytes + 256;
   static_assert(kMmaN % 16 == 0 && kMmaN <= 256, "UMMA N");
-  static_assert(kTmemCols <= 512, "TMEM");
+  static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
+                "TMEM allocation: a power of two in [32, 512] columns");
 };
 
 __device__ __forceinline__ void tile_of(int tile, const int32_t *s_tstart, const int32_t *s_off,
@@ -265,11 +268,11 @@ __device__ __forceinline__ void tile_of(int tile, const int32_t *s_tstart, const
   m = local - n * mt;
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, int SPANS>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
                    const __grid_constant__ CUtensorMap tmB3, const Params p) {
-  using S = Shape<SWIGLU>;
+  using S = Shape<SWIGLU, SPANS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -485,13 +488,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_uint4(w[0], w[1], w[2], w[3]);
               }
             }
-          } else {  // y: fp32 (the combine rounds once), 8 x 16-byte stores
+          } else {  // fp32 (+ bias), 8 x 16-byte stores
             float *orow = static_cast<float *>(p.out) + (size_t)row * p.N;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              if (col + q * 4 < p.N)
-                *reinterpret_cast<float4 *>(orow + col + q * 4) =
-                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              if (col + q * 4 < p.N) {
+                float4 o = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                if (p.bias) {  // the bias is only 4-byte aligned: scalar loads
+                  const float *b = p.bias + col + q * 4;
+                  o.x += b[0];
+                  o.y += b[1];
+                  o.z += b[2];
+                  o.w += b[3];
+                }
+                *reinterpret_cast<float4 *>(orow + col + q * 4) = o;
+              }
             }
           }
         }
@@ -559,11 +570,11 @@ bool make_map_b(CUtensorMap *m, const void *B, int G, int K, int N) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, int SPANS>
 cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, int fixed_rows,
-                   const void *A, const void *B1, const void *B3, void *out, uint32_t *err,
-                   cudaStream_t s) {
-  using S = Shape<SWIGLU>;
+                   const void *A, const void *B1, const void *B3, void *out, const float *bias,
+                   uint32_t *err, cudaStream_t s) {
+  using S = Shape<SWIGLU, SPANS>;
   CUtensorMap ma, mb1, mb3;
   if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
       !make_map_b(&mb3, SWIGLU ? B3 : B1, G, K, N))
@@ -574,14 +585,18 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
   static bool attr_set[64] = {};  // per device
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(
-        k_grouped_gemm<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        k_grouped_gemm<SWIGLU, SPANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
         (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, err};
-  k_grouped_gemm<SWIGLU><<<sms, kThreads, smem, s>>>(ma, mb1, mb3, p);
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, bias, err};
+  // never more CTAs than tiles can exist (a group holds at most rows_cap rows)
+  const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
+                              ((N + S::BN - 1) / S::BN);
+  const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
+  k_grouped_gemm<SWIGLU, SPANS><<<grid, kThreads, smem, s>>>(ma, mb1, mb3, p);
   return cudaGetLastError();
 }
 
@@ -593,9 +608,21 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                      cudaStream_t s) {
   if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if (rows_cap == 0) return cudaSuccess;
-  return swiglu ? tc::launch<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out, err, s)
-                : tc::launch<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out, err,
-                                    s);
+  return swiglu ? tc::launch<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
+                                      nullptr, err, s)
+                : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
+                                       nullptr, err, s);
+}
+
+cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,
+                             const float *bias, float *logits, uint32_t *err, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  // one group of T rows; B = Wr viewed as [1, d, E]; tile width follows E
+  if (E <= 64)
+    return tc::launch<false, 1>(T, d, E, 1, nullptr, T, x, Wr, Wr, logits, bias, err, s);
+  if (E <= 128)
+    return tc::launch<false, 2>(T, d, E, 1, nullptr, T, x, Wr, Wr, logits, bias, err, s);
+  return tc::launch<false, 4>(T, d, E, 1, nullptr, T, x, Wr, Wr, logits, bias, err, s);
 }
 
 }  // namespace moe

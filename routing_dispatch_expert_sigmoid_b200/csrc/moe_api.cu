@@ -147,7 +147,16 @@ T *at(void *ws, size_t off) {
 moe_status route_impl(const moe_config &c, const void *x, const void *Wr, const float *logit_bias,
                       const float *sel_bias, const int32_t *k_per_token, const moe_route_out &o,
                       void *cap_scratch, uint32_t *err, cudaStream_t s) {
-  MOE_TRY_CUDA(launch_router(c, x, Wr, logit_bias, o.logits, s));
+  // The router is a dense contraction: bf16 layers whose logit rows are a
+  // multiple of 16 bytes (E % 8 == 0, a TMA stride rule) run it on the tensor
+  // cores (its epilogue writes 16-byte vectors, so the logits buffer must be
+  // 16-byte aligned too); fp32 layers keep plain fp32 FMA (TF32 would miss
+  // the logit tolerance).
+  if (c.dtype == MOE_BF16 && c.E % 8 == 0 && aligned16(o.logits)) {
+    MOE_TRY_CUDA(launch_router_tc(c.T, c.d, c.E, x, Wr, logit_bias, o.logits, err, s));
+  } else {
+    MOE_TRY_CUDA(launch_router(c, x, Wr, logit_bias, o.logits, s));
+  }
   MOE_TRY_CUDA(launch_gating(c, o.logits, sel_bias, k_per_token, o.topk_idx, o.topk_w, err, s));
   MOE_TRY_CUDA(launch_capacity(c, o.topk_idx, o.counts, o.kept, o.offsets, o.slot_row, o.row_src,
                                o.n_dropped, cap_scratch, err, s));

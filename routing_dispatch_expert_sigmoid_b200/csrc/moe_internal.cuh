@@ -86,4 +86,9 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                      const void *B1, const void *B3, void *out, uint32_t *err,
                                      cudaStream_t s);
 
+// K1 on the tensor cores (bf16 layers with E % 8 == 0): logits[T,E] =
+// x[T,d] . Wr[d,E] (+ bias), fp32 accumulation in tensor memory, fp32 out.
+cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,
+                             const float *bias, float *logits, uint32_t *err, cudaStream_t s);
+
 }  // namespace moe
