@@ -24,7 +24,9 @@
 //               hands finished accumulators to the epilogue;
 //   warps 2-5   epilogue: tcgen05.ld of the 128 x 256 fp32 accumulator (warp w
 //               reads TMEM lanes 32*(w%4)...), SiLU-gate multiply for K5,
-//               bf16 conversion, masked 16-byte stores of the group's rows.
+//               bf16 conversion; each 32 x 32 chunk is staged in shared
+//               memory and written back row-wise (whole 64/128-byte row
+//               segments per warp store), masked to the group's rows.
 // The accumulator is double-buffered in tensor memory (2 x 256 columns) so
 // the epilogue of one tile overlaps the main loop of the next.
 // For SWIGLU the W1 and W3 tiles of the same 128 output columns sit next to
@@ -244,7 +246,13 @@ struct Shape {
   static constexpr uint32_t kAccCols = kMmaN;         // fp32 columns per accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccCols; // 512
   static constexpr uint32_t kIdesc = instr_desc(BM, kMmaN);
-  static constexpr size_t kSmemFixed = 1024 /*align slack*/ + kStages * kStageBytes + 256;
+  // epilogue staging: per epilogue warp a 32-row x 32-column fp32 chunk, rows
+  // padded to 36 words so both the row-wise writes and the column-wise reads
+  // are free of bank conflicts
+  static constexpr uint32_t kStageRowWords = 36;
+  static constexpr uint32_t kEpiBytes = 4 * 32 * kStageRowWords * 4;  // 18 KB
+  static constexpr size_t kSmemFixed =
+      1024 /*align slack*/ + kStages * kStageBytes + 256 + kEpiBytes;
   static_assert(kMmaN % 16 == 0 && kMmaN <= 256, "UMMA N");
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                 "TMEM allocation: a power of two in [32, 512] columns");
@@ -281,7 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // bars: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain[1]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S::kStages + 5);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kStages * S::kStageBytes + 256);
+  float *s_epi = reinterpret_cast<float *>(ring + S::kStages * S::kStageBytes + 256);
+  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kStages * S::kStageBytes + 256 +
+                                               S::kEpiBytes);
   int32_t *s_tstart = s_off + (p.G + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -457,11 +467,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ready = __shfl_sync(0xffffffffu, ready, 0);
       if (!ready) break;
       tc_fence_after();
-      const int row = s_off[g] + m * BM + quarter * 32 + lane;
-      const bool row_ok = row < s_off[g + 1];
+      // This warp owns rows row0 .. row0+31 of the tile (TMEM lanes 32*quarter ..).
+      const int row0 = s_off[g] + m * BM + quarter * 32;
+      const int row_end = s_off[g + 1];
       const uint32_t tb = tmem_base + buf * S::kAccCols + ((uint32_t)(quarter * 32) << 16);
+      float *stg = s_epi + (warp - 2) * 32 * S::kStageRowWords;
 #pragma unroll 1
       for (int c = 0; c < S::BN; c += 32) {
+        // lane = row: 32 consecutive columns of its row from tensor memory
         float v[32];
         tmem_ld32(tb + c, v);
         if (SWIGLU) {
@@ -471,41 +484,56 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
         }
         const int col = n * S::BN + c;
-        if (row_ok) {
-          if (SWIGLU) {  // h: bf16, 4 x 16-byte stores
-            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.out) + (size_t)row * p.N;
+        // Stage the 32 x 32 chunk in shared memory, then write it back row by
+        // row so that each warp store covers whole 64/128-byte row segments.
+        if (SWIGLU) {  // h: bf16, a row is 16 words
+          uint32_t *st = reinterpret_cast<uint32_t *>(stg);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (col + q * 8 < p.N) {
-                uint32_t w[4];
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  __nv_bfloat162 b2 =
-                      __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
-                  w[i] = *reinterpret_cast<uint32_t *>(&b2);
-                }
-                *reinterpret_cast<uint4 *>(orow + col + q * 8) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-              }
+            for (int i = 0; i < 4; ++i) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+              w[i] = *reinterpret_cast<uint32_t *>(&b2);
             }
-          } else {  // fp32 (+ bias), 8 x 16-byte stores
-            float *orow = static_cast<float *>(p.out) + (size_t)row * p.N;
+            *reinterpret_cast<uint4 *>(st + lane * S::kStageRowWords + 4 * q) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          __syncwarp();
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              if (col + q * 4 < p.N) {
-                float4 o = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                if (p.bias) {  // the bias is only 4-byte aligned: scalar loads
-                  const float *b = p.bias + col + q * 4;
-                  o.x += b[0];
-                  o.y += b[1];
-                  o.z += b[2];
-                  o.w += b[3];
-                }
-                *reinterpret_cast<float4 *>(orow + col + q * 4) = o;
+          for (int i = 0; i < 4; ++i) {  // 8 rows x 64 bytes per instruction
+            const int r = i * 8 + (lane >> 2), q = lane & 3;
+            const int grow = row0 + r, gcol = col + q * 8;
+            const uint4 val = *reinterpret_cast<const uint4 *>(st + r * S::kStageRowWords + 4 * q);
+            if (grow < row_end && gcol < p.N)
+              *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) +
+                                         (size_t)grow * p.N + gcol) = val;
+          }
+        } else {  // fp32 (+ bias), a row is 32 words
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4 *>(stg + lane * S::kStageRowWords + 4 * q) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {  // 4 rows x 128 bytes per instruction
+            const int r = i * 4 + (lane >> 3), q = lane & 7;
+            const int grow = row0 + r, gcol = col + q * 4;
+            float4 o = *reinterpret_cast<const float4 *>(stg + r * S::kStageRowWords + 4 * q);
+            if (grow < row_end && gcol < p.N) {
+              if (p.bias) {  // the bias is only 4-byte aligned: scalar loads
+                const float *b = p.bias + gcol;
+                o.x += b[0];
+                o.y += b[1];
+                o.z += b[2];
+                o.w += b[3];
               }
+              *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)grow * p.N +
+                                          gcol) = o;
             }
           }
         }
+        __syncwarp();  // the next chunk overwrites the staging buffer
       }
       tc_fence_before();
       __syncwarp();

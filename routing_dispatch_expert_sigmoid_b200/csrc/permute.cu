@@ -9,9 +9,9 @@
 // on one GPU, so they are a gather into expert-contiguous rows and a weighted
 // gather back.
 //
-// Both kernels are HBM-bound row copies: one warp per row (dispatch) or per
-// token (combine), 16-byte vector loads and stores, rows of d*s bytes with
-// d*s a multiple of 16.  The number of rows R lives on the device
+// Both kernels are HBM-bound row copies with 16-byte vector loads and stores
+// (rows of d*s bytes, d*s a multiple of 16); a warp takes a chunk of one row
+// (dispatch) or of one token's output (combine) at a time.  The number of rows R lives on the device
 // (offsets[E]); a fixed grid strides over the row space and stops at R.
 #include "moe_internal.cuh"
 
@@ -26,6 +26,10 @@ __device__ __forceinline__ uint4 ldg_nc(const uint4 *p) {
   return v;
 }
 
+// Work items are (row, 2 KB chunk of the row): a batch of a few rows still
+// spreads over the whole GPU, a large one keeps every warp on long streams.
+constexpr int kChunkVecs = 128;  // 16-byte vectors per chunk (4 per lane)
+
 __global__ void __launch_bounds__(256)
     k_dispatch(const uint4 *__restrict__ x, const int32_t *__restrict__ offsets,
                const int32_t *__restrict__ row_src, uint4 *__restrict__ x_perm, int E,
@@ -36,8 +40,12 @@ __global__ void __launch_bounds__(256)
     R = R < 0 ? 0 : rows_cap;
   }
   const int lane = threadIdx.x % 32;
-  const int warps = gridDim.x * (blockDim.x / 32);
-  for (int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; row < R; row += warps) {
+  const int chunks = (row_vecs + kChunkVecs - 1) / kChunkVecs;
+  const long long items = (long long)R * chunks;
+  const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+  for (long long it = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; it < items;
+       it += warps) {
+    const int row = (int)(it / chunks), ch = (int)(it % chunks);
     const int a = row_src[row];
     const int t = a / k_max;
     if (a < 0 || t >= T) {
@@ -46,16 +54,14 @@ __global__ void __launch_bounds__(256)
     }
     const uint4 *src = x + (size_t)t * row_vecs;
     uint4 *dst = x_perm + (size_t)row * row_vecs;
-    int v = lane;
-    for (; v + 96 < row_vecs; v += 128) {
-      const uint4 a0 = ldg_nc(src + v), a1 = ldg_nc(src + v + 32);
-      const uint4 a2 = ldg_nc(src + v + 64), a3 = ldg_nc(src + v + 96);
-      dst[v] = a0;
-      dst[v + 32] = a1;
-      dst[v + 64] = a2;
-      dst[v + 96] = a3;
-    }
-    for (; v < row_vecs; v += 32) dst[v] = ldg_nc(src + v);
+    const int v0 = ch * kChunkVecs + lane;
+    uint4 u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (v0 + 32 * i < row_vecs) u[i] = ldg_nc(src + v0 + 32 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (v0 + 32 * i < row_vecs) dst[v0 + 32 * i] = u[i];
   }
 }
 
@@ -98,22 +104,27 @@ struct Vec<__nv_bfloat16> {
   }
 };
 
-// y and shared_y are fp32 rows (row_vecs4 16-byte vectors of 4 values); out
-// rows are T (row_vecs_out vectors of Vec<T>::N values).
+// y and shared_y are fp32 rows (Q 16-byte vectors per output vector); out
+// rows are T (row_vecs vectors of Vec<T>::N values).  Work items are (token,
+// 32 consecutive output vectors): lane l of the item's warp owns one output
+// vector and sums the token's kept slots for it in slot order.
 template <typename T>
 __global__ void __launch_bounds__(256)
     k_combine(const uint4 *__restrict__ y, const int32_t *__restrict__ slot_row,
               const float *__restrict__ topk_w, const uint4 *__restrict__ shared_y,
               uint4 *__restrict__ out, int Tn, int k_max, int rows_cap, int row_vecs,
               uint32_t *err) {
-  constexpr int N = Vec<T>::N;   // output values per 16-byte vector
-  constexpr int Q = N / 4;       // fp32 input vectors per output vector
-  // Per warp: the token's kept slots, compacted in slot order.
+  constexpr int N = Vec<T>::N;  // output values per 16-byte vector
+  constexpr int Q = N / 4;      // fp32 input vectors per output vector
   __shared__ int32_t s_row[8][32];
   __shared__ float s_w[8][32];
   const int lane = threadIdx.x % 32, wib = threadIdx.x / 32;
-  const int warps = gridDim.x * (blockDim.x / 32);
-  for (int t = blockIdx.x * (blockDim.x / 32) + wib; t < Tn; t += warps) {
+  const int chunks = (row_vecs + 31) / 32;
+  const long long items = (long long)Tn * chunks;
+  const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+  const size_t in_vecs = (size_t)row_vecs * Q;  // fp32 vectors per row
+  for (long long it = (long long)blockIdx.x * (blockDim.x / 32) + wib; it < items; it += warps) {
+    const int t = (int)(it / chunks), ch = (int)(it % chunks);
     int my_row = -1;
     float my_w = 0.f;
     if (lane < k_max) {
@@ -126,14 +137,14 @@ __global__ void __launch_bounds__(256)
     }
     const unsigned live = __ballot_sync(0xffffffffu, my_row >= 0);
     const int n_live = __popc(live);
-    if (my_row >= 0) {
+    if (my_row >= 0) {  // compact the kept slots, in slot order
       const int pos = __popc(live & ((1u << lane) - 1u));
       s_row[wib][pos] = my_row;
       s_w[wib][pos] = my_w;
     }
     __syncwarp();
-    const size_t in_vecs = (size_t)row_vecs * Q;  // fp32 vectors per row
-    for (int v = lane; v < row_vecs; v += 32) {
+    const int v = ch * 32 + lane;
+    if (v < row_vecs) {
       float acc[N];
       if (shared_y) {
 #pragma unroll
@@ -188,7 +199,8 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *o
   const int rows_cap = c.T * c.k_max;
   if (rows_cap == 0) return cudaSuccess;
   const int row_vecs = c.d * esz / 16;
-  k_dispatch<<<grid_for(rows_cap), 256, 0, s>>>(
+  const long long items = (long long)rows_cap * ((row_vecs + kChunkVecs - 1) / kChunkVecs);
+  k_dispatch<<<grid_for(items), 256, 0, s>>>(
       static_cast<const uint4 *>(x), offsets, row_src, static_cast<uint4 *>(x_perm), c.E,
       c.k_max, c.T, rows_cap, row_vecs, err);
   return cudaGetLastError();
@@ -201,7 +213,7 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
   const int esz = c.dtype == MOE_F32 ? 4 : 2;
   const int row_vecs = c.d * esz / 16;
   const int rows_cap = c.T * c.k_max;
-  const int grid = grid_for(c.T);
+  const int grid = grid_for((long long)c.T * ((row_vecs + 31) / 32));
   if (c.dtype == MOE_F32)
     k_combine<float><<<grid, 256, 0, s>>>(
         static_cast<const uint4 *>(y_perm), slot_row, topk_w,
