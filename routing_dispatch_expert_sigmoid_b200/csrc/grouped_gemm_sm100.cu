@@ -44,6 +44,7 @@
 // waits (again bounded) for its own copies and MMAs in flight, frees its
 // tensor memory and returns.  No TMA multicast is used.
 #include <cuda.h>
+#include <stdlib.h>
 
 #include "moe_internal.cuh"
 
@@ -552,6 +553,433 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// The same grouped GEMM on CTA pairs (tcgen05 cta_group::2)
+//
+// A cluster of two CTAs (two SMs of one TPC) computes a 256-row tile: CTA r
+// loads rows r*128.. of the tile's A and half of the B columns (SWIGLU: CTA 0
+// the W1 span pair, CTA 1 the W3 span pair; PLAIN: columns r*128..r*128+127
+// of the 256), so each SM streams 32 KB per k-block instead of 48 KB and the
+// same shared-memory ring covers 1.5 times the tensor-core time.  CTA 0 (the
+// leader) issues one M=256, N=256, K=16 MMA per step for both SMs; each
+// CTA's tensor memory receives its own 128 rows of the accumulator.
+// Barriers: both CTAs' TMA loads complete on the leader's "full" barrier
+// (cta_group::2 form), the leader's commits arrive on "empty" and
+// "accumulator full" in both CTAs (cluster multicast of the commit, not of
+// any load), and both CTAs' epilogue warps arrive on the leader's
+// "accumulator empty" barrier.
+// ---------------------------------------------------------------------------
+constexpr int BM2 = 256;  // rows per pair tile
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map,
+                                                 uint32_t leader_bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(leader_bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap *map,
+                                                 uint32_t leader_bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(leader_bar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   slot_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` (same shared-memory offset) in both CTAs of the pair when
+// every tcgen05 operation issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\t"
+      "mov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], m;\n\t}\n" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_self(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+template <bool SWIGLU>
+struct Shape2 {
+  static constexpr int BN = SWIGLU ? 128 : 256;       // output columns per tile
+  static constexpr int kSpansPerCta = 2;              // 64-column B spans each CTA loads
+  static constexpr uint32_t kABytes = 128 * BK * 2;   // 16 KB: this CTA's 128 rows
+  static constexpr uint32_t kSpanBytes = BK * 128;    // 8 KB
+  static constexpr uint32_t kBBytes = kSpansPerCta * kSpanBytes;  // 16 KB
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;      // 32 KB per CTA
+  static constexpr int kStages = 6;
+  static constexpr int kMmaN = 256;                   // N of the pair instruction
+  static constexpr uint32_t kAccCols = 256;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kIdesc = instr_desc(BM2, kMmaN);
+  static constexpr uint32_t kStageRowWords = 36;
+  static constexpr uint32_t kEpiBytes = 4 * 32 * kStageRowWords * 4;
+  static constexpr size_t kSmemFixed =
+      1024 + kStages * kStageBytes + 256 + kEpiBytes;
+};
+
+template <bool SWIGLU>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB1,
+                        const __grid_constant__ CUtensorMap tmB3, const Params p) {
+  using S = Shape2<SWIGLU>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *ring = smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + S::kStages * S::kStageBytes);
+  // bars: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain[1]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S::kStages + 5);
+  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+  float *s_epi = reinterpret_cast<float *>(ring + S::kStages * S::kStageBytes + 256);
+  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kStages * S::kStageBytes + 256 +
+                                               S::kEpiBytes);
+  int32_t *s_tstart = s_off + (p.G + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x / 2, npairs = gridDim.x / 2;
+  const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + S::kStages);
+  const uint32_t accf0 = smem_addr(bars + 2 * S::kStages);
+  const uint32_t acce0 = smem_addr(bars + 2 * S::kStages + 2);
+  const uint32_t drain = smem_addr(bars + 2 * S::kStages + 4);
+  const Ctl ctl{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);   // the leader's arrive.expect_tx (both CTAs' bytes)
+      mbar_init(empty0 + 8 * s, 1);  // the leader's multicast commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf0 + 8 * b, 1);   // the leader's multicast commit
+      mbar_init(acce0 + 8 * b, 8);   // 4 epilogue warps x 2 CTAs (leader's copy is used)
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB1);
+    if (SWIGLU) prefetch_tmap(&tmB3);
+  }
+  bool bad = false;
+  for (int g = threadIdx.x; g <= p.G; g += kThreads) {
+    const int v = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.fixed_rows);
+    s_off[g] = v;
+    if (v < 0 || v > p.rows_cap) bad = true;
+  }
+  if (warp == 1) tmem_alloc_pair(smem_addr(tmem_slot), S::kTmemCols);
+  __syncthreads();
+  const int n_tiles = (p.N + S::BN - 1) / S::BN;
+  for (int g = threadIdx.x; g < p.G; g += kThreads) {
+    const int rows = s_off[g + 1] - s_off[g];
+    if (rows < 0) bad = true;
+    s_tstart[g] = rows > 0 ? ((rows + BM2 - 1) / BM2) * n_tiles : 0;
+  }
+  if (bad) {
+    *abort_flag = 1;
+    raise_error(p.err, kErrIndex);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < p.G; base += 32) {
+      const int g = base + lane;
+      const int v = g < p.G ? s_tstart[g] : 0;
+      int incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (g < p.G) s_tstart[g] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_tstart[p.G] = carry;
+  }
+  if (warp == 1) tmem_relinquish_pair();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // Both CTAs see the same offsets, so they agree on the tile list; a CTA
+  // that found bad offsets stops, and its peer's waits time out.
+  const int total = *abort_flag ? 0 : s_tstart[p.G];
+  const int num_kb = (p.K + BK - 1) / BK;
+  const uint32_t leader_full0 = mapa_shared(full0, 0);
+  const uint32_t leader_acce0 = mapa_shared(acce0, 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producers (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        int g, m, n;
+        {
+          int lo = 0, hi = p.G - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+          }
+          g = lo;
+          const int mt = (s_off[g + 1] - s_off[g] + BM2 - 1) / BM2;
+          const int local = tile - s_tstart[g];
+          n = local / mt;
+          m = local - n * mt;
+        }
+        const int row = s_off[g] + m * BM2 + (int)rank * 128;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+          const uint32_t lfb = leader_full0 + 8 * s;
+          if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * S::kStageBytes);
+          tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
+          if (SWIGLU) {
+            const CUtensorMap *mb = rank == 0 ? &tmB1 : &tmB3;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb,
+                               n * S::BN + j * 64, kb * BK, g);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, &tmB1, lfb,
+                               n * S::BN + (int)rank * 128 + j * 64, kb * BK, g);
+          }
+          ++issued;
+          if (++s == S::kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok && issued > 0) {
+        // Stopped early.  The leader waits for the stages it armed; both CTAs'
+        // copies complete there.  The peer gives its copies a moment to land.
+        if (rank == 0) {
+          for (int q = 0; q < S::kStages && q < issued; ++q) {
+            int st_i = s - 1 - q;
+            uint32_t par = ph;
+            if (st_i < 0) {
+              st_i += S::kStages;
+              par ^= 1;
+            }
+            wait_drain(full0 + 8 * st_i, par, p.err);
+          }
+        } else {
+          const uint64_t t0 = global_timer();
+          while (global_timer() - t0 < 2000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (rank == 0 && lane == 0) {
+      int s = 0, buf = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool ok = true, any = false;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        if (!wait(acce0 + 8 * buf, acc_ph ^ 1, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * S::kAccCols;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait(full0 + 8 * s, ph, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc(st + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc(st + S::kABytes + kk * 2048, S::kSpanBytes, 1024);
+            umma_pair(d_tmem, ad, bd, S::kIdesc, (kb | kk) != 0);
+          }
+          any = true;
+          umma_commit_pair_both(empty0 + 8 * s);
+          if (++s == S::kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_both(accf0 + 8 * buf);
+        buf ^= 1;
+        if (buf == 0) acc_ph ^= 1;
+      }
+      if (!ok && any) {
+        umma_commit_pair_self(drain);
+        wait_drain(drain, 0, p.err);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    int buf = 0;
+    uint32_t acc_ph = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      int g, m, n;
+      {
+        int lo = 0, hi = p.G - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+        }
+        g = lo;
+        const int mt = (s_off[g + 1] - s_off[g] + BM2 - 1) / BM2;
+        const int local = tile - s_tstart[g];
+        n = local / mt;
+        m = local - n * mt;
+      }
+      int ready = 0;
+      if (lane == 0) ready = wait(accf0 + 8 * buf, acc_ph, ctl) ? 1 : 0;
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (!ready) break;
+      tc_fence_after();
+      const int row0 = s_off[g] + m * BM2 + (int)rank * 128 + quarter * 32;
+      const int row_end = s_off[g + 1];
+      const uint32_t tb = tmem_base + buf * S::kAccCols + ((uint32_t)(quarter * 32) << 16);
+      float *stg = s_epi + (warp - 2) * 32 * S::kStageRowWords;
+#pragma unroll 1
+      for (int c = 0; c < S::BN; c += 32) {
+        float v[32];
+        tmem_ld32(tb + c, v);
+        if (SWIGLU) {
+          float u[32];
+          tmem_ld32(tb + S::BN + c, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
+        }
+        const int col = n * S::BN + c;
+        if (SWIGLU) {
+          uint32_t *st = reinterpret_cast<uint32_t *>(stg);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+              w[i] = *reinterpret_cast<uint32_t *>(&b2);
+            }
+            *reinterpret_cast<uint4 *>(st + lane * S::kStageRowWords + 4 * q) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = i * 8 + (lane >> 2), q = lane & 3;
+            const int grow = row0 + r, gcol = col + q * 8;
+            const uint4 val = *reinterpret_cast<const uint4 *>(st + r * S::kStageRowWords + 4 * q);
+            if (grow < row_end && gcol < p.N)
+              *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) +
+                                         (size_t)grow * p.N + gcol) = val;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4 *>(stg + lane * S::kStageRowWords + 4 * q) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = i * 4 + (lane >> 3), q = lane & 7;
+            const int grow = row0 + r, gcol = col + q * 4;
+            float4 o = *reinterpret_cast<const float4 *>(stg + r * S::kStageRowWords + 4 * q);
+            if (grow < row_end && gcol < p.N) {
+              if (p.bias) {
+                const float *b = p.bias + gcol;
+                o.x += b[0];
+                o.y += b[1];
+                o.z += b[2];
+                o.w += b[3];
+              }
+              *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)grow * p.N +
+                                          gcol) = o;
+            }
+          }
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(acce0 + 8 * buf);
+        else
+          mbar_arrive_cluster(leader_acce0 + 8 * buf);
+      }
+      buf ^= 1;
+      if (buf == 0) acc_ph ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the pair's MMAs may still use its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, S::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -628,7 +1056,49 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
   return cudaGetLastError();
 }
 
+template <bool SWIGLU>
+cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offsets,
+                        int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
+                        uint32_t *err, cudaStream_t s) {
+  using S = Shape2<SWIGLU>;
+  CUtensorMap ma, mb1, mb3;
+  if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
+      !make_map_b(&mb3, SWIGLU ? B3 : B1, G, K, N))
+    return cudaErrorInvalidValue;
+  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool attr_set[64] = {};
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(
+        k_grouped_gemm_pair<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, err};
+  const long long max_tiles = (long long)((rows_cap + BM2 - 1) / BM2 + (offsets ? G : 0)) *
+                              ((N + S::BN - 1) / S::BN);
+  long long pairs = sms / 2;
+  if (max_tiles < pairs) pairs = max_tiles < 1 ? 1 : max_tiles;
+  k_grouped_gemm_pair<SWIGLU><<<(int)(2 * pairs), kThreads, smem, s>>>(ma, mb1, mb3, p);
+  return cudaGetLastError();
+}
+
 }  // namespace tc
+
+// CTA pairs pay off when groups are large: a pair tile is 256 rows, so a
+// group's last tile wastes up to 255 rows instead of 127.  The host knows the
+// mean rows per group (the true counts live on the device); MOE_GEMM_PAIR=0/1
+// forces one engine (tests run both on every shape).
+static bool use_pair_tiles(int rows_cap, int G, const int32_t *offsets, int fixed_rows) {
+  const char *env = getenv("MOE_GEMM_PAIR");
+  if (env && env[0] == '0') return false;
+  if (env && env[0] == '1') return true;
+  const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
+  return mean_rows >= 2048;
+}
 
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
                                      const int32_t *offsets, int fixed_rows, const void *A,
@@ -636,6 +1106,19 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                      cudaStream_t s) {
   if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if (rows_cap == 0) return cudaSuccess;
+  if (use_pair_tiles(rows_cap, G, offsets, fixed_rows))
+    return swiglu ? tc::launch_pair<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
+                                          err, s)
+                  : tc::launch_pair<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
+                                           out, err, s);
+  // Decode-sized groups (a few rows each) stream weights: every tile costs
+  // the same, so the tile count decides how evenly the last wave fills the
+  // GPU.  Half-width up-projection tiles (64 columns of gate and of up)
+  // double the count and shrink that tail.
+  const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
+  if (swiglu && mean_rows <= 32)
+    return tc::launch<true, 1>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out, nullptr,
+                               err, s);
   return swiglu ? tc::launch<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
                                       nullptr, err, s)
                 : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
