@@ -301,6 +301,19 @@ def run_e2e(layer: Layer, steps: int, warmup: int, dist) -> dict:
     return {"ms": t0.elapsed_time(t1), "h2d": nbytes, "d2h": out_host.numel() * out_host.element_size()}
 
 
+def kernel_roofline(alg: dict, ms: float, peak_tf: float, peak_gbs: float, traffic, tf_src: str,
+                    bw_src: str) -> dict:
+    """Roofline of K5: bound by whichever of its algorithmic FLOPs at the bf16
+    peak or its algorithmic bytes at the HBM peak takes longer."""
+    t_flops = alg["up_flops"] / (peak_tf * 1e12)
+    t_bytes = alg["up_bytes"] / (peak_gbs * 1e9)
+    if t_flops >= t_bytes:
+        return roofline_obj("tensor", alg["up_flops"] / (ms * 1e-3) / 1e12, peak_tf, "TFLOP/s",
+                            traffic, tf_src)
+    return roofline_obj("hbm", alg["up_bytes"] / (ms * 1e-3) / 1e9, peak_gbs, "GB/s", traffic,
+                        bw_src)
+
+
 def roofline_obj(kind: str, achieved: float, peak: float, unit: str, traffic, peak_src: str):
     return {"bound": kind, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src}
@@ -409,9 +422,10 @@ def main():
     # power cap (or for more than a second); the burst figure otherwise.
     sustained = rp["ms"] > 1000.0 or "sw_power_cap" in rp["clocks"]["reasons"]
     peak_tf = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
-    roof_pre = roofline_obj("tensor", alg["up_flops"] / (up_ms * 1e-3) / 1e12, peak_tf, "TFLOP/s",
-                            traffic_from_profile(a.workload) if a.T <= 0 else None,
-                            f"{pk_src} bf16 {'sustained' if sustained else 'burst'}")
+    roof_pre = kernel_roofline(alg, up_ms, peak_tf, pk["hbm_gbs"],
+                               traffic_from_profile(a.workload) if a.T <= 0 else None,
+                               f"{pk_src} bf16 {'sustained' if sustained else 'burst'}",
+                               f"{pk_src} copy bandwidth")
     layer_roof_ms = max(alg["layer_flops"] / (pk["bf16_tflops"] * 1e12),
                         alg["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
     del pre
@@ -426,9 +440,11 @@ def main():
         d_ms_max, d_tokens = aggregate(rd["ms"], wd.T * dsteps, dist)
         algd = algorithmic(wd, rd["R"], rd["touched"])
         d_up_ms = rd["stage_ms"]["up_swiglu"]
-        roof_dec = roofline_obj("hbm", algd["up_bytes"] / (d_up_ms * 1e-3) / 1e9, pk["hbm_gbs"],
-                                "GB/s", traffic_from_profile(a.decode_workload),
-                                f"{pk_src} copy bandwidth")
+        sustained_d = "sw_power_cap" in rd["clocks"]["reasons"]
+        roof_dec = kernel_roofline(
+            algd, d_up_ms, pk["bf16_tflops_sustained"] if sustained_d else pk["bf16_tflops"],
+            pk["hbm_gbs"], traffic_from_profile(a.decode_workload),
+            f"{pk_src} bf16 {'sustained' if sustained_d else 'burst'}", f"{pk_src} copy bandwidth")
         d_layer_roof_ms = max(algd["layer_flops"] / (pk["bf16_tflops"] * 1e12),
                               algd["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
         dec_obj = {
