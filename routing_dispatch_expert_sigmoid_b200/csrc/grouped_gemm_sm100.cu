@@ -980,6 +980,334 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Small groups: the same products with the operands swapped ("swap-AB")
+//
+// When most groups hold a few rows (decode, or thousands of fine-grained
+// experts), a 128-row tile is mostly padding.  Here a tile is 128 output
+// columns x at most 128 rows of one group: the weights are the MMA's M
+// operand (MN-major, the same 64 x 64 TMA boxes as above), the group's rows
+// are its N operand (K-major, loaded in 32-row boxes, only as many as the tile
+// has rows), and N is the row count rounded up to 16, set per tile in the
+// instruction descriptor.  Tensor memory then holds the transposed tile
+// (lane = output column, column = row); the epilogue transposes it back
+// through its shared-memory stage.
+//   SWIGLU: two MMAs per step, gate = W1^T.x^T and up = W3^T.x^T, into TMEM
+//           columns [0,128) and [128,256) of the accumulator buffer;
+//   PLAIN:  one MMA per step, y^T = W^T.h^T.
+// ---------------------------------------------------------------------------
+constexpr int kRowBox = 32;  // rows per TMA box of the N operand
+
+template <bool SWIGLU>
+struct ShapeSwap {
+  static constexpr int kCols = 128;                      // output columns per tile (MMA M)
+  static constexpr int kMaxRows = 128;                   // rows per tile (MMA N <= 128)
+  static constexpr int kWOps = SWIGLU ? 2 : 1;
+  static constexpr uint32_t kSpanBytes = BK * 128;       // 8 KB: 64 K-rows x 64 columns
+  static constexpr uint32_t kWBytes = kWOps * 2 * kSpanBytes;   // 16 or 32 KB
+  static constexpr uint32_t kRowBoxBytes = kRowBox * BK * 2;    // 4 KB
+  static constexpr uint32_t kXBytes = kMaxRows * BK * 2;        // 16 KB
+  static constexpr uint32_t kStageBytes = kWBytes + kXBytes;
+  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  static constexpr uint32_t kAccCols = SWIGLU ? 256 : 128;
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;
+  static constexpr uint32_t kStageRowWords = 36;
+  static constexpr uint32_t kEpiBytes = 4 * 32 * kStageRowWords * 4;
+  static constexpr size_t kSmemFixed = 1024 + kStages * kStageBytes + 256 + kEpiBytes;
+};
+
+// kind::f16 descriptor: fp32 accumulator, bf16 A and B, A MN-major, B K-major.
+__device__ __forceinline__ uint32_t instr_desc_swap(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_grouped_gemm_swap(const __grid_constant__ CUtensorMap tmX,
+                        const __grid_constant__ CUtensorMap tmW1,
+                        const __grid_constant__ CUtensorMap tmW3, const Params p) {
+  using S = ShapeSwap<SWIGLU>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *ring = smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + S::kStages * S::kStageBytes);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S::kStages + 5);
+  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+  float *s_epi = reinterpret_cast<float *>(ring + S::kStages * S::kStageBytes + 256);
+  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kStages * S::kStageBytes + 256 +
+                                               S::kEpiBytes);
+  int32_t *s_tstart = s_off + (p.G + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + S::kStages);
+  const uint32_t accf0 = smem_addr(bars + 2 * S::kStages);
+  const uint32_t acce0 = smem_addr(bars + 2 * S::kStages + 2);
+  const uint32_t drain = smem_addr(bars + 2 * S::kStages + 4);
+  const Ctl ctl{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf0 + 8 * b, 1);
+      mbar_init(acce0 + 8 * b, 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmW1);
+    if (SWIGLU) prefetch_tmap(&tmW3);
+  }
+  bool bad = false;
+  for (int g = threadIdx.x; g <= p.G; g += kThreads) {
+    const int v = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.fixed_rows);
+    s_off[g] = v;
+    if (v < 0 || v > p.rows_cap) bad = true;
+  }
+  if (warp == 1) tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
+  __syncthreads();
+  const int col_tiles = (p.N + S::kCols - 1) / S::kCols;
+  for (int g = threadIdx.x; g < p.G; g += kThreads) {
+    const int rows = s_off[g + 1] - s_off[g];
+    if (rows < 0) bad = true;
+    s_tstart[g] = rows > 0 ? ((rows + S::kMaxRows - 1) / S::kMaxRows) * col_tiles : 0;
+  }
+  if (bad) {
+    *abort_flag = 1;
+    raise_error(p.err, kErrIndex);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < p.G; base += 32) {
+      const int g = base + lane;
+      const int v = g < p.G ? s_tstart[g] : 0;
+      int incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (g < p.G) s_tstart[g] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_tstart[p.G] = carry;
+  }
+  if (warp == 1) tmem_relinquish();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = *abort_flag ? 0 : s_tstart[p.G];
+  const int num_kb = (p.K + BK - 1) / BK;
+
+  // tile -> (group g, column tile c, row tile r); rows fastest, so CTAs
+  // running together share a weight tile
+  auto tile_coords = [&](int tile, int &g, int &c, int &r, int &row0, int &nr) {
+    int lo = 0, hi = p.G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const int rows = s_off[g + 1] - s_off[g];
+    const int rt = (rows + S::kMaxRows - 1) / S::kMaxRows;
+    const int local = tile - s_tstart[g];
+    c = local / rt;
+    r = local - c * rt;
+    row0 = s_off[g] + r * S::kMaxRows;
+    nr = min(S::kMaxRows, rows - r * S::kMaxRows);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int g, c, r, row0, nr;
+        tile_coords(tile, g, c, r, row0, nr);
+        const int boxes = (nr + kRowBox - 1) / kRowBox;
+        const uint32_t bytes = S::kWBytes + boxes * S::kRowBoxBytes;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+          const uint32_t fb = full0 + 8 * s;
+          mbar_expect_tx(fb, bytes);
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            tma_load_3d(st + j * S::kSpanBytes, &tmW1, fb, c * S::kCols + j * 64, kb * BK, g);
+          if (SWIGLU) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_3d(st + (2 + j) * S::kSpanBytes, &tmW3, fb, c * S::kCols + j * 64,
+                          kb * BK, g);
+          }
+          for (int q = 0; q < boxes; ++q)
+            tma_load_2d(st + S::kWBytes + q * S::kRowBoxBytes, &tmX, fb, kb * BK,
+                        row0 + q * kRowBox);
+          issued_mask |= 1u << s;
+          issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
+          if (++s == S::kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        for (int q = 0; q < S::kStages; ++q)
+          if ((issued_mask >> q) & 1u) wait_drain(full0 + 8 * q, (issued_parity >> q) & 1u, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0, buf = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool ok = true, any = false;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int g, c, r, row0, nr;
+        tile_coords(tile, g, c, r, row0, nr);
+        const uint32_t idesc = instr_desc_swap(S::kCols, (nr + 15) & ~15);
+        if (!wait(acce0 + 8 * buf, acc_ph ^ 1, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * S::kAccCols;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait(full0 + 8 * s, ph, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // weights: MN-major spans (LBO = span stride), rows: K-major 128-byte rows
+            const uint64_t xd = smem_desc(st + S::kWBytes + kk * 32, 16, 1024);
+            const uint64_t w1d = smem_desc(st + kk * 2048, S::kSpanBytes, 1024);
+            umma(d_tmem, w1d, xd, idesc, (kb | kk) != 0);
+            if (SWIGLU) {
+              const uint64_t w3d = smem_desc(st + 2 * S::kSpanBytes + kk * 2048, S::kSpanBytes,
+                                             1024);
+              umma(d_tmem + 128, w3d, xd, idesc, (kb | kk) != 0);
+            }
+          }
+          any = true;
+          umma_commit(empty0 + 8 * s);
+          if (++s == S::kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(accf0 + 8 * buf);
+        buf ^= 1;
+        if (buf == 0) acc_ph ^= 1;
+      }
+      if (!ok && any) {
+        umma_commit(drain);
+        wait_drain(drain, 0, p.err);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // TMEM lane = output column (this warp: columns 32*quarter ..), TMEM
+    // column = row of the tile.
+    const int quarter = warp & 3;
+    int buf = 0;
+    uint32_t acc_ph = 0;
+    float *stg = s_epi + (warp - 2) * 32 * S::kStageRowWords;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int g, c, r, row0, nr;
+      tile_coords(tile, g, c, r, row0, nr);
+      int ready = 0;
+      if (lane == 0) ready = wait(accf0 + 8 * buf, acc_ph, ctl) ? 1 : 0;
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (!ready) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + buf * S::kAccCols + ((uint32_t)(quarter * 32) << 16);
+      const int col0 = c * S::kCols + quarter * 32;  // this warp's 32 output columns
+#pragma unroll 1
+      for (int j0 = 0; j0 < nr; j0 += 32) {
+        float v[32];
+        tmem_ld32(tb + j0, v);  // v[j] = out[row j0 + j][col0 + lane]
+        if (SWIGLU) {
+          float u[32];
+          tmem_ld32(tb + 128 + j0, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
+        }
+        // transpose through shared memory: stage[row j][column lane]
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stg[j * S::kStageRowWords + lane] = v[j];
+        __syncwarp();
+        if (SWIGLU) {  // bf16 rows: 8 lanes x 8 bytes per 64-byte row segment, 4 rows per step
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = i * 4 + (lane >> 3), q = lane & 7;
+            const int grow = row0 + j0 + j, gcol = col0 + q * 4;
+            const float4 f = *reinterpret_cast<const float4 *>(stg + j * S::kStageRowWords + 4 * q);
+            if (j0 + j < nr && gcol < p.N) {
+              __nv_bfloat162 lo = __floats2bfloat162_rn(f.x, f.y);
+              __nv_bfloat162 hi = __floats2bfloat162_rn(f.z, f.w);
+              uint2 w;
+              w.x = *reinterpret_cast<uint32_t *>(&lo);
+              w.y = *reinterpret_cast<uint32_t *>(&hi);
+              *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) +
+                                         (size_t)grow * p.N + gcol) = w;
+            }
+          }
+        } else {  // fp32 (+ bias) rows: 8 lanes x 16 bytes, 4 rows per step
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = i * 4 + (lane >> 3), q = lane & 7;
+            const int grow = row0 + j0 + j, gcol = col0 + q * 4;
+            float4 o = *reinterpret_cast<const float4 *>(stg + j * S::kStageRowWords + 4 * q);
+            if (j0 + j < nr && gcol < p.N) {
+              if (p.bias) {
+                const float *b = p.bias + gcol;
+                o.x += b[0];
+                o.y += b[1];
+                o.z += b[2];
+                o.w += b[3];
+              }
+              *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)grow * p.N +
+                                          gcol) = o;
+            }
+          }
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce0 + 8 * buf);
+      buf ^= 1;
+      if (buf == 0) acc_ph ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -1007,6 +1335,19 @@ bool make_map_a(CUtensorMap *m, const void *A, int rows, int K) {
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)(rows > 0 ? rows : 1)};
   cuuint64_t strides[1] = {(cuuint64_t)K * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)BM};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over rows [rows, K] with a box of `box_rows` rows.
+bool make_map_rows(CUtensorMap *m, const void *A, int rows, int K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1086,18 +1427,62 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   return cudaGetLastError();
 }
 
+template <bool SWIGLU>
+cudaError_t launch_swap(int rows_cap, int K, int N, int G, const int32_t *offsets,
+                        int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
+                        uint32_t *err, cudaStream_t s) {
+  using S = ShapeSwap<SWIGLU>;
+  CUtensorMap mx, mw1, mw3;
+  if (!make_map_rows(&mx, A, rows_cap, K, kRowBox) || !make_map_b(&mw1, B1, G, K, N) ||
+      !make_map_b(&mw3, SWIGLU ? B3 : B1, G, K, N))
+    return cudaErrorInvalidValue;
+  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool attr_set[64] = {};
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(
+        k_grouped_gemm_swap<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, err};
+  const long long max_tiles = (long long)((rows_cap + S::kMaxRows - 1) / S::kMaxRows +
+                                          (offsets ? G : 0)) *
+                              ((N + S::kCols - 1) / S::kCols);
+  const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
+  k_grouped_gemm_swap<SWIGLU><<<grid, kThreads, smem, s>>>(mx, mw1, mw3, p);
+  return cudaGetLastError();
+}
+
 }  // namespace tc
 
-// CTA pairs pay off when groups are large: a pair tile is 256 rows, so a
-// group's last tile wastes up to 255 rows instead of 127.  The host knows the
-// mean rows per group (the true counts live on the device); MOE_GEMM_PAIR=0/1
-// forces one engine (tests run both on every shape).
-static bool use_pair_tiles(int rows_cap, int G, const int32_t *offsets, int fixed_rows) {
-  const char *env = getenv("MOE_GEMM_PAIR");
-  if (env && env[0] == '0') return false;
-  if (env && env[0] == '1') return true;
+// Three engines, all correct for every shape (the tests run each):
+//   single  one CTA per 128-row tile; up projection 128 columns of gate and of
+//           up (N=256 MMA), down projection 256 columns;
+//   narrow  the same with 64-column up-projection tiles (twice the tiles);
+//   pair    CTA pairs on 256-row tiles (tcgen05 cta_group::2);
+//   swap    weights as the M operand, rows in steps of 16 (swap-AB).
+// Measured on B200 with the engines interleaved in one process (best of four
+// rounds), the single-CTA engine is fastest or tied on every workload here,
+// except the up projection of decode-sized groups (at most 32 rows per group
+// on average), where swap-AB loads only the valid rows instead of 128-row
+// boxes (Mixtral-shaped decode: 0.298 vs 0.320 ms).  Those are the defaults;
+// MOE_GEMM_ENGINE=single|narrow|pair|swap selects one engine for every GEMM.
+enum class Engine { kSingle, kNarrow, kPair, kSwap };
+
+static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offsets,
+                          int fixed_rows) {
+  const char *env = getenv("MOE_GEMM_ENGINE");
+  if (env && env[0] == 's' && env[1] == 'i') return Engine::kSingle;
+  if (env && env[0] == 'n') return Engine::kNarrow;
+  if (env && env[0] == 'p') return Engine::kPair;
+  if (env && env[0] == 's' && env[1] == 'w') return Engine::kSwap;
   const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
-  return mean_rows >= 2048;
+  if (swiglu && mean_rows <= 32) return Engine::kSwap;
+  return Engine::kSingle;
 }
 
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
@@ -1106,23 +1491,28 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                      cudaStream_t s) {
   if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if (rows_cap == 0) return cudaSuccess;
-  if (use_pair_tiles(rows_cap, G, offsets, fixed_rows))
-    return swiglu ? tc::launch_pair<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
-                                          err, s)
-                  : tc::launch_pair<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
-                                           out, err, s);
-  // Decode-sized groups (a few rows each) stream weights: every tile costs
-  // the same, so the tile count decides how evenly the last wave fills the
-  // GPU.  Half-width up-projection tiles (64 columns of gate and of up)
-  // double the count and shrink that tail.
-  const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
-  if (swiglu && mean_rows <= 32)
-    return tc::launch<true, 1>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out, nullptr,
-                               err, s);
-  return swiglu ? tc::launch<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
-                                      nullptr, err, s)
-                : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
-                                       nullptr, err, s);
+  switch (pick_engine(swiglu, rows_cap, G, offsets, fixed_rows)) {
+    case Engine::kPair:
+      return swiglu ? tc::launch_pair<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
+                                            out, err, s)
+                    : tc::launch_pair<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
+                                             out, err, s);
+    case Engine::kSwap:
+      return swiglu ? tc::launch_swap<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
+                                            out, err, s)
+                    : tc::launch_swap<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
+                                             out, err, s);
+    case Engine::kNarrow:
+      if (swiglu)
+        return tc::launch<true, 1>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
+                                   nullptr, err, s);
+      [[fallthrough]];
+    default:
+      return swiglu ? tc::launch<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
+                                          out, nullptr, err, s)
+                    : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
+                                           out, nullptr, err, s);
+  }
 }
 
 cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,

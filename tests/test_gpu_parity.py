@@ -25,13 +25,13 @@ pytestmark = pytest.mark.gpu
 SMALL = {
     "tiny_f32": WORKLOADS["tiny_f32"],
     "mixtral_small": WORKLOADS["mixtral_prefill"].scaled(T=300, d=256, f=384),
-    # at most 32 rows per expert on average: the half-width up-projection tiles
+    # a handful of rows per expert
     "qwen3_decode_small": WORKLOADS["qwen3_prefill"].scaled(T=50, d=192, E=16, k_max=4, f=200),
     "qwen3_small": WORKLOADS["qwen3_prefill"].scaled(T=257, d=192, E=16, k_max=4, f=200),
     "dsv3_small": WORKLOADS["dsv3_prefill"].scaled(T=130, d=256, E=64, f=136, f_shared=72),
     "gptoss_small": WORKLOADS["gptoss_sub"].scaled(T=211, d=200, E=32, k_max=6, k_min=2, f=72),
     "mixtral_decode_small": WORKLOADS["mixtral_decode"].scaled(T=5, d=512, f=1024),
-    # more than 32 rows per expert on average: the wide up-projection tiles
+    # more rows per expert on average than the small cases
     "qwen3_medium": WORKLOADS["qwen3_prefill"].scaled(T=1100, d=192, E=16, k_max=4, f=200),
     "dsv3_medium": WORKLOADS["dsv3_prefill"].scaled(T=1200, d=256, E=64, f=136, f_shared=72),
 }
@@ -236,18 +236,18 @@ def test_sigmoid_grouped_near_ties_bit_exact(dev):
 
 
 # ---------------------------------------------------------------------------
-# Both grouped-GEMM engines (single-CTA tiles, CTA-pair tiles) on every shape
+# Every grouped-GEMM engine (single-CTA, CTA-pair and swap-AB tiles) on every shape
 # ---------------------------------------------------------------------------
-@pytest.fixture(params=["0", "1"], ids=["single_cta", "cta_pair"])
+@pytest.fixture(params=["single", "narrow", "pair", "swap"])
 def gemm_engine(request):
     import os
-    old = os.environ.get("MOE_GEMM_PAIR")
-    os.environ["MOE_GEMM_PAIR"] = request.param
+    old = os.environ.get("MOE_GEMM_ENGINE")
+    os.environ["MOE_GEMM_ENGINE"] = request.param
     yield request.param
     if old is None:
-        os.environ.pop("MOE_GEMM_PAIR", None)
+        os.environ.pop("MOE_GEMM_ENGINE", None)
     else:
-        os.environ["MOE_GEMM_PAIR"] = old
+        os.environ["MOE_GEMM_ENGINE"] = old
 
 
 BF16_SMALL = [n for n, w in SMALL.items() if w.dtype == "bf16"]
@@ -263,7 +263,7 @@ def test_layer_each_engine(name, gemm_engine, dev):
     test_layer_matches_oracle(name, dev)
 
 
-@pytest.mark.parametrize("T", [1, 255, 257, 600])
-def test_pair_tiles_across_256_row_edges(T, gemm_engine, dev):
+@pytest.mark.parametrize("T", [1, 15, 17, 255, 257, 600])
+def test_tile_row_edges(T, gemm_engine, dev):
     w = SMALL["mixtral_small"].scaled(T=T)
     _layer_vs_oracle(w, _host_inputs(w, seed=T), dev)
