@@ -138,6 +138,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
 }
+// Four rows (r0..r3) of 64 columns starting at column c0 into 4 consecutive
+// 128-byte rows of shared memory (the map's box is one row high).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(bar)
+      : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -229,6 +240,11 @@ struct Params {
   int K, N;
   void *out;  // [rows_cap, N]: bf16 for SWIGLU (h), fp32 for PLAIN (y, logits)
   const float *bias;  // PLAIN only: [N] added to every row (router logit bias), or nullptr
+  // Gathered A rows: when row_src is set, row r of A is row row_src[r] / k_max
+  // of the tensor map (the token rows x), fetched with TMA gather4; this fuses
+  // the dispatch copy into the GEMM.
+  const int32_t *row_src;
+  int k_max;
   uint32_t *err;
 };
 
@@ -367,23 +383,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int g, m, n;
-        tile_of(tile, s_tstart, s_off, p.G, g, m, n);
-        const int row = s_off[g] + m * BM;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
-            ok = false;
-            break;
-          }
-          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
-          const uint32_t fb = full0 + 8 * s;
-          mbar_expect_tx(fb, S::kStageBytes);
-          tma_load_2d(st, &tmA, fb, kb * BK, row);
+    // Lane 0 waits and issues the tiled loads; when the A rows are gathered,
+    // every lane issues one gather4 (4 of the tile's 128 rows).
+    const bool gather = p.row_src != nullptr;
+    int s = 0;
+    uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      int g, m, n;
+      tile_of(tile, s_tstart, s_off, p.G, g, m, n);
+      const int row = s_off[g] + m * BM;
+      int tok[4] = {0, 0, 0, 0};  // rows past the group read token 0 (masked later)
+      if (gather) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int r = row + 4 * lane + q;
+          if (r < s_off[g + 1]) tok[q] = p.row_src[r] / p.k_max;
+        }
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
+        int okw = 1;
+        if (lane == 0) okw = wait(empty0 + 8 * s, ph ^ 1, ctl) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) {
+          ok = false;
+          break;
+        }
+        const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+        const uint32_t fb = full0 + 8 * s;
+        if (lane == 0) mbar_expect_tx(fb, S::kStageBytes);
+        if (gather)
+          tma_gather4(st + lane * 4 * 128, &tmA, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
+        if (lane == 0) {
+          if (!gather) tma_load_2d(st, &tmA, fb, kb * BK, row);
 #pragma unroll
           for (int j = 0; j < S::kSpans; ++j)
             tma_load_3d(st + S::kABytes + j * S::kSpanBytes, &tmB1, fb, n * S::BN + j * 64,
@@ -394,18 +426,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d(st + S::kABytes + (S::kSpans + j) * S::kSpanBytes, &tmB3, fb,
                           n * S::BN + j * 64, kb * BK, g);
           }
-          issued_mask |= 1u << s;
-          issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
-          if (++s == S::kStages) {
-            s = 0;
-            ph ^= 1;
-          }
+        }
+        issued_mask |= 1u << s;
+        issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
+        if (++s == S::kStages) {
+          s = 0;
+          ph ^= 1;
         }
       }
-      if (!ok) {  // stopped early: let the copies already issued land first
-        for (int q = 0; q < S::kStages; ++q)
-          if ((issued_mask >> q) & 1u) wait_drain(full0 + 8 * q, (issued_parity >> q) & 1u, p.err);
-      }
+    }
+    if (!ok && lane == 0) {  // stopped early: let the copies already issued land first
+      for (int q = 0; q < S::kStages; ++q)
+        if ((issued_mask >> q) & 1u) wait_drain(full0 + 8 * q, (issued_parity >> q) & 1u, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -1127,23 +1159,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int g, c, r, row0, nr;
-        tile_coords(tile, g, c, r, row0, nr);
-        const int boxes = (nr + kRowBox - 1) / kRowBox;
-        const uint32_t bytes = S::kWBytes + boxes * S::kRowBoxBytes;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
-            ok = false;
-            break;
-          }
-          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
-          const uint32_t fb = full0 + 8 * s;
-          mbar_expect_tx(fb, bytes);
+    const bool gather = p.row_src != nullptr;
+    int s = 0;
+    uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      int g, c, r, row0, nr;
+      tile_coords(tile, g, c, r, row0, nr);
+      // rows loaded: 32-row boxes, or (gathering) gather4s up to the MMA's N
+      const int nq = gather ? ((nr + 15) & ~15) / 4 : (nr + kRowBox - 1) / kRowBox;
+      const uint32_t bytes = S::kWBytes + (gather ? nq * 512 : nq * S::kRowBoxBytes);
+      int tok[4] = {0, 0, 0, 0};
+      if (gather && lane < nq) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int rr = 4 * lane + q;
+          if (rr < nr) tok[q] = p.row_src[row0 + rr] / p.k_max;
+        }
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
+        int okw = 1;
+        if (lane == 0) okw = wait(empty0 + 8 * s, ph ^ 1, ctl) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) {
+          ok = false;
+          break;
+        }
+        const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+        const uint32_t fb = full0 + 8 * s;
+        if (lane == 0) mbar_expect_tx(fb, bytes);
+        if (gather && lane < nq)
+          tma_gather4(st + S::kWBytes + lane * 4 * 128, &tmX, fb, kb * BK, tok[0], tok[1],
+                      tok[2], tok[3]);
+        if (lane == 0) {
 #pragma unroll
           for (int j = 0; j < 2; ++j)
             tma_load_3d(st + j * S::kSpanBytes, &tmW1, fb, c * S::kCols + j * 64, kb * BK, g);
@@ -1153,21 +1201,22 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d(st + (2 + j) * S::kSpanBytes, &tmW3, fb, c * S::kCols + j * 64,
                           kb * BK, g);
           }
-          for (int q = 0; q < boxes; ++q)
-            tma_load_2d(st + S::kWBytes + q * S::kRowBoxBytes, &tmX, fb, kb * BK,
-                        row0 + q * kRowBox);
-          issued_mask |= 1u << s;
-          issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
-          if (++s == S::kStages) {
-            s = 0;
-            ph ^= 1;
-          }
+          if (!gather)
+            for (int q = 0; q < nq; ++q)
+              tma_load_2d(st + S::kWBytes + q * S::kRowBoxBytes, &tmX, fb, kb * BK,
+                          row0 + q * kRowBox);
+        }
+        issued_mask |= 1u << s;
+        issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
+        if (++s == S::kStages) {
+          s = 0;
+          ph ^= 1;
         }
       }
-      if (!ok) {
-        for (int q = 0; q < S::kStages; ++q)
-          if ((issued_mask >> q) & 1u) wait_drain(full0 + 8 * q, (issued_parity >> q) & 1u, p.err);
-      }
+    }
+    if (!ok && lane == 0) {
+      for (int q = 0; q < S::kStages; ++q)
+        if ((issued_mask >> q) & 1u) wait_drain(full0 + 8 * q, (issued_parity >> q) & 1u, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -1370,10 +1419,12 @@ bool make_map_b(CUtensorMap *m, const void *B, int G, int K, int N) {
 template <bool SWIGLU, int SPANS>
 cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, int fixed_rows,
                    const void *A, const void *B1, const void *B3, void *out, const float *bias,
-                   uint32_t *err, cudaStream_t s) {
+                   uint32_t *err, cudaStream_t s, const int32_t *row_src = nullptr,
+                   int k_max = 1, int a_rows = 0) {
   using S = Shape<SWIGLU, SPANS>;
   CUtensorMap ma, mb1, mb3;
-  if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
+  const bool map_ok = row_src ? make_map_rows(&ma, A, a_rows, K, 1) : make_map_a(&ma, A, rows_cap, K);
+  if (!map_ok || !make_map_b(&mb1, B1, G, K, N) ||
       !make_map_b(&mb3, SWIGLU ? B3 : B1, G, K, N))
     return cudaErrorInvalidValue;
   const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
@@ -1388,7 +1439,7 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
     attr_set[dev] = true;
   }
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, bias, err};
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, bias, row_src, k_max, err};
   // never more CTAs than tiles can exist (a group holds at most rows_cap rows)
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
@@ -1418,7 +1469,7 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, err};
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
   const long long max_tiles = (long long)((rows_cap + BM2 - 1) / BM2 + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
   long long pairs = sms / 2;
@@ -1430,10 +1481,13 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
 template <bool SWIGLU>
 cudaError_t launch_swap(int rows_cap, int K, int N, int G, const int32_t *offsets,
                         int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
-                        uint32_t *err, cudaStream_t s) {
+                        uint32_t *err, cudaStream_t s, const int32_t *row_src = nullptr,
+                        int k_max = 1, int a_rows = 0) {
   using S = ShapeSwap<SWIGLU>;
   CUtensorMap mx, mw1, mw3;
-  if (!make_map_rows(&mx, A, rows_cap, K, kRowBox) || !make_map_b(&mw1, B1, G, K, N) ||
+  const bool map_ok = row_src ? make_map_rows(&mx, A, a_rows, K, 1)
+                              : make_map_rows(&mx, A, rows_cap, K, kRowBox);
+  if (!map_ok || !make_map_b(&mw1, B1, G, K, N) ||
       !make_map_b(&mw3, SWIGLU ? B3 : B1, G, K, N))
     return cudaErrorInvalidValue;
   const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
@@ -1448,7 +1502,7 @@ cudaError_t launch_swap(int rows_cap, int K, int N, int G, const int32_t *offset
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, err};
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, row_src, k_max, err};
   const long long max_tiles = (long long)((rows_cap + S::kMaxRows - 1) / S::kMaxRows +
                                           (offsets ? G : 0)) *
                               ((N + S::kCols - 1) / S::kCols);
@@ -1485,13 +1539,21 @@ static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offse
   return Engine::kSingle;
 }
 
+bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *offsets,
+                             int fixed_rows) {
+  return swiglu && pick_engine(swiglu, rows_cap, G, offsets, fixed_rows) != Engine::kPair;
+}
+
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
                                      const int32_t *offsets, int fixed_rows, const void *A,
                                      const void *B1, const void *B3, void *out, uint32_t *err,
-                                     cudaStream_t s) {
+                                     cudaStream_t s, const int32_t *row_src, int k_max,
+                                     int a_rows) {
   if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if (rows_cap == 0) return cudaSuccess;
-  switch (pick_engine(swiglu, rows_cap, G, offsets, fixed_rows)) {
+  const Engine e = pick_engine(swiglu, rows_cap, G, offsets, fixed_rows);
+  if (row_src && (!swiglu || e == Engine::kPair)) return cudaErrorInvalidValue;
+  switch (e) {
     case Engine::kPair:
       return swiglu ? tc::launch_pair<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                             out, err, s)
@@ -1499,17 +1561,17 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                              out, err, s);
     case Engine::kSwap:
       return swiglu ? tc::launch_swap<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
-                                            out, err, s)
+                                            out, err, s, row_src, k_max, a_rows)
                     : tc::launch_swap<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                              out, err, s);
     case Engine::kNarrow:
       if (swiglu)
         return tc::launch<true, 1>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
-                                   nullptr, err, s);
+                                   nullptr, err, s, row_src, k_max, a_rows);
       [[fallthrough]];
     default:
       return swiglu ? tc::launch<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
-                                          out, nullptr, err, s)
+                                          out, nullptr, err, s, row_src, k_max, a_rows)
                     : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                            out, nullptr, err, s);
   }

@@ -80,11 +80,17 @@ cudaError_t launch_ffn_simt_f32(int rows_cap, int d, int f, int G, const int32_t
 //   swiglu: out[r, :] = silu(A[r].B1[g]) * (A[r].B3[g])  bf16 out   (B*: [G, K, N])
 //   plain:  out[r, :] = A[r].B1[g]                       fp32 out
 // Rows of group g are offsets[g]..offsets[g+1]-1 of A (rows_cap rows, K
-// columns); offsets == nullptr means one group of fixed_rows rows.
+// columns); offsets == nullptr means one group of fixed_rows rows.  With
+// row_src (swiglu only, when grouped_gemm_can_gather says so), row r of A is
+// row row_src[r] / k_max of A itself ([a_rows, K], the token rows): the
+// dispatch gather is fused into the GEMM's loads.
+bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *offsets,
+                             int fixed_rows);
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
                                      const int32_t *offsets, int fixed_rows, const void *A,
                                      const void *B1, const void *B3, void *out, uint32_t *err,
-                                     cudaStream_t s);
+                                     cudaStream_t s, const int32_t *row_src = nullptr,
+                                     int k_max = 1, int a_rows = 0);
 
 // K1 on the tensor cores (bf16 layers with E % 8 == 0): logits[T,E] =
 // x[T,d] . Wr[d,E] (+ bias), fp32 accumulation in tensor memory, fp32 out.

@@ -267,3 +267,26 @@ def test_layer_each_engine(name, gemm_engine, dev):
 def test_tile_row_edges(T, gemm_engine, dev):
     w = SMALL["mixtral_small"].scaled(T=T)
     _layer_vs_oracle(w, _host_inputs(w, seed=T), dev)
+
+
+@pytest.fixture
+def fused_dispatch():
+    import os
+    old = os.environ.get("MOE_FUSED_DISPATCH")
+    os.environ["MOE_FUSED_DISPATCH"] = "1"
+    yield
+    if old is None:
+        os.environ.pop("MOE_FUSED_DISPATCH", None)
+    else:
+        os.environ["MOE_FUSED_DISPATCH"] = old
+
+
+@pytest.mark.parametrize("name", BF16_SMALL)
+def test_layer_with_dispatch_fused_into_gemm(name, fused_dispatch, dev):
+    """The layer with the up projection gathering token rows itself (TMA gather4)."""
+    test_layer_matches_oracle(name, dev)
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "dsv3_small", "gptoss_small"])
+def test_fused_dispatch_each_engine(name, fused_dispatch, gemm_engine, dev):
+    test_layer_matches_oracle(name, dev)
