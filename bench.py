@@ -110,7 +110,8 @@ def barrier(dist):
 # ---------------------------------------------------------------------------
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+                "enforced.power.limit")
 
 
 class ClockSampler:
@@ -148,7 +149,7 @@ class ClockSampler:
             rows = [r for r in csv.reader(io.StringIO(fh.read())) if len(r) >= 9]
         os.unlink(self.file.name)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        sm, mx, pw, reasons = [], [], [], set()
+        sm, mx, pw, lim, reasons = [], [], [], [], set()
         for r in rows:
             try:
                 sm.append(float(r[1]))
@@ -156,14 +157,21 @@ class ClockSampler:
                 pw.append(float(r[3]))
             except ValueError:
                 continue
+            try:  # the enforced power limit, read (never set) alongside the clocks
+                lim.append(float(r[9]))
+            except (IndexError, ValueError):
+                pass
             for name, v in zip(names, r[5:9]):
                 if v.strip().lower() == "active":
                     reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": sorted(reasons), "samples": 0}
         hot = [s for s, p in zip(sm, pw) if p > 0.3 * max(pw)] or sm
-        return {"sm_mhz": statistics.median(hot), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(hot), "sm_max_mhz": max(mx),
+               "reasons": sorted(reasons), "samples": len(sm), "power_max_w": max(pw)}
+        if lim:
+            out["power_limit_w"] = statistics.median(lim)
+        return out
 
 
 # ---------------------------------------------------------------------------
@@ -176,9 +184,18 @@ def peaks() -> tuple[dict, str]:
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def small_batch_routing(w) -> bool:
+    """Decode-sized bf16 batches (E % 8 == 0, T <= 128) route with two launches:
+    the split-K router and one fused gating/ranking kernel."""
+    return (w.dtype == "bf16" and w.E % 8 == 0 and 1 <= w.T <= 128
+            and not os.environ.get("MOE_SMALL_ROUTE", "1").startswith("0"))
+
+
 def launches_per_layer(w) -> int:
     """Kernel launches of one moe_layer call (see the C ABI's launch order)."""
-    n = 1 + 1 + 3 + 1 + 2 + 1  # router, gating, hist+scan+rank, dispatch, 2 FFN passes, combine
+    # router, gating, hist+scan+rank -- or the two small-batch launches
+    routing = 2 if small_batch_routing(w) else 1 + 1 + 3
+    n = routing + 1 + 2 + 1  # + dispatch, 2 FFN passes, combine
     if w.f_shared > 0:
         n += 2
     return n

@@ -24,221 +24,22 @@
 //   log2(e) rounded to binary32; ln 2 rounded to 12 significant bits
 //   (2839/4096, so n * hi is exact); the binary32 rounding of
 //   ln 2 - 2839/4096; and 1/k! rounded to binary32 for k = 2..7.
-#include <math.h>
-
-#include "moe_internal.cuh"
+#include "gating.cuh"
 
 namespace moe {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ float spec_expf(float z) {
-  const float kLog2e = 1.44269502162933349609375f;   // 0x3FB8AA3B
-  const float kLn2Hi = 0.693115234375f;              // 2839 / 4096 = 0x3F317000
-  const float kLn2Lo = 3.19461832987144589424133e-05f; // 0x3805FDF4
-  const float kC7 = 1.98412701138295233249664e-04f;  // 1/5040 -> 0x39500D01
-  const float kC6 = 1.38888892251998186111450e-03f;  // 1/720  -> 0x3AB60B61
-  const float kC5 = 8.33333376795053482055664e-03f;  // 1/120  -> 0x3C088889
-  const float kC4 = 4.16666679084300994873047e-02f;  // 1/24   -> 0x3D2AAAAB
-  const float kC3 = 1.66666671633720397949219e-01f;  // 1/6    -> 0x3E2AAAAB
-  z = z > 87.0f ? 87.0f : z;
-  z = z < -87.0f ? -87.0f : z;
-  const float n = rintf(__fmul_rn(z, kLog2e));
-  float r = __fmaf_rn(-n, kLn2Hi, z);
-  r = __fmaf_rn(-n, kLn2Lo, r);
-  float p = kC7;
-  p = __fmaf_rn(p, r, kC6);
-  p = __fmaf_rn(p, r, kC5);
-  p = __fmaf_rn(p, r, kC4);
-  p = __fmaf_rn(p, r, kC3);
-  p = __fmaf_rn(p, r, 0.5f);
-  p = __fmaf_rn(p, r, 1.0f);
-  p = __fmaf_rn(p, r, 1.0f);
-  const int ni = static_cast<int>(n);
-  return __fmul_rn(p, __int_as_float((ni + 127) << 23));
-}
-
-__device__ __forceinline__ float spec_sigmoidf(float z) {
-  return __fdiv_rn(1.0f, __fadd_rn(1.0f, spec_expf(-z)));
-}
-
-// Is candidate (k1, i1) ranked ahead of (k0, i0)?
-__device__ __forceinline__ bool ahead(float k1, int i1, float k0, int i0) {
-  return k1 > k0 || (k1 == k0 && i1 < i0);
-}
-
-__device__ __forceinline__ void warp_argmax(float &key, int &idx) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    float ok = __shfl_xor_sync(kFull, key, off);
-    int oi = __shfl_xor_sync(kFull, idx, off);
-    if (ahead(ok, oi, key, idx)) {
-      key = ok;
-      idx = oi;
-    }
-  }
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-  return v;
-}
-
-struct GatingArgs {
-  const float *logits;
-  const float *sel_bias;
-  const int32_t *k_per_token;
-  int32_t *topk_idx;
-  float *topk_w;
-  int T, E, k_max, mode, n_groups, topk_groups, group_score_topk;
-  float routed_scale;
-  uint32_t *err;
-};
+using gating::GatingArgs;
 
 constexpr int kWarpsPerBlock = 4;
 
 template <int NPL>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_gating(GatingArgs g) {
   extern __shared__ float s_u_all[];  // [kWarpsPerBlock][E], sigmoid mode only
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int warp = threadIdx.x / 32;
   const int t = blockIdx.x * kWarpsPerBlock + warp;
   if (t >= g.T) return;  // whole warp leaves together
-  const int E = g.E;
-  const float *l = g.logits + (size_t)t * E;
-
-  float key[NPL], val[NPL];  // val: logit (softmax modes) or sigmoid score
-  uint32_t alive = 0;
-#pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    const int e = i * 32 + lane;
-    key[i] = -INFINITY;
-    val[i] = 0.f;
-    if (e < E) {
-      const float v = l[e];
-      alive |= 1u << i;
-      if (g.mode == MOE_SIGMOID_GROUPED) {
-        const float s = spec_sigmoidf(v);
-        val[i] = s;
-        key[i] = __fadd_rn(s, g.sel_bias ? g.sel_bias[e] : 0.0f);
-      } else {
-        val[i] = v;
-        key[i] = v;
-      }
-    }
-  }
-
-  int kt = g.k_per_token ? g.k_per_token[t] : g.k_max;
-  if (kt < 1 || kt > g.k_max) {
-    if (lane == 0) raise_error(g.err, kErrRouting);
-    kt = kt < 1 ? 1 : g.k_max;
-  }
-
-  if (g.mode == MOE_SIGMOID_GROUPED) {
-    // Group scores: lane g sums, in descending order, the group_score_topk
-    // largest biased scores of group g; then keep the topk_groups best groups.
-    float *s_u = s_u_all + warp * E;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E) s_u[e] = key[i];
-    }
-    __syncwarp();
-    const int gsz = E / g.n_groups, m = g.group_score_topk;
-    float gscore = -INFINITY;
-    int gidx = 0x7fffffff;
-    if (lane < g.n_groups) {
-      float top[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) top[q] = -INFINITY;
-      for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) {
-        float v = s_u[e];
-        // insert v into the descending list top[0..m-1]
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (q < m && v > top[q]) {
-            const float tmp = top[q];
-            top[q] = v;
-            v = tmp;
-          }
-        }
-      }
-      float sc = top[0];
-#pragma unroll
-      for (int q = 1; q < 8; ++q)
-        if (q < m) sc = __fadd_rn(sc, top[q]);
-      gscore = sc;
-      gidx = lane;
-    }
-    uint32_t kept_groups = 0;
-    for (int r = 0; r < g.topk_groups; ++r) {
-      float bk = gscore;
-      int bi = gidx;
-      warp_argmax(bk, bi);
-      kept_groups |= 1u << bi;
-      if (bi == lane) {
-        gscore = -INFINITY;
-        gidx = 0x7fffffff;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E && !((kept_groups >> (e / gsz)) & 1u)) alive &= ~(1u << i);
-    }
-  }
-
-  // k_t rounds of warp argmax; lane j keeps slot j.
-  int my_idx = -1;
-  float my_val = 0.f;
-  for (int j = 0; j < kt; ++j) {
-    float bk = -INFINITY;
-    int bi = 0x7fffffff;
-    float bv = 0.f;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      if (((alive >> i) & 1u) && (key[i] > bk || bi == 0x7fffffff)) {
-        bk = key[i];
-        bi = i * 32 + lane;
-        bv = val[i];
-      }
-    }
-    warp_argmax(bk, bi);
-    if (bi == 0x7fffffff) break;  // fewer candidates than k_t (rejected on the host)
-    const int owner = bi & 31;
-    const float v = __shfl_sync(kFull, bv, owner);
-    if (lane == owner) alive &= ~(1u << (bi >> 5));
-    if (lane == j) {
-      my_idx = bi;
-      my_val = v;
-    }
-  }
-
-  // Weights.
-  float w = 0.f;
-  const bool mine = lane < kt;
-  if (g.mode == MOE_TOPK_SOFTMAX) {
-    const float top = __shfl_sync(kFull, my_val, 0);
-    const float ex = mine ? expf(my_val - top) : 0.f;
-    w = ex / warp_sum(ex);
-  } else if (g.mode == MOE_SOFTMAX_TOPK_RENORM) {
-    const float top = __shfl_sync(kFull, my_val, 0);  // the largest logit of the row
-    float z = 0.f;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i)
-      if (i * 32 + lane < E) z += expf(l[i * 32 + lane] - top);
-    z = warp_sum(z);
-    const float p = mine ? expf(my_val - top) / z : 0.f;
-    w = p / warp_sum(p);
-  } else {
-    const float s = mine ? my_val : 0.f;
-    w = g.routed_scale * s / warp_sum(s);
-  }
-  if (lane < g.k_max) {
-    g.topk_idx[(size_t)t * g.k_max + lane] = mine ? my_idx : -1;
-    g.topk_w[(size_t)t * g.k_max + lane] = mine ? w : 0.f;
-  }
+  gating::gate_token<NPL>(g, t, g.logits + (size_t)t * g.E, s_u_all + warp * g.E);
 }
 
 template <int NPL>

@@ -246,6 +246,14 @@ struct Params {
   const int32_t *row_src;
   int k_max;
   uint32_t *err;
+  // Split K (single engine, PLAIN, offsets == nullptr): group g multiplies
+  // the same fixed_rows rows of A by K columns g*k_split .. g*k_split+k_split-1
+  // (B is one [K, N] matrix) and writes its partial product to output rows
+  // g*fixed_rows .. ; columns past K read the TMA zero fill.
+  int k_split = 0;
+  // Word set to zero by the first thread of block 0 (a ticket the next
+  // launch on the stream counts with), or nullptr.
+  int32_t *clear = nullptr;
 };
 
 template <bool SWIGLU, int SPANS>
@@ -339,8 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Group table: row offsets, then tile starts (exclusive scan of the
   // per-group tile counts), checked against the buffer size.
   bool bad = false;
+  if (p.clear && blockIdx.x == 0 && threadIdx.x == 0) *p.clear = 0;
   for (int g = threadIdx.x; g <= p.G; g += kThreads) {
-    const int v = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.fixed_rows);
+    const int v = p.offsets ? p.offsets[g]
+                            : (p.k_split ? g * p.fixed_rows : (g == 0 ? 0 : p.fixed_rows));
     s_off[g] = v;
     if (v < 0 || v > p.rows_cap) bad = true;
   }
@@ -379,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = *abort_flag ? 0 : s_tstart[p.G];
-  const int num_kb = (p.K + BK - 1) / BK;
+  const int num_kb = p.k_split ? p.k_split / BK : (p.K + BK - 1) / BK;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -392,7 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       int g, m, n;
       tile_of(tile, s_tstart, s_off, p.G, g, m, n);
-      const int row = s_off[g] + m * BM;
+      // split K: every group reads the same A rows, at its own K offset
+      const int row = p.k_split ? m * BM : s_off[g] + m * BM;
+      const int k0 = p.k_split ? g * p.k_split : 0;
+      const int gb = p.k_split ? 0 : g;  // B's group coordinate
       int tok[4] = {0, 0, 0, 0};  // rows past the group read token 0 (masked later)
       if (gather) {
 #pragma unroll
@@ -415,16 +428,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (gather)
           tma_gather4(st + lane * 4 * 128, &tmA, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
         if (lane == 0) {
-          if (!gather) tma_load_2d(st, &tmA, fb, kb * BK, row);
+          if (!gather) tma_load_2d(st, &tmA, fb, k0 + kb * BK, row);
 #pragma unroll
           for (int j = 0; j < S::kSpans; ++j)
             tma_load_3d(st + S::kABytes + j * S::kSpanBytes, &tmB1, fb, n * S::BN + j * 64,
-                        kb * BK, g);
+                        k0 + kb * BK, gb);
           if (SWIGLU) {
 #pragma unroll
             for (int j = 0; j < S::kSpans; ++j)
               tma_load_3d(st + S::kABytes + (S::kSpans + j) * S::kSpanBytes, &tmB3, fb,
-                          n * S::BN + j * 64, kb * BK, g);
+                          n * S::BN + j * 64, k0 + kb * BK, gb);
           }
         }
         issued_mask |= 1u << s;
@@ -1575,6 +1588,34 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                     : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                            out, nullptr, err, s);
   }
+}
+
+cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const void *x,
+                                const void *Wr, float *partials, int32_t *clear, uint32_t *err,
+                                cudaStream_t s) {
+  using Sh = tc::Shape<false, 1>;
+  if (T <= 0 || S < 1 || S > tc::kMaxGroups || k_split <= 0 || k_split % tc::BK)
+    return cudaErrorInvalidValue;
+  CUtensorMap ma, mb;
+  if (!tc::make_map_a(&ma, x, T, d) || !tc::make_map_b(&mb, Wr, 1, d, E))
+    return cudaErrorInvalidValue;
+  const size_t smem = Sh::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(S + 1);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  static bool attr_set[64] = {};
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(
+        tc::k_grouped_gemm<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(Sh::kSmemFixed + sizeof(int32_t) * 2 * (tc::kMaxGroups + 1)));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  tc::Params p{nullptr, S, T, S * T, d, E, partials, nullptr, nullptr, 1, err, k_split, clear};
+  const long long tiles = (long long)S * ((T + tc::BM - 1) / tc::BM) * ((E + Sh::BN - 1) / Sh::BN);
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  tc::k_grouped_gemm<false, 1><<<grid, tc::kThreads, smem, s>>>(ma, mb, mb, p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,

@@ -80,7 +80,7 @@ Layout layout(const moe_config &c, int kind) {
     L.row_src = take(sizeof(int32_t) * slots);
     L.n_dropped = take(sizeof(int32_t));
   }
-  if (kind == MOE_WS_LAYER || kind == MOE_WS_ROUTE) L.cap_scratch = take(capacity_scratch_bytes(c));
+  if (kind == MOE_WS_LAYER || kind == MOE_WS_ROUTE) L.cap_scratch = take(route_scratch_bytes(c));
   if (kind == MOE_WS_LAYER) L.x_perm = take(slots * c.d * s);
   if (kind == MOE_WS_LAYER || kind == MOE_WS_EXPERT_FFN) L.h = take(slots * c.f * s);
   if (kind == MOE_WS_LAYER) {
@@ -148,6 +148,13 @@ T *at(void *ws, size_t off) {
 moe_status route_impl(const moe_config &c, const void *x, const void *Wr, const float *logit_bias,
                       const float *sel_bias, const int32_t *k_per_token, const moe_route_out &o,
                       void *cap_scratch, uint32_t *err, cudaStream_t s) {
+  // Decode-sized batches: split-K router plus one fused gating/ranking kernel.
+  const SmallRoutePlan plan = small_route_plan(c);
+  if (plan.use) {
+    MOE_TRY_CUDA(launch_route_small(c, plan, x, Wr, logit_bias, sel_bias, k_per_token, o,
+                                    cap_scratch, err, s));
+    return MOE_OK;
+  }
   // The router is a dense contraction: bf16 layers whose logit rows are a
   // multiple of 16 bytes (E % 8 == 0, a TMA stride rule) run it on the tensor
   // cores (its epilogue writes 16-byte vectors, so the logits buffer must be
@@ -326,8 +333,10 @@ moe_status moe_route(const moe_config *cfg, const void *x, const void *Wr,
 // with a static memory plan in which every byte of HBM is already assigned
 // (weights, caches) and a stray cudaMalloc would fail or fragment the pool, or
 // a latency-critical path that must not pay for an allocator call.  For them,
-// moe_route_static_scratch keeps the capacity step's scratch (per-chunk
-// expert histograms and their prefix sums) in the fixed device array below.
+// moe_route_static_scratch keeps the routing step's scratch (per-chunk
+// expert histograms and their prefix sums; for decode-sized batches, the
+// split-K router's partial logits, at most 768 KiB, and a ticket word) in the
+// fixed device array below.
 //
 // The array is kStaticScratchBytes (1 MiB) on every GPU that loads this
 // library, held until the process exits.  In host code its name is only a
@@ -365,7 +374,7 @@ moe_status moe_route_static_scratch(const moe_config *cfg, const void *x, const 
   MOE_TRY(need4_opt(sel_bias));
   MOE_TRY(need4_opt(k_per_token));
   MOE_TRY(check_route_out(out));
-  if (capacity_scratch_bytes(c) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
+  if (route_scratch_bytes(c) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
   void *scratch = route_scratch_address();
   uint32_t *err = device_error_word();
   if (!scratch || !err) return MOE_ERR_CUDA;

@@ -97,4 +97,27 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
 cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,
                              const float *bias, float *logits, uint32_t *err, cudaStream_t s);
 
+// K1 split along K: partials[g][T][E] = x[:, g*k_split ..] . Wr[g*k_split .., :]
+// for g < S (k_split a multiple of 64; the last slice may run past d).  The
+// first thread of block 0 sets *clear to zero.
+cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const void *x,
+                                const void *Wr, float *partials, int32_t *clear, uint32_t *err,
+                                cudaStream_t s);
+
+// Routing of small batches (decode): split-K router, then one kernel that
+// sums the partials, gates and ranks (see route_small.cu).  The plan depends
+// on the layer's shape only.
+struct SmallRoutePlan {
+  bool use = false;
+  int S = 0, k_split = 0;
+  size_t partial_bytes = 0, scratch_bytes = 0;
+};
+SmallRoutePlan small_route_plan(const moe_config &c);
+// Scratch of the routing step: the small-batch plan's, else the capacity step's.
+size_t route_scratch_bytes(const moe_config &c);
+cudaError_t launch_route_small(const moe_config &c, const SmallRoutePlan &plan, const void *x,
+                               const void *Wr, const float *logit_bias, const float *sel_bias,
+                               const int32_t *k_per_token, const moe_route_out &o, void *scratch,
+                               uint32_t *err, cudaStream_t s);
+
 }  // namespace moe

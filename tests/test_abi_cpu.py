@@ -160,7 +160,7 @@ def test_gpu_sigmoid_constants_are_the_rounded_definitions():
     from decimal import Decimal, getcontext
     getcontext().prec = 60
     ln2 = Fraction(Decimal(2).ln())
-    src = open(os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc", "gating.cu")).read()
+    src = open(os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc", "gating.cuh")).read()
     lits = dict(re.findall(r"const float (k\w+) = ([0-9.e+-]+)f;", src))
 
     def bits(name):

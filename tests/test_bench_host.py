@@ -56,6 +56,10 @@ def test_launch_count_and_algorithmic_work():
     w = WORKLOADS["mixtral_prefill"]
     assert bench.launches_per_layer(w) == 9
     assert bench.launches_per_layer(WORKLOADS["dsv3_prefill"]) == 11
+    # decode batches: split-K router + fused gating/ranking instead of 5 launches
+    assert bench.launches_per_layer(WORKLOADS["mixtral_decode"]) == 6
+    assert bench.launches_per_layer(WORKLOADS["dsv3_decode"]) == 8
+    assert bench.launches_per_layer(WORKLOADS["tiny_f32"]) == 9
     a = bench.algorithmic(w, R=16384, touched=8)
     assert a["up_flops"] == 4 * 16384 * 4096 * 14336
     assert a["layer_flops"] == 2 * 8192 * 4096 * 8 + 6 * 4096 * 14336 * 16384
@@ -83,10 +87,11 @@ def test_clock_summary_parses_reasons():
     c = bench.ClockSampler(0)
     import tempfile
     c.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-    c.file.write("0, 1920, 1965, 900.1, 0x4, Not Active, Not Active, Not Active, Active\n"
-                 "0, 1900, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active\n"
-                 "0, 600, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    c.file.write("0, 1920, 1965, 900.1, 0x4, Not Active, Not Active, Not Active, Active, 1000.00\n"
+                 "0, 1900, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active, 1000.00\n"
+                 "0, 600, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active, 1000.00\n")
     c.file.flush()
     s = c.summary()
     assert s["sm_mhz"] == pytest.approx(1910.0) and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+    assert s["power_limit_w"] == 1000.0 and s["power_max_w"] == 950.0

@@ -204,10 +204,47 @@ def test_empty_batch(dev):
     ops.moe_check_errors()
 
 
-def test_sigmoid_grouped_near_ties_bit_exact(dev):
+# Decode-sized batches (bf16, E % 8 == 0, T <= 128) route with the split-K
+# router and the fused gating/ranking kernel; T = 129 is the first batch on
+# the separate kernels.  Cases: one token; the largest batch with a ragged last
+# K slice (d = 448 is 7 steps of 64); 512 experts with variable k and padded
+# slots; 1024 experts with k = 32 (4096 slots ranked by one CTA) and capacity
+# drops; a small capacity factor.
+SMALL_BATCH = {
+    "t1_mixtral": WORKLOADS["mixtral_decode"].scaled(T=1, d=512, f=128),
+    "t128_dsv3_ragged_k": WORKLOADS["dsv3_decode"].scaled(T=128, d=448, f=64, f_shared=64),
+    "t129_dsv3": WORKLOADS["dsv3_decode"].scaled(T=129, d=448, f=64, f_shared=64),
+    "gptoss_e512_var_k": WORKLOADS["gptoss_sub"].scaled(T=100, d=200, f=72),
+    "e1024_k32_drops": WORKLOADS["qwen3_prefill"].scaled(T=128, d=128, E=1024, k_max=32, f=64),
+    "qwen3_cf_half": WORKLOADS["qwen3_prefill"].scaled(T=96, d=192, E=16, k_max=4, f=64,
+                                                       capacity_factor=0.5),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL_BATCH))
+def test_small_batch_route_bit_exact(name, dev):
+    w = SMALL_BATCH[name]
+    hin = _host_inputs(w, seed=3)
+    inp = gpu_inputs(w, 3, dev, hin)
+    cfg, out = run_route(w, inp)
+    ref = oracle.router_logits(to_numpy(hin["x"]), to_numpy(hin["Wr"]),
+                               to_numpy(hin["logit_bias"]))
+    assert_logits_close(out["logits"], ref)
+    check_routing_bit_exact(w, hin, out)
+
+
+@pytest.mark.parametrize("name", list(SMALL_BATCH))
+def test_small_batch_layer(name, dev):
+    w = SMALL_BATCH[name]
+    _layer_vs_oracle(w, _host_inputs(w, seed=4), dev)
+
+
+@pytest.mark.parametrize("T", [512, 128])
+def test_sigmoid_grouped_near_ties_bit_exact(T, dev):
     """Logits on a fine grid with many exact and one-ulp ties in the biased
-    scores: selection must follow the specified sigmoid bit for bit."""
-    w = SMALL["dsv3_small"].scaled(T=512)
+    scores: selection must follow the specified sigmoid bit for bit (T = 128
+    goes through the fused small-batch routing kernel)."""
+    w = SMALL["dsv3_small"].scaled(T=T)
     hin = _host_inputs(w)
     cfg = ops.config(w)
     g = torch.Generator().manual_seed(5)
