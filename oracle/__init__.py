@@ -6,7 +6,8 @@ does, and the two implementations share no code.
 
 Each function is a thin numpy <-> C marshaller around oracle/moe_oracle.c,
 where the arithmetic and its citations live.  Floating tensors are passed as
-numpy arrays of float32, or of uint16 holding bf16 bit patterns (dtype="bf16").
+numpy arrays of float32, or of uint16 holding bf16 bit patterns (dtype="bf16");
+the FFN and layer functions also take float64 weights (dequantised fp8).
 """
 from __future__ import annotations
 
@@ -17,7 +18,7 @@ import numpy as np
 
 from . import build as _build
 
-F32, BF16 = 0, 1
+F32, BF16, F64 = 0, 1, 2
 TOPK_SOFTMAX, SOFTMAX_TOPK_RENORM, SIGMOID_GROUPED = 0, 1, 2
 GATING = {"topk_softmax": TOPK_SOFTMAX, "softmax_topk_renorm": SOFTMAX_TOPK_RENORM,
           "sigmoid_grouped": SIGMOID_GROUPED}
@@ -57,7 +58,10 @@ def _declare(L):
     L.oracle_combine.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P]
     L.oracle_combine_rows.argtypes = [_I, _I, _I, _P, _P, _P, _P, _I, _P]
     L.oracle_layer_tokens.argtypes = [_I, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
-                                      _I, _P, _P, _P, _P]
+                                      _I, _I, _P, _P, _P, _P]
+    L.oracle_e4m3_decode_n.argtypes = [ctypes.c_longlong, _P, _P]
+    L.oracle_e4m3_encode_n.argtypes = [ctypes.c_longlong, _P, _P]
+    L.oracle_quantize_fp8.argtypes = [_I, _I, _I, _P, _P, _P]
 
 
 def _ptr(a):
@@ -73,7 +77,9 @@ def _dt(a) -> int:
         return F32
     if a.dtype == np.uint16:
         return BF16
-    raise TypeError(f"oracle tensors are float32 or uint16 (bf16 bits), got {a.dtype}")
+    if a.dtype == np.float64:
+        return F64
+    raise TypeError(f"oracle tensors are float32, uint16 (bf16 bits) or float64, got {a.dtype}")
 
 
 # --------------------------------------------------------------------------
@@ -226,8 +232,10 @@ def layer_tokens(tokens, x, W1, W3, W2, topk_idx, topk_w, slot_row, Ws1=None, Ws
     if Ws1 is not None:
         Ws1, Ws3, Ws2 = (np.ascontiguousarray(a) for a in (Ws1, Ws3, Ws2))
     out = np.empty((tok.size, d), np.float64)
+    if Ws1 is not None:
+        assert Ws1.dtype == W1.dtype, "routed and shared weights share one storage type"
     lib().oracle_layer_tokens(tok.size, _ptr(tok), d, E, k_max, f, fs, _ptr(x), _ptr(W1),
-                              _ptr(W3), _ptr(W2), _ptr(Ws1), _ptr(Ws3), _ptr(Ws2), _dt(x),
+                              _ptr(W3), _ptr(W2), _ptr(Ws1), _ptr(Ws3), _ptr(Ws2), _dt(x), _dt(W1),
                               _ptr(_c(topk_idx, np.int32)), _ptr(_c(topk_w, np.float64)),
                               _ptr(_c(slot_row, np.int32)), _ptr(out))
     return out
@@ -253,3 +261,41 @@ def layer(x, Wr, W1, W3, W2, *, k_max, gating_mode="topk_softmax", capacity_fact
     out = layer_tokens(np.arange(T, dtype=np.int32), x, W1, W3, W2, idx, w, disp["slot_row"],
                        Ws1, Ws3, Ws2)
     return dict(logits=logits, topk_idx=idx, topk_w=w, out=out, **disp)
+
+
+# --------------------------------------------------------------------------
+# FP8 expert weights ("LLM MoE Expert Parallel 生产实战", sections 5 and 10:
+# DeepSeek-V3 served with fp8 quantisation, router head kept in precision).
+# e4m3 codes with one fp32 scale per output column of each expert matrix.
+def e4m3_decode(codes) -> np.ndarray:
+    """The value of every e4m3 code (NaN for the two NaN codes), as float64."""
+    c = _c(codes, np.uint8)
+    out = np.empty(c.shape, np.float64)
+    lib().oracle_e4m3_decode_n(c.size, _ptr(c), _ptr(out))
+    return out
+
+
+def e4m3_encode(values) -> np.ndarray:
+    """Nearest e4m3 code of every float32 value, ties to even, saturating at 448."""
+    v = _c(values, np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().oracle_e4m3_encode_n(v.size, _ptr(v), _ptr(out))
+    return out
+
+
+def quantize_fp8(W):
+    """W: [G, K, N] bf16 bits (uint16).  Returns (codes uint8 [G, K, N],
+    scales float32 [G, N]): per output column s = max|W| / 448 in fp32 (1 for
+    an all-zero column) and codes e4m3(W / s) of the fp32 quotient."""
+    W = _c(W, np.uint16)
+    G, K, N = W.shape
+    q = np.empty((G, K, N), np.uint8)
+    s = np.empty((G, N), np.float32)
+    lib().oracle_quantize_fp8(G, K, N, _ptr(W), _ptr(q), _ptr(s))
+    return q, s
+
+
+def dequantize_fp8(q, s) -> np.ndarray:
+    """The weights the quantised layer computes with: e4m3_decode(q) * s per
+    output column, exact in float64 ([G, K, N])."""
+    return e4m3_decode(q) * np.asarray(s, np.float64)[:, None, :]

@@ -58,6 +58,7 @@
 
 #define OR_F32 0
 #define OR_BF16 1
+#define OR_F64 2 /* dequantised fp8 weights, exact in double */
 
 #define OR_TOPK_SOFTMAX 0
 #define OR_SOFTMAX_TOPK_RENORM 1
@@ -67,6 +68,7 @@
  * bf16 is the upper half of an IEEE binary32, so widening is a shift. */
 static double ld(const void *p, int dtype, size_t i) {
   if (dtype == OR_F32) return (double)((const float *)p)[i];
+  if (dtype == OR_F64) return ((const double *)p)[i];
   uint32_t bits = ((uint32_t)((const uint16_t *)p)[i]) << 16;
   float v;
   memcpy(&v, &bits, sizeof v);
@@ -443,7 +445,8 @@ void oracle_combine_rows(int T, int k_max, int d, const double *w, const int *sl
 }
 
 /* ------------------------------------------------------------------------ */
-/* Whole layer on a subset of tokens, for a given routing.                   */
+/* Whole layer on a subset of tokens, for a given routing.  x is stored in   */
+/* `dtype`, every weight in `w_dtype` (the same, or fp64 dequantised fp8).   */
 /* For each listed token t: out[i] = sum_j w[t,j] * FFN_{idx[t,j]}(x[t])      */
 /* over slots with slot_row >= 0, plus the shared expert's FFN(x[t]) when     */
 /* Ws1 is given.  W1, W3: [E, d, f]; W2: [E, f, d]; Ws1, Ws3: [d, fs];        */
@@ -452,10 +455,10 @@ void oracle_combine_rows(int T, int k_max, int d, const double *w, const int *sl
 void oracle_layer_tokens(int n_tok, const int *tok, int d, int E, int k_max, int f, int fs,
                          const void *x, const void *W1, const void *W3, const void *W2,
                          const void *Ws1, const void *Ws3, const void *Ws2, int dtype,
-                         const int *topk_idx, const double *topk_w, const int *slot_row,
-                         double *out) {
+                         int w_dtype, const int *topk_idx, const double *topk_w,
+                         const int *slot_row, double *out) {
   (void)E;
-  size_t esz = dtype == OR_F32 ? 4 : 2;
+  size_t esz = w_dtype == OR_F64 ? 8 : (w_dtype == OR_F32 ? 4 : 2);
   int fmax = f > fs ? f : fs;
 #pragma omp parallel
   {
@@ -469,7 +472,7 @@ void oracle_layer_tokens(int n_tok, const int *tok, int d, int E, int k_max, int
       double *o = out + (size_t)i * d;
       for (int c = 0; c < d; ++c) o[c] = 0.0;
       if (Ws1 && fs > 0) {
-        ffn_row(d, fs, x, dtype, (size_t)t * d, Ws1, Ws3, Ws2, dtype, xr, g, u, y);
+        ffn_row(d, fs, x, dtype, (size_t)t * d, Ws1, Ws3, Ws2, w_dtype, xr, g, u, y);
         for (int c = 0; c < d; ++c) o[c] += y[c];
       }
       for (int j = 0; j < k_max; ++j) {
@@ -478,7 +481,7 @@ void oracle_layer_tokens(int n_tok, const int *tok, int d, int E, int k_max, int
         int e = topk_idx[a];
         ffn_row(d, f, x, dtype, (size_t)t * d, (const char *)W1 + (size_t)e * d * f * esz,
                 (const char *)W3 + (size_t)e * d * f * esz,
-                (const char *)W2 + (size_t)e * f * d * esz, dtype, xr, g, u, y);
+                (const char *)W2 + (size_t)e * f * d * esz, w_dtype, xr, g, u, y);
         for (int c = 0; c < d; ++c) o[c] += topk_w[a] * y[c];
       }
     }
@@ -486,6 +489,85 @@ void oracle_layer_tokens(int n_tok, const int *tok, int d, int E, int k_max, int
     free(g);
     free(u);
     free(y);
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 expert weights.                                                       */
+/* "LLM MoE Expert Parallel 生产实战", section 5 (DeepSeek-V3 served with     */
+/* --quantization fp8) and section 10 (check that fp8 quantisation does not   */
+/* disturb the router head): the experts' weights are stored in 8-bit        */
+/* floating point while the router keeps its precision.  Reading: e4m3        */
+/* codes (OCP FP8 E4M3, the finite-only variant) with one fp32 scale per      */
+/* output column of each expert matrix; activations stay in the layer dtype. */
+/*                                                                          */
+/* e4m3: sign, 4 exponent bits (bias 7), 3 fraction bits.  Exponent field 0  */
+/* holds the subnormals m * 2^-9; 1..15 hold (1 + m/8) * 2^(e-7); the code   */
+/* with every exponent and fraction bit set is NaN, so the largest finite    */
+/* magnitude is 1.75 * 2^8 = 448.  There is no infinity.                     */
+/* ------------------------------------------------------------------------ */
+double oracle_e4m3_decode(uint8_t c) {
+  const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+/* Nearest e4m3 value, ties to the even code; finite magnitudes above 448
+ * saturate to 448; NaN maps to the NaN code. */
+uint8_t oracle_e4m3_encode(float v) {
+  if (isnan(v)) return 0x7F;
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  const double a = fabs((double)v);
+  if (a >= 448.0) return sign | 0x7E;
+  if (a == 0.0) return sign;
+  int ex;
+  frexp(a, &ex); /* a = f * 2^ex, f in [0.5, 1): floor(log2 a) = ex - 1 */
+  int E = ex - 1;
+  if (E < -6) E = -6; /* below the smallest normal the grid step stays 2^-9 */
+  const double step = ldexp(1.0, E - 3);
+  const double q = a / step; /* exact: division by a power of two */
+  double n = floor(q);
+  const double rem = q - n;
+  if (rem > 0.5 || (rem == 0.5 && fmod(n, 2.0) == 1.0)) n += 1.0;
+  const double val = n * step; /* the chosen grid point, <= 448 */
+  if (val == 0.0) return sign;
+  frexp(val, &ex);
+  const int Ev = ex - 1;
+  if (Ev < -6) return sign | (uint8_t)(val / ldexp(1.0, -9)); /* subnormal */
+  const int m = (int)(val / ldexp(1.0, Ev - 3)) - 8;
+  return sign | (uint8_t)((Ev + 7) << 3) | (uint8_t)m;
+}
+
+void oracle_e4m3_decode_n(long long n, const uint8_t *c, double *out) {
+  for (long long i = 0; i < n; ++i) out[i] = oracle_e4m3_decode(c[i]);
+}
+
+void oracle_e4m3_encode_n(long long n, const float *v, uint8_t *out) {
+  for (long long i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(v[i]);
+}
+
+/* Quantise W[g][k][n] (bf16 bits) per output column (g, n):
+ *   amax = max_k |W[g][k][n]|;  s = amax / 448 in fp32 (1 when amax = 0);
+ *   q[g][k][n] = e4m3(W[g][k][n] / s), the quotient rounded to fp32 first.
+ * The dequantised weight is e4m3_decode(q) * s. */
+void oracle_quantize_fp8(int G, int K, int N, const uint16_t *W, uint8_t *q, float *scale) {
+#pragma omp parallel for schedule(static)
+  for (long long gn = 0; gn < (long long)G * N; ++gn) {
+    const int g = (int)(gn / N), n = (int)(gn % N);
+    const size_t base = (size_t)g * K * N + n;
+    float amax = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      const double w = ld(W, OR_BF16, base + (size_t)k * N);
+      const float a = (float)fabs(w);
+      if (a > amax) amax = a;
+    }
+    const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+    scale[gn] = s;
+    for (int k = 0; k < K; ++k) {
+      const float w = (float)ld(W, OR_BF16, base + (size_t)k * N);
+      q[base + (size_t)k * N] = oracle_e4m3_encode(w / s);
+    }
   }
 }
 

@@ -34,6 +34,10 @@ MUTANTS = {
     "shared_expert_dropped": ("for (int c = 0; c < d; ++c) o[c] += y[c];",
                               "for (int c = 0; c < d; ++c) o[c] += 0.0 * y[c];"),
     "exp_lo_term_missing": ("r = fmaf(-n, OR_LN2_LO, r);", "r = r;"),
+    "e4m3_ties_away_from_zero": ("if (rem > 0.5 || (rem == 0.5 && fmod(n, 2.0) == 1.0)) n += 1.0;",
+                                 "if (rem >= 0.5) n += 1.0;"),
+    "e4m3_exponent_bias_8": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "fp8_scale_for_e5m2_range": ("amax / 448.0f : 1.0f", "amax / 57344.0f : 1.0f"),
 }
 
 

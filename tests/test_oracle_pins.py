@@ -417,3 +417,112 @@ def test_combine_worked_example():
     km = (sr >= 0).astype(np.int32)
     ys = np.where(km[..., None] > 0, y[np.maximum(sr, 0)], 0).astype(np.float64)
     assert oracle.combine(w, km, ys).tolist() == g["expect_no_shared"]
+
+
+# --------------------------------------------------------------------------
+# FP8 expert weights: e4m3 codes, per-output-column scales
+# --------------------------------------------------------------------------
+def _bf16_bits(a) -> np.ndarray:
+    return to_numpy(torch.as_tensor(np.asarray(a, np.float32)).to(torch.bfloat16))
+
+
+def test_e4m3_decode_known_codes():
+    """Values fixed by the format: bias 7, 3 fraction bits, subnormals m*2^-9,
+    the all-ones exponent-and-fraction code is NaN, no infinity."""
+    code = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6,
+            0x38: 1.0, 0x39: 1.125, 0x3C: 1.5, 0x40: 2.0, 0x77: 240.0, 0x78: 256.0,
+            0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0}
+    v = oracle.e4m3_decode(np.array(list(code), np.uint8))
+    assert v.tolist() == list(code.values())
+    assert np.isnan(oracle.e4m3_decode(np.uint8([0x7F, 0xFF]))).all()
+    neg0 = oracle.e4m3_decode(np.uint8([0x80]))[0]
+    assert neg0 == 0.0 and math.copysign(1.0, neg0) == -1.0
+    pos = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    assert (np.diff(pos) > 0).all()                      # codes 0..126 increase
+    assert (oracle.e4m3_decode(np.arange(0x80, 0xFF, dtype=np.uint8)) == -pos).all()
+
+
+def test_e4m3_encode_round_trip_ties_and_saturation():
+    c = np.arange(256, dtype=np.uint8)
+    v = oracle.e4m3_decode(c)
+    fin = ~np.isnan(v)
+    assert (oracle.e4m3_encode(v[fin].astype(np.float32)) == c[fin]).all()
+    pos = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    mid = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)  # exact in float32
+    got = oracle.e4m3_encode(mid).astype(int)
+    lower = np.arange(0x7E)
+    assert (got == np.where(lower % 2 == 0, lower, lower + 1)).all()  # ties to even
+    up = np.nextafter(mid, np.float32(np.inf))
+    dn = np.nextafter(mid, np.float32(0))
+    assert (oracle.e4m3_encode(up).astype(int) == lower + 1).all()
+    assert (oracle.e4m3_encode(dn).astype(int) == lower).all()
+    sat = oracle.e4m3_encode(np.float32([449, 464, 1e6, 3e38, -500, -np.inf, np.inf]))
+    assert sat.tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7E]
+    assert oracle.e4m3_encode(np.float32([np.nan]))[0] == 0x7F
+    assert oracle.e4m3_encode(np.float32([-0.0]))[0] == 0x80
+
+
+def test_e4m3_encode_matches_library_conversion_in_range():
+    """Inside the finite range, round-to-nearest-even to e4m3 is what torch's
+    float8_e4m3fn conversion does (out of range it saturates here, NaN there)."""
+    g = torch.Generator().manual_seed(21)
+    x = torch.cat([torch.randn(200000, generator=g) * s for s in (1e-3, 0.05, 1.0, 60.0)])
+    x = x[x.abs() < 448]
+    lib = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert (oracle.e4m3_encode(x.numpy()) == lib).all()
+
+
+def test_quantize_fp8_per_column_scales_and_error_bound():
+    rng = np.random.default_rng(22)
+    G, K, N = 3, 40, 24
+    W = rng.standard_normal((G, K, N)).astype(np.float32) * rng.uniform(0.01, 3, (G, 1, N))
+    W[1, :, 5] = 0.0                                       # an all-zero column
+    Wb = _bf16_bits(W)
+    q, s = oracle.quantize_fp8(Wb)
+    Wf = torch.from_numpy(Wb.astype(np.int32) << 16).view(torch.float32).numpy()
+    amax = np.abs(Wf).max(axis=1)
+    exp_s = np.where(amax > 0, (amax / np.float32(448)).astype(np.float32), np.float32(1))
+    assert (s == exp_s).all()
+    assert (q[1, :, 5] == 0).all() and s[1, 5] == 1.0
+    # the largest magnitude of every column maps to the largest code
+    kmax = np.abs(Wf).argmax(axis=1)
+    top = np.take_along_axis(q, kmax[:, None, :], axis=1)[:, 0, :]
+    nz = amax > 0
+    assert ((top[nz] & 0x7F) == 0x7E).all()
+    # dequantised weights are within half a grid step of the weight
+    deq = oracle.dequantize_fp8(q, s)
+    qv = Wf / s[:, None, :]
+    step = np.where(np.abs(qv) < 2.0 ** -6, 2.0 ** -9,
+                    2.0 ** (np.floor(np.log2(np.maximum(np.abs(qv), 1e-30))) - 3))
+    assert (np.abs(deq - Wf) <= 0.5 * step * s[:, None, :] * (1 + 1e-6)).all()
+
+
+def test_fp8_layer_equals_layer_on_representable_weights():
+    """Weights that are e4m3 values times a power-of-two column scale with the
+    column maximum at 448 * scale quantise exactly, so the layer on the
+    dequantised fp64 weights equals the layer on the bf16 weights."""
+    w, inp = _small_inputs("bf16", T=20, d=32, E=4, k=2, f=48, seed=23, fs=16)
+    rng = np.random.default_rng(24)
+    grid = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+
+    def representable(shape):
+        v = rng.choice(np.concatenate([grid, -grid]), size=shape)
+        G, K, N = shape
+        v[:, 0, :] = 448.0                              # column maximum
+        scale = 2.0 ** rng.integers(-12, -6, size=(G, 1, N))
+        return _bf16_bits(v * scale)
+
+    Wq = {k: representable(inp[k].shape) for k in ("W1", "W3", "W2")}
+    Sq = {k: representable((1,) + inp[k].shape) for k in ("Ws1", "Ws3", "Ws2")}
+    deq = {k: oracle.dequantize_fp8(*oracle.quantize_fp8(v)) for k, v in Wq.items()}
+    sdeq = {k: oracle.dequantize_fp8(*oracle.quantize_fp8(v))[0] for k, v in Sq.items()}
+    for k, v in Wq.items():  # the quantisation is exact
+        assert (deq[k] == torch.from_numpy(v.astype(np.int32) << 16).view(torch.float32)
+                .numpy()).all()
+    r = oracle.layer(inp["x"], inp["Wr"], Wq["W1"], Wq["W3"], Wq["W2"], k_max=2,
+                     Ws1=Sq["Ws1"][0], Ws3=Sq["Ws3"][0], Ws2=Sq["Ws2"][0])
+    tok = np.arange(w.T)
+    got = oracle.layer_tokens(tok, inp["x"], deq["W1"], deq["W3"], deq["W2"], r["topk_idx"],
+                              r["topk_w"], r["slot_row"], sdeq["Ws1"], sdeq["Ws3"],
+                              sdeq["Ws2"])
+    assert (got == r["out"]).all()
