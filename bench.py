@@ -23,7 +23,10 @@ Extra keys of the JSON line:
                of the layer output are inside the timed region;
   cpu_baseline the CPU oracle as it stands, on a bounded sample of the same
                workload, on the host cores (rank 0, N=1 only);
-  clocks       nvidia-smi samples taken during the timed region.
+  clocks       nvidia-smi samples taken during the timed region;
+  decode       the same layer at decode size (T=64), same keys;
+  fp8_weights  the decode-size layer with e4m3 expert weights and per-column
+               scales (quantised before timing), same keys.
 `--impl reference` times the CPU oracle alone on the same workload (the
 reference arm: there is no other implementation of this layer to run).
 """
@@ -201,17 +204,22 @@ def launches_per_layer(w) -> int:
     return n
 
 
-def algorithmic(w, R: int, touched: int) -> dict:
-    """Algorithmic work of the layer and of the up-projection grouped GEMM."""
+def algorithmic(w, R: int, touched: int, fp8: bool = False) -> dict:
+    """Algorithmic work of the layer and of the up-projection grouped GEMM.
+    With fp8 expert weights each weight is one byte plus its column's fp32
+    scale; the router stays in the layer dtype."""
     s = w.elem_bytes
+    ws = 1 if fp8 else s                              # bytes per expert weight
+    sc = 4 if fp8 else 0                              # bytes per column scale
     return {
         "layer_flops": 2 * w.T * w.d * w.E + 6 * w.d * w.f * R + 6 * w.d * w.f_shared * w.T,
-        "layer_bytes": (touched * 3 * w.d * w.f * s + 3 * w.d * w.f_shared * s + w.d * w.E * s
-                        + 2 * w.T * w.d * s),
+        "layer_bytes": (touched * (3 * w.d * w.f * ws + (2 * w.f + w.d) * sc)
+                        + 3 * w.d * w.f_shared * ws + (2 * w.f_shared + w.d) * sc * (w.f_shared > 0)
+                        + w.d * w.E * s + 2 * w.T * w.d * s),
         # K5: gate and up GEMMs over the R kept rows; reads the touched experts'
         # W1 and W3 and the R dispatched rows, writes h
         "up_flops": 4 * R * w.d * w.f,
-        "up_bytes": touched * 2 * w.d * w.f * s + R * w.d * s + R * w.f * s,
+        "up_bytes": touched * 2 * (w.d * w.f * ws + w.f * sc) + R * w.d * s + R * w.f * s,
     }
 
 
@@ -231,7 +239,7 @@ def traffic_from_profile(workload: str):
 
 
 class Layer:
-    def __init__(self, name: str, dev, seed: int, T: int = 0):
+    def __init__(self, name: str, dev, seed: int, T: int = 0, fp8: bool = False):
         from routing_dispatch_expert_sigmoid_b200 import ops
         self.ops = ops
         self.w = WORKLOADS[name] if T <= 0 else WORKLOADS[name].scaled(T=T)
@@ -240,6 +248,15 @@ class Layer:
         self.ws = ops.workspace(self.cfg, ops.WS_LAYER, device=dev)
         self.rb = ops.route_buffers(self.cfg, device=dev)
         self.out = torch.empty_like(self.inp["x"])
+        self.fp8 = None
+        if fp8:  # weight preparation, outside any timed region
+            i = self.inp
+            self.fp8 = (ops.fp8_weight_set(i["W1"], i["W3"], i["W2"]),
+                        ops.fp8_weight_set(i["Ws1"], i["Ws3"], i["Ws2"]) if self.w.f_shared
+                        else None)
+            for k in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2"):
+                i[k] = None  # the bf16 copies are not used by this layer
+            torch.cuda.empty_cache()
 
     def args(self, x=None, out=None):
         i = self.inp
@@ -248,10 +265,22 @@ class Layer:
                 self.out if out is None else out, self.rb, self.ws)
 
     def step(self, x=None, out=None):
-        self.ops.moe_layer(*self.args(x, out))
+        if self.fp8:
+            self._fp8_layer(x, out, None)
+        else:
+            self.ops.moe_layer(*self.args(x, out))
 
     def timed_step(self, events):
-        self.ops.moe_layer_timed(*self.args(), events)
+        if self.fp8:
+            self._fp8_layer(None, None, events)
+        else:
+            self.ops.moe_layer_timed(*self.args(), events)
+
+    def _fp8_layer(self, x, out, events):
+        i = self.inp
+        self.ops.moe_layer_fp8(self.cfg, i["x"] if x is None else x, i["Wr"], i["logit_bias"],
+                               i["sel_bias"], i["k_per_token"], self.fp8[0], self.fp8[1],
+                               self.out if out is None else out, self.rb, self.ws, events=events)
 
 
 def run_device(layer: Layer, steps: int, warmup: int, dist, gpu_index: int) -> dict:
@@ -392,6 +421,8 @@ def main():
     ap.add_argument("--T", type=int, default=0, help="override the main leg's token count")
     ap.add_argument("--decode-workload", default=DECODE,
                     choices=sorted(WORKLOADS) + ["none"], help="workload of the decode leg")
+    ap.add_argument("--fp8-workload", default=DECODE, choices=sorted(WORKLOADS) + ["none"],
+                    help="workload of the leg with fp8 expert weights")
     a = ap.parse_args()
     rank, local_rank, world = dist_env()
     warmup = max(a.warmup, 3)
@@ -478,6 +509,34 @@ def main():
         del dec
         torch.cuda.empty_cache()
 
+    fp8_obj = None
+    if a.fp8_workload != "none":
+        q = Layer(a.fp8_workload, dev, seed=rank, fp8=True)
+        qsteps = max(a.steps, 50)
+        rq = run_device(q, qsteps, warmup, dist, local_rank)
+        wq = q.w
+        q_ms_max, q_tokens = aggregate(rq["ms"], wq.T * qsteps, dist)
+        algq = algorithmic(wq, rq["R"], rq["touched"], fp8=True)
+        sustained_q = "sw_power_cap" in rq["clocks"]["reasons"]
+        roof_q = kernel_roofline(
+            algq, rq["stage_ms"]["up_swiglu"],
+            pk["bf16_tflops_sustained"] if sustained_q else pk["bf16_tflops"], pk["hbm_gbs"],
+            None, f"{pk_src} bf16 {'sustained' if sustained_q else 'burst'}",
+            f"{pk_src} copy bandwidth")
+        q_layer_roof_ms = max(algq["layer_flops"] / (pk["bf16_tflops"] * 1e12),
+                              algq["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
+        fp8_obj = {
+            "workload": f"{a.fp8_workload} with e4m3 expert weights (per-column fp32 scales)",
+            "steps": qsteps, "value": round(q_tokens / (q_ms_max * 1e-3), 1),
+            "unit": "tokens/s", "ms_per_step": round(q_ms_max / qsteps, 4),
+            "stage_ms": {k: round(v, 4) for k, v in rq["stage_ms"].items()},
+            "layer_roofline_ms": round(q_layer_roof_ms, 4),
+            "layer_roofline_frac": round(q_layer_roof_ms / (q_ms_max / qsteps), 4),
+            "roofline": roof_q, "gpu_launches": launches_per_layer(wq) * qsteps,
+        }
+        del q
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         n_tok = cpu_sample_tokens(a.workload, a.cpu_budget_s)
@@ -509,11 +568,13 @@ def main():
             "layer_roofline_frac": round(layer_roof_ms / (ms_max / a.steps), 4),
             "roofline": roof_pre,
             "decode": dec_obj,
+            "fp8_weights": fp8_obj,
             "e2e": None if e2e is None else {
                 "value": round(tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
             "gpu_launches": (launches_per_layer(w) * a.steps * (1 if e2e is None else 2)
-                             + (dec_obj["gpu_launches"] if dec_obj else 0)),
+                             + (dec_obj["gpu_launches"] if dec_obj else 0)
+                             + (fp8_obj["gpu_launches"] if fp8_obj else 0)),
             "clocks": rp["clocks"],
             "cpu_baseline": cpu,
         }

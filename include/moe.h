@@ -174,11 +174,13 @@ MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *W
  * outputs, a runtime whose device memory is fully planned in advance, a path
  * that must not call an allocator).  The pages have no counterpart: this is
  * an interface convenience, not a step of the method.  Results are those of
- * moe_route.  The scratch of the capacity step lives in a fixed 1 MiB device
- * array inside this library, held on every GPU that loads it until exit; a
- * configuration that needs more (8 * ceil(T*k_max/1024) * E bytes rounded up
- * to a multiple of 256, plus 256) is rejected with MOE_ERR_WORKSPACE before
- * anything is enqueued.  No
+ * moe_route.  The routing step's scratch lives in a fixed 1 MiB device array
+ * inside this library, held on every GPU that loads it until exit.  That
+ * scratch is the capacity step's 8 * ceil(T*k_max/1024) * E bytes (rounded up
+ * to a multiple of 256, plus 256), or, for bf16 layers with E % 8 == 0 and
+ * T <= 128, the split-K router's partial logits (at most 768 KiB) plus 256
+ * bytes.  A configuration that needs more than the array is rejected with
+ * MOE_ERR_WORKSPACE before anything is enqueued.  No
  * call allocates or frees memory.  The first call on a device looks up the
  * array's device address with that device current.  All calls share the
  * array, so calls whose work overlaps on the GPU (other streams or host
@@ -239,6 +241,48 @@ MOE_API moe_status moe_layer_timed(const moe_config *cfg, const void *x, const v
                                    const void *Ws2, void *out, const moe_route_out *route_out,
                                    void *ws, size_t ws_bytes, void *stream,
                                    void *const *events, int32_t n_events);
+
+/* ---- FP8 expert weights ----------------------------------------------------
+ * "LLM MoE Expert Parallel 生产实战" serves DeepSeek-V3 with fp8 quantisation
+ * (section 5) and warns to check that it leaves the router head alone
+ * (section 10).  Here the experts' matrices, routed and shared, are e4m3
+ * codes (OCP FP8 E4M3, the finite-only variant: bias 7, 3 fraction bits,
+ * largest magnitude 448) with one fp32 scale per output column: the weight
+ * the layer computes with is e4m3_value(code) * scale[column].  The router
+ * weights, activations and outputs stay in the layer dtype, which must be
+ * MOE_BF16; d, f and f_shared must be multiples of 16.  Codes are bytes in
+ * the bf16 weights' layout; every pointer is a device pointer, 16-byte
+ * aligned, owned by the caller. */
+typedef struct {
+  const void *W1, *W3;  /* [G, d, f] e4m3 codes */
+  const void *W2;       /* [G, f, d] e4m3 codes */
+  const float *s1, *s3; /* [G, f] column scales of W1, W3 */
+  const float *s2;      /* [G, d] column scales of W2 */
+} moe_fp8_weights;
+
+/* Weight preparation (not a hot call): W [G, K, N] bf16 -> Wq [G, K, N] e4m3
+ * codes and scale [G, N], with scale = max_k |W[g,k,n]| / 448 (fp32
+ * division; 1 for an all-zero column) and Wq = e4m3(W / scale) of the fp32
+ * quotient, rounded to nearest even, saturating at 448.  N % 16 == 0. */
+MOE_API moe_status moe_quantize_fp8(const void *W, int32_t G, int32_t K, int32_t N, void *Wq,
+                                    float *scale, void *stream);
+
+/* moe_expert_ffn with fp8 expert weights w (G = E).  ws: moe_workspace_size(
+ * cfg, MOE_WS_EXPERT_FFN). */
+MOE_API moe_status moe_expert_ffn_fp8(const moe_config *cfg, const void *x_perm,
+                                      const int32_t *offsets, const moe_fp8_weights *w,
+                                      void *y_perm, void *ws, size_t ws_bytes, void *stream);
+
+/* moe_layer with fp8 expert weights: `experts` (G = E) and, when
+ * cfg->f_shared > 0, `shared` (G = 1, f = f_shared; NULL otherwise).  Wr
+ * stays in cfg->dtype.  events / n_events as in moe_layer_timed (NULL / 0:
+ * none).  ws: moe_workspace_size(cfg, MOE_WS_LAYER). */
+MOE_API moe_status moe_layer_fp8(const moe_config *cfg, const void *x, const void *Wr,
+                                 const float *logit_bias, const float *sel_bias,
+                                 const int32_t *k_per_token, const moe_fp8_weights *experts,
+                                 const moe_fp8_weights *shared, void *out,
+                                 const moe_route_out *route_out, void *ws, size_t ws_bytes,
+                                 void *stream, void *const *events, int32_t n_events);
 
 /* Synchronises `stream`, then reads and clears the device error flags of the
  * current device.  *flags (may be NULL) receives them: bit 0 an index out of

@@ -39,6 +39,15 @@
 // once and A stays in L2.  All tiles of a launch have the same K, so the
 // deal is balanced to within one tile.
 //
+// FP8 weights (single engine, FP8W): B holds e4m3 codes and one fp32 scale
+// per output column of each group.  TMA brings the codes (64 x 64 bytes per
+// span) into a staging area of the stage; warps 6-9 widen them to bf16 --
+// exact, every e4m3 value is a bf16 value; integer bit moves and one packed
+// multiply, see e4m3x2_to_bf16x2 -- into the swizzled B layout the
+// MMA reads, fence the generic-proxy stores for the tensor cores and arrive
+// on the stage's "converted" barrier, which the MMA thread waits on instead
+// of "full".  The epilogue multiplies each column by its scale before SiLU.
+//
 // Every wait on an mbarrier is bounded (by %globaltimer): on expiry the CTA
 // records kErrWait in the device error word, tells its other roles to stop,
 // waits (again bounded) for its own copies and MMAs in flight, frees its
@@ -254,9 +263,11 @@ struct Params {
   // Word set to zero by the first thread of block 0 (a ticket the next
   // launch on the stream counts with), or nullptr.
   int32_t *clear = nullptr;
+  // FP8 weights: per-column scales of B1 and B3, [G, N] fp32
+  const float *scale1 = nullptr, *scale3 = nullptr;
 };
 
-template <bool SWIGLU, int SPANS>
+template <bool SWIGLU, int SPANS, bool FP8W = false>
 struct Shape {
   static constexpr int kSpans = SPANS;                // 64-column spans per B operand
   static constexpr int BN = 64 * SPANS;               // output columns per tile
@@ -264,9 +275,30 @@ struct Shape {
   static constexpr uint32_t kABytes = BM * BK * 2;    // 16 KB
   static constexpr uint32_t kSpanBytes = BK * 128;    // 8 KB: 64 K-rows x 128 B
   static constexpr uint32_t kBBytes = kBOps * kSpans * kSpanBytes;
+  // compute ring: A and (widened) B of one k-block per stage
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  // as many stages as fit in ~192 KB of the ring, at most 8
-  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  // bf16: as many stages as fit in ~192 KB, at most 8.  FP8W: two compute
+  // stages; the rest of the 192 KB is a deeper ring of e4m3 codes (64 K-rows
+  // x 64 bytes per span), the HBM stream, at most 8 deep.
+  static constexpr int kStages =
+      FP8W ? 2 : ((196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes));
+  static constexpr uint32_t kQSpanBytes = BK * 64;    // 4 KB
+  static constexpr uint32_t kQBytes = FP8W ? kBOps * kSpans * kQSpanBytes : 0;
+  // codes arrive in boxes of 128 columns (128-byte rows) where the tile is
+  // that wide, else 64
+  static constexpr int kQBox = SPANS >= 2 ? 128 : 64;
+  static constexpr uint32_t kQBoxBytes = BK * kQBox;
+  static constexpr int kQBoxesPerOp = 64 * SPANS / kQBox;
+  static constexpr int kQStages =
+      !FP8W ? 0
+            : ((196608 - kStages * kStageBytes) / kQBytes > 8
+                   ? 8
+                   : (196608 - kStages * kStageBytes) / kQBytes);
+  static constexpr uint32_t kRingBytes = kStages * kStageBytes + kQStages * kQBytes;
+  static constexpr uint32_t kTxBytes = FP8W ? kABytes : kStageBytes;  // TMA bytes per stage
+  // FP8W: + 4 converter warps (6-9) and an A-loading warp (10)
+  static constexpr int kCtaThreads = FP8W ? 352 : 192;
+  static constexpr int kConvThreads = 128;
   static constexpr int kMmaN = kBOps * BN;            // 256
   static constexpr uint32_t kAccCols = kMmaN;         // fp32 columns per accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccCols; // 512
@@ -277,7 +309,13 @@ struct Shape {
   static constexpr uint32_t kStageRowWords = 36;
   static constexpr uint32_t kEpiBytes = 4 * 32 * kStageRowWords * 4;  // 18 KB
   static constexpr size_t kSmemFixed =
-      1024 /*align slack*/ + kStages * kStageBytes + 256 + kEpiBytes;
+      1024 /*align slack*/ + kRingBytes + 256 + kEpiBytes;
+  // barriers: full, empty per stage, 2 + 2 accumulator, drain; FP8W also
+  // converted per stage and code-full, code-empty per code stage
+  static constexpr int kBars = FP8W ? 3 * kStages + 2 * kQStages + 5 : 2 * kStages + 5;
+  static_assert(kBars * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit 256 bytes");
+  static_assert(!FP8W || kQStages >= 2, "code ring");
+  static_assert(kQBytes % (16 * kConvThreads) == 0, "whole 16-byte chunks per converter");
   static_assert(kMmaN % 16 == 0 && kMmaN <= 256, "UMMA N");
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                 "TMEM allocation: a power of two in [32, 512] columns");
@@ -301,22 +339,114 @@ __device__ __forceinline__ void tile_of(int tile, const int32_t *s_tstart, const
   m = local - n * mt;
 }
 
-template <bool SWIGLU, int SPANS>
-__global__ void __launch_bounds__(kThreads, 1)
+// Two e4m3 codes (bytes 0 and 1 of `two`) to two bf16 values (the low half
+// from byte 0), on the integer and FMA pipes (the conversion instructions'
+// pipe is the narrow one).  Each byte goes to the top of a 16-bit half, so
+// its sign sits on the bf16 sign bit and its 4 exponent and 3 fraction bits,
+// shifted right by 4, on the low end of the bf16 exponent and the top of the
+// fraction.  Read as bf16 that is value * 2^-120 (exponent bias 127 instead
+// of 7) -- for e4m3 subnormals a bf16 subnormal of the same significand -- so
+// one exact multiply by 2^120 gives the value.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+  const uint32_t y = __byte_perm(two, 0u, 0x1404);  // bytes: 0, b0, 0, b1
+  const uint32_t bits = ((y >> 4) & 0x07F007F0u) | (y & 0x80008000u);
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&bits);
+  const __nv_bfloat162 k = __floats2bfloat162_rn(0x1p120f, 0x1p120f);  // exact in bf16
+  v = __hmul2(v, k);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+__device__ __forceinline__ void e4m3x16_to_bf16(uint4 c, uint4 &lo, uint4 &hi) {
+  lo = make_uint4(e4m3x2_to_bf16x2(c.x & 0xffffu), e4m3x2_to_bf16x2(c.x >> 16),
+                  e4m3x2_to_bf16x2(c.y & 0xffffu), e4m3x2_to_bf16x2(c.y >> 16));
+  hi = make_uint4(e4m3x2_to_bf16x2(c.z & 0xffffu), e4m3x2_to_bf16x2(c.z >> 16),
+                  e4m3x2_to_bf16x2(c.w & 0xffffu), e4m3x2_to_bf16x2(c.w >> 16));
+}
+// Shared-memory stores of this thread become visible to the tensor cores'
+// (async proxy) reads that are ordered after it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Widen one k-block of e4m3 codes (kQ bytes at q: boxes of 64 K-rows x QB
+// bytes, QB = 64 or 128 columns, box b covering 64-column spans QB/64 * b ..)
+// into 64-column bf16 spans of 64 K-rows x 128 bytes, 8 KB apart, with the
+// 128-byte swizzle TMA would apply (16-byte slot XOR K-row mod 8).  `ct` is
+// the thread's index among the 128 converter threads.  With 128-column boxes
+// a quarter warp takes the first half of one K-row and the second half of
+// the next (or the reverse), so both its loads and its stores hit 32
+// distinct banks.
+template <int QB, uint32_t kQ>
+__device__ __forceinline__ void widen_codes(const uint8_t *__restrict__ q,
+                                            uint8_t *__restrict__ w, int ct) {
+  constexpr int kIt = kQ >= 16 * 128 ? (int)(kQ / 16 / 128) : 1;
+  if (kQ < 16 * 128) return;  // bf16 instantiations: no codes
+  int off_q[kIt], off_w[kIt], kr[kIt], jj[kIt];
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) {
+    const int c = it * 128 + ct;  // 16-byte code chunk
+    int blk, k, span, j;
+    if (QB == 64) {
+      blk = c >> 8;
+      k = (c >> 2) & 63;
+      span = 0;
+      j = c & 3;
+    } else {
+      blk = c >> 9;  // 64 K-rows x 8 chunks per box
+      const int r = c & 511, t = r & 31, qq = t >> 3, i = (t >> 2) & 1;
+      j = t & 3;
+      k = (r >> 5) * 4 + 2 * (qq >> 1) + i;
+      span = i ^ (qq & 1);
+    }
+    off_q[it] = blk * (64 * QB) + k * QB + (span * 4 + j) * 16;
+    off_w[it] = (blk * (QB / 64) + span) * 8192 + k * 128;
+    kr[it] = k & 7;
+    jj[it] = j;
+  }
+  // every load first, so their latencies overlap; then widen and store
+  uint4 codes[kIt];
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) codes[it] = *reinterpret_cast<const uint4 *>(q + off_q[it]);
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) {
+    uint4 lo, hi;
+    e4m3x16_to_bf16(codes[it], lo, hi);
+    uint8_t *rowp = w + off_w[it];
+    *reinterpret_cast<uint4 *>(rowp + (((2 * jj[it]) ^ kr[it]) << 4)) = lo;
+    *reinterpret_cast<uint4 *>(rowp + (((2 * jj[it] + 1) ^ kr[it]) << 4)) = hi;
+  }
+}
+
+// v[i] *= scale[col + i] for the columns below N (N a multiple of 16, col a
+// multiple of 32, scale 16-byte aligned: a float4 is whole or absent).
+__device__ __forceinline__ void scale_cols(float (&v)[32], const float *scale, int col, int N) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    if (col + 4 * q < N) {
+      const float4 sc = __ldg(reinterpret_cast<const float4 *>(scale + col + 4 * q));
+      v[4 * q] *= sc.x;
+      v[4 * q + 1] *= sc.y;
+      v[4 * q + 2] *= sc.z;
+      v[4 * q + 3] *= sc.w;
+    }
+  }
+}
+
+template <bool SWIGLU, int SPANS, bool FP8W = false>
+__global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
                    const __grid_constant__ CUtensorMap tmB3, const Params p) {
-  using S = Shape<SWIGLU, SPANS>;
+  using S = Shape<SWIGLU, SPANS, FP8W>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *ring = smem;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + S::kStages * S::kStageBytes);
-  // bars: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain[1]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S::kStages + 5);
+  uint8_t *ring = smem;                                  // compute stages
+  uint8_t *qring = ring + S::kStages * S::kStageBytes;   // FP8W: code stages
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + S::kRingBytes);
+  // bars: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain[1];
+  // FP8W: converted[kStages], code_full[kQStages], code_empty[kQStages]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + S::kBars);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-  float *s_epi = reinterpret_cast<float *>(ring + S::kStages * S::kStageBytes + 256);
-  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kStages * S::kStageBytes + 256 +
-                                               S::kEpiBytes);
+  float *s_epi = reinterpret_cast<float *>(ring + S::kRingBytes + 256);
+  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kRingBytes + 256 + S::kEpiBytes);
   int32_t *s_tstart = s_off + (p.G + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -324,6 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t accf0 = smem_addr(bars + 2 * S::kStages);
   const uint32_t acce0 = smem_addr(bars + 2 * S::kStages + 2);
   const uint32_t drain = smem_addr(bars + 2 * S::kStages + 4);
+  const uint32_t conv0 = smem_addr(bars + 2 * S::kStages + 5);
+  const uint32_t qfull0 = smem_addr(bars + 3 * S::kStages + 5);
+  const uint32_t qempty0 = smem_addr(bars + 3 * S::kStages + 5 + S::kQStages);
   const Ctl ctl{abort_flag, p.err};
 
   if (threadIdx.x == 0) {
@@ -336,6 +469,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(acce0 + 8 * b, 4);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
+    if (FP8W) {
+      for (int s = 0; s < S::kStages; ++s) mbar_init(conv0 + 8 * s, S::kConvThreads / 32);
+      for (int s = 0; s < S::kQStages; ++s) {
+        mbar_init(qfull0 + 8 * s, 1);
+        mbar_init(qempty0 + 8 * s, S::kConvThreads / 32);
+      }
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -348,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // per-group tile counts), checked against the buffer size.
   bool bad = false;
   if (p.clear && blockIdx.x == 0 && threadIdx.x == 0) *p.clear = 0;
-  for (int g = threadIdx.x; g <= p.G; g += kThreads) {
+  for (int g = threadIdx.x; g <= p.G; g += S::kCtaThreads) {
     const int v = p.offsets ? p.offsets[g]
                             : (p.k_split ? g * p.fixed_rows : (g == 0 ? 0 : p.fixed_rows));
     s_off[g] = v;
@@ -357,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
   __syncthreads();
   const int n_tiles = (p.N + S::BN - 1) / S::BN;
-  for (int g = threadIdx.x; g < p.G; g += kThreads) {
+  for (int g = threadIdx.x; g < p.G; g += S::kCtaThreads) {
     const int rows = s_off[g + 1] - s_off[g];
     if (rows < 0) bad = true;
     s_tstart[g] = rows > 0 ? ((rows + BM - 1) / BM) * n_tiles : 0;
@@ -391,11 +531,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = *abort_flag ? 0 : s_tstart[p.G];
   const int num_kb = p.k_split ? p.k_split / BK : (p.K + BK - 1) / BK;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || (FP8W && warp == 10)) {
+    // ------------------------------------------------------------ producers
     // Lane 0 waits and issues the tiled loads; when the A rows are gathered,
-    // every lane issues one gather4 (4 of the tile's 128 rows).
+    // every lane issues one gather4 (4 of the tile's 128 rows).  With fp8
+    // weights warp 0 streams the e4m3 codes through the code ring and warp
+    // 10 loads the A tiles into the compute ring, so the code stream runs
+    // ahead of the compute stages.
+    const bool codes = FP8W && warp == 0;
+    const bool load_a = !FP8W || warp == 10;
     const bool gather = p.row_src != nullptr;
+    const int nst = codes ? S::kQStages : S::kStages;
+    const uint32_t fullb = codes ? qfull0 : full0, emptyb = codes ? qempty0 : empty0;
     int s = 0;
     uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
     bool ok = true;
@@ -416,41 +563,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int kb = 0; kb < num_kb; ++kb) {
         int okw = 1;
-        if (lane == 0) okw = wait(empty0 + 8 * s, ph ^ 1, ctl) ? 1 : 0;
+        if (lane == 0) okw = wait(emptyb + 8 * s, ph ^ 1, ctl) ? 1 : 0;
         okw = __shfl_sync(0xffffffffu, okw, 0);
         if (!okw) {
           ok = false;
           break;
         }
-        const uint32_t st = smem_addr(ring + s * S::kStageBytes);
-        const uint32_t fb = full0 + 8 * s;
-        if (lane == 0) mbar_expect_tx(fb, S::kStageBytes);
-        if (gather)
-          tma_gather4(st + lane * 4 * 128, &tmA, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
-        if (lane == 0) {
-          if (!gather) tma_load_2d(st, &tmA, fb, k0 + kb * BK, row);
+        const uint32_t fb = fullb + 8 * s;
+        if (codes) {
+          const uint32_t qt = smem_addr(qring + s * S::kQBytes);
+          if (lane == 0) {
+            mbar_expect_tx(fb, S::kQBytes);
 #pragma unroll
-          for (int j = 0; j < S::kSpans; ++j)
-            tma_load_3d(st + S::kABytes + j * S::kSpanBytes, &tmB1, fb, n * S::BN + j * 64,
-                        k0 + kb * BK, gb);
-          if (SWIGLU) {
+            for (int b = 0; b < S::kQBoxesPerOp; ++b)
+              tma_load_3d(qt + b * S::kQBoxBytes, &tmB1, fb, n * S::BN + b * S::kQBox,
+                          k0 + kb * BK, gb);
+            if (SWIGLU) {
 #pragma unroll
-            for (int j = 0; j < S::kSpans; ++j)
-              tma_load_3d(st + S::kABytes + (S::kSpans + j) * S::kSpanBytes, &tmB3, fb,
-                          n * S::BN + j * 64, k0 + kb * BK, gb);
+              for (int b = 0; b < S::kQBoxesPerOp; ++b)
+                tma_load_3d(qt + (S::kQBoxesPerOp + b) * S::kQBoxBytes, &tmB3, fb,
+                            n * S::BN + b * S::kQBox, k0 + kb * BK, gb);
+            }
+          }
+        } else {
+          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+          if (lane == 0) mbar_expect_tx(fb, S::kTxBytes);
+          if (gather)
+            tma_gather4(st + lane * 4 * 128, &tmA, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
+          if (lane == 0) {
+            if (!gather && load_a) tma_load_2d(st, &tmA, fb, k0 + kb * BK, row);
+            if (!FP8W) {
+#pragma unroll
+              for (int j = 0; j < S::kSpans; ++j)
+                tma_load_3d(st + S::kABytes + j * S::kSpanBytes, &tmB1, fb, n * S::BN + j * 64,
+                            k0 + kb * BK, gb);
+              if (SWIGLU) {
+#pragma unroll
+                for (int j = 0; j < S::kSpans; ++j)
+                  tma_load_3d(st + S::kABytes + (S::kSpans + j) * S::kSpanBytes, &tmB3, fb,
+                              n * S::BN + j * 64, k0 + kb * BK, gb);
+              }
+            }
           }
         }
         issued_mask |= 1u << s;
         issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
-        if (++s == S::kStages) {
+        if (++s == nst) {
           s = 0;
           ph ^= 1;
         }
       }
     }
     if (!ok && lane == 0) {  // stopped early: let the copies already issued land first
-      for (int q = 0; q < S::kStages; ++q)
-        if ((issued_mask >> q) & 1u) wait_drain(full0 + 8 * q, (issued_parity >> q) & 1u, p.err);
+      for (int q = 0; q < nst; ++q)
+        if ((issued_mask >> q) & 1u) wait_drain(fullb + 8 * q, (issued_parity >> q) & 1u, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -466,7 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * S::kAccCols;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait(full0 + 8 * s, ph, ctl)) {
+          // FP8W: the A tile has landed and the converters have filled B
+          if (!wait(full0 + 8 * s, ph, ctl) || (FP8W && !wait(conv0 + 8 * s, ph, ctl))) {
             ok = false;
             break;
           }
@@ -499,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     int buf = 0;
@@ -523,13 +690,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lane = row: 32 consecutive columns of its row from tensor memory
         float v[32];
         tmem_ld32(tb + c, v);
+        const int col = n * S::BN + c;
+        if (FP8W) scale_cols(v, p.scale1 + (size_t)g * p.N, col, p.N);
         if (SWIGLU) {
           float u[32];
           tmem_ld32(tb + S::BN + c, u);
+          if (FP8W) scale_cols(u, p.scale3 + (size_t)g * p.N, col, p.N);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
         }
-        const int col = n * S::BN + c;
         // Stage the 32 x 32 chunk in shared memory, then write it back row by
         // row so that each warp store covers whole 64/128-byte row segments.
         if (SWIGLU) {  // h: bf16, a row is 16 words
@@ -586,6 +755,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(acce0 + 8 * buf);
       buf ^= 1;
       if (buf == 0) acc_ph ^= 1;
+    }
+  } else if (FP8W && warp >= 6 && warp < 10) {
+    // ------------------------------------------------------------ fp8 converters
+    // Per k-block: wait for its codes (code stage qs) and for a free compute
+    // stage s, widen them into the stage's B tile, release the code stage and
+    // mark the compute stage converted.
+    const int ct = threadIdx.x - 192;
+    int s = 0, qs = 0;
+    uint32_t ph = 0, qph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < num_kb; ++kb) {
+        int okw = 1;
+        if (lane == 0)
+          okw = (wait(qfull0 + 8 * qs, qph, ctl) && wait(empty0 + 8 * s, ph ^ 1, ctl)) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) {
+          ok = false;
+          break;
+        }
+        widen_codes<S::kQBox, S::kQBytes>(qring + qs * S::kQBytes,
+                                          ring + s * S::kStageBytes + S::kABytes, ct);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(qempty0 + 8 * qs);
+          mbar_arrive(conv0 + 8 * s);
+        }
+        if (++qs == S::kQStages) {
+          qs = 0;
+          qph ^= 1;
+        }
+        if (++s == S::kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
     }
   }
 
@@ -1042,22 +1248,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 constexpr int kRowBox = 32;  // rows per TMA box of the N operand
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool FP8W = false>
 struct ShapeSwap {
   static constexpr int kCols = 128;                      // output columns per tile (MMA M)
-  static constexpr int kMaxRows = 128;                   // rows per tile (MMA N <= 128)
+  // rows per tile (MMA N): fp8 weights keep decode-sized row tiles so that
+  // a stage stays small and the code stream can run deep
+  static constexpr int kMaxRows = FP8W ? 32 : 128;
   static constexpr int kWOps = SWIGLU ? 2 : 1;
   static constexpr uint32_t kSpanBytes = BK * 128;       // 8 KB: 64 K-rows x 64 columns
-  static constexpr uint32_t kWBytes = kWOps * 2 * kSpanBytes;   // 16 or 32 KB
+  static constexpr uint32_t kWBytes = kWOps * 2 * kSpanBytes;   // 16 or 32 KB (bf16)
   static constexpr uint32_t kRowBoxBytes = kRowBox * BK * 2;    // 4 KB
-  static constexpr uint32_t kXBytes = kMaxRows * BK * 2;        // 16 KB
-  static constexpr uint32_t kStageBytes = kWBytes + kXBytes;
-  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  static constexpr uint32_t kXBytes = kMaxRows * BK * 2;        // 16 KB (fp8: 4 KB)
+  static constexpr uint32_t kQSpanBytes = BK * 64;              // e4m3 codes of a span
+  static constexpr uint32_t kQBytes = FP8W ? kWOps * 2 * kQSpanBytes : 0;
+  static constexpr int kQBox = 128;                             // one code box per operand
+  static constexpr uint32_t kQBoxBytes = BK * kQBox;
+  // a stage: the weights (bf16, or e4m3 codes) and the rows of one k-block;
+  // FP8W adds kCStages compute stages of widened bf16 weights
+  static constexpr uint32_t kStageBytes = (FP8W ? kQBytes : kWBytes) + kXBytes;
+  static constexpr int kCStages = FP8W ? 3 : 0;  // 3 measured faster than 2 on decode
+  static constexpr uint32_t kCBytes = FP8W ? kWBytes : 0;
+  static constexpr int kStages = ((196608 - kCStages * kCBytes) / kStageBytes) > 8
+                                     ? 8
+                                     : ((196608 - kCStages * kCBytes) / kStageBytes);
+  static constexpr uint32_t kRingBytes = kStages * kStageBytes + kCStages * kCBytes;
+  static constexpr int kCtaThreads = FP8W ? 320 : 192;  // + 4 converter warps
+  static constexpr int kConvThreads = 128;
   static constexpr uint32_t kAccCols = SWIGLU ? 256 : 128;
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static constexpr uint32_t kStageRowWords = 36;
   static constexpr uint32_t kEpiBytes = 4 * 32 * kStageRowWords * 4;
-  static constexpr size_t kSmemFixed = 1024 + kStages * kStageBytes + 256 + kEpiBytes;
+  static constexpr size_t kSmemFixed = 1024 + kRingBytes + 256 + kEpiBytes;
+  static constexpr int kBars = 2 * kStages + 2 * kCStages + 5;
+  static_assert(kBars * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit 256 bytes");
+  static_assert((kStages * kStageBytes) % 1024 == 0 && (FP8W ? kQBytes : kWBytes) % 1024 == 0,
+                "128-byte swizzled tiles start on 1024-byte boundaries");
+  static_assert(kQBytes % (16 * kConvThreads) == 0, "whole 16-byte chunks per converter");
 };
 
 // kind::f16 descriptor: fp32 accumulator, bf16 A and B, A MN-major, B K-major.
@@ -1066,22 +1292,22 @@ __device__ __forceinline__ uint32_t instr_desc_swap(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-template <bool SWIGLU>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool SWIGLU, bool FP8W = false>
+__global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
     k_grouped_gemm_swap(const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmW1,
                         const __grid_constant__ CUtensorMap tmW3, const Params p) {
-  using S = ShapeSwap<SWIGLU>;
+  using S = ShapeSwap<SWIGLU, FP8W>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *ring = smem;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + S::kStages * S::kStageBytes);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S::kStages + 5);
+  uint8_t *cring = ring + S::kStages * S::kStageBytes;  // FP8W: widened weights
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + S::kRingBytes);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + S::kBars);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-  float *s_epi = reinterpret_cast<float *>(ring + S::kStages * S::kStageBytes + 256);
-  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kStages * S::kStageBytes + 256 +
-                                               S::kEpiBytes);
+  float *s_epi = reinterpret_cast<float *>(ring + S::kRingBytes + 256);
+  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kRingBytes + 256 + S::kEpiBytes);
   int32_t *s_tstart = s_off + (p.G + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -1089,6 +1315,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t accf0 = smem_addr(bars + 2 * S::kStages);
   const uint32_t acce0 = smem_addr(bars + 2 * S::kStages + 2);
   const uint32_t drain = smem_addr(bars + 2 * S::kStages + 4);
+  // FP8W: converted[kCStages], compute-stage empty[kCStages]
+  const uint32_t conv0 = smem_addr(bars + 2 * S::kStages + 5);
+  const uint32_t cempty0 = smem_addr(bars + 2 * S::kStages + 5 + S::kCStages);
   const Ctl ctl{abort_flag, p.err};
 
   if (threadIdx.x == 0) {
@@ -1101,6 +1330,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(acce0 + 8 * b, 4);
     }
     mbar_init(drain, 1);
+    for (int c = 0; c < S::kCStages; ++c) {
+      mbar_init(conv0 + 8 * c, S::kConvThreads / 32);
+      mbar_init(cempty0 + 8 * c, 1);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1110,7 +1343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (SWIGLU) prefetch_tmap(&tmW3);
   }
   bool bad = false;
-  for (int g = threadIdx.x; g <= p.G; g += kThreads) {
+  for (int g = threadIdx.x; g <= p.G; g += S::kCtaThreads) {
     const int v = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.fixed_rows);
     s_off[g] = v;
     if (v < 0 || v > p.rows_cap) bad = true;
@@ -1118,7 +1351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
   __syncthreads();
   const int col_tiles = (p.N + S::kCols - 1) / S::kCols;
-  for (int g = threadIdx.x; g < p.G; g += kThreads) {
+  for (int g = threadIdx.x; g < p.G; g += S::kCtaThreads) {
     const int rows = s_off[g + 1] - s_off[g];
     if (rows < 0) bad = true;
     s_tstart[g] = rows > 0 ? ((rows + S::kMaxRows - 1) / S::kMaxRows) * col_tiles : 0;
@@ -1181,7 +1414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_coords(tile, g, c, r, row0, nr);
       // rows loaded: 32-row boxes, or (gathering) gather4s up to the MMA's N
       const int nq = gather ? ((nr + 15) & ~15) / 4 : (nr + kRowBox - 1) / kRowBox;
-      const uint32_t bytes = S::kWBytes + (gather ? nq * 512 : nq * S::kRowBoxBytes);
+      const uint32_t wbytes = FP8W ? S::kQBytes : S::kWBytes;  // where the rows start
+      const uint32_t bytes = wbytes + (gather ? nq * 512 : nq * S::kRowBoxBytes);
       int tok[4] = {0, 0, 0, 0};
       if (gather && lane < nq) {
 #pragma unroll
@@ -1202,21 +1436,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = full0 + 8 * s;
         if (lane == 0) mbar_expect_tx(fb, bytes);
         if (gather && lane < nq)
-          tma_gather4(st + S::kWBytes + lane * 4 * 128, &tmX, fb, kb * BK, tok[0], tok[1],
-                      tok[2], tok[3]);
+          tma_gather4(st + wbytes + lane * 4 * 128, &tmX, fb, kb * BK, tok[0], tok[1], tok[2],
+                      tok[3]);
         if (lane == 0) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-            tma_load_3d(st + j * S::kSpanBytes, &tmW1, fb, c * S::kCols + j * 64, kb * BK, g);
-          if (SWIGLU) {
+          if (FP8W) {  // one 128-column box of codes per operand
+            tma_load_3d(st, &tmW1, fb, c * S::kCols, kb * BK, g);
+            if (SWIGLU) tma_load_3d(st + S::kQBoxBytes, &tmW3, fb, c * S::kCols, kb * BK, g);
+          } else {
 #pragma unroll
             for (int j = 0; j < 2; ++j)
-              tma_load_3d(st + (2 + j) * S::kSpanBytes, &tmW3, fb, c * S::kCols + j * 64,
-                          kb * BK, g);
+              tma_load_3d(st + j * S::kSpanBytes, &tmW1, fb, c * S::kCols + j * 64, kb * BK, g);
+            if (SWIGLU) {
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                tma_load_3d(st + (2 + j) * S::kSpanBytes, &tmW3, fb, c * S::kCols + j * 64,
+                            kb * BK, g);
+            }
           }
           if (!gather)
             for (int q = 0; q < nq; ++q)
-              tma_load_2d(st + S::kWBytes + q * S::kRowBoxBytes, &tmX, fb, kb * BK,
+              tma_load_2d(st + wbytes + q * S::kRowBoxBytes, &tmX, fb, kb * BK,
                           row0 + q * kRowBox);
         }
         issued_mask |= 1u << s;
@@ -1234,8 +1473,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int s = 0, buf = 0;
-      uint32_t ph = 0, acc_ph = 0;
+      int s = 0, buf = 0, cs = 0;
+      uint32_t ph = 0, acc_ph = 0, cph = 0;
       bool ok = true, any = false;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int g, c, r, row0, nr;
@@ -1248,29 +1487,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * S::kAccCols;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!wait(full0 + 8 * s, ph, ctl)) {
+          // FP8W: the rows have landed and the converters have filled the weights
+          if (!wait(full0 + 8 * s, ph, ctl) || (FP8W && !wait(conv0 + 8 * cs, cph, ctl))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+          const uint32_t wt = FP8W ? smem_addr(cring + cs * S::kCBytes) : st;
+          const uint32_t xt = st + (FP8W ? S::kQBytes : S::kWBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             // weights: MN-major spans (LBO = span stride), rows: K-major 128-byte rows
-            const uint64_t xd = smem_desc(st + S::kWBytes + kk * 32, 16, 1024);
-            const uint64_t w1d = smem_desc(st + kk * 2048, S::kSpanBytes, 1024);
+            const uint64_t xd = smem_desc(xt + kk * 32, 16, 1024);
+            const uint64_t w1d = smem_desc(wt + kk * 2048, S::kSpanBytes, 1024);
             umma(d_tmem, w1d, xd, idesc, (kb | kk) != 0);
             if (SWIGLU) {
-              const uint64_t w3d = smem_desc(st + 2 * S::kSpanBytes + kk * 2048, S::kSpanBytes,
+              const uint64_t w3d = smem_desc(wt + 2 * S::kSpanBytes + kk * 2048, S::kSpanBytes,
                                              1024);
               umma(d_tmem + 128, w3d, xd, idesc, (kb | kk) != 0);
             }
           }
           any = true;
           umma_commit(empty0 + 8 * s);
+          if (FP8W) umma_commit(cempty0 + 8 * cs);
           if (++s == S::kStages) {
             s = 0;
             ph ^= 1;
+          }
+          if (FP8W && ++cs == S::kCStages) {
+            cs = 0;
+            cph ^= 1;
           }
         }
         if (!ok) break;
@@ -1284,7 +1531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------ epilogue
     // TMEM lane = output column (this warp: columns 32*quarter ..), TMEM
     // column = row of the tile.
@@ -1302,13 +1549,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + buf * S::kAccCols + ((uint32_t)(quarter * 32) << 16);
       const int col0 = c * S::kCols + quarter * 32;  // this warp's 32 output columns
+      // FP8W: this lane's column scales (lane = column)
+      float sc1 = 1.f, sc3 = 1.f;
+      if (FP8W && col0 + lane < p.N) {
+        sc1 = p.scale1[(size_t)g * p.N + col0 + lane];
+        if (SWIGLU) sc3 = p.scale3[(size_t)g * p.N + col0 + lane];
+      }
 #pragma unroll 1
       for (int j0 = 0; j0 < nr; j0 += 32) {
         float v[32];
         tmem_ld32(tb + j0, v);  // v[j] = out[row j0 + j][col0 + lane]
+        if (FP8W) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= sc1;
+        }
         if (SWIGLU) {
           float u[32];
           tmem_ld32(tb + 128 + j0, u);
+          if (FP8W) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] *= sc3;
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
         }
@@ -1358,6 +1619,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(acce0 + 8 * buf);
       buf ^= 1;
       if (buf == 0) acc_ph ^= 1;
+    }
+  } else if (FP8W) {
+    // ------------------------------------------------------------ fp8 converters
+    // Per k-block: wait for its codes (stage s) and a free compute stage cs,
+    // widen the codes into the swizzled bf16 weight tiles the MMA reads (see
+    // the single engine's converters; same layout), mark cs converted.
+    const int ct = threadIdx.x - 192;
+    int s = 0, cs = 0;
+    uint32_t ph = 0, cph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < num_kb; ++kb) {
+        int okw = 1;
+        if (lane == 0)
+          okw = (wait(full0 + 8 * s, ph, ctl) && wait(cempty0 + 8 * cs, cph ^ 1, ctl)) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) {
+          ok = false;
+          break;
+        }
+        widen_codes<S::kQBox, S::kQBytes>(ring + s * S::kStageBytes, cring + cs * S::kCBytes,
+                                          ct);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(conv0 + 8 * cs);
+        if (++s == S::kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+        if (++cs == S::kCStages) {
+          cs = 0;
+          cph ^= 1;
+        }
+      }
     }
   }
 
@@ -1427,6 +1722,53 @@ bool make_map_b(CUtensorMap *m, const void *B, int G, int K, int N) {
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(B), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over e4m3 codes B [G, K, N] (one byte each, N contiguous), box
+// box_cols (N) x 64 (K) x 1, no swizzle: the converter warps apply the
+// 128-byte swizzle when they write the widened bf16 tile.
+bool make_map_b_q8(CUtensorMap *m, const void *B, int G, int K, int N, int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)G};
+  cuuint64_t strides[2] = {(cuuint64_t)N, (cuuint64_t)K * N};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)BK, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(B), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The single engine on e4m3 weights with per-column scales.
+template <bool SWIGLU, int SPANS>
+cudaError_t launch_q8(int rows_cap, int K, int N, int G, const int32_t *offsets, int fixed_rows,
+                      const void *A, const void *B1, const void *B3, const float *s1,
+                      const float *s3, void *out, uint32_t *err, cudaStream_t s) {
+  using S = Shape<SWIGLU, SPANS, true>;
+  CUtensorMap ma, mb1, mb3;
+  if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b_q8(&mb1, B1, G, K, N, S::kQBox) ||
+      !make_map_b_q8(&mb3, SWIGLU ? B3 : B1, G, K, N, S::kQBox))
+    return cudaErrorInvalidValue;
+  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  static bool attr_set[64] = {};
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(
+        k_grouped_gemm<SWIGLU, SPANS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
+  p.scale1 = s1;
+  p.scale3 = SWIGLU ? s3 : nullptr;
+  const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
+                              ((N + S::BN - 1) / S::BN);
+  const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
+  k_grouped_gemm<SWIGLU, SPANS, true><<<grid, S::kCtaThreads, smem, s>>>(ma, mb1, mb3, p);
+  return cudaGetLastError();
 }
 
 template <bool SWIGLU, int SPANS>
@@ -1524,6 +1866,41 @@ cudaError_t launch_swap(int rows_cap, int K, int N, int G, const int32_t *offset
   return cudaGetLastError();
 }
 
+// The swap-AB engine on e4m3 weights with per-column scales.
+template <bool SWIGLU>
+cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *offsets,
+                           int fixed_rows, const void *A, const void *B1, const void *B3,
+                           const float *s1, const float *s3, void *out, uint32_t *err,
+                           cudaStream_t s) {
+  using S = ShapeSwap<SWIGLU, true>;
+  CUtensorMap mx, mw1, mw3;
+  if (!make_map_rows(&mx, A, rows_cap, K, kRowBox) ||
+      !make_map_b_q8(&mw1, B1, G, K, N, S::kQBox) ||
+      !make_map_b_q8(&mw3, SWIGLU ? B3 : B1, G, K, N, S::kQBox))
+    return cudaErrorInvalidValue;
+  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool attr_set[64] = {};
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(
+        k_grouped_gemm_swap<SWIGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
+  p.scale1 = s1;
+  p.scale3 = SWIGLU ? s3 : nullptr;
+  const long long max_tiles = (long long)((rows_cap + S::kMaxRows - 1) / S::kMaxRows +
+                                          (offsets ? G : 0)) *
+                              ((N + S::kCols - 1) / S::kCols);
+  const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
+  k_grouped_gemm_swap<SWIGLU, true><<<grid, S::kCtaThreads, smem, s>>>(mx, mw1, mw3, p);
+  return cudaGetLastError();
+}
+
 }  // namespace tc
 
 // Three engines, all correct for every shape (the tests run each):
@@ -1588,6 +1965,33 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                     : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                            out, nullptr, err, s);
   }
+}
+
+cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int G,
+                                    const int32_t *offsets, int fixed_rows, const void *A,
+                                    const void *B1, const void *B3, const float *s1,
+                                    const float *s3, void *out, uint32_t *err, cudaStream_t s) {
+  if (rows_cap <= 0) return cudaSuccess;
+  if (G <= 0 || G > tc::kMaxGroups || N % 16 != 0) return cudaErrorInvalidValue;
+  // fp8 weights: swap-AB for decode-sized groups (at most 32 rows per group
+  // on average, as for bf16), the single engine otherwise;
+  // MOE_GEMM_ENGINE=single|narrow|swap forces one (narrow: 64-column up
+  // projection tiles on the single engine)
+  const char *env = getenv("MOE_GEMM_ENGINE");
+  const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
+  const bool swap = env ? (env[0] == 's' && env[1] == 'w') : mean_rows <= 32;
+  if (swap)
+    return swiglu ? tc::launch_swap_q8<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
+                                             s1, s3, out, err, s)
+                  : tc::launch_swap_q8<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1,
+                                              B1, s1, nullptr, out, err, s);
+  if (swiglu && env && env[0] == 'n')
+    return tc::launch_q8<true, 1>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, s1, s3,
+                                  out, err, s);
+  return swiglu ? tc::launch_q8<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, s1,
+                                         s3, out, err, s)
+                : tc::launch_q8<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B1, s1,
+                                          nullptr, out, err, s);
 }
 
 cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const void *x,

@@ -180,28 +180,77 @@ struct Events {
   }
 };
 
+// One set of expert matrices: in the layer dtype, or e4m3 codes with
+// per-column scales (fp8 set).
+struct Weights {
+  const void *W1 = nullptr, *W3 = nullptr, *W2 = nullptr;
+  const float *s1 = nullptr, *s3 = nullptr, *s2 = nullptr;
+  bool fp8 = false;
+};
+Weights plain_weights(const void *W1, const void *W3, const void *W2) {
+  Weights w;
+  w.W1 = W1;
+  w.W3 = W3;
+  w.W2 = W2;
+  return w;
+}
+Weights fp8_weights(const moe_fp8_weights &q) {
+  Weights w;
+  w.W1 = q.W1;
+  w.W3 = q.W3;
+  w.W2 = q.W2;
+  w.s1 = q.s1;
+  w.s3 = q.s3;
+  w.s2 = q.s2;
+  w.fp8 = true;
+  return w;
+}
+moe_status check_weights(const Weights &w) {
+  MOE_TRY(need(w.W1));
+  MOE_TRY(need(w.W3));
+  MOE_TRY(need(w.W2));
+  if (w.fp8) {  // the scales are read as float4 vectors
+    MOE_TRY(need(w.s1));
+    MOE_TRY(need(w.s3));
+    MOE_TRY(need(w.s2));
+  }
+  return MOE_OK;
+}
+// Layers with fp8 weights: bf16 activations, rows of codes in 16-byte steps.
+moe_status check_fp8_config(const moe_config &c) {
+  if (c.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (c.d % 16 || c.f % 16 || c.f_shared % 16) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
 // Routed experts (G = E groups over rows_cap rows) or the shared expert
 // (offsets == nullptr: one group of T rows).  `mid` is recorded between the
 // up projection (with SwiGLU) and the down projection.  With row_src, A is
 // the token rows x and the up projection gathers its rows itself.
 moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixed_rows,
-                    int rows_cap, int f, const void *A, const void *W1, const void *W3,
-                    const void *W2, void *h, void *y, uint32_t *err, cudaStream_t s,
-                    const Events &ev = Events(), int mid = -1,
+                    int rows_cap, int f, const void *A, const Weights &w, void *h, void *y,
+                    uint32_t *err, cudaStream_t s, const Events &ev = Events(), int mid = -1,
                     const int32_t *row_src = nullptr) {
+  if (w.fp8) {
+    MOE_TRY_CUDA(launch_grouped_gemm_fp8(true, rows_cap, c.d, f, G, offsets, fixed_rows, A, w.W1,
+                                         w.W3, w.s1, w.s3, h, err, s));
+    MOE_TRY_CUDA(ev.mark(mid, s));
+    MOE_TRY_CUDA(launch_grouped_gemm_fp8(false, rows_cap, f, c.d, G, offsets, fixed_rows, h,
+                                         w.W2, nullptr, w.s2, nullptr, y, err, s));
+    return MOE_OK;
+  }
   if (c.dtype == MOE_F32) {
-    MOE_TRY_CUDA(launch_ffn_simt_f32(rows_cap, c.d, f, G, offsets, fixed_rows,
-                                     static_cast<const float *>(A), static_cast<const float *>(W1),
-                                     static_cast<const float *>(W3),
-                                     static_cast<const float *>(W2), static_cast<float *>(h),
-                                     static_cast<float *>(y), s));
+    MOE_TRY_CUDA(launch_ffn_simt_f32(
+        rows_cap, c.d, f, G, offsets, fixed_rows, static_cast<const float *>(A),
+        static_cast<const float *>(w.W1), static_cast<const float *>(w.W3),
+        static_cast<const float *>(w.W2), static_cast<float *>(h), static_cast<float *>(y), s));
     MOE_TRY_CUDA(ev.mark(mid, s));
     return MOE_OK;
   }
-  MOE_TRY_CUDA(launch_grouped_gemm_bf16(true, rows_cap, c.d, f, G, offsets, fixed_rows, A, W1, W3,
-                                        h, err, s, row_src, c.k_max, c.T));
+  MOE_TRY_CUDA(launch_grouped_gemm_bf16(true, rows_cap, c.d, f, G, offsets, fixed_rows, A, w.W1,
+                                        w.W3, h, err, s, row_src, c.k_max, c.T));
   MOE_TRY_CUDA(ev.mark(mid, s));
-  MOE_TRY_CUDA(launch_grouped_gemm_bf16(false, rows_cap, f, c.d, G, offsets, fixed_rows, h, W2,
+  MOE_TRY_CUDA(launch_grouped_gemm_bf16(false, rows_cap, f, c.d, G, offsets, fixed_rows, h, w.W2,
                                         nullptr, y, err, s));
   return MOE_OK;
 }
@@ -225,11 +274,11 @@ using namespace moe;
 
 static moe_status layer_impl(const moe_config *cfg, const void *x, const void *Wr,
                              const float *logit_bias, const float *sel_bias,
-                             const int32_t *k_per_token, const void *W1, const void *W3,
-                             const void *W2, const void *Ws1, const void *Ws3, const void *Ws2,
+                             const int32_t *k_per_token, const Weights &we, const Weights &wsh,
                              void *out, const moe_route_out *route_out, void *ws, size_t ws_bytes,
                              void *stream, const Events &ev) {
   MOE_TRY(check_config(cfg));
+  if (we.fp8) MOE_TRY(check_fp8_config(*cfg));
   if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
   const moe_config &c = *cfg;
   MOE_TRY(need(x));
@@ -237,14 +286,8 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   MOE_TRY(need4_opt(logit_bias));
   MOE_TRY(need4_opt(sel_bias));
   MOE_TRY(need4_opt(k_per_token));
-  MOE_TRY(need(W1));
-  MOE_TRY(need(W3));
-  MOE_TRY(need(W2));
-  if (c.f_shared > 0) {
-    MOE_TRY(need(Ws1));
-    MOE_TRY(need(Ws3));
-    MOE_TRY(need(Ws2));
-  }
+  MOE_TRY(check_weights(we));
+  if (c.f_shared > 0) MOE_TRY(check_weights(wsh));
   MOE_TRY(need(out));
   if (route_out) MOE_TRY(check_route_out(route_out));
   MOE_TRY(check_ws(c, MOE_WS_LAYER, ws, ws_bytes));
@@ -272,20 +315,20 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   MOE_TRY_CUDA(ev.mark(1, s));
   const int rows_cap = c.T * c.k_max;
   void *x_perm = at<void>(ws, L.x_perm), *y_perm = at<void>(ws, L.y_perm);
-  if (fuse_dispatch(c, rows_cap, r.offsets)) {
+  if (!we.fp8 && fuse_dispatch(c, rows_cap, r.offsets)) {
     MOE_TRY_CUDA(ev.mark(2, s));
-    MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x, W1, W3, W2, at<void>(ws, L.h),
-                     y_perm, err, s, ev, 3, r.row_src));
+    MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x, we, at<void>(ws, L.h), y_perm, err,
+                     s, ev, 3, r.row_src));
   } else {
     MOE_TRY_CUDA(launch_dispatch(c, x, r.offsets, r.row_src, x_perm, err, s));
     MOE_TRY_CUDA(ev.mark(2, s));
-    MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x_perm, W1, W3, W2, at<void>(ws, L.h),
-                     y_perm, err, s, ev, 3));
+    MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x_perm, we, at<void>(ws, L.h), y_perm,
+                     err, s, ev, 3));
   }
   MOE_TRY_CUDA(ev.mark(4, s));
   const void *shared_y = nullptr;
   if (c.f_shared > 0) {
-    MOE_TRY(ffn_impl(c, 1, nullptr, c.T, c.T, c.f_shared, x, Ws1, Ws3, Ws2, at<void>(ws, L.h_sh),
+    MOE_TRY(ffn_impl(c, 1, nullptr, c.T, c.T, c.f_shared, x, wsh, at<void>(ws, L.h_sh),
                      at<void>(ws, L.y_sh), err, s));
     shared_y = at<void>(ws, L.y_sh);
   }
@@ -413,8 +456,42 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32
   if (!err) return MOE_ERR_CUDA;
   const Layout L = layout(c, MOE_WS_EXPERT_FFN);
   const int rows_cap = c.T * c.k_max;
-  return ffn_impl(c, c.E, offsets, 0, rows_cap, c.f, x_perm, W1, W3, W2, at<void>(ws, L.h), y_perm,
+  return ffn_impl(c, c.E, offsets, 0, rows_cap, c.f, x_perm, plain_weights(W1, W3, W2),
+                  at<void>(ws, L.h), y_perm, err, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_ffn_fp8(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                              const moe_fp8_weights *w, void *y_perm, void *ws, size_t ws_bytes,
+                              void *stream) {
+  MOE_TRY(check_config(cfg));
+  MOE_TRY(check_fp8_config(*cfg));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to do, pointers unused
+  const moe_config &c = *cfg;
+  if (!w) return MOE_ERR_INVALID_ARG;
+  const Weights we = fp8_weights(*w);
+  MOE_TRY(need(x_perm));
+  MOE_TRY(need4(offsets));
+  MOE_TRY(check_weights(we));
+  MOE_TRY(need(y_perm));
+  MOE_TRY(check_ws(c, MOE_WS_EXPERT_FFN, ws, ws_bytes));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  const Layout L = layout(c, MOE_WS_EXPERT_FFN);
+  return ffn_impl(c, c.E, offsets, 0, c.T * c.k_max, c.f, x_perm, we, at<void>(ws, L.h), y_perm,
                   err, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_quantize_fp8(const void *W, int32_t G, int32_t K, int32_t N, void *Wq,
+                            float *scale, void *stream) {
+  if (G < 0 || K < 0 || N < 0) return MOE_ERR_INVALID_ARG;
+  if ((long long)G * K * N == 0) return MOE_OK;
+  if (N % 16) return MOE_ERR_ALIGNMENT;
+  if (G > 65535) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(need(W));
+  MOE_TRY(need(Wq));
+  MOE_TRY(need(scale));
+  return cuda_status(launch_quantize_fp8(G, K, N, W, static_cast<uint8_t *>(Wq), scale,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *slot_row,
@@ -437,8 +514,8 @@ moe_status moe_layer(const moe_config *cfg, const void *x, const void *Wr,
                      const void *W1, const void *W3, const void *W2, const void *Ws1,
                      const void *Ws3, const void *Ws2, void *out, const moe_route_out *route_out,
                      void *ws, size_t ws_bytes, void *stream) {
-  return layer_impl(cfg, x, Wr, logit_bias, sel_bias, k_per_token, W1, W3, W2, Ws1, Ws3, Ws2, out,
-                    route_out, ws, ws_bytes, stream, Events());
+  return layer_impl(cfg, x, Wr, logit_bias, sel_bias, k_per_token, plain_weights(W1, W3, W2),
+                    plain_weights(Ws1, Ws3, Ws2), out, route_out, ws, ws_bytes, stream, Events());
 }
 
 moe_status moe_layer_timed(const moe_config *cfg, const void *x, const void *Wr,
@@ -451,8 +528,26 @@ moe_status moe_layer_timed(const moe_config *cfg, const void *x, const void *Wr,
   Events ev;
   ev.ev = reinterpret_cast<cudaEvent_t const *>(events);
   ev.n = n_events;
-  return layer_impl(cfg, x, Wr, logit_bias, sel_bias, k_per_token, W1, W3, W2, Ws1, Ws3, Ws2, out,
-                    route_out, ws, ws_bytes, stream, ev);
+  return layer_impl(cfg, x, Wr, logit_bias, sel_bias, k_per_token, plain_weights(W1, W3, W2),
+                    plain_weights(Ws1, Ws3, Ws2), out, route_out, ws, ws_bytes, stream, ev);
+}
+
+moe_status moe_layer_fp8(const moe_config *cfg, const void *x, const void *Wr,
+                         const float *logit_bias, const float *sel_bias,
+                         const int32_t *k_per_token, const moe_fp8_weights *experts,
+                         const moe_fp8_weights *shared, void *out,
+                         const moe_route_out *route_out, void *ws, size_t ws_bytes, void *stream,
+                         void *const *events, int32_t n_events) {
+  if (n_events < 0 || (n_events > 0 && !events)) return MOE_ERR_INVALID_ARG;
+  if (!experts || (cfg && cfg->f_shared > 0 && !shared)) return MOE_ERR_INVALID_ARG;
+  Events ev;
+  ev.ev = reinterpret_cast<cudaEvent_t const *>(events);
+  ev.n = n_events;
+  Weights wsh;
+  if (shared) wsh = fp8_weights(*shared);
+  wsh.fp8 = true;
+  return layer_impl(cfg, x, Wr, logit_bias, sel_bias, k_per_token, fp8_weights(*experts), wsh,
+                    out, route_out, ws, ws_bytes, stream, ev);
 }
 
 moe_status moe_check_errors(void *stream, uint32_t *flags) {

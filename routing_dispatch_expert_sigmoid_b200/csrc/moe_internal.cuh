@@ -92,6 +92,21 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                      cudaStream_t s, const int32_t *row_src = nullptr,
                                      int k_max = 1, int a_rows = 0);
 
+// K5/K6 with fp8 weights: B1, B3 are e4m3 codes [G, K, N] (N % 16 == 0) with
+// per-column fp32 scales s1, s3 [G, N] (16-byte aligned); the codes are
+// widened to bf16 in shared memory and the scales applied in the epilogue.
+// Output types as for launch_grouped_gemm_bf16.
+cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int G,
+                                    const int32_t *offsets, int fixed_rows, const void *A,
+                                    const void *B1, const void *B3, const float *s1,
+                                    const float *s3, void *out, uint32_t *err, cudaStream_t s);
+
+// Per-column e4m3 quantisation of bf16 weights W [G, K, N]: scale[g, n] =
+// max_k |W| / 448 (1 for an all-zero column), Wq = e4m3(W / scale), rounded
+// to nearest even with saturation.
+cudaError_t launch_quantize_fp8(int G, int K, int N, const void *W, uint8_t *Wq, float *scale,
+                                cudaStream_t s);
+
 // K1 on the tensor cores (bf16 layers with E % 8 == 0): logits[T,E] =
 // x[T,d] . Wr[d,E] (+ bias), fp32 accumulation in tensor memory, fp32 out.
 cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,

@@ -13,8 +13,8 @@
 //   * the router GEMM x[T,d] . Wr[d,E] runs as S independent K slices (the
 //     grouped GEMM's split-K mode), each writing fp32 partial logits
 //     [S][T][E]; S is a function of the layer's shape alone;
-//   * k_route_small: one warp per token adds the S partials in slice order
-//     (then the logit bias), stores the logits row and gates the token; each
+//   * k_route_small: one warp per token adds the S partials (then the logit
+//     bias) in a fixed order, stores the logits row and gates the token; each
 //     CTA then takes a ticket, and the CTA holding the last ticket ranks all
 //     T*k_max slots in shared memory.  No CTA waits for another: the ticket
 //     only decides which CTA continues.
@@ -34,7 +34,7 @@ constexpr size_t kPartialBudget = 768u << 10;  // fp32 partial logits, bytes
 constexpr int kSplitTarget = 148;           // CTAs to aim for (SMs of a B200)
 constexpr int kBK = 64;                     // K per pipeline stage of the GEMM
 constexpr int kBN = 64;                     // output columns per GEMM tile
-constexpr int kBatch = 16;                  // partial-logit loads in flight per lane
+constexpr int kBatch = 8;                   // slices loaded per step (columns of <= 16)
 
 struct SmallArgs {
   gating::GatingArgs g;  // g.logits is the row this kernel writes
@@ -173,33 +173,56 @@ __global__ void __launch_bounds__(kWarps * 32) k_route_small(SmallArgs a) {
     float *row = a.logits + (size_t)t * E;
     const float *pt = a.partials + (size_t)t * E;
     const size_t slab = (size_t)T * E;
+    const int S = a.S;
+    if (NPL == 1 && E <= 16) {
+      // 32/E lanes share a column: lane l sums slices l/E, l/E + 32/E, ...
+      // of column l % E, then the column's lanes are added in lane order.
+      const int lpc = 32 / E, e = lane % E, sub = lane / E;
+      float v = 0.f;
+      for (int s0 = sub; s0 < S; s0 += kBatch * lpc) {
+        float b[kBatch];
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E) {
-        // kBatch independent loads in flight, then added in slice order
-        float v = 0.f;
-        for (int s0 = 0; s0 < a.S; s0 += kBatch) {
-          float buf[kBatch];
+        for (int j = 0; j < kBatch; ++j)  // clamped address: every load is issued
+          b[j] = pt[(size_t)min(s0 + j * lpc, S - 1) * slab + e];
 #pragma unroll
-          for (int j = 0; j < kBatch; ++j)
-            buf[j] = s0 + j < a.S ? __ldcg(pt + (size_t)(s0 + j) * slab + e) : 0.f;
+        for (int j = 0; j < kBatch; ++j)
+          if (s0 + j * lpc < S) v += b[j];
+      }
+      float tot = __shfl_sync(0xffffffffu, v, e);
+      for (int q = 1; q < lpc; ++q) tot += __shfl_sync(0xffffffffu, v, e + q * E);
+      if (lane < E) row[e] = a.logit_bias ? tot + a.logit_bias[e] : tot;
+    } else {
+      // lane l owns columns l, l+32, ...: per step, kSteps slices x NPL
+      // columns of independent loads, added in slice order per column
+      constexpr int kSteps = NPL >= 16 ? 1 : 16 / NPL;
+      float acc[NPL];
 #pragma unroll
-          for (int j = 0; j < kBatch; ++j)
-            if (s0 + j < a.S) v += buf[j];
-        }
-        if (a.logit_bias) v += a.logit_bias[e];
-        row[e] = v;
+      for (int i = 0; i < NPL; ++i) acc[i] = 0.f;
+      for (int s0 = 0; s0 < S; s0 += kSteps) {
+        float b[kSteps][NPL];
+#pragma unroll
+        for (int j = 0; j < kSteps; ++j)
+#pragma unroll
+          for (int i = 0; i < NPL; ++i)
+            b[j][i] = pt[(size_t)min(s0 + j, S - 1) * slab + min(i * 32 + lane, E - 1)];
+#pragma unroll
+        for (int j = 0; j < kSteps; ++j)
+#pragma unroll
+          for (int i = 0; i < NPL; ++i)
+            if (s0 + j < S) acc[i] += b[j][i];
+      }
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = i * 32 + lane;
+        if (e < E) row[e] = a.logit_bias ? acc[i] + a.logit_bias[e] : acc[i];
       }
     }
     __syncwarp();  // a lane reads back only its own entries; this orders the warp
     gating::gate_token<NPL>(a.g, t, row, reinterpret_cast<float *>(s_dyn) + warp * E);
   }
+  __threadfence();  // every thread's topk_idx stores before the CTA's ticket
   __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();  // this CTA's topk_idx stores before its ticket
-    s_last = atomicAdd(a.ticket, 1) == (int)gridDim.x - 1;
-  }
+  if (threadIdx.x == 0) s_last = atomicAdd(a.ticket, 1) == (int)gridDim.x - 1;
   __syncthreads();
   if (!s_last) return;
   __threadfence();  // every other CTA's stores are visible past its ticket

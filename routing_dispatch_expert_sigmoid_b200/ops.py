@@ -43,6 +43,10 @@ class MoeRouteOut(ctypes.Structure):
                  "row_src", "n_dropped")]
 
 
+class MoeFp8Weights(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in ("W1", "W3", "W2", "s1", "s3", "s2")]
+
+
 _lib = None
 
 
@@ -65,12 +69,18 @@ def lib() -> ctypes.CDLL:
         L.moe_layer.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, outp, P, S, P]
         L.moe_layer_timed.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, outp, P, S, P,
                                       ctypes.POINTER(ctypes.c_void_p), I]
+        fp8p = ctypes.POINTER(MoeFp8Weights)
+        L.moe_quantize_fp8.argtypes = [P, I, I, I, P, P, P]
+        L.moe_expert_ffn_fp8.argtypes = [cfgp, P, P, fp8p, P, P, S, P]
+        L.moe_layer_fp8.argtypes = [cfgp, P, P, P, P, P, fp8p, fp8p, P, outp, P, S, P,
+                                    ctypes.POINTER(ctypes.c_void_p), I]
         L.moe_check_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         for fn in ("moe_workspace_size", "moe_route", "moe_route_static_scratch", "moe_dispatch",
                    "moe_expert_ffn",
-                   "moe_combine", "moe_layer", "moe_layer_timed", "moe_check_errors"):
+                   "moe_combine", "moe_layer", "moe_layer_timed", "moe_check_errors",
+                   "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_layer_fp8"):
             getattr(L, fn).restype = I
         _lib = L
     return _lib
@@ -197,3 +207,57 @@ def moe_check_errors(stream=None) -> int:
     if flags.value:
         raise MoeError(st, f"moe_check_errors: device flags {flags.value:#x}")
     return 0
+
+
+# ---- fp8 expert weights -----------------------------------------------------
+def moe_quantize_fp8(W: torch.Tensor, stream=None):
+    """W [G, K, N] (or [K, N]) bf16 -> (codes uint8 of W's shape, scales fp32
+    [G, N] (or [N])), computed by the library."""
+    Wg = W if W.dim() == 3 else W.unsqueeze(0)
+    G, K, N = Wg.shape
+    q = torch.empty(Wg.shape, dtype=torch.uint8, device=W.device)
+    sc = torch.empty((G, N), dtype=torch.float32, device=W.device)
+    _check(lib().moe_quantize_fp8(_p(Wg), G, K, N, _p(q), _p(sc), _stream(stream)),
+           "moe_quantize_fp8")
+    if W.dim() == 2:
+        return q[0], sc[0]
+    return q, sc
+
+
+def fp8_weight_set(W1, W3, W2, stream=None) -> dict:
+    """Quantise one set of expert matrices (routed [E, ...] or shared [d, f])."""
+    out = {}
+    for name, W in (("W1", W1), ("W3", W3), ("W2", W2)):
+        q, sc = moe_quantize_fp8(W, stream)
+        out[name], out["s" + name[1]] = q, sc
+    return out
+
+
+def _fp8_struct(ws: dict | None):
+    if ws is None:
+        return None
+    return MoeFp8Weights(*[ws[k].data_ptr() for k in ("W1", "W3", "W2", "s1", "s3", "s2")])
+
+
+def moe_expert_ffn_fp8(cfg, x_perm, offsets, weights: dict, y_perm, ws, stream=None):
+    wq = _fp8_struct(weights)
+    _check(lib().moe_expert_ffn_fp8(ctypes.byref(cfg), _p(x_perm), _p(offsets), ctypes.byref(wq),
+                                    _p(y_perm), _p(ws), 0 if ws is None else ws.numel(),
+                                    _stream(stream)), "moe_expert_ffn_fp8")
+
+
+def moe_layer_fp8(cfg, x, Wr, logit_bias, sel_bias, k_per_token, experts: dict,
+                  shared: dict | None, out, route_out: dict | None, ws, events=None,
+                  stream=None):
+    """moe_layer with fp8 expert weights (dicts from fp8_weight_set); events as
+    in moe_layer_timed, or None."""
+    r = None if route_out is None else ctypes.byref(_route_struct(route_out))
+    we, wsh = _fp8_struct(experts), _fp8_struct(shared)
+    n = 0 if events is None else len(events)
+    handles = None if events is None else (ctypes.c_void_p * n)(
+        *[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib().moe_layer_fp8(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias),
+                               _p(k_per_token), ctypes.byref(we),
+                               None if wsh is None else ctypes.byref(wsh), _p(out), r, _p(ws),
+                               0 if ws is None else ws.numel(), _stream(stream), handles, n),
+           "moe_layer_fp8")

@@ -171,3 +171,69 @@ def test_gpu_sigmoid_constants_are_the_rounded_definitions():
     assert bits("kLn2Lo") == _exact_f32(ln2 - Fraction(2839, 4096))
     for k in range(3, 8):
         assert bits(f"kC{k}") == _exact_f32(Fraction(1, math.factorial(k))), k
+
+
+# ---- fp8 expert weights: host-side checks (nothing reaches the device) -------
+_FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: rejected first
+
+
+def _fp8_set(**kw):
+    v = dict(W1=_FAKE, W3=_FAKE, W2=_FAKE, s1=_FAKE, s3=_FAKE, s2=_FAKE)
+    v.update(kw)
+    return ops.MoeFp8Weights(*[v[k] for k in ("W1", "W3", "W2", "s1", "s3", "s2")])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dtype=ops.MOE_F32), -2),   # fp8 weights need bf16 activations
+    (dict(d=7160), -4),              # d a multiple of 8 but not of 16
+    (dict(f=2040), -4),
+    (dict(f_shared=2040), -4),
+])
+def test_fp8_layer_config_checks(kw, expect):
+    c = _cfg(**kw)
+    w = _fp8_set()
+    st = ops.lib().moe_layer_fp8(ctypes.byref(c), _FAKE, _FAKE, None, None, None, ctypes.byref(w),
+                                 ctypes.byref(w), _FAKE, None, _FAKE, 1 << 40, None, None, 0)
+    assert st == expect
+
+
+def test_fp8_layer_argument_checks():
+    c = _cfg()
+    w = _fp8_set()
+    lib = ops.lib()
+    args = lambda we, ws, ev=None, n=0: (ctypes.byref(c), _FAKE, _FAKE, None, None, None, we, ws,
+                                         _FAKE, None, _FAKE, 1 << 40, None, ev, n)
+    assert lib.moe_layer_fp8(*args(None, ctypes.byref(w))) == -1           # no experts
+    assert lib.moe_layer_fp8(*args(ctypes.byref(w), None)) == -1           # shared expert missing
+    assert lib.moe_layer_fp8(*args(ctypes.byref(w), ctypes.byref(w), None, 3)) == -1  # events
+    bad = _fp8_set(s2=_FAKE + 4)                                            # scales need 16 B
+    assert lib.moe_layer_fp8(*args(ctypes.byref(bad), ctypes.byref(w))) == -4
+    bad = _fp8_set(W3=0)
+    assert lib.moe_layer_fp8(*args(ctypes.byref(bad), ctypes.byref(w))) == -1
+    assert lib.moe_expert_ffn_fp8(ctypes.byref(c), _FAKE, _FAKE, None, _FAKE, _FAKE, 1 << 40,
+                                  None) == -1
+
+
+def test_fp8_quantize_checks():
+    lib = ops.lib()
+    assert lib.moe_quantize_fp8(_FAKE, 2, 64, 24, _FAKE, _FAKE, None) == -4   # N % 16
+    assert lib.moe_quantize_fp8(_FAKE, -1, 64, 32, _FAKE, _FAKE, None) == -1
+    assert lib.moe_quantize_fp8(_FAKE, 0, 64, 32, _FAKE, _FAKE, None) == 0    # nothing to do
+    assert lib.moe_quantize_fp8(_FAKE + 8, 2, 64, 32, _FAKE, _FAKE, None) == -4
+
+
+def test_fp8_widening_bit_formula_gives_every_code():
+    """The GEMM widens e4m3 codes to bf16 by moving bits -- the byte to the
+    top of a 16-bit half, exponent and fraction shifted right by 4, sign kept
+    -- and one multiply by 2^120.  Emulated here for every finite code against
+    the oracle's decoding (the GPU tests cover the hardware's multiply)."""
+    import numpy as np
+
+    import oracle
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint32)
+    y = codes << 8
+    bits = ((y >> 4) & 0x07F0) | (y & 0x8000)
+    val = (bits << 16).astype(np.uint32).view(np.float32).astype(np.float64) * 2.0 ** 120
+    ref = oracle.e4m3_decode(codes.astype(np.uint8))
+    assert (val == ref).all()
+    assert (np.signbit(val) == np.signbit(ref)).all()

@@ -95,3 +95,14 @@ def test_clock_summary_parses_reasons():
     assert s["sm_mhz"] == pytest.approx(1910.0) and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
     assert s["power_limit_w"] == 1000.0 and s["power_max_w"] == 950.0
+
+
+def test_algorithmic_bytes_with_fp8_weights():
+    w = WORKLOADS["mixtral_decode"]
+    b = bench.algorithmic(w, R=128, touched=8)
+    q = bench.algorithmic(w, R=128, touched=8, fp8=True)
+    d, f = w.d, w.f
+    assert q["up_bytes"] == 8 * 2 * (d * f + 4 * f) + 128 * d * 2 + 128 * f * 2
+    assert q["up_flops"] == b["up_flops"]
+    # one byte per expert weight plus the column scales; router, x and out unchanged
+    assert b["layer_bytes"] - q["layer_bytes"] == 8 * (3 * d * f - 4 * (2 * f + d))
