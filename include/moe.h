@@ -250,20 +250,23 @@ MOE_API moe_status moe_layer_timed(const moe_config *cfg, const void *x, const v
  * largest magnitude 448) with one fp32 scale per output column: the weight
  * the layer computes with is e4m3_value(code) * scale[column].  The router
  * weights, activations and outputs stay in the layer dtype, which must be
- * MOE_BF16; d, f and f_shared must be multiples of 16.  Codes are bytes in
- * the bf16 weights' layout; every pointer is a device pointer, 16-byte
- * aligned, owned by the caller. */
+ * MOE_BF16; d, f and f_shared must be multiples of 16.  The codes are stored
+ * transposed, K contiguous (one byte each): the codes of one output column
+ * of the bf16 matrix [G, K, N] are the contiguous row [g, n, :] -- the order
+ * in which the GEMMs widen them.  moe_quantize_fp8 writes this layout.
+ * Every pointer is a device pointer, 16-byte aligned, owned by the caller. */
 typedef struct {
-  const void *W1, *W3;  /* [G, d, f] e4m3 codes */
-  const void *W2;       /* [G, f, d] e4m3 codes */
+  const void *W1, *W3;  /* [G, f, d] e4m3 codes of the [G, d, f] matrices */
+  const void *W2;       /* [G, d, f] e4m3 codes of the [G, f, d] matrix */
   const float *s1, *s3; /* [G, f] column scales of W1, W3 */
   const float *s2;      /* [G, d] column scales of W2 */
 } moe_fp8_weights;
 
-/* Weight preparation (not a hot call): W [G, K, N] bf16 -> Wq [G, K, N] e4m3
- * codes and scale [G, N], with scale = max_k |W[g,k,n]| / 448 (fp32
- * division; 1 for an all-zero column) and Wq = e4m3(W / scale) of the fp32
- * quotient, rounded to nearest even, saturating at 448.  N % 16 == 0. */
+/* Weight preparation (not a hot call): W [G, K, N] bf16 -> Wq [G, N, K] e4m3
+ * codes (transposed) and scale [G, N], with scale = max_k |W[g,k,n]| / 448
+ * (fp32 division; 1 for an all-zero column) and Wq[g,n,k] = e4m3(W[g,k,n] /
+ * scale[g,n]) of the fp32 quotient, rounded to nearest even, saturating at
+ * 448.  K and N multiples of 16. */
 MOE_API moe_status moe_quantize_fp8(const void *W, int32_t G, int32_t K, int32_t N, void *Wq,
                                     float *scale, void *stream);
 

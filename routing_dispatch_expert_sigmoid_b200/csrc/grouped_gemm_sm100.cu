@@ -194,6 +194,45 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a_desc, uint64_t 
 }
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
+// The same MMA with A read from tensor memory (a_tmem: lane = row of A,
+// 32-bit column c = K elements 2c, 2c+1).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 consecutive 32-bit columns of this warp's 32 lanes; completion is
+// waited for with tmem_wait_st.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -235,6 +274,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 // K-major, B MN-major, N >> 3 at bit 17, M >> 4 at bit 24.
 constexpr uint32_t instr_desc(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+// The same with B K-major too (the widened fp8 weight tiles).
+__host__ __device__ constexpr uint32_t instr_desc_kk(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
 }
 
@@ -282,13 +326,10 @@ struct Shape {
   // x 64 bytes per span), the HBM stream, at most 8 deep.
   static constexpr int kStages =
       FP8W ? 2 : ((196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes));
-  static constexpr uint32_t kQSpanBytes = BK * 64;    // 4 KB
-  static constexpr uint32_t kQBytes = FP8W ? kBOps * kSpans * kQSpanBytes : 0;
-  // codes arrive in boxes of 128 columns (128-byte rows) where the tile is
-  // that wide, else 64
-  static constexpr int kQBox = SPANS >= 2 ? 128 : 64;
-  static constexpr uint32_t kQBoxBytes = BK * kQBox;
-  static constexpr int kQBoxesPerOp = 64 * SPANS / kQBox;
+  // FP8W codes are K-contiguous ([G, N, K]): per operand one box of BN
+  // columns x 64 K-codes, 64-byte rows with the 64-byte swizzle
+  static constexpr uint32_t kQOpBytes = FP8W ? BN * BK : 0;
+  static constexpr uint32_t kQBytes = kBOps * kQOpBytes;
   static constexpr int kQStages =
       !FP8W ? 0
             : ((196608 - kStages * kStageBytes) / kQBytes > 8
@@ -302,7 +343,8 @@ struct Shape {
   static constexpr int kMmaN = kBOps * BN;            // 256
   static constexpr uint32_t kAccCols = kMmaN;         // fp32 columns per accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccCols; // 512
-  static constexpr uint32_t kIdesc = instr_desc(BM, kMmaN);
+  // bf16 weights are an MN-major B tile; widened fp8 weights a K-major one
+  static constexpr uint32_t kIdesc = FP8W ? instr_desc_kk(BM, kMmaN) : instr_desc(BM, kMmaN);
   // epilogue staging: per epilogue warp a 32-row x 32-column fp32 chunk, rows
   // padded to 36 words so both the row-wise writes and the column-wise reads
   // are free of bank conflicts
@@ -315,7 +357,7 @@ struct Shape {
   static constexpr int kBars = FP8W ? 3 * kStages + 2 * kQStages + 5 : 2 * kStages + 5;
   static_assert(kBars * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit 256 bytes");
   static_assert(!FP8W || kQStages >= 2, "code ring");
-  static_assert(kQBytes % (16 * kConvThreads) == 0, "whole 16-byte chunks per converter");
+  static_assert(!FP8W || (kMmaN % kConvThreads == 0 && BN <= 256), "whole B rows per converter");
   static_assert(kMmaN % 16 == 0 && kMmaN <= 256, "UMMA N");
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                 "TMEM allocation: a power of two in [32, 512] columns");
@@ -366,52 +408,51 @@ __device__ __forceinline__ void e4m3x16_to_bf16(uint4 c, uint4 &lo, uint4 &hi) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Widen one k-block of e4m3 codes (kQ bytes at q: boxes of 64 K-rows x QB
-// bytes, QB = 64 or 128 columns, box b covering 64-column spans QB/64 * b ..)
-// into 64-column bf16 spans of 64 K-rows x 128 bytes, 8 KB apart, with the
-// 128-byte swizzle TMA would apply (16-byte slot XOR K-row mod 8).  `ct` is
-// the thread's index among the 128 converter threads.  With 128-column boxes
-// a quarter warp takes the first half of one K-row and the second half of
-// the next (or the reverse), so both its loads and its stores hit 32
-// distinct banks.
-template <int QB, uint32_t kQ>
-__device__ __forceinline__ void widen_codes(const uint8_t *__restrict__ q,
-                                            uint8_t *__restrict__ w, int ct) {
-  constexpr int kIt = kQ >= 16 * 128 ? (int)(kQ / 16 / 128) : 1;
-  if (kQ < 16 * 128) return;  // bf16 instantiations: no codes
-  int off_q[kIt], off_w[kIt], kr[kIt], jj[kIt];
+// The 64 codes of one column of a code box (64-byte rows, 64-byte TMA
+// swizzle: 16-byte chunk j of row r sits in slot j ^ ((r >> 1) & 3)), widened
+// to 32 bf16 pairs, K ascending (pair i = K elements 2i, 2i+1).  Eight
+// threads on consecutive rows read 8 distinct bank groups.
+// NC of the 4 16-code chunks of row r, from chunk j0 (K = 16*j0 ..).
+template <int NC>
+__device__ __forceinline__ void widen_chunks(const uint8_t *__restrict__ box, int r, int j0,
+                                             uint32_t (&out)[8 * NC]) {
+  const uint8_t *row = box + r * 64;
+  uint4 c[NC];
 #pragma unroll
-  for (int it = 0; it < kIt; ++it) {
-    const int c = it * 128 + ct;  // 16-byte code chunk
-    int blk, k, span, j;
-    if (QB == 64) {
-      blk = c >> 8;
-      k = (c >> 2) & 63;
-      span = 0;
-      j = c & 3;
-    } else {
-      blk = c >> 9;  // 64 K-rows x 8 chunks per box
-      const int r = c & 511, t = r & 31, qq = t >> 3, i = (t >> 2) & 1;
-      j = t & 3;
-      k = (r >> 5) * 4 + 2 * (qq >> 1) + i;
-      span = i ^ (qq & 1);
+  for (int j = 0; j < NC; ++j)
+    c[j] = *reinterpret_cast<const uint4 *>(row + (((j0 + j) ^ ((r >> 1) & 3)) << 4));
+#pragma unroll
+  for (int j = 0; j < NC; ++j) {
+    const uint32_t w[4] = {c[j].x, c[j].y, c[j].z, c[j].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      out[8 * j + 2 * i] = e4m3x2_to_bf16x2(w[i] & 0xffffu);
+      out[8 * j + 2 * i + 1] = e4m3x2_to_bf16x2(w[i] >> 16);
     }
-    off_q[it] = blk * (64 * QB) + k * QB + (span * 4 + j) * 16;
-    off_w[it] = (blk * (QB / 64) + span) * 8192 + k * 128;
-    kr[it] = k & 7;
-    jj[it] = j;
   }
-  // every load first, so their latencies overlap; then widen and store
-  uint4 codes[kIt];
+}
+__device__ __forceinline__ void widen_column(const uint8_t *__restrict__ box, int r,
+                                             uint32_t (&out)[32]) {
+  widen_chunks<4>(box, r, 0, out);
+}
+
+// Single engine: widen the stage's codes (per operand a box of BN columns x
+// 64 K) into the K-major B tile the MMA reads: row r (operand r / BN, column
+// r % BN) holds 64 bf16 = 128 bytes, 16-byte chunk c in slot c ^ (r & 7)
+// (the 128-byte swizzle).  Thread ct widens rows ct, ct + 128, ...
+template <int kRowsPerThread>
+__device__ __forceinline__ void widen_rows(const uint8_t *__restrict__ q, uint8_t *__restrict__ b,
+                                           int ct, int BN) {
 #pragma unroll
-  for (int it = 0; it < kIt; ++it) codes[it] = *reinterpret_cast<const uint4 *>(q + off_q[it]);
+  for (int i = 0; i < kRowsPerThread; ++i) {
+    const int r = ct + 128 * i, op = r / BN, rn = r - op * BN;
+    uint32_t v[32];
+    widen_column(q + op * BN * 64, rn, v);
+    uint8_t *row = b + r * 128;
 #pragma unroll
-  for (int it = 0; it < kIt; ++it) {
-    uint4 lo, hi;
-    e4m3x16_to_bf16(codes[it], lo, hi);
-    uint8_t *rowp = w + off_w[it];
-    *reinterpret_cast<uint4 *>(rowp + (((2 * jj[it]) ^ kr[it]) << 4)) = lo;
-    *reinterpret_cast<uint4 *>(rowp + (((2 * jj[it] + 1) ^ kr[it]) << 4)) = hi;
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) =
+          make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
   }
 }
 
@@ -572,18 +613,10 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
         const uint32_t fb = fullb + 8 * s;
         if (codes) {
           const uint32_t qt = smem_addr(qring + s * S::kQBytes);
-          if (lane == 0) {
+          if (lane == 0) {  // codes [G, N, K]: coordinates (k, n, group)
             mbar_expect_tx(fb, S::kQBytes);
-#pragma unroll
-            for (int b = 0; b < S::kQBoxesPerOp; ++b)
-              tma_load_3d(qt + b * S::kQBoxBytes, &tmB1, fb, n * S::BN + b * S::kQBox,
-                          k0 + kb * BK, gb);
-            if (SWIGLU) {
-#pragma unroll
-              for (int b = 0; b < S::kQBoxesPerOp; ++b)
-                tma_load_3d(qt + (S::kQBoxesPerOp + b) * S::kQBoxBytes, &tmB3, fb,
-                            n * S::BN + b * S::kQBox, k0 + kb * BK, gb);
-            }
+            tma_load_3d(qt, &tmB1, fb, k0 + kb * BK, n * S::BN, gb);
+            if (SWIGLU) tma_load_3d(qt + S::kQOpBytes, &tmB3, fb, k0 + kb * BK, n * S::BN, gb);
           }
         } else {
           const uint32_t st = smem_addr(ring + s * S::kStageBytes);
@@ -644,8 +677,10 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
             // A: K-major, 128-byte rows, 8-row groups 1024 B apart; step K by 32 B.
             const uint64_t ad = smem_desc(st + kk * 32, 16, 1024);
             // B: MN-major, 64-column spans kSpanBytes apart (LBO), 8-row K
-            // groups 1024 B apart (SBO); step K by 16 rows = 2048 B.
-            const uint64_t bd = smem_desc(st + S::kABytes + kk * 2048, S::kSpanBytes, 1024);
+            // groups 1024 B apart (SBO); step K by 16 rows = 2048 B.  Widened
+            // fp8 weights: K-major like A.
+            const uint64_t bd = FP8W ? smem_desc(st + S::kABytes + kk * 32, 16, 1024)
+                                     : smem_desc(st + S::kABytes + kk * 2048, S::kSpanBytes, 1024);
             umma(d_tmem, ad, bd, S::kIdesc, (kb | kk) != 0);
           }
           any = true;
@@ -775,8 +810,9 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
           ok = false;
           break;
         }
-        widen_codes<S::kQBox, S::kQBytes>(qring + qs * S::kQBytes,
-                                          ring + s * S::kStageBytes + S::kABytes, ct);
+        widen_rows<S::kMmaN / S::kConvThreads>(qring + qs * S::kQBytes,
+                                                ring + s * S::kStageBytes + S::kABytes, ct,
+                                                S::BN);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -1254,36 +1290,46 @@ struct ShapeSwap {
   // rows per tile (MMA N): fp8 weights keep decode-sized row tiles so that
   // a stage stays small and the code stream can run deep
   static constexpr int kMaxRows = FP8W ? 32 : 128;
-  static constexpr int kWOps = SWIGLU ? 2 : 1;
+  // fp8 down projection: 256-column tiles as two 128-column halves (the MMA's
+  // M is 128), so that decode-sized layers fill the GPU in one wave
+  static constexpr bool kWide = FP8W && !SWIGLU;
+  static constexpr int kTileCols = kWide ? 256 : 128;
+  static constexpr int kWOps = (SWIGLU || kWide) ? 2 : 1;  // operands or column halves
   static constexpr uint32_t kSpanBytes = BK * 128;       // 8 KB: 64 K-rows x 64 columns
   static constexpr uint32_t kWBytes = kWOps * 2 * kSpanBytes;   // 16 or 32 KB (bf16)
   static constexpr uint32_t kRowBoxBytes = kRowBox * BK * 2;    // 4 KB
   static constexpr uint32_t kXBytes = kMaxRows * BK * 2;        // 16 KB (fp8: 4 KB)
-  static constexpr uint32_t kQSpanBytes = BK * 64;              // e4m3 codes of a span
-  static constexpr uint32_t kQBytes = FP8W ? kWOps * 2 * kQSpanBytes : 0;
-  static constexpr int kQBox = 128;                             // one code box per operand
-  static constexpr uint32_t kQBoxBytes = BK * kQBox;
-  // a stage: the weights (bf16, or e4m3 codes) and the rows of one k-block;
-  // FP8W adds kCStages compute stages of widened bf16 weights
+  // FP8W codes are K-contiguous ([G, N, K]): per operand one box of 128
+  // columns x 64 K-codes (64-byte rows, 64-byte TMA swizzle)
+  static constexpr uint32_t kQOpBytes = FP8W ? kCols * BK : 0;
+  static constexpr uint32_t kQBytes = kWOps * kQOpBytes;
+  // a stage: the weights (bf16, or e4m3 codes) and the rows of one k-block
   static constexpr uint32_t kStageBytes = (FP8W ? kQBytes : kWBytes) + kXBytes;
-  static constexpr int kCStages = FP8W ? 3 : 0;  // 3 measured faster than 2 on decode
-  static constexpr uint32_t kCBytes = FP8W ? kWBytes : 0;
-  static constexpr int kStages = ((196608 - kCStages * kCBytes) / kStageBytes) > 8
-                                     ? 8
-                                     : ((196608 - kCStages * kCBytes) / kStageBytes);
-  static constexpr uint32_t kRingBytes = kStages * kStageBytes + kCStages * kCBytes;
-  static constexpr int kCtaThreads = FP8W ? 320 : 192;  // + 4 converter warps
-  static constexpr int kConvThreads = 128;
-  static constexpr uint32_t kAccCols = SWIGLU ? 256 : 128;
-  static constexpr uint32_t kTmemCols = 2 * kAccCols;
+  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  static constexpr uint32_t kRingBytes = kStages * kStageBytes;
+  // FP8W: + 8 converter warps (6-13), two per tensor-memory lane quarter
+  static constexpr int kCtaThreads = FP8W ? 448 : 192;
+  static constexpr int kConvThreads = 256;
+  // Tensor memory: two accumulators (W1 [and W3] x rows), and with fp8
+  // weights kASlots k-blocks of widened weights, the MMA's A operand
+  // (lane = output column, 32 columns = 64 bf16 K-values per operand).
+  static constexpr uint32_t kW3Off = FP8W ? kMaxRows : 128;     // W3 accumulator columns
+  static constexpr uint32_t kAccCols = kWOps * kW3Off;
+  static constexpr int kASlots = FP8W ? 6 : 0;
+  static constexpr uint32_t kACol0 = 2 * kAccCols;
+  static constexpr uint32_t kASlotCols = kWOps * 32;
+  static constexpr uint32_t kTmemCols = FP8W ? 512 : 2 * kAccCols;
   static constexpr uint32_t kStageRowWords = 36;
   static constexpr uint32_t kEpiBytes = 4 * 32 * kStageRowWords * 4;
-  static constexpr size_t kSmemFixed = 1024 + kRingBytes + 256 + kEpiBytes;
-  static constexpr int kBars = 2 * kStages + 2 * kCStages + 5;
-  static_assert(kBars * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit 256 bytes");
-  static_assert((kStages * kStageBytes) % 1024 == 0 && (FP8W ? kQBytes : kWBytes) % 1024 == 0,
-                "128-byte swizzled tiles start on 1024-byte boundaries");
-  static_assert(kQBytes % (16 * kConvThreads) == 0, "whole 16-byte chunks per converter");
+  static constexpr uint32_t kBarBytes = FP8W ? 512 : 256;
+  static constexpr size_t kSmemFixed = 1024 + kRingBytes + kBarBytes + kEpiBytes;
+  // barriers: full, empty per stage, 2 + 2 accumulator, drain; FP8W also
+  // converted and free per A slot
+  static constexpr int kBars = 2 * kStages + 2 * kASlots + 5;
+  static_assert(kBars * 8 + 8 <= kBarBytes, "barriers, TMEM slot and abort flag fit");
+  static_assert(kACol0 + kASlots * kASlotCols <= kTmemCols, "tensor memory");
+  static_assert(kStageBytes % 1024 == 0 && (FP8W ? kQBytes : kWBytes) % 1024 == 0,
+                "swizzled tiles start on 1024-byte boundaries");
 };
 
 // kind::f16 descriptor: fp32 accumulator, bf16 A and B, A MN-major, B K-major.
@@ -1302,12 +1348,12 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *ring = smem;
-  uint8_t *cring = ring + S::kStages * S::kStageBytes;  // FP8W: widened weights
   uint64_t *bars = reinterpret_cast<uint64_t *>(ring + S::kRingBytes);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + S::kBars);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-  float *s_epi = reinterpret_cast<float *>(ring + S::kRingBytes + 256);
-  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kRingBytes + 256 + S::kEpiBytes);
+  float *s_epi = reinterpret_cast<float *>(ring + S::kRingBytes + S::kBarBytes);
+  int32_t *s_off =
+      reinterpret_cast<int32_t *>(ring + S::kRingBytes + S::kBarBytes + S::kEpiBytes);
   int32_t *s_tstart = s_off + (p.G + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -1315,9 +1361,9 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
   const uint32_t accf0 = smem_addr(bars + 2 * S::kStages);
   const uint32_t acce0 = smem_addr(bars + 2 * S::kStages + 2);
   const uint32_t drain = smem_addr(bars + 2 * S::kStages + 4);
-  // FP8W: converted[kCStages], compute-stage empty[kCStages]
+  // FP8W: A slot converted[kASlots], A slot free[kASlots]
   const uint32_t conv0 = smem_addr(bars + 2 * S::kStages + 5);
-  const uint32_t cempty0 = smem_addr(bars + 2 * S::kStages + 5 + S::kCStages);
+  const uint32_t cempty0 = smem_addr(bars + 2 * S::kStages + 5 + S::kASlots);
   const Ctl ctl{abort_flag, p.err};
 
   if (threadIdx.x == 0) {
@@ -1330,8 +1376,8 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
       mbar_init(acce0 + 8 * b, 4);
     }
     mbar_init(drain, 1);
-    for (int c = 0; c < S::kCStages; ++c) {
-      mbar_init(conv0 + 8 * c, S::kConvThreads / 32);
+    for (int c = 0; c < S::kASlots; ++c) {
+      mbar_init(conv0 + 8 * c, 4);  // the 4 warps of the group converting that k-block
       mbar_init(cempty0 + 8 * c, 1);
     }
     *abort_flag = 0;
@@ -1350,7 +1396,7 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
   }
   if (warp == 1) tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
   __syncthreads();
-  const int col_tiles = (p.N + S::kCols - 1) / S::kCols;
+  const int col_tiles = (p.N + S::kTileCols - 1) / S::kTileCols;
   for (int g = threadIdx.x; g < p.G; g += S::kCtaThreads) {
     const int rows = s_off[g + 1] - s_off[g];
     if (rows < 0) bad = true;
@@ -1439,9 +1485,11 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
           tma_gather4(st + wbytes + lane * 4 * 128, &tmX, fb, kb * BK, tok[0], tok[1], tok[2],
                       tok[3]);
         if (lane == 0) {
-          if (FP8W) {  // one 128-column box of codes per operand
-            tma_load_3d(st, &tmW1, fb, c * S::kCols, kb * BK, g);
-            if (SWIGLU) tma_load_3d(st + S::kQBoxBytes, &tmW3, fb, c * S::kCols, kb * BK, g);
+          if (FP8W) {  // codes [G, N, K]: one box (64 K x 128 columns) per operand / half
+            tma_load_3d(st, &tmW1, fb, kb * BK, c * S::kTileCols, g);
+            if (SWIGLU) tma_load_3d(st + S::kQOpBytes, &tmW3, fb, kb * BK, c * S::kTileCols, g);
+            if (S::kWide)
+              tma_load_3d(st + S::kQOpBytes, &tmW1, fb, kb * BK, c * S::kTileCols + 128, g);
           } else {
 #pragma unroll
             for (int j = 0; j < 2; ++j)
@@ -1479,7 +1527,10 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int g, c, r, row0, nr;
         tile_coords(tile, g, c, r, row0, nr);
-        const uint32_t idesc = instr_desc_swap(S::kCols, (nr + 15) & ~15);
+        // bf16: weights an MN-major smem A; fp8: the widened weights in
+        // tensor memory (K-major); the rows K-major in both
+        const uint32_t idesc = FP8W ? instr_desc_kk(S::kCols, (nr + 15) & ~15)
+                                    : instr_desc_swap(S::kCols, (nr + 15) & ~15);
         if (!wait(acce0 + 8 * buf, acc_ph ^ 1, ctl)) {
           ok = false;
           break;
@@ -1494,18 +1545,25 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
           }
           tc_fence_after();
           const uint32_t st = smem_addr(ring + s * S::kStageBytes);
-          const uint32_t wt = FP8W ? smem_addr(cring + cs * S::kCBytes) : st;
           const uint32_t xt = st + (FP8W ? S::kQBytes : S::kWBytes);
+          const uint32_t at = tmem_base + S::kACol0 + cs * S::kASlotCols;  // FP8W
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            // weights: MN-major spans (LBO = span stride), rows: K-major 128-byte rows
+            // rows: K-major 128-byte rows; bf16 weights: MN-major spans (LBO
+            // = span stride); fp8: 8 tensor-memory columns per 16 K-values
             const uint64_t xd = smem_desc(xt + kk * 32, 16, 1024);
-            const uint64_t w1d = smem_desc(wt + kk * 2048, S::kSpanBytes, 1024);
-            umma(d_tmem, w1d, xd, idesc, (kb | kk) != 0);
-            if (SWIGLU) {
-              const uint64_t w3d = smem_desc(wt + 2 * S::kSpanBytes + kk * 2048, S::kSpanBytes,
-                                             1024);
-              umma(d_tmem + 128, w3d, xd, idesc, (kb | kk) != 0);
+            const uint32_t acc = (kb | kk) != 0;
+            if (FP8W) {
+              umma_ts(d_tmem, at + kk * 8, xd, idesc, acc);
+              if (S::kWOps == 2) umma_ts(d_tmem + S::kW3Off, at + 32 + kk * 8, xd, idesc, acc);
+            } else {
+              const uint64_t w1d = smem_desc(st + kk * 2048, S::kSpanBytes, 1024);
+              umma(d_tmem, w1d, xd, idesc, acc);
+              if (SWIGLU) {
+                const uint64_t w3d =
+                    smem_desc(st + 2 * S::kSpanBytes + kk * 2048, S::kSpanBytes, 1024);
+                umma(d_tmem + S::kW3Off, w3d, xd, idesc, acc);
+              }
             }
           }
           any = true;
@@ -1515,7 +1573,7 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
             s = 0;
             ph ^= 1;
           }
-          if (FP8W && ++cs == S::kCStages) {
+          if (FP8W && ++cs == S::kASlots) {
             cs = 0;
             cph ^= 1;
           }
@@ -1547,8 +1605,11 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
       ready = __shfl_sync(0xffffffffu, ready, 0);
       if (!ready) break;
       tc_fence_after();
-      const uint32_t tb = tmem_base + buf * S::kAccCols + ((uint32_t)(quarter * 32) << 16);
-      const int col0 = c * S::kCols + quarter * 32;  // this warp's 32 output columns
+      // wide fp8 tiles: two 128-column halves, each its own accumulator
+      for (int h = 0; h < (S::kWide ? 2 : 1); ++h) {
+      const uint32_t tb = tmem_base + buf * S::kAccCols + h * S::kW3Off +
+                          ((uint32_t)(quarter * 32) << 16);
+      const int col0 = c * S::kTileCols + h * 128 + quarter * 32;  // this warp's 32 columns
       // FP8W: this lane's column scales (lane = column)
       float sc1 = 1.f, sc3 = 1.f;
       if (FP8W && col0 + lane < p.N) {
@@ -1565,7 +1626,7 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
         }
         if (SWIGLU) {
           float u[32];
-          tmem_ld32(tb + 128 + j0, u);
+          tmem_ld32(tb + S::kW3Off + j0, u);
           if (FP8W) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) u[i] *= sc3;
@@ -1614,6 +1675,7 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
         }
         __syncwarp();
       }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce0 + 8 * buf);
@@ -1622,33 +1684,48 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
     }
   } else if (FP8W) {
     // ------------------------------------------------------------ fp8 converters
-    // Per k-block: wait for its codes (stage s) and a free compute stage cs,
-    // widen the codes into the swizzled bf16 weight tiles the MMA reads (see
-    // the single engine's converters; same layout), mark cs converted.
-    const int ct = threadIdx.x - 192;
-    int s = 0, cs = 0;
+    // Per k-block: wait for its codes (stage s) and a free A slot cs; each
+    // thread widens the 64 codes of its weight column (= its tensor-memory
+    // lane, warp w holding lanes 32*(w%4)..) per operand and stores them as
+    // 32 tensor-memory columns, then the slot is marked converted.  Warps 6-9
+    // take the even k-blocks and warps 10-13 the odd ones, so that two
+    // k-blocks are in flight at a time.
+    const int quarter = warp & 3, half = (warp - 6) >> 2;
+    const int m = quarter * 32 + lane;  // weight column within the tile
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    int s = 0, cs = 0, it = 0;
     uint32_t ph = 0, cph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < num_kb; ++kb) {
-        int okw = 1;
-        if (lane == 0)
-          okw = (wait(full0 + 8 * s, ph, ctl) && wait(cempty0 + 8 * cs, cph ^ 1, ctl)) ? 1 : 0;
-        okw = __shfl_sync(0xffffffffu, okw, 0);
-        if (!okw) {
-          ok = false;
-          break;
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        if ((it & 1) == half) {
+          int okw = 1;
+          if (lane == 0)
+            okw = (wait(full0 + 8 * s, ph, ctl) && wait(cempty0 + 8 * cs, cph ^ 1, ctl)) ? 1 : 0;
+          okw = __shfl_sync(0xffffffffu, okw, 0);
+          if (!okw) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t *q = ring + s * S::kStageBytes;
+          const uint32_t at = tmem_base + lane_base + S::kACol0 + cs * S::kASlotCols;
+#pragma unroll
+          for (int op = 0; op < S::kWOps; ++op) {
+            uint32_t v[32];
+            widen_column(q + op * S::kQOpBytes, m, v);
+            tmem_st32(at + op * 32, v);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(conv0 + 8 * cs);
         }
-        widen_codes<S::kQBox, S::kQBytes>(ring + s * S::kStageBytes, cring + cs * S::kCBytes,
-                                          ct);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(conv0 + 8 * cs);
         if (++s == S::kStages) {
           s = 0;
           ph ^= 1;
         }
-        if (++cs == S::kCStages) {
+        if (++cs == S::kASlots) {
           cs = 0;
           cph ^= 1;
         }
@@ -1724,18 +1801,18 @@ bool make_map_b(CUtensorMap *m, const void *B, int G, int K, int N) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over e4m3 codes B [G, K, N] (one byte each, N contiguous), box
-// box_cols (N) x 64 (K) x 1, no swizzle: the converter warps apply the
-// 128-byte swizzle when they write the widened bf16 tile.
-bool make_map_b_q8(CUtensorMap *m, const void *B, int G, int K, int N, int box_cols) {
+// 3-D map over e4m3 codes Q [G, N, K] (one byte each, K contiguous: the
+// transposed weights), box 64 (K) x box_n (N) x 1, 64-byte swizzle (the
+// converters read one column's 64 codes per thread without bank conflicts).
+bool make_map_codes(CUtensorMap *m, const void *Q, int G, int N, int K, int box_n) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)G};
-  cuuint64_t strides[2] = {(cuuint64_t)N, (cuuint64_t)K * N};
-  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)BK, 1};
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)N, (cuuint64_t)G};
+  cuuint64_t strides[2] = {(cuuint64_t)K, (cuuint64_t)N * K};
+  cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)box_n, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(B), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(Q), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1746,8 +1823,8 @@ cudaError_t launch_q8(int rows_cap, int K, int N, int G, const int32_t *offsets,
                       const float *s3, void *out, uint32_t *err, cudaStream_t s) {
   using S = Shape<SWIGLU, SPANS, true>;
   CUtensorMap ma, mb1, mb3;
-  if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b_q8(&mb1, B1, G, K, N, S::kQBox) ||
-      !make_map_b_q8(&mb3, SWIGLU ? B3 : B1, G, K, N, S::kQBox))
+  if (!make_map_a(&ma, A, rows_cap, K) || !make_map_codes(&mb1, B1, G, N, K, S::BN) ||
+      !make_map_codes(&mb3, SWIGLU ? B3 : B1, G, N, K, S::BN))
     return cudaErrorInvalidValue;
   const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
   int dev = 0, sms = 148;
@@ -1875,8 +1952,8 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
   using S = ShapeSwap<SWIGLU, true>;
   CUtensorMap mx, mw1, mw3;
   if (!make_map_rows(&mx, A, rows_cap, K, kRowBox) ||
-      !make_map_b_q8(&mw1, B1, G, K, N, S::kQBox) ||
-      !make_map_b_q8(&mw3, SWIGLU ? B3 : B1, G, K, N, S::kQBox))
+      !make_map_codes(&mw1, B1, G, N, K, S::kCols) ||
+      !make_map_codes(&mw3, SWIGLU ? B3 : B1, G, N, K, S::kCols))
     return cudaErrorInvalidValue;
   const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
   int dev = 0, sms = 148;
@@ -1895,7 +1972,7 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
   p.scale3 = SWIGLU ? s3 : nullptr;
   const long long max_tiles = (long long)((rows_cap + S::kMaxRows - 1) / S::kMaxRows +
                                           (offsets ? G : 0)) *
-                              ((N + S::kCols - 1) / S::kCols);
+                              ((N + S::kTileCols - 1) / S::kTileCols);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
   k_grouped_gemm_swap<SWIGLU, true><<<grid, S::kCtaThreads, smem, s>>>(mx, mw1, mw3, p);
   return cudaGetLastError();

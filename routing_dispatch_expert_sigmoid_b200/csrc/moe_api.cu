@@ -485,7 +485,7 @@ moe_status moe_quantize_fp8(const void *W, int32_t G, int32_t K, int32_t N, void
                             float *scale, void *stream) {
   if (G < 0 || K < 0 || N < 0) return MOE_ERR_INVALID_ARG;
   if ((long long)G * K * N == 0) return MOE_OK;
-  if (N % 16) return MOE_ERR_ALIGNMENT;
+  if (N % 16 || K % 16) return MOE_ERR_ALIGNMENT;
   if (G > 65535) return MOE_ERR_UNSUPPORTED;
   MOE_TRY(need(W));
   MOE_TRY(need(Wq));

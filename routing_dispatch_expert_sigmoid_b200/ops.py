@@ -211,11 +211,11 @@ def moe_check_errors(stream=None) -> int:
 
 # ---- fp8 expert weights -----------------------------------------------------
 def moe_quantize_fp8(W: torch.Tensor, stream=None):
-    """W [G, K, N] (or [K, N]) bf16 -> (codes uint8 of W's shape, scales fp32
-    [G, N] (or [N])), computed by the library."""
+    """W [G, K, N] (or [K, N]) bf16 -> (codes uint8 [G, N, K] (or [N, K]),
+    scales fp32 [G, N] (or [N])), computed by the library."""
     Wg = W if W.dim() == 3 else W.unsqueeze(0)
     G, K, N = Wg.shape
-    q = torch.empty(Wg.shape, dtype=torch.uint8, device=W.device)
+    q = torch.empty((G, N, K), dtype=torch.uint8, device=W.device)
     sc = torch.empty((G, N), dtype=torch.float32, device=W.device)
     _check(lib().moe_quantize_fp8(_p(Wg), G, K, N, _p(q), _p(sc), _stream(stream)),
            "moe_quantize_fp8")

@@ -217,6 +217,7 @@ def test_fp8_layer_argument_checks():
 def test_fp8_quantize_checks():
     lib = ops.lib()
     assert lib.moe_quantize_fp8(_FAKE, 2, 64, 24, _FAKE, _FAKE, None) == -4   # N % 16
+    assert lib.moe_quantize_fp8(_FAKE, 2, 40, 32, _FAKE, _FAKE, None) == -4   # K % 16
     assert lib.moe_quantize_fp8(_FAKE, -1, 64, 32, _FAKE, _FAKE, None) == -1
     assert lib.moe_quantize_fp8(_FAKE, 0, 64, 32, _FAKE, _FAKE, None) == 0    # nothing to do
     assert lib.moe_quantize_fp8(_FAKE + 8, 2, 64, 32, _FAKE, _FAKE, None) == -4

@@ -74,23 +74,26 @@ def _assert_same_quantisation(gpu_set, oracle_set, names):
         gq = gpu_set["W" + k[-1]].cpu().numpy()  # a set's keys: W1 W3 W2 s1 s3 s2
         gs = gpu_set["s" + k[-1]].cpu().numpy()
         gq, gs = (gq, gs) if gq.ndim == 3 else (gq[None], gs[None])
+        gq = gq.swapaxes(1, 2)  # the library stores the codes K-contiguous
         assert (gq == q).all(), f"{k}: codes differ at {np.argwhere(gq != q)[:3].tolist()}"
         assert (gs == s).all(), f"{k}: scales differ"
 
 
 def test_quantizer_matches_oracle_bit_for_bit(dev):
     g = torch.Generator().manual_seed(31)
-    W = torch.randn(3, 100, 48, generator=g) * torch.rand(3, 1, 48, generator=g) * 4
+    W = torch.randn(3, 112, 48, generator=g) * torch.rand(3, 1, 48, generator=g) * 4
     W[0, :, 7] = 0                            # all-zero column: scale 1, codes 0
     W[1, 3, 9] = 3e4                          # one large weight dominates its column
     W[2, :, 11] = 1e-39                       # subnormal in fp32 and bf16
     Wb = W.to(torch.bfloat16)
     q, s = ops.moe_quantize_fp8(Wb.to(dev))
     oq, os_ = oracle.quantize_fp8(to_numpy(Wb))
-    assert (q.cpu().numpy() == oq).all() and (s.cpu().numpy() == os_).all()
+    # the library stores the codes transposed ([G, N, K]); the values must match
+    assert q.shape == (3, 48, 112)
+    assert (q.cpu().numpy().swapaxes(1, 2) == oq).all() and (s.cpu().numpy() == os_).all()
     # a 2-D matrix is one group
     q2, s2 = ops.moe_quantize_fp8(Wb[1].to(dev))
-    assert (q2.cpu().numpy() == oq[1]).all() and (s2.cpu().numpy() == os_[1]).all()
+    assert (q2.cpu().numpy().T == oq[1]).all() and (s2.cpu().numpy() == os_[1]).all()
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -160,8 +163,8 @@ def test_fp8_every_code_through_the_ffn(fp8_engine, dev):
         sc = (g.uniform(0.5, 2.0, (w.E, N)) / (448 * np.sqrt(K))).astype(np.float32)
         sets[k] = (q, sc)
     gpu = {}
-    for k, (q, sc) in sets.items():
-        gpu[k] = torch.from_numpy(q).to(dev)
+    for k, (q, sc) in sets.items():  # the library takes the codes K-contiguous
+        gpu[k] = torch.from_numpy(np.ascontiguousarray(q.swapaxes(1, 2))).to(dev)
         gpu["s" + k[-1]] = torch.from_numpy(sc).to(dev)
     offsets = np.array([0, 50, 50, 192], np.int32)  # an empty expert in the middle
     xb = torch.randn(192, w.d, generator=torch.Generator().manual_seed(42)).to(torch.bfloat16)
