@@ -30,6 +30,12 @@ CASES = {
     "qwen3_small": WORKLOADS["qwen3_prefill"].scaled(T=257, d=192, E=16, k_max=4, f=208),
     "dsv3_small": WORKLOADS["dsv3_prefill"].scaled(T=130, d=256, E=64, f=144, f_shared=80),
     "gptoss_small": WORKLOADS["gptoss_sub"].scaled(T=211, d=208, E=32, k_max=6, k_min=2, f=80),
+    # capacity drops (a quarter of the slots kept), renormalised softmax
+    "qwen3_heavy_drops": WORKLOADS["qwen3_prefill"].scaled(T=150, d=192, E=16, k_max=4, f=208,
+                                                           capacity_factor=0.25),
+    # one expert, k = 1: the dense FFN on fp8 weights
+    "single_expert": WORKLOADS["mixtral_prefill"].scaled(T=77, d=256, E=1, k_max=1, f=384,
+                                                         zipf_s=0.0),
 }
 
 
@@ -175,3 +181,15 @@ def test_fp8_every_code_through_the_ffn(fp8_engine, dev):
     deq = {k: oracle.dequantize_fp8(q, sc) for k, (q, sc) in sets.items()}
     ref = oracle.grouped_ffn(to_numpy(xb), offsets, deq["W1"], deq["W3"], deq["W2"])
     assert_out_close(f64(y), ref, "fp8 FFN over every code", "f32")
+
+
+def test_fp8_empty_batch_is_a_no_op(dev):
+    w = CASES["dsv3_small"]
+    inp = make_inputs(w.scaled(T=1), 0, device=dev)
+    cfg = ops.config(w, T=0)
+    experts = ops.fp8_weight_set(inp["W1"], inp["W3"], inp["W2"])
+    shared = ops.fp8_weight_set(inp["Ws1"], inp["Ws3"], inp["Ws2"])
+    out = torch.empty((0, w.d), dtype=inp["x"].dtype, device=dev)
+    ops.moe_layer_fp8(cfg, inp["x"][:0], inp["Wr"], None, inp["sel_bias"], None, experts, shared,
+                      out, None, ops.workspace(cfg, ops.WS_LAYER))
+    ops.moe_check_errors()
