@@ -309,6 +309,16 @@ struct Params {
   int32_t *clear = nullptr;
   // FP8 weights: per-column scales of B1 and B3, [G, N] fp32
   const float *scale1 = nullptr, *scale3 = nullptr;
+  // PLAIN: output row r is multiplied by row_w[w_row_src[r]] (the gate weight
+  // of the slot the row serves), or nothing when row_w is nullptr
+  const float *row_w = nullptr;
+  const int32_t *w_row_src = nullptr;
+};
+
+// Gate weights to apply in the down projection's epilogue (both nullptr: none).
+struct RowWeights {
+  const float *w = nullptr;
+  const int32_t *row_src = nullptr;
 };
 
 template <bool SWIGLU, int SPANS, bool FP8W = false>
@@ -778,6 +788,13 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
                 o.z += b[2];
                 o.w += b[3];
               }
+              if (p.row_w) {  // the slot's gate weight, applied here instead of in combine
+                const float wr = p.row_w[p.w_row_src[grow]];
+                o.x *= wr;
+                o.y *= wr;
+                o.z *= wr;
+                o.w *= wr;
+              }
               *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)grow * p.N +
                                           gcol) = o;
             }
@@ -1237,6 +1254,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 o.z += b[2];
                 o.w += b[3];
               }
+              if (p.row_w) {  // the slot's gate weight, applied here instead of in combine
+                const float wr = p.row_w[p.w_row_src[grow]];
+                o.x *= wr;
+                o.y *= wr;
+                o.z *= wr;
+                o.w *= wr;
+              }
               *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)grow * p.N +
                                           gcol) = o;
             }
@@ -1668,6 +1692,13 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
                 o.z += b[2];
                 o.w += b[3];
               }
+              if (p.row_w) {  // the slot's gate weight, applied here instead of in combine
+                const float wr = p.row_w[p.w_row_src[grow]];
+                o.x *= wr;
+                o.y *= wr;
+                o.z *= wr;
+                o.w *= wr;
+              }
               *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)grow * p.N +
                                           gcol) = o;
             }
@@ -1820,7 +1851,8 @@ bool make_map_codes(CUtensorMap *m, const void *Q, int G, int N, int K, int box_
 template <bool SWIGLU, int SPANS>
 cudaError_t launch_q8(int rows_cap, int K, int N, int G, const int32_t *offsets, int fixed_rows,
                       const void *A, const void *B1, const void *B3, const float *s1,
-                      const float *s3, void *out, uint32_t *err, cudaStream_t s) {
+                      const float *s3, void *out, uint32_t *err, cudaStream_t s,
+                      RowWeights rw = RowWeights()) {
   using S = Shape<SWIGLU, SPANS, true>;
   CUtensorMap ma, mb1, mb3;
   if (!make_map_a(&ma, A, rows_cap, K) || !make_map_codes(&mb1, B1, G, N, K, S::BN) ||
@@ -1839,6 +1871,8 @@ cudaError_t launch_q8(int rows_cap, int K, int N, int G, const int32_t *offsets,
   }
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
+  p.row_w = rw.w;
+  p.w_row_src = rw.row_src;
   p.scale1 = s1;
   p.scale3 = SWIGLU ? s3 : nullptr;
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
@@ -1852,7 +1886,7 @@ template <bool SWIGLU, int SPANS>
 cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, int fixed_rows,
                    const void *A, const void *B1, const void *B3, void *out, const float *bias,
                    uint32_t *err, cudaStream_t s, const int32_t *row_src = nullptr,
-                   int k_max = 1, int a_rows = 0) {
+                   int k_max = 1, int a_rows = 0, RowWeights rw = RowWeights()) {
   using S = Shape<SWIGLU, SPANS>;
   CUtensorMap ma, mb1, mb3;
   const bool map_ok = row_src ? make_map_rows(&ma, A, a_rows, K, 1) : make_map_a(&ma, A, rows_cap, K);
@@ -1872,6 +1906,8 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
   }
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, bias, row_src, k_max, err};
+  p.row_w = rw.w;
+  p.w_row_src = rw.row_src;
   // never more CTAs than tiles can exist (a group holds at most rows_cap rows)
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
@@ -1883,7 +1919,7 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
 template <bool SWIGLU>
 cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offsets,
                         int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
-                        uint32_t *err, cudaStream_t s) {
+                        uint32_t *err, cudaStream_t s, RowWeights rw = RowWeights()) {
   using S = Shape2<SWIGLU>;
   CUtensorMap ma, mb1, mb3;
   if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
@@ -1902,6 +1938,8 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
     attr_set[dev] = true;
   }
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
+  p.row_w = rw.w;
+  p.w_row_src = rw.row_src;
   const long long max_tiles = (long long)((rows_cap + BM2 - 1) / BM2 + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
   long long pairs = sms / 2;
@@ -1914,7 +1952,7 @@ template <bool SWIGLU>
 cudaError_t launch_swap(int rows_cap, int K, int N, int G, const int32_t *offsets,
                         int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
                         uint32_t *err, cudaStream_t s, const int32_t *row_src = nullptr,
-                        int k_max = 1, int a_rows = 0) {
+                        int k_max = 1, int a_rows = 0, RowWeights rw = RowWeights()) {
   using S = ShapeSwap<SWIGLU>;
   CUtensorMap mx, mw1, mw3;
   const bool map_ok = row_src ? make_map_rows(&mx, A, a_rows, K, 1)
@@ -1935,6 +1973,8 @@ cudaError_t launch_swap(int rows_cap, int K, int N, int G, const int32_t *offset
     attr_set[dev] = true;
   }
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, row_src, k_max, err};
+  p.row_w = rw.w;
+  p.w_row_src = rw.row_src;
   const long long max_tiles = (long long)((rows_cap + S::kMaxRows - 1) / S::kMaxRows +
                                           (offsets ? G : 0)) *
                               ((N + S::kCols - 1) / S::kCols);
@@ -1948,7 +1988,7 @@ template <bool SWIGLU>
 cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *offsets,
                            int fixed_rows, const void *A, const void *B1, const void *B3,
                            const float *s1, const float *s3, void *out, uint32_t *err,
-                           cudaStream_t s) {
+                           cudaStream_t s, RowWeights rw = RowWeights()) {
   using S = ShapeSwap<SWIGLU, true>;
   CUtensorMap mx, mw1, mw3;
   if (!make_map_rows(&mx, A, rows_cap, K, kRowBox) ||
@@ -1968,6 +2008,8 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
     attr_set[dev] = true;
   }
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
+  p.row_w = rw.w;
+  p.w_row_src = rw.row_src;
   p.scale1 = s1;
   p.scale3 = SWIGLU ? s3 : nullptr;
   const long long max_tiles = (long long)((rows_cap + S::kMaxRows - 1) / S::kMaxRows +
@@ -2015,22 +2057,27 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                      const int32_t *offsets, int fixed_rows, const void *A,
                                      const void *B1, const void *B3, void *out, uint32_t *err,
                                      cudaStream_t s, const int32_t *row_src, int k_max,
-                                     int a_rows) {
+                                     int a_rows, const float *row_w,
+                                     const int32_t *w_row_src) {
   if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if (rows_cap == 0) return cudaSuccess;
   const Engine e = pick_engine(swiglu, rows_cap, G, offsets, fixed_rows);
   if (row_src && (!swiglu || e == Engine::kPair)) return cudaErrorInvalidValue;
+  if (row_w && swiglu) return cudaErrorInvalidValue;  // gate weights: the down projection only
+  tc::RowWeights rw;
+  rw.w = row_w;
+  rw.row_src = w_row_src;
   switch (e) {
     case Engine::kPair:
       return swiglu ? tc::launch_pair<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                             out, err, s)
                     : tc::launch_pair<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
-                                             out, err, s);
+                                             out, err, s, rw);
     case Engine::kSwap:
       return swiglu ? tc::launch_swap<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                             out, err, s, row_src, k_max, a_rows)
                     : tc::launch_swap<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
-                                             out, err, s);
+                                             out, err, s, nullptr, 1, 0, rw);
     case Engine::kNarrow:
       if (swiglu)
         return tc::launch<true, 1>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out,
@@ -2040,16 +2087,21 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
       return swiglu ? tc::launch<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                           out, nullptr, err, s, row_src, k_max, a_rows)
                     : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
-                                           out, nullptr, err, s);
+                                           out, nullptr, err, s, nullptr, 1, 0, rw);
   }
 }
 
 cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int G,
                                     const int32_t *offsets, int fixed_rows, const void *A,
                                     const void *B1, const void *B3, const float *s1,
-                                    const float *s3, void *out, uint32_t *err, cudaStream_t s) {
+                                    const float *s3, void *out, uint32_t *err, cudaStream_t s,
+                                    const float *row_w, const int32_t *w_row_src) {
   if (rows_cap <= 0) return cudaSuccess;
   if (G <= 0 || G > tc::kMaxGroups || N % 16 != 0) return cudaErrorInvalidValue;
+  if (row_w && swiglu) return cudaErrorInvalidValue;  // gate weights: the down projection only
+  tc::RowWeights rw;
+  rw.w = row_w;
+  rw.row_src = w_row_src;
   // fp8 weights: swap-AB for decode-sized groups (at most 32 rows per group
   // on average, as for bf16), the single engine otherwise;
   // MOE_GEMM_ENGINE=single|narrow|swap forces one (narrow: 64-column up
@@ -2061,14 +2113,14 @@ cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int
     return swiglu ? tc::launch_swap_q8<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                              s1, s3, out, err, s)
                   : tc::launch_swap_q8<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1,
-                                              B1, s1, nullptr, out, err, s);
+                                              B1, s1, nullptr, out, err, s, rw);
   if (swiglu && env && env[0] == 'n')
     return tc::launch_q8<true, 1>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, s1, s3,
                                   out, err, s);
   return swiglu ? tc::launch_q8<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, s1,
                                          s3, out, err, s)
                 : tc::launch_q8<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B1, s1,
-                                          nullptr, out, err, s);
+                                          nullptr, out, err, s, rw);
 }
 
 cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const void *x,

@@ -227,16 +227,20 @@ moe_status check_fp8_config(const moe_config &c) {
 // (offsets == nullptr: one group of T rows).  `mid` is recorded between the
 // up projection (with SwiGLU) and the down projection.  With row_src, A is
 // the token rows x and the up projection gathers its rows itself.
+// gate_w / gate_src (routed experts, bf16 layers): the down projection
+// multiplies output row r by gate_w[gate_src[r]], its slot's gate weight.
 moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixed_rows,
                     int rows_cap, int f, const void *A, const Weights &w, void *h, void *y,
                     uint32_t *err, cudaStream_t s, const Events &ev = Events(), int mid = -1,
-                    const int32_t *row_src = nullptr) {
+                    const int32_t *row_src = nullptr, const float *gate_w = nullptr,
+                    const int32_t *gate_src = nullptr) {
   if (w.fp8) {
     MOE_TRY_CUDA(launch_grouped_gemm_fp8(true, rows_cap, c.d, f, G, offsets, fixed_rows, A, w.W1,
                                          w.W3, w.s1, w.s3, h, err, s));
     MOE_TRY_CUDA(ev.mark(mid, s));
     MOE_TRY_CUDA(launch_grouped_gemm_fp8(false, rows_cap, f, c.d, G, offsets, fixed_rows, h,
-                                         w.W2, nullptr, w.s2, nullptr, y, err, s));
+                                         w.W2, nullptr, w.s2, nullptr, y, err, s, gate_w,
+                                         gate_src));
     return MOE_OK;
   }
   if (c.dtype == MOE_F32) {
@@ -251,8 +255,17 @@ moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixe
                                         w.W3, h, err, s, row_src, c.k_max, c.T));
   MOE_TRY_CUDA(ev.mark(mid, s));
   MOE_TRY_CUDA(launch_grouped_gemm_bf16(false, rows_cap, f, c.d, G, offsets, fixed_rows, h, w.W2,
-                                        nullptr, y, err, s));
+                                        nullptr, y, err, s, nullptr, 1, 0, gate_w, gate_src));
   return MOE_OK;
+}
+
+// The gate weights can be applied by the down projection's epilogue (each
+// row of y_perm scaled by its slot's weight), leaving the combine a plain
+// sum of the kept rows.  MOE_WEIGHTS_IN_GEMM=1 selects it for bf16 layers;
+// by default the combine applies them.
+bool weights_in_gemm(const moe_config &c) {
+  const char *env = getenv("MOE_WEIGHTS_IN_GEMM");
+  return c.dtype == MOE_BF16 && env && env[0] == '1';
 }
 
 // The dispatch copy can be fused into the up projection (bf16 layers, engines
@@ -315,15 +328,18 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   MOE_TRY_CUDA(ev.mark(1, s));
   const int rows_cap = c.T * c.k_max;
   void *x_perm = at<void>(ws, L.x_perm), *y_perm = at<void>(ws, L.y_perm);
+  const bool wig = weights_in_gemm(c);
+  const float *gate_w = wig ? r.topk_w : nullptr;
+  const int32_t *gate_src = wig ? r.row_src : nullptr;
   if (!we.fp8 && fuse_dispatch(c, rows_cap, r.offsets)) {
     MOE_TRY_CUDA(ev.mark(2, s));
     MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x, we, at<void>(ws, L.h), y_perm, err,
-                     s, ev, 3, r.row_src));
+                     s, ev, 3, r.row_src, gate_w, gate_src));
   } else {
     MOE_TRY_CUDA(launch_dispatch(c, x, r.offsets, r.row_src, x_perm, err, s));
     MOE_TRY_CUDA(ev.mark(2, s));
     MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x_perm, we, at<void>(ws, L.h), y_perm,
-                     err, s, ev, 3));
+                     err, s, ev, 3, nullptr, gate_w, gate_src));
   }
   MOE_TRY_CUDA(ev.mark(4, s));
   const void *shared_y = nullptr;
@@ -333,7 +349,8 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
     shared_y = at<void>(ws, L.y_sh);
   }
   MOE_TRY_CUDA(ev.mark(5, s));
-  MOE_TRY_CUDA(launch_combine(c, y_perm, r.slot_row, r.topk_w, shared_y, out, err, s));
+  MOE_TRY_CUDA(launch_combine(c, y_perm, r.slot_row, wig ? nullptr : r.topk_w, shared_y, out,
+                               err, s));
   MOE_TRY_CUDA(ev.mark(6, s));
   return MOE_OK;
 }

@@ -65,7 +65,8 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *o
                             const int32_t *row_src, void *x_perm, uint32_t *err, cudaStream_t s);
 
 // K7: out[t] = sum_j w[t,j] y_perm[slot_row[t,j]] (+ shared[t]); y_perm and
-// shared are fp32, out is in the layer dtype.
+// shared are fp32, out is in the layer dtype.  topk_w == nullptr: the rows
+// already carry their gate weights (applied by the down projection).
 cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                            const float *topk_w, const void *shared_y, void *out, uint32_t *err,
                            cudaStream_t s);
@@ -86,11 +87,15 @@ cudaError_t launch_ffn_simt_f32(int rows_cap, int d, int f, int G, const int32_t
 // dispatch gather is fused into the GEMM's loads.
 bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *offsets,
                              int fixed_rows);
+// row_w (plain only): output row r is multiplied by row_w[w_row_src[r]], the
+// gate weight of the slot it serves (the combine then only sums).
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
                                      const int32_t *offsets, int fixed_rows, const void *A,
                                      const void *B1, const void *B3, void *out, uint32_t *err,
                                      cudaStream_t s, const int32_t *row_src = nullptr,
-                                     int k_max = 1, int a_rows = 0);
+                                     int k_max = 1, int a_rows = 0,
+                                     const float *row_w = nullptr,
+                                     const int32_t *w_row_src = nullptr);
 
 // K5/K6 with fp8 weights: B1, B3 are e4m3 codes [G, K, N] (N % 16 == 0) with
 // per-column fp32 scales s1, s3 [G, N] (16-byte aligned); the codes are
@@ -99,7 +104,9 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
 cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int G,
                                     const int32_t *offsets, int fixed_rows, const void *A,
                                     const void *B1, const void *B3, const float *s1,
-                                    const float *s3, void *out, uint32_t *err, cudaStream_t s);
+                                    const float *s3, void *out, uint32_t *err, cudaStream_t s,
+                                    const float *row_w = nullptr,
+                                    const int32_t *w_row_src = nullptr);
 
 // Per-column e4m3 quantisation of bf16 weights W [G, K, N]: scale[g, n] =
 // max_k |W| / 448 (1 for an all-zero column), Wq = e4m3(W / scale), rounded

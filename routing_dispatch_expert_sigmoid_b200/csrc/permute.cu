@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(256)
     float my_w = 0.f;
     if (lane < k_max) {
       my_row = slot_row[(size_t)t * k_max + lane];
-      my_w = topk_w[(size_t)t * k_max + lane];
+      my_w = topk_w ? topk_w[(size_t)t * k_max + lane] : 1.0f;  // fmaf(1, y, acc) = y + acc
       if (my_row >= rows_cap) {
         raise_error(err, kErrIndex);
         my_row = -1;

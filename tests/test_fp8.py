@@ -193,3 +193,18 @@ def test_fp8_empty_batch_is_a_no_op(dev):
     ops.moe_layer_fp8(cfg, inp["x"][:0], inp["Wr"], None, inp["sel_bias"], None, experts, shared,
                       out, None, ops.workspace(cfg, ops.WS_LAYER))
     ops.moe_check_errors()
+
+
+@pytest.mark.parametrize("name", ["mixtral_decode_small", "dsv3_small", "qwen3_heavy_drops"])
+def test_fp8_layer_with_weights_in_gemm(name, fp8_engine, dev):
+    """Gate weights applied by the down projection's epilogue on fp8 weights."""
+    import os
+    old = os.environ.get("MOE_WEIGHTS_IN_GEMM")
+    os.environ["MOE_WEIGHTS_IN_GEMM"] = "1"
+    try:
+        test_fp8_layer_matches_oracle(name, fp8_engine, dev)
+    finally:
+        if old is None:
+            os.environ.pop("MOE_WEIGHTS_IN_GEMM", None)
+        else:
+            os.environ["MOE_WEIGHTS_IN_GEMM"] = old

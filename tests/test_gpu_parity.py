@@ -327,3 +327,34 @@ def test_layer_with_dispatch_fused_into_gemm(name, fused_dispatch, dev):
 @pytest.mark.parametrize("name", ["mixtral_small", "dsv3_small", "gptoss_small"])
 def test_fused_dispatch_each_engine(name, fused_dispatch, gemm_engine, dev):
     test_layer_matches_oracle(name, dev)
+
+
+# ---------------------------------------------------------------------------
+# Gate weights applied by the down projection's epilogue (combine only sums)
+# ---------------------------------------------------------------------------
+@pytest.fixture
+def weights_in_gemm():
+    import os
+    old = os.environ.get("MOE_WEIGHTS_IN_GEMM")
+    os.environ["MOE_WEIGHTS_IN_GEMM"] = "1"
+    yield
+    if old is None:
+        os.environ.pop("MOE_WEIGHTS_IN_GEMM", None)
+    else:
+        os.environ["MOE_WEIGHTS_IN_GEMM"] = old
+
+
+@pytest.mark.parametrize("name", BF16_SMALL)
+def test_layer_with_weights_in_gemm(name, weights_in_gemm, dev):
+    test_layer_matches_oracle(name, dev)
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "dsv3_small", "qwen3_small",
+                                  "mixtral_decode_small"])
+def test_weights_in_gemm_each_engine(name, weights_in_gemm, gemm_engine, dev):
+    test_layer_matches_oracle(name, dev)
+
+
+@pytest.mark.parametrize("name", ["t128_dsv3_ragged_k", "e1024_k32_drops"])
+def test_small_batch_layer_with_weights_in_gemm(name, weights_in_gemm, dev):
+    test_small_batch_layer(name, dev)
