@@ -407,6 +407,21 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
   v = __hmul2(v, k);
   return *reinterpret_cast<const uint32_t *>(&v);
 }
+// Four e4m3 codes (one 32-bit word, byte i = K element i) to four bf16 values
+// (two bf16 pairs, low halves first), with fewer integer-pipe operations: the
+// magnitudes' exponent and fraction bits reach their bf16 positions by a byte
+// permute and a multiply by 16 (the FMA pipe), the exact multiply by 2^120
+// rebiases them, and the signs are or-ed back in by a second byte permute.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t &p01, uint32_t &p23) {
+  const uint32_t mag = w & 0x7F7F7F7Fu;
+  const uint32_t m01 = __byte_perm(mag, 0u, 0x4140) * 16u;  // |b0| -> bits 4-10, |b1| -> 20-26
+  const uint32_t m23 = __byte_perm(mag, 0u, 0x4342) * 16u;
+  const __nv_bfloat162 k = __floats2bfloat162_rn(0x1p120f, 0x1p120f);
+  __nv_bfloat162 v01 = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&m01), k);
+  __nv_bfloat162 v23 = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&m23), k);
+  p01 = *reinterpret_cast<const uint32_t *>(&v01) | (__byte_perm(w, 0u, 0x1404) & 0x80008000u);
+  p23 = *reinterpret_cast<const uint32_t *>(&v23) | (__byte_perm(w, 0u, 0x3424) & 0x80008000u);
+}
 __device__ __forceinline__ void e4m3x16_to_bf16(uint4 c, uint4 &lo, uint4 &hi) {
   lo = make_uint4(e4m3x2_to_bf16x2(c.x & 0xffffu), e4m3x2_to_bf16x2(c.x >> 16),
                   e4m3x2_to_bf16x2(c.y & 0xffffu), e4m3x2_to_bf16x2(c.y >> 16));
@@ -435,10 +450,7 @@ __device__ __forceinline__ void widen_chunks(const uint8_t *__restrict__ box, in
   for (int j = 0; j < NC; ++j) {
     const uint32_t w[4] = {c[j].x, c[j].y, c[j].z, c[j].w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      out[8 * j + 2 * i] = e4m3x2_to_bf16x2(w[i] & 0xffffu);
-      out[8 * j + 2 * i + 1] = e4m3x2_to_bf16x2(w[i] >> 16);
-    }
+    for (int i = 0; i < 4; ++i) e4m3x4_to_bf16x4(w[i], out[8 * j + 2 * i], out[8 * j + 2 * i + 1]);
   }
 }
 __device__ __forceinline__ void widen_column(const uint8_t *__restrict__ box, int r,
@@ -2028,29 +2040,39 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
 //   narrow  the same with 64-column up-projection tiles (twice the tiles);
 //   pair    CTA pairs on 256-row tiles (tcgen05 cta_group::2);
 //   swap    weights as the M operand, rows in steps of 16 (swap-AB).
-// Measured on B200 with the engines interleaved in one process (best of four
-// rounds), the single-CTA engine is fastest or tied on every workload here,
-// except the up projection of decode-sized groups (at most 32 rows per group
-// on average), where swap-AB loads only the valid rows instead of 128-row
-// boxes (Mixtral-shaped decode: 0.298 vs 0.320 ms).  Those are the defaults;
+// Defaults, from B200 measurements with the engines alternated call by call
+// in one process:
+//   - decode-sized groups (at most 32 rows per group on average): swap-AB for
+//     the up projection, which loads only the valid rows (Mixtral-shaped
+//     decode: 0.298 vs 0.320 ms single-CTA), single-CTA for the down
+//     projection (CTA pairs: 0.171 vs 0.146 ms);
+//   - larger groups: CTA pairs for the up projection, and for the down
+//     projection when it is at least 4096 columns wide.  Sharing each B tile
+//     between two SMs cuts the shared-memory and L2 traffic per FLOP by a
+//     third, which under the 1 kW power cap keeps the clock up: Mixtral
+//     prefill 4.22 vs 6.31 ms, DeepSeek-V3 prefill 5.89 vs 6.36, Qwen3 up
+//     0.54 vs 0.67 ms (down, 2048 wide: 0.43 vs 0.40, single kept).  On
+//     boxes that did not reach the cap the single-CTA engine was ahead by
+//     6% on Mixtral prefill.
 // MOE_GEMM_ENGINE=single|narrow|pair|swap selects one engine for every GEMM.
 enum class Engine { kSingle, kNarrow, kPair, kSwap };
 
 static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offsets,
-                          int fixed_rows) {
+                          int fixed_rows, int N) {
   const char *env = getenv("MOE_GEMM_ENGINE");
   if (env && env[0] == 's' && env[1] == 'i') return Engine::kSingle;
   if (env && env[0] == 'n') return Engine::kNarrow;
   if (env && env[0] == 'p') return Engine::kPair;
   if (env && env[0] == 's' && env[1] == 'w') return Engine::kSwap;
   const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
-  if (swiglu && mean_rows <= 32) return Engine::kSwap;
+  if (mean_rows <= 32) return swiglu ? Engine::kSwap : Engine::kSingle;
+  if (swiglu || N >= 4096) return Engine::kPair;
   return Engine::kSingle;
 }
 
 bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *offsets,
                              int fixed_rows) {
-  return swiglu && pick_engine(swiglu, rows_cap, G, offsets, fixed_rows) != Engine::kPair;
+  return swiglu && pick_engine(swiglu, rows_cap, G, offsets, fixed_rows, 0) != Engine::kPair;
 }
 
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
@@ -2061,7 +2083,7 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                      const int32_t *w_row_src) {
   if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if (rows_cap == 0) return cudaSuccess;
-  const Engine e = pick_engine(swiglu, rows_cap, G, offsets, fixed_rows);
+  const Engine e = pick_engine(swiglu, rows_cap, G, offsets, fixed_rows, N);
   if (row_src && (!swiglu || e == Engine::kPair)) return cudaErrorInvalidValue;
   if (row_w && swiglu) return cudaErrorInvalidValue;  // gate weights: the down projection only
   tc::RowWeights rw;

@@ -224,17 +224,27 @@ def test_fp8_quantize_checks():
 
 
 def test_fp8_widening_bit_formula_gives_every_code():
-    """The GEMM widens e4m3 codes to bf16 by moving bits -- the byte to the
-    top of a 16-bit half, exponent and fraction shifted right by 4, sign kept
-    -- and one multiply by 2^120.  Emulated here for every finite code against
-    the oracle's decoding (the GPU tests cover the hardware's multiply)."""
+    """The GEMM widens four e4m3 codes (one 32-bit word) to bf16 by moving
+    bits: signs cleared, each pair's bytes placed 16 bits apart and multiplied
+    by 16 (exponent and fraction land in the bf16 field), one multiply by
+    2^120, then the signs or-ed back in.  Emulated here for every finite code
+    in every byte position against the oracle's decoding (the GPU tests cover
+    the hardware's multiply)."""
     import numpy as np
 
     import oracle
-    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint32)
-    y = codes << 8
-    bits = ((y >> 4) & 0x07F0) | (y & 0x8000)
-    val = (bits << 16).astype(np.uint32).view(np.float32).astype(np.float64) * 2.0 ** 120
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint64)
     ref = oracle.e4m3_decode(codes.astype(np.uint8))
-    assert (val == ref).all()
-    assert (np.signbit(val) == np.signbit(ref)).all()
+    other = np.uint64(0x38)  # the code of 1.0 in the other byte positions
+    for pos in range(4):
+        words = np.full(codes.shape, 0, np.uint64)
+        for q in range(4):
+            words |= (codes if q == pos else other) << np.uint64(8 * q)
+        mag = words & np.uint64(0x7F7F7F7F)
+        byte = (mag >> np.uint64(8 * pos)) & np.uint64(0xFF)
+        field = (byte * np.uint64(16)) & np.uint64(0xFFFF)   # this half's 16 bits
+        sign = (words >> np.uint64(8 * pos + 7)) & np.uint64(1)
+        val = (field.astype(np.uint32) << 16).view(np.float32).astype(np.float64) * 2.0 ** 120
+        val = np.where(sign == 1, -val, val)
+        assert (val == ref).all(), pos
+        assert (np.signbit(val) == np.signbit(ref)).all(), pos
