@@ -13,11 +13,13 @@
 //   K3a  one CTA per chunk of kChunk slots: per-chunk expert histogram
 //        (shared-memory atomics; counts do not depend on order);
 //   K3b  one CTA: per expert, exclusive scan of the chunk histograms (the
-//        chunk's first rank), totals, C = ceil(cf * sum k_t / E) in double,
+//        chunk's first rank; each expert's chunks split into ranges summed
+//        by separate threads), totals, C = ceil(cf * sum k_t / E) in double,
 //        kept = min(count, C), offsets = exclusive scan of kept, drops;
-//   K3c  one warp per chunk walks its slots 32 at a time in order; lanes
-//        with the same expert find each other with __match_any_sync and rank
-//        themselves by lane order on top of the chunk's running count.
+//   K3c  one warp per chunk loads the chunk's expert ids, then walks them
+//        32 at a time in order; lanes with the same expert find each other
+//        with __match_any_sync and rank themselves by lane order on top of
+//        the chunk's running count.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -53,6 +55,7 @@ __global__ void __launch_bounds__(256) k_hist(const int32_t *__restrict__ idx, l
 }
 
 constexpr int kScanThreads = 1024;
+constexpr int kScanBatch = 16;  // chunk histograms loaded before they are summed
 
 __global__ void __launch_bounds__(kScanThreads)
     k_scan(const int32_t *__restrict__ chunk_counts, int n_chunks, int E, double cf,
@@ -62,18 +65,53 @@ __global__ void __launch_bounds__(kScanThreads)
   __shared__ long long s_part[kScanThreads / 32];
   __shared__ long long s_total;
   __shared__ int32_t s_cnt[1024];
+  __shared__ int32_t s_sum[kScanThreads];  // [part][expert] chunk-range sums
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
-  // E <= 1024 = blockDim: thread e owns expert e.
+  // E <= 1024 = blockDim.  Expert e's chunks are split into P contiguous
+  // ranges, one thread (part, e) each: the ranges are summed, each thread
+  // takes the sum of the earlier ranges as its base and writes its chunks'
+  // bases.
+  int P = kScanThreads / E;
+  if (P > n_chunks) P = n_chunks;
+  if (P < 1) P = 1;
+  const int per = (n_chunks + P - 1) / P;
+  const int e = tid % E, part = tid / E;
+  const bool active = part < P;
+  const int c0 = active ? min(part * per, n_chunks) : 0;
+  const int c1 = active ? min(c0 + per, n_chunks) : 0;
+  int sum = 0;
+  for (int c = c0; c < c1; c += kScanBatch) {
+    int v[kScanBatch];
+#pragma unroll
+    for (int i = 0; i < kScanBatch; ++i)
+      v[i] = c + i < c1 ? chunk_counts[(size_t)(c + i) * E + e] : 0;
+#pragma unroll
+    for (int i = 0; i < kScanBatch; ++i) sum += v[i];
+  }
+  if (active) s_sum[tid] = sum;
+  __syncthreads();
+  if (active) {
+    int run = 0;
+    for (int q = 0; q < part; ++q) run += s_sum[q * E + e];
+    for (int c = c0; c < c1; c += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+        v[i] = c + i < c1 ? chunk_counts[(size_t)(c + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+        if (c + i < c1) {
+          chunk_base[(size_t)(c + i) * E + e] = run;
+          run += v[i];
+        }
+    }
+    if (part == P - 1) s_cnt[e] = run;
+  }
+  __syncthreads();
   long long my = 0;
   if (tid < E) {
-    int run = 0;
-    for (int c = 0; c < n_chunks; ++c) {
-      chunk_base[(size_t)c * E + tid] = run;
-      run += chunk_counts[(size_t)c * E + tid];
-    }
-    counts[tid] = run;
-    s_cnt[tid] = run;
-    my = run;
+    my = s_cnt[tid];
+    counts[tid] = (int32_t)my;
   }
   // block sum of counts = sum over tokens of k_t
   long long v = my;
@@ -128,17 +166,30 @@ __global__ void __launch_bounds__(32)
            const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ offsets,
            const int32_t *__restrict__ cap, int32_t *__restrict__ slot_row,
            int32_t *__restrict__ row_src) {
-  extern __shared__ int32_t run[];
+  extern __shared__ int32_t s_rank[];  // run[E] (running count), off[E] (first row)
+  int32_t *run = s_rank, *off = s_rank + E;
   const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) run[e] = chunk_base[(size_t)blockIdx.x * E + e];
-  __syncwarp();
-  const int C = cap[0];
   const long long a0 = (long long)blockIdx.x * kChunk;
   const long long a1 = min(a0 + kChunk, n_slots);
-  for (long long base = a0; base < a1; base += 32) {
-    const long long a = base + lane;
+  // Every load is issued before the ordered walk, which then only touches
+  // registers and shared memory.
+  int ev[kChunk / 32];
+#pragma unroll
+  for (int i = 0; i < kChunk / 32; ++i) {
+    const long long a = a0 + 32 * i + lane;
+    ev[i] = a < a1 ? idx[a] : -1;
+  }
+  for (int e = lane; e < E; e += 32) {
+    run[e] = chunk_base[(size_t)blockIdx.x * E + e];
+    off[e] = offsets[e];
+  }
+  const int C = cap[0];
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < kChunk / 32; ++i) {
+    const long long a = a0 + 32 * i + lane;
     const bool valid = a < a1;
-    const int e = valid ? idx[a] : -1;
+    const int e = ev[i];
     const bool real = valid && e >= 0 && e < E;
     const unsigned peers = __match_any_sync(0xffffffffu, real ? e : E + lane);
     const int before = __popc(peers & ((1u << lane) - 1u));
@@ -150,7 +201,7 @@ __global__ void __launch_bounds__(32)
       if (C >= 0 && rho >= C) {
         slot_row[a] = -1;
       } else {
-        const int row = offsets[e] + rho;
+        const int row = off[e] + rho;
         slot_row[a] = row;
         row_src[row] = (int32_t)a;
       }
@@ -185,7 +236,8 @@ cudaError_t launch_capacity(const moe_config &c, const int32_t *topk_idx, int32_
   k_scan<<<1, kScanThreads, 0, s>>>(chunk_counts, nch, c.E, (double)c.capacity_factor, chunk_base,
                                     counts, kept, offsets, n_dropped, cap);
   if (nch > 0)
-    k_rank<<<nch, 32, eb, s>>>(topk_idx, slots, c.E, chunk_base, offsets, cap, slot_row, row_src);
+    k_rank<<<nch, 32, 2 * eb, s>>>(topk_idx, slots, c.E, chunk_base, offsets, cap, slot_row,
+                                   row_src);
   return cudaGetLastError();
 }
 

@@ -5,7 +5,7 @@
 // g are offsets[g]..offsets[g+1]-1 (the expert-contiguous layout of the
 // dispatch step).  fp32 tensors have no bf16 tensor-core path; the fp32
 // workload is the small correctness configuration, so a tiled fp32 FMA GEMM
-// (64 x 64 tiles, 4 x 4 outputs per thread) is enough.
+// is enough.
 //   pass 1 (swiglu): h[r, n] = silu(sum_k A[r,k] W1[g,k,n]) * (sum_k A[r,k] W3[g,k,n])
 //   pass 2 (plain):  y[r, n] = sum_k h[r,k] W2[g,k,n]
 #include "moe_internal.cuh"
@@ -13,14 +13,18 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 64, BN = 64, BK = 16;
+// 32 x 32 output tiles (2 x 2 per thread) so that the few rows of a small
+// layer still spread over the SMs; the next K slice is loaded into registers
+// while the current one is multiplied from shared memory.
+constexpr int BM = 32, BN = 32, BK = 32;
+constexpr int kPer = BM * BK / 256;  // elements of a tile each thread loads (4)
 
 template <bool SWIGLU>
 __global__ void __launch_bounds__(256)
     k_ffn_f32(const float *__restrict__ A, const float *__restrict__ B1,
               const float *__restrict__ B3, float *__restrict__ C, const int32_t *offsets,
               int fixed_rows, int K, int N) {
-  __shared__ float as[BK][BM + 4];
+  __shared__ float as[BK][BM + 1];
   __shared__ float b1s[BK][BN];
   __shared__ float b3s[SWIGLU ? BK : 1][BN];
   const int g = blockIdx.z;
@@ -31,52 +35,57 @@ __global__ void __launch_bounds__(256)
   const float *Bg1 = B1 + (size_t)g * K * N;
   const float *Bg3 = SWIGLU ? B3 + (size_t)g * K * N : nullptr;
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-  float acc1[4][4], acc3[4][4];
+  float ra[kPer], rb1[kPer], rb3[kPer];
+  // element i of this thread's share: A (row i*8 + tid/32, k tid%32), B (k i*8 + tid/32, col tid%32)
+  auto load = [&](int k0) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc1[i][j] = acc3[i][j] = 0.f;
-  for (int k0 = 0; k0 < K; k0 += BK) {
-    for (int i = tid; i < BM * BK; i += 256) {
-      const int r = i / BK, kk = i % BK;
+    for (int i = 0; i < kPer; ++i) {
+      const int r = i * 8 + tid / 32, kk = tid % 32;
       const int m = m0 + r, k = k0 + kk;
-      as[kk][r] = (m < rows && k < K) ? A[(size_t)(r0 + m) * K + k] : 0.f;
+      ra[i] = (m < rows && k < K) ? A[(size_t)(r0 + m) * K + k] : 0.f;
+      const int kb = k0 + r, n = n0 + kk;
+      const bool in = kb < K && n < N;
+      rb1[i] = in ? Bg1[(size_t)kb * N + n] : 0.f;
+      if (SWIGLU) rb3[i] = in ? Bg3[(size_t)kb * N + n] : 0.f;
     }
-    for (int i = tid; i < BK * BN; i += 256) {
-      const int kk = i / BN, c = i % BN;
-      const int k = k0 + kk, n = n0 + c;
-      const bool in = k < K && n < N;
-      b1s[kk][c] = in ? Bg1[(size_t)k * N + n] : 0.f;
-      if (SWIGLU) b3s[kk][c] = in ? Bg3[(size_t)k * N + n] : 0.f;
+  };
+  float acc1[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, acc3[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  load(0);
+  for (int k0 = 0; k0 < K; k0 += BK) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int r = i * 8 + tid / 32, kk = tid % 32;
+      as[kk][r] = ra[i];
+      b1s[r][kk] = rb1[i];
+      if (SWIGLU) b3s[r][kk] = rb3[i];
     }
     __syncthreads();
+    if (k0 + BK < K) load(k0 + BK);
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
-      float a[4], b1[4], b3[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = as[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        b1[j] = b1s[kk][tx * 4 + j];
-        if (SWIGLU) b3[j] = b3s[kk][tx * 4 + j];
+      const float a0 = as[kk][ty * 2], a1 = as[kk][ty * 2 + 1];
+      const float b0 = b1s[kk][tx * 2], b1 = b1s[kk][tx * 2 + 1];
+      acc1[0][0] = fmaf(a0, b0, acc1[0][0]);
+      acc1[0][1] = fmaf(a0, b1, acc1[0][1]);
+      acc1[1][0] = fmaf(a1, b0, acc1[1][0]);
+      acc1[1][1] = fmaf(a1, b1, acc1[1][1]);
+      if (SWIGLU) {
+        const float c0 = b3s[kk][tx * 2], c1 = b3s[kk][tx * 2 + 1];
+        acc3[0][0] = fmaf(a0, c0, acc3[0][0]);
+        acc3[0][1] = fmaf(a0, c1, acc3[0][1]);
+        acc3[1][0] = fmaf(a1, c0, acc3[1][0]);
+        acc3[1][1] = fmaf(a1, c1, acc3[1][1]);
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc1[i][j] = fmaf(a[i], b1[j], acc1[i][j]);
-          if (SWIGLU) acc3[i][j] = fmaf(a[i], b3[j], acc3[i][j]);
-        }
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
+  for (int i = 0; i < 2; ++i) {
+    const int m = m0 + ty * 2 + i;
     if (m >= rows) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
+    for (int j = 0; j < 2; ++j) {
+      const int n = n0 + tx * 2 + j;
       if (n >= N) continue;
       float v = acc1[i][j];
       if (SWIGLU) v = (v / (1.0f + expf(-v))) * acc3[i][j];

@@ -43,21 +43,24 @@ __device__ __forceinline__ float spec_sigmoidf(float z) {
   return __fdiv_rn(1.0f, __fadd_rn(1.0f, spec_expf(-z)));
 }
 
-// Is candidate (k1, i1) ranked ahead of (k0, i0)?
-__device__ __forceinline__ bool ahead(float k1, int i1, float k0, int i0) {
-  return k1 > k0 || (k1 == k0 && i1 < i0);
+// Selection keys as unsigned integers in the fp32 order of the keys, -0 and
+// +0 equal (both rank as +0).  0 is below every key and stands for "no
+// candidate" (a negative NaN that would map there is moved up to 1).
+__device__ __forceinline__ uint32_t order_key(float k) {
+  uint32_t b = __float_as_uint(k);
+  if (b == 0x80000000u) b = 0u;
+  const uint32_t u = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return u ? u : 1u;
 }
 
-__device__ __forceinline__ void warp_argmax(float &key, int &idx) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    float ok = __shfl_xor_sync(kFull, key, off);
-    int oi = __shfl_xor_sync(kFull, idx, off);
-    if (ahead(ok, oi, key, idx)) {
-      key = ok;
-      idx = oi;
-    }
-  }
+// The warp's best candidate: lane candidates (ordered key u, index i; u == 0
+// for none) are ranked by larger key, then lower index.  Two warp reductions
+// (the largest key, then the lowest index holding it).  -1 if no lane has a
+// candidate.
+__device__ __forceinline__ int warp_best(uint32_t u, int i) {
+  const uint32_t top = __reduce_max_sync(kFull, u);
+  if (top == 0u) return -1;
+  return __reduce_min_sync(kFull, u == top ? i : 0x7fffffff);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -86,6 +89,7 @@ __device__ __forceinline__ void gate_token(const GatingArgs &g, int t, const flo
   const int E = g.E;
 
   float key[NPL], val[NPL];  // val: logit (softmax modes) or sigmoid score
+  uint32_t ku[NPL];          // key[i] as an ordered integer
   uint32_t alive = 0;
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
@@ -104,6 +108,7 @@ __device__ __forceinline__ void gate_token(const GatingArgs &g, int t, const flo
         key[i] = v;
       }
     }
+    ku[i] = order_key(key[i]);
   }
 
   int kt = g.k_per_token ? g.k_per_token[t] : g.k_max;
@@ -122,8 +127,7 @@ __device__ __forceinline__ void gate_token(const GatingArgs &g, int t, const flo
     }
     __syncwarp();
     const int gsz = E / g.n_groups, m = g.group_score_topk;
-    float gscore = -INFINITY;
-    int gidx = 0x7fffffff;
+    uint32_t gu = 0;  // this lane's group score, ordered (0: no group)
     if (lane < g.n_groups) {
       float top[8];
 #pragma unroll
@@ -144,19 +148,14 @@ __device__ __forceinline__ void gate_token(const GatingArgs &g, int t, const flo
 #pragma unroll
       for (int q = 1; q < 8; ++q)
         if (q < m) sc = __fadd_rn(sc, top[q]);
-      gscore = sc;
-      gidx = lane;
+      gu = order_key(sc);
     }
     uint32_t kept_groups = 0;
     for (int r = 0; r < g.topk_groups; ++r) {
-      float bk = gscore;
-      int bi = gidx;
-      warp_argmax(bk, bi);
-      kept_groups |= 1u << bi;
-      if (bi == lane) {
-        gscore = -INFINITY;
-        gidx = 0x7fffffff;
-      }
+      const int win = warp_best(gu, lane);
+      if (win < 0) break;
+      kept_groups |= 1u << win;
+      if (win == lane) gu = 0;
     }
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
@@ -169,24 +168,24 @@ __device__ __forceinline__ void gate_token(const GatingArgs &g, int t, const flo
   int my_idx = -1;
   float my_val = 0.f;
   for (int j = 0; j < kt; ++j) {
-    float bk = -INFINITY;
+    uint32_t bu = 0;  // this lane's best alive candidate (the lowest i among equals)
     int bi = 0x7fffffff;
     float bv = 0.f;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
-      if (((alive >> i) & 1u) && (key[i] > bk || bi == 0x7fffffff)) {
-        bk = key[i];
+      if (((alive >> i) & 1u) && ku[i] > bu) {
+        bu = ku[i];
         bi = i * 32 + lane;
         bv = val[i];
       }
     }
-    warp_argmax(bk, bi);
-    if (bi == 0x7fffffff) break;  // fewer candidates than k_t (rejected on the host)
-    const int owner = bi & 31;
+    const int win = warp_best(bu, bi);
+    if (win < 0) break;  // fewer candidates than k_t (rejected on the host)
+    const int owner = win & 31;
     const float v = __shfl_sync(kFull, bv, owner);
-    if (lane == owner) alive &= ~(1u << (bi >> 5));
+    if (lane == owner) alive &= ~(1u << (win >> 5));
     if (lane == j) {
-      my_idx = bi;
+      my_idx = win;
       my_val = v;
     }
   }

@@ -748,11 +748,12 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
         float v[32];
         tmem_ld32(tb + c, v);
         const int col = n * S::BN + c;
-        if (FP8W) scale_cols(v, p.scale1 + (size_t)g * p.N, col, p.N);
+        // split K: every split is the same weight group 0
+        if (FP8W) scale_cols(v, p.scale1 + (size_t)(p.k_split ? 0 : g) * p.N, col, p.N);
         if (SWIGLU) {
           float u[32];
           tmem_ld32(tb + S::BN + c, u);
-          if (FP8W) scale_cols(u, p.scale3 + (size_t)g * p.N, col, p.N);
+          if (FP8W) scale_cols(u, p.scale3 + (size_t)(p.k_split ? 0 : g) * p.N, col, p.N);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
         }
@@ -2145,14 +2146,22 @@ cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int
                                           nullptr, out, err, s, rw);
 }
 
-cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const void *x,
-                                const void *Wr, float *partials, int32_t *clear, uint32_t *err,
-                                cudaStream_t s) {
-  using Sh = tc::Shape<false, 1>;
-  if (T <= 0 || S < 1 || S > tc::kMaxGroups || k_split <= 0 || k_split % tc::BK)
+namespace tc {
+
+// Split-K launch of the single engine without SwiGLU (fp32 output): S groups
+// of the same T rows, group s at K offset s*k_split (its tiles read past K as
+// zeros).  The A map holds exactly T rows, so a tile's rows past T read as
+// zeros too.
+template <int SPANS, bool FP8W>
+cudaError_t launch_split(int T, int K, int N, int S, int k_split, const void *A, const void *B,
+                         const float *scale, float *out, int32_t *clear, uint32_t *err,
+                         cudaStream_t s) {
+  using Sh = Shape<false, SPANS, FP8W>;
+  if (T <= 0 || S < 1 || S > kMaxGroups || k_split <= 0 || k_split % BK)
     return cudaErrorInvalidValue;
   CUtensorMap ma, mb;
-  if (!tc::make_map_a(&ma, x, T, d) || !tc::make_map_b(&mb, Wr, 1, d, E))
+  if (!make_map_a(&ma, A, T, K)) return cudaErrorInvalidValue;
+  if (FP8W ? !make_map_codes(&mb, B, 1, N, K, Sh::BN) : !make_map_b(&mb, B, 1, K, N))
     return cudaErrorInvalidValue;
   const size_t smem = Sh::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(S + 1);
   int dev = 0, sms = 148;
@@ -2160,26 +2169,65 @@ cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const v
   static bool attr_set[64] = {};
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(
-        tc::k_grouped_gemm<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(Sh::kSmemFixed + sizeof(int32_t) * 2 * (tc::kMaxGroups + 1)));
+        k_grouped_gemm<false, SPANS, FP8W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(Sh::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  tc::Params p{nullptr, S, T, S * T, d, E, partials, nullptr, nullptr, 1, err, k_split, clear};
-  const long long tiles = (long long)S * ((T + tc::BM - 1) / tc::BM) * ((E + Sh::BN - 1) / Sh::BN);
+  Params p{nullptr, S, T, S * T, K, N, out, nullptr, nullptr, 1, err, k_split, clear};
+  p.scale1 = scale;
+  const long long tiles = (long long)S * ((T + BM - 1) / BM) * ((N + Sh::BN - 1) / Sh::BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
-  tc::k_grouped_gemm<false, 1><<<grid, tc::kThreads, smem, s>>>(ma, mb, mb, p);
+  k_grouped_gemm<false, SPANS, FP8W><<<grid, Sh::kCtaThreads, smem, s>>>(ma, mb, mb, p);
   return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const void *x,
+                                const void *Wr, float *partials, int32_t *clear, uint32_t *err,
+                                cudaStream_t s) {
+  return tc::launch_split<1, false>(T, d, E, S, k_split, x, Wr, nullptr, partials, clear, err, s);
+}
+
+// Tile widths: 64 columns (bf16), 128 (fp8: the converters widen whole
+// 128-column rows).
+cudaError_t launch_gemm_split(bool fp8, int T, int K, int N, int S, const void *A, const void *B,
+                              const float *scale, float *out, uint32_t *err, cudaStream_t s) {
+  if (S < 1 || K % (S * tc::BK)) return cudaErrorInvalidValue;
+  if (fp8) {
+    if (N % 16) return cudaErrorInvalidValue;
+    return tc::launch_split<2, true>(T, K, N, S, K / S, A, B, scale, out, nullptr, err, s);
+  }
+  return tc::launch_split<1, false>(T, K, N, S, K / S, A, B, nullptr, out, nullptr, err, s);
 }
 
 cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,
                              const float *bias, float *logits, uint32_t *err, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  // one group of T rows; B = Wr viewed as [1, d, E]; tile width follows E
-  if (E <= 64)
+  // One group of T rows; B = Wr viewed as [1, d, E].  A tile is 128 rows by
+  // 64 x spans columns.  Wide tiles read a block of x once for all experts,
+  // narrow ones give more CTAs when T is short: take the width with the
+  // fewest waves x spans (the time of the busiest CTA), ties to the widest.
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long row_tiles = (T + tc::BM - 1) / tc::BM;
+  int spans = 1;
+  long long best = -1;
+  for (int sp = 4; sp >= 1; sp /= 2) {
+    if (sp > 1 && E <= 64 * sp / 2) continue;  // wider than E needs
+    const long long tiles = row_tiles * ((E + 64 * sp - 1) / (64 * sp));
+    const long long cost = (tiles + sms - 1) / sms * sp;
+    if (best < 0 || cost < best) {
+      best = cost;
+      spans = sp;
+    }
+  }
+  if (spans == 1)
     return tc::launch<false, 1>(T, d, E, 1, nullptr, T, x, Wr, Wr, logits, bias, err, s);
-  if (E <= 128)
+  if (spans == 2)
     return tc::launch<false, 2>(T, d, E, 1, nullptr, T, x, Wr, Wr, logits, bias, err, s);
   return tc::launch<false, 4>(T, d, E, 1, nullptr, T, x, Wr, Wr, logits, bias, err, s);
 }

@@ -57,7 +57,7 @@ moe_status check_config(const moe_config *c) {
 // Workspace regions, each 256-byte aligned.
 struct Layout {
   size_t logits, topk_idx, topk_w, counts, kept, offsets, slot_row, row_src, n_dropped;
-  size_t cap_scratch, x_perm, h, y_perm, h_sh, y_sh, total;
+  size_t cap_scratch, x_perm, h, y_perm, h_sh, y_sh, sh_part, total;
 };
 
 Layout layout(const moe_config &c, int kind) {
@@ -88,6 +88,8 @@ Layout layout(const moe_config &c, int kind) {
     if (c.f_shared > 0) {
       L.h_sh = take((size_t)c.T * c.f_shared * s);
       L.y_sh = take((size_t)c.T * c.d * sizeof(float));
+      const size_t part = shared_split_bytes(c);  // decode-sized batches only
+      if (part) L.sh_part = take(part);
     }
   }
   L.total = o;
@@ -343,14 +345,24 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   }
   MOE_TRY_CUDA(ev.mark(4, s));
   const void *shared_y = nullptr;
+  int shared_parts = 1;
   if (c.f_shared > 0) {
-    MOE_TRY(ffn_impl(c, 1, nullptr, c.T, c.T, c.f_shared, x, wsh, at<void>(ws, L.h_sh),
-                     at<void>(ws, L.y_sh), err, s));
-    shared_y = at<void>(ws, L.y_sh);
+    const SharedSplitPlan sp = shared_split_plan(c, wsh.fp8);
+    if (sp.use) {
+      const float *parts = nullptr;
+      MOE_TRY_CUDA(launch_shared_split(c, sp, wsh.fp8, x, wsh.W1, wsh.W3, wsh.W2, wsh.s1, wsh.s3,
+                                       wsh.s2, at<void>(ws, L.h_sh), at<float>(ws, L.y_sh),
+                                       at<void>(ws, L.sh_part), &parts, &shared_parts, err, s));
+      shared_y = parts;
+    } else {
+      MOE_TRY(ffn_impl(c, 1, nullptr, c.T, c.T, c.f_shared, x, wsh, at<void>(ws, L.h_sh),
+                       at<void>(ws, L.y_sh), err, s));
+      shared_y = at<void>(ws, L.y_sh);
+    }
   }
   MOE_TRY_CUDA(ev.mark(5, s));
   MOE_TRY_CUDA(launch_combine(c, y_perm, r.slot_row, wig ? nullptr : r.topk_w, shared_y, out,
-                               err, s));
+                               err, s, shared_parts));
   MOE_TRY_CUDA(ev.mark(6, s));
   return MOE_OK;
 }

@@ -67,9 +67,11 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *o
 // K7: out[t] = sum_j w[t,j] y_perm[slot_row[t,j]] (+ shared[t]); y_perm and
 // shared are fp32, out is in the layer dtype.  topk_w == nullptr: the rows
 // already carry their gate weights (applied by the down projection).
+// shared_y: shared_parts fp32 blocks [T, d] (partial sums of the shared
+// expert, added in order), or nullptr.
 cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                            const float *topk_w, const void *shared_y, void *out, uint32_t *err,
-                           cudaStream_t s);
+                           cudaStream_t s, int shared_parts = 1);
 
 // K9: fp32 SIMT grouped SwiGLU FFN (fp32 layers).  h: [rows_cap, f] fp32.
 cudaError_t launch_ffn_simt_f32(int rows_cap, int d, int f, int G, const int32_t *offsets,
@@ -125,6 +127,28 @@ cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,
 cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const void *x,
                                 const void *Wr, float *partials, int32_t *clear, uint32_t *err,
                                 cudaStream_t s);
+
+// Split-K GEMM of one group of T rows (bf16 A [T, K]): out [S][T][N] fp32,
+// split s over K columns s*K/S .. (s+1)*K/S-1 (K a multiple of 64*S).  B is
+// [K, N] bf16, or with fp8 the e4m3 codes [N, K] and column scales [N].
+cudaError_t launch_gemm_split(bool fp8, int T, int K, int N, int S, const void *A, const void *B,
+                              const float *scale, float *out, uint32_t *err, cudaStream_t s);
+
+// The shared expert of a decode-sized batch, split along K (shared_expert.cu).
+struct SharedSplitPlan {
+  bool use = false;
+  int s_up = 1, s_down = 1;
+};
+SharedSplitPlan shared_split_plan(const moe_config &c, bool fp8);
+// Scratch for the partial sums (the larger of the bf16 and fp8 plans; 0 if neither).
+size_t shared_split_bytes(const moe_config &c);
+// h: [T, f_shared] bf16; y_sh: [T, d] fp32.  On return *shared_y / *shared_parts
+// describe the partial sums the combine adds.
+cudaError_t launch_shared_split(const moe_config &c, const SharedSplitPlan &p, bool fp8,
+                                const void *x, const void *W1, const void *W3, const void *W2,
+                                const float *s1, const float *s3, const float *s2, void *h,
+                                float *y_sh, void *scratch, const float **shared_y,
+                                int *shared_parts, uint32_t *err, cudaStream_t s);
 
 // Routing of small batches (decode): split-K router, then one kernel that
 // sums the partials, gates and ranks (see route_small.cu).  The plan depends

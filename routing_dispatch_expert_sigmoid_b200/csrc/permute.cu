@@ -112,8 +112,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
     k_combine(const uint4 *__restrict__ y, const int32_t *__restrict__ slot_row,
               const float *__restrict__ topk_w, const uint4 *__restrict__ shared_y,
-              uint4 *__restrict__ out, int Tn, int k_max, int rows_cap, int row_vecs,
-              uint32_t *err) {
+              int shared_parts, uint4 *__restrict__ out, int Tn, int k_max, int rows_cap,
+              int row_vecs, uint32_t *err) {
   constexpr int N = Vec<T>::N;  // output values per 16-byte vector
   constexpr int Q = N / 4;      // fp32 input vectors per output vector
   __shared__ int32_t s_row[8][32];
@@ -150,6 +150,16 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int q = 0; q < Q; ++q)
           Vec<float>::load(ldg_nc(shared_y + (size_t)t * in_vecs + (size_t)v * Q + q), acc + 4 * q);
+        for (int sp = 1; sp < shared_parts; ++sp) {  // further partial sums, in order
+          const uint4 *part = shared_y + (size_t)sp * Tn * in_vecs + (size_t)t * in_vecs;
+#pragma unroll
+          for (int q = 0; q < Q; ++q) {
+            float f[4];
+            Vec<float>::load(ldg_nc(part + (size_t)v * Q + q), f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[4 * q + i] += f[i];
+          }
+        }
       } else {
 #pragma unroll
         for (int i = 0; i < N; ++i) acc[i] = 0.f;
@@ -208,7 +218,7 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *o
 
 cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                            const float *topk_w, const void *shared_y, void *out, uint32_t *err,
-                           cudaStream_t s) {
+                           cudaStream_t s, int shared_parts) {
   if (c.T == 0) return cudaSuccess;
   const int esz = c.dtype == MOE_F32 ? 4 : 2;
   const int row_vecs = c.d * esz / 16;
@@ -217,13 +227,13 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
   if (c.dtype == MOE_F32)
     k_combine<float><<<grid, 256, 0, s>>>(
         static_cast<const uint4 *>(y_perm), slot_row, topk_w,
-        static_cast<const uint4 *>(shared_y), static_cast<uint4 *>(out), c.T, c.k_max, rows_cap,
-        row_vecs, err);
+        static_cast<const uint4 *>(shared_y), shared_parts, static_cast<uint4 *>(out), c.T,
+        c.k_max, rows_cap, row_vecs, err);
   else
     k_combine<__nv_bfloat16><<<grid, 256, 0, s>>>(
         static_cast<const uint4 *>(y_perm), slot_row, topk_w,
-        static_cast<const uint4 *>(shared_y), static_cast<uint4 *>(out), c.T, c.k_max, rows_cap,
-        row_vecs, err);
+        static_cast<const uint4 *>(shared_y), shared_parts, static_cast<uint4 *>(out), c.T,
+        c.k_max, rows_cap, row_vecs, err);
   return cudaGetLastError();
 }
 

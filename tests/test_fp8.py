@@ -29,6 +29,9 @@ CASES = {
     "ragged_n_k": WORKLOADS["mixtral_prefill"].scaled(T=200, d=272, f=400),
     "qwen3_small": WORKLOADS["qwen3_prefill"].scaled(T=257, d=192, E=16, k_max=4, f=208),
     "dsv3_small": WORKLOADS["dsv3_prefill"].scaled(T=130, d=256, E=64, f=144, f_shared=80),
+    # decode-sized batch: the shared expert split along K (8 up, 2 down splits)
+    "dsv3_decode_shared_split": WORKLOADS["dsv3_decode"].scaled(T=100, d=512, E=64, f=144,
+                                                                f_shared=128),
     "gptoss_small": WORKLOADS["gptoss_sub"].scaled(T=211, d=208, E=32, k_max=6, k_min=2, f=80),
     # capacity drops (a quarter of the slots kept), renormalised softmax
     "qwen3_heavy_drops": WORKLOADS["qwen3_prefill"].scaled(T=150, d=192, E=16, k_max=4, f=208,

@@ -209,7 +209,8 @@ def test_empty_batch(dev):
 # the separate kernels.  Cases: one token; the largest batch with a ragged last
 # K slice (d = 448 is 7 steps of 64); 512 experts with variable k and padded
 # slots; 1024 experts with k = 32 (4096 slots ranked by one CTA) and capacity
-# drops; a small capacity factor.
+# drops; a small capacity factor; a shared expert whose projections are both
+# split along K (7 up splits, 4 down splits added by the combine).
 SMALL_BATCH = {
     "t1_mixtral": WORKLOADS["mixtral_decode"].scaled(T=1, d=512, f=128),
     "t128_dsv3_ragged_k": WORKLOADS["dsv3_decode"].scaled(T=128, d=448, f=64, f_shared=64),
@@ -218,6 +219,7 @@ SMALL_BATCH = {
     "e1024_k32_drops": WORKLOADS["qwen3_prefill"].scaled(T=128, d=128, E=1024, k_max=32, f=64),
     "qwen3_cf_half": WORKLOADS["qwen3_prefill"].scaled(T=96, d=192, E=16, k_max=4, f=64,
                                                        capacity_factor=0.5),
+    "t64_dsv3_shared_split": WORKLOADS["dsv3_decode"].scaled(T=64, d=448, f=64, f_shared=256),
 }
 
 
