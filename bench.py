@@ -20,7 +20,10 @@ Extra keys of the JSON line:
                during the timed region, the burst figure otherwise;
   e2e          the same metric through the C ABI with host buffers: per step a
                pinned-host -> device copy of x and a device -> pinned-host copy
-               of the layer output are inside the timed region;
+               of the layer output are inside the timed region, double-buffered
+               on two copy streams so that they overlap the neighbouring steps'
+               layers (serial_value: the same with copies and layer in one
+               stream, one after the other);
   cpu_baseline the CPU oracle as it stands, on a bounded sample of the same
                workload, on the host cores (rank 0, N=1 only);
   clocks       nvidia-smi samples taken during the timed region;
@@ -194,13 +197,27 @@ def small_batch_routing(w) -> bool:
             and not os.environ.get("MOE_SMALL_ROUTE", "1").startswith("0"))
 
 
+def shared_split_k(w) -> bool:
+    """Whether the layer splits its shared expert along K (a decode-sized
+    batch: at most two 128-row tiles, 256-column output tiles, splits that
+    divide the 64-deep K blocks, at most one wave of 148 CTAs)."""
+    if w.f_shared <= 0 or w.dtype != "bf16":
+        return False
+    row_tiles = (w.T + 127) // 128
+    if row_tiles > 2 or w.d % 64 or w.f_shared % 64:
+        return False
+    kb, tiles = w.d // 64, row_tiles * ((w.f_shared + 255) // 256)
+    s_up = max(s for s in range(1, min(16, kb) + 1) if kb % s == 0 and s * tiles <= 148)
+    return s_up >= 2
+
+
 def launches_per_layer(w) -> int:
     """Kernel launches of one moe_layer call (see the C ABI's launch order)."""
     # router, gating, hist+scan+rank -- or the two small-batch launches
     routing = 2 if small_batch_routing(w) else 1 + 1 + 3
     n = routing + 1 + 2 + 1  # + dispatch, 2 FFN passes, combine
-    if w.f_shared > 0:
-        n += 2
+    if w.f_shared > 0:  # two FFN passes, or gate, up, SwiGLU and down split along K
+        n += 4 if shared_split_k(w) else 2
     return n
 
 
@@ -320,31 +337,69 @@ def run_device(layer: Layer, steps: int, warmup: int, dist, gpu_index: int) -> d
 
 
 def run_e2e(layer: Layer, steps: int, warmup: int, dist) -> dict:
-    """Host buffers through the C ABI: H2D of x and D2H of the output inside the timed region."""
+    """Host buffers through the C ABI, double-buffered the way a serving loop
+    runs: every step copies its x from pinned host memory and its output back
+    to pinned host memory, on two copy streams, so that the input copy of step
+    i+1 and the output copy of step i-1 overlap the layer of step i.  The timed
+    region runs from before the first input copy to after the last output
+    copy."""
     x_host = layer.inp["x"].cpu().pin_memory()
-    out_host = torch.empty_like(x_host).pin_memory()
-    x_dev = torch.empty_like(layer.inp["x"])
-    out_dev = torch.empty_like(layer.out)
-    stream = torch.cuda.current_stream()
+    out_host = [torch.empty_like(x_host).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(layer.inp["x"]) for _ in range(2)]
+    out_dev = [torch.empty_like(layer.out) for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    x_free = [torch.cuda.Event() for _ in range(2)]     # the layer is done with x_dev[b]
+    out_ready = [torch.cuda.Event() for _ in range(2)]
+    out_free = [torch.cuda.Event() for _ in range(2)]   # out_dev[b] has been copied out
 
-    def one():
-        x_dev.copy_(x_host, non_blocking=True)
-        layer.step(x_dev, out_dev)
-        out_host.copy_(out_dev, non_blocking=True)
+    def load(b):
+        with torch.cuda.stream(h2d):
+            h2d.wait_event(x_free[b])
+            x_dev[b].copy_(x_host, non_blocking=True)
+            in_ready[b].record(h2d)
 
-    for _ in range(warmup):
-        one()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    barrier(dist)
-    t0.record(stream)
-    for _ in range(steps):
-        one()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier(dist)
+    def run(n):
+        h2d.wait_stream(comp)
+        d2h.wait_stream(comp)
+        load(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                load(1 - b)
+            comp.wait_event(in_ready[b])
+            comp.wait_event(out_free[b])
+            layer.step(x_dev[b], out_dev[b])
+            x_free[b].record(comp)
+            out_ready[b].record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(out_ready[b])
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                out_free[b].record(d2h)
+        comp.wait_stream(d2h)
+
+    def serial(n):  # the same copies and layer, one after the other on one stream
+        for _ in range(n):
+            x_dev[0].copy_(x_host, non_blocking=True)
+            layer.step(x_dev[0], out_dev[0])
+            out_host[0].copy_(out_dev[0], non_blocking=True)
+
+    ms = {}
+    for kind, fn in (("overlapped", run), ("serial", serial)):
+        fn(max(warmup, 2))
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier(dist)
+        t0.record(comp)
+        fn(steps)
+        t1.record(comp)
+        torch.cuda.synchronize()
+        barrier(dist)
+        ms[kind] = t0.elapsed_time(t1)
     nbytes = x_host.numel() * x_host.element_size()
-    return {"ms": t0.elapsed_time(t1), "h2d": nbytes, "d2h": out_host.numel() * out_host.element_size()}
+    return {"ms": ms["overlapped"], "ms_serial": ms["serial"], "h2d": nbytes,
+            "d2h": out_host[0].numel() * out_host[0].element_size()}
 
 
 def kernel_roofline(alg: dict, ms: float, peak_tf: float, peak_gbs: float, traffic, tf_src: str,
@@ -464,6 +519,7 @@ def main():
     w = pre.w
     ms_max, tokens = aggregate(rp["ms"], w.T * a.steps, dist)
     e2e_ms = None if e2e is None else aggregate(e2e["ms"], w.T * a.steps, dist)[0]
+    e2e_serial_ms = None if e2e is None else aggregate(e2e["ms_serial"], w.T * a.steps, dist)[0]
     alg = algorithmic(w, rp["R"], rp["touched"])
     up_ms = rp["stage_ms"]["up_swiglu"]
     # The sustained bf16 figure applies when the timed region ran under the
@@ -571,8 +627,11 @@ def main():
             "fp8_weights": fp8_obj,
             "e2e": None if e2e is None else {
                 "value": round(tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
-            "gpu_launches": (launches_per_layer(w) * a.steps * (1 if e2e is None else 2)
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "copies": "pinned host buffers; each step's input and output copies run on two "
+                          "copy streams, overlapping the neighbouring steps' layers",
+                "serial_value": round(tokens / (e2e_serial_ms * 1e-3), 1)},
+            "gpu_launches": (launches_per_layer(w) * a.steps * (1 if e2e is None else 3)
                              + (dec_obj["gpu_launches"] if dec_obj else 0)
                              + (fp8_obj["gpu_launches"] if fp8_obj else 0)),
             "clocks": rp["clocks"],

@@ -2055,6 +2055,11 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
 //     0.54 vs 0.67 ms (down, 2048 wide: 0.43 vs 0.40, single kept).  On
 //     boxes that did not reach the cap the single-CTA engine was ahead by
 //     6% on Mixtral prefill.
+//   - except for the up projection of ragged groups of at most 256 rows on
+//     average (routed experts only), where a 256-row pair tile is often
+//     half empty: single-CTA (DeepSeek-V3-shaped prefill, 128 rows per expert
+//     on average: 3.52 vs 3.74 ms; GPT-OSS-shaped sub-experts: 1.27 vs
+//     1.35 ms).
 // MOE_GEMM_ENGINE=single|narrow|pair|swap selects one engine for every GEMM.
 enum class Engine { kSingle, kNarrow, kPair, kSwap };
 
@@ -2067,8 +2072,8 @@ static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offse
   if (env && env[0] == 's' && env[1] == 'w') return Engine::kSwap;
   const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
   if (mean_rows <= 32) return swiglu ? Engine::kSwap : Engine::kSingle;
-  if (swiglu || N >= 4096) return Engine::kPair;
-  return Engine::kSingle;
+  if (swiglu) return (offsets && mean_rows <= 256) ? Engine::kSingle : Engine::kPair;
+  return N >= 4096 ? Engine::kPair : Engine::kSingle;
 }
 
 bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *offsets,
@@ -2191,16 +2196,15 @@ cudaError_t launch_router_split(int T, int d, int E, int S, int k_split, const v
   return tc::launch_split<1, false>(T, d, E, S, k_split, x, Wr, nullptr, partials, clear, err, s);
 }
 
-// Tile widths: 64 columns (bf16), 128 (fp8: the converters widen whole
-// 128-column rows).
+// 256-column output tiles (the down projection's single-engine shapes).
 cudaError_t launch_gemm_split(bool fp8, int T, int K, int N, int S, const void *A, const void *B,
                               const float *scale, float *out, uint32_t *err, cudaStream_t s) {
   if (S < 1 || K % (S * tc::BK)) return cudaErrorInvalidValue;
   if (fp8) {
     if (N % 16) return cudaErrorInvalidValue;
-    return tc::launch_split<2, true>(T, K, N, S, K / S, A, B, scale, out, nullptr, err, s);
+    return tc::launch_split<4, true>(T, K, N, S, K / S, A, B, scale, out, nullptr, err, s);
   }
-  return tc::launch_split<1, false>(T, K, N, S, K / S, A, B, nullptr, out, nullptr, err, s);
+  return tc::launch_split<4, false>(T, K, N, S, K / S, A, B, nullptr, out, nullptr, err, s);
 }
 
 cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,

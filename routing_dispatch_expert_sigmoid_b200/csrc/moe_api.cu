@@ -347,7 +347,7 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   const void *shared_y = nullptr;
   int shared_parts = 1;
   if (c.f_shared > 0) {
-    const SharedSplitPlan sp = shared_split_plan(c, wsh.fp8);
+    const SharedSplitPlan sp = shared_split_plan(c);
     if (sp.use) {
       const float *parts = nullptr;
       MOE_TRY_CUDA(launch_shared_split(c, sp, wsh.fp8, x, wsh.W1, wsh.W3, wsh.W2, wsh.s1, wsh.s3,

@@ -139,8 +139,8 @@ struct SharedSplitPlan {
   bool use = false;
   int s_up = 1, s_down = 1;
 };
-SharedSplitPlan shared_split_plan(const moe_config &c, bool fp8);
-// Scratch for the partial sums (the larger of the bf16 and fp8 plans; 0 if neither).
+SharedSplitPlan shared_split_plan(const moe_config &c);
+// Scratch for the partial sums (0 without a plan).
 size_t shared_split_bytes(const moe_config &c);
 // h: [T, f_shared] bf16; y_sh: [T, d] fp32.  On return *shared_y / *shared_parts
 // describe the partial sums the combine adds.

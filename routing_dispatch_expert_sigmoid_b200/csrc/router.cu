@@ -9,7 +9,8 @@
 // owning TM x TN outputs; x and Wr tiles of BK along d are staged through
 // shared memory (x transposed so a thread's TM rows are one broadcast read).
 // The expert tile width BN follows E so that small-E layers do not waste
-// lanes on empty columns.
+// lanes on empty columns.  Short batches with at most 16 experts take one
+// warp per token instead.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -69,6 +70,47 @@ __global__ void __launch_bounds__(256) k_router(const T *__restrict__ x, const T
   }
 }
 
+// Short batches with few experts: one warp per token, lane l accumulating
+// the products of K positions l, l+32, ... for every expert, then a
+// butterfly sum across the warp (a fixed order).  The tiled kernel above
+// would give a 256-token batch only four CTAs.
+template <typename T, int EMAX>
+__global__ void __launch_bounds__(256)
+    k_router_warp(const T *__restrict__ x, const T *__restrict__ Wr, const float *__restrict__ bias,
+                  float *__restrict__ logits, int Tn, int d, int E) {
+  const int t = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (t >= Tn) return;  // whole warp leaves together
+  float acc[EMAX];
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
+  const T *xr = x + (size_t)t * d;
+#pragma unroll 4
+  for (int k = lane; k < d; k += 32) {
+    const float xv = to_f32(xr[k]);
+    const T *w = Wr + (size_t)k * E;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e)
+      if (e < E) acc[e] = fmaf(xv, to_f32(w[e]), acc[e]);
+  }
+  float mine = 0.f;
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) {
+    float v = acc[e];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == e) mine = v;
+  }
+  if (lane < E) logits[(size_t)t * E + lane] = mine + (bias ? bias[lane] : 0.f);
+}
+
+template <typename T, int EMAX>
+cudaError_t run_warp(const moe_config &c, const void *x, const void *Wr, const float *bias,
+                     float *logits, cudaStream_t s) {
+  k_router_warp<T, EMAX><<<(c.T + 7) / 8, 256, 0, s>>>(
+      static_cast<const T *>(x), static_cast<const T *>(Wr), bias, logits, c.T, c.d, c.E);
+  return cudaGetLastError();
+}
+
 template <typename T, int BM, int BN, int BK, int TM, int TN>
 cudaError_t run(const moe_config &c, const void *x, const void *Wr, const float *bias,
                 float *logits, cudaStream_t s) {
@@ -81,6 +123,8 @@ cudaError_t run(const moe_config &c, const void *x, const void *Wr, const float 
 template <typename T>
 cudaError_t dispatch_tile(const moe_config &c, const void *x, const void *Wr, const float *bias,
                           float *logits, cudaStream_t s) {
+  if (c.T <= 2048 && c.E <= 8) return run_warp<T, 8>(c, x, Wr, bias, logits, s);
+  if (c.T <= 2048 && c.E <= 16) return run_warp<T, 16>(c, x, Wr, bias, logits, s);
   if (c.E <= 8) return run<T, 64, 8, 32, 2, 1>(c, x, Wr, bias, logits, s);
   if (c.E <= 16) return run<T, 64, 16, 32, 2, 2>(c, x, Wr, bias, logits, s);
   if (c.E <= 32) return run<T, 64, 32, 32, 2, 4>(c, x, Wr, bias, logits, s);

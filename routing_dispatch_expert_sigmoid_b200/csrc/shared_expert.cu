@@ -65,13 +65,14 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-SharedSplitPlan shared_split_plan(const moe_config &c, bool fp8) {
+SharedSplitPlan shared_split_plan(const moe_config &c) {
   SharedSplitPlan p;
   if (c.f_shared <= 0 || c.dtype != MOE_BF16 || env_disabled()) return p;
   const long long row_tiles = (c.T + 127) / 128;
   if (row_tiles > 2 || c.d % 64 || c.f_shared % 64) return p;
-  // output tile widths of the split GEMMs: 64 columns (bf16), 128 (fp8)
-  const int bn = fp8 ? 128 : 64;
+  // 256-column output tiles: each CTA reads its slice of x once for 256
+  // columns (narrower tiles would re-read it from L2 once per 64 columns)
+  const int bn = 256;
   const long long up_tiles = row_tiles * ((c.f_shared + bn - 1) / bn);
   const long long dn_tiles = row_tiles * ((c.d + bn - 1) / bn);
   p.s_up = pick_splits(c.d / 64, up_tiles);
@@ -81,15 +82,11 @@ SharedSplitPlan shared_split_plan(const moe_config &c, bool fp8) {
 }
 
 size_t shared_split_bytes(const moe_config &c) {
-  size_t most = 0;
-  for (int fp8 = 0; fp8 < 2; ++fp8) {
-    const SharedSplitPlan p = shared_split_plan(c, fp8 != 0);
-    if (!p.use) continue;
-    size_t b = 2 * (size_t)p.s_up * c.T * c.f_shared * sizeof(float);
-    if (p.s_down > 1) b += (size_t)p.s_down * c.T * c.d * sizeof(float);
-    most = b > most ? b : most;
-  }
-  return most;
+  const SharedSplitPlan p = shared_split_plan(c);
+  if (!p.use) return 0;
+  size_t b = 2 * (size_t)p.s_up * c.T * c.f_shared * sizeof(float);
+  if (p.s_down > 1) b += (size_t)p.s_down * c.T * c.d * sizeof(float);
+  return b;
 }
 
 cudaError_t launch_shared_split(const moe_config &c, const SharedSplitPlan &p, bool fp8,

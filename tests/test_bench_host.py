@@ -58,7 +58,8 @@ def test_launch_count_and_algorithmic_work():
     assert bench.launches_per_layer(WORKLOADS["dsv3_prefill"]) == 11
     # decode batches: split-K router + fused gating/ranking instead of 5 launches
     assert bench.launches_per_layer(WORKLOADS["mixtral_decode"]) == 6
-    assert bench.launches_per_layer(WORKLOADS["dsv3_decode"]) == 8
+    # decode-sized shared expert: gate, up, SwiGLU and down, split along K
+    assert bench.launches_per_layer(WORKLOADS["dsv3_decode"]) == 10
     assert bench.launches_per_layer(WORKLOADS["tiny_f32"]) == 9
     a = bench.algorithmic(w, R=16384, touched=8)
     assert a["up_flops"] == 4 * 16384 * 4096 * 14336

@@ -61,6 +61,29 @@ def test_route_bit_exact_and_logits(name, dev):
     check_routing_bit_exact(w, hin, out)
 
 
+# The CUDA-core router (fp32 layers, and bf16 layers whose E is not a multiple
+# of 8): one warp per token for short batches with at most 16 experts, the
+# tiled kernel beyond 2048 tokens or 16 experts.
+SIMT_ROUTER = {
+    "bf16_e12_warp": WORKLOADS["qwen3_prefill"].scaled(T=300, d=200, E=12, k_max=3, f=64),
+    "bf16_e12_tiled": WORKLOADS["qwen3_prefill"].scaled(T=2100, d=200, E=12, k_max=3, f=64),
+    "bf16_e20_tiled": WORKLOADS["qwen3_prefill"].scaled(T=300, d=136, E=20, k_max=3, f=64),
+    "f32_e8_tiled": WORKLOADS["tiny_f32"].scaled(T=2049),
+}
+
+
+@pytest.mark.parametrize("name", list(SIMT_ROUTER))
+def test_simt_router_bit_exact_and_logits(name, dev):
+    w = SIMT_ROUTER[name]
+    hin = _host_inputs(w, seed=6)
+    inp = gpu_inputs(w, 6, dev, hin)
+    cfg, out = run_route(w, inp)
+    ref = oracle.router_logits(to_numpy(hin["x"]), to_numpy(hin["Wr"]),
+                               to_numpy(hin["logit_bias"]))
+    assert_logits_close(out["logits"], ref)
+    check_routing_bit_exact(w, hin, out)
+
+
 @pytest.mark.parametrize("name", list(SMALL))
 def test_dispatch_bit_exact(name, dev):
     w = SMALL[name]
