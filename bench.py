@@ -12,6 +12,11 @@ per GPU) every rank runs its own replica of the layer on its own batch and
 the time is the max over ranks (weak scaling, no collective on the data path).
 
 Extra keys of the JSON line:
+  layer_roofline_frac          max(F / bf16 peak, B / HBM peak) of the whole layer
+                               over its measured time, against the measured
+                               peaks (MEASURED_PEAKS.json, burst figures);
+  layer_roofline_frac_nominal  the same against nominal B200 peaks (8 TB/s,
+                               2.25 PFLOP/s dense bf16);
   roofline     the up-projection + SwiGLU grouped GEMM (the dominant kernel):
                algorithmic FLOPs (prefill) or bytes (decode) per launch over its
                mean launch time, from CUDA events recorded on the launching
@@ -58,6 +63,15 @@ from routing_dispatch_expert_sigmoid_b200.workloads import WORKLOADS, make_input
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Nominal B200 figures, the second denominator of the layer roofline: 8 TB/s
+# HBM3e and 2.25 PFLOP/s dense bf16.
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+def layer_roofline_ms(alg: dict, peaks: dict) -> float:
+    """max(F / bf16 peak, B / HBM peak) of the whole layer, in ms."""
+    return max(alg["layer_flops"] / (peaks["bf16_tflops"] * 1e12),
+               alg["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
 PROFILES = os.path.join(ROOT, "profiles")
 GEMM_SRC = os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc",
                         "grouped_gemm_sm100.cu")
@@ -530,8 +544,7 @@ def main():
                                traffic_from_profile(a.workload) if a.T <= 0 else None,
                                f"{pk_src} bf16 {'sustained' if sustained else 'burst'}",
                                f"{pk_src} copy bandwidth")
-    layer_roof_ms = max(alg["layer_flops"] / (pk["bf16_tflops"] * 1e12),
-                        alg["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
+    layer_roof_ms = layer_roofline_ms(alg, pk)
     del pre
     torch.cuda.empty_cache()
 
@@ -549,8 +562,7 @@ def main():
             algd, d_up_ms, pk["bf16_tflops_sustained"] if sustained_d else pk["bf16_tflops"],
             pk["hbm_gbs"], traffic_from_profile(a.decode_workload),
             f"{pk_src} bf16 {'sustained' if sustained_d else 'burst'}", f"{pk_src} copy bandwidth")
-        d_layer_roof_ms = max(algd["layer_flops"] / (pk["bf16_tflops"] * 1e12),
-                              algd["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
+        d_layer_roof_ms = layer_roofline_ms(algd, pk)
         dec_obj = {
             "workload": f"{a.decode_workload}: T={wd.T}, d={wd.d}, E={wd.E}, top-{wd.k_max}, "
                         f"f={wd.f}", "steps": dsteps,
@@ -559,6 +571,8 @@ def main():
             "stage_ms": {k: round(v, 4) for k, v in rd["stage_ms"].items()},
             "layer_roofline_ms": round(d_layer_roof_ms, 4),
             "layer_roofline_frac": round(d_layer_roof_ms / (d_ms_max / dsteps), 4),
+            "layer_roofline_frac_nominal": round(
+                layer_roofline_ms(algd, NOMINAL_PEAKS) / (d_ms_max / dsteps), 4),
             "roofline": roof_dec, "kept_rows": rd["R"], "experts_touched": rd["touched"],
             "gpu_launches": launches_per_layer(wd) * dsteps,
         }
@@ -579,8 +593,7 @@ def main():
             pk["bf16_tflops_sustained"] if sustained_q else pk["bf16_tflops"], pk["hbm_gbs"],
             None, f"{pk_src} bf16 {'sustained' if sustained_q else 'burst'}",
             f"{pk_src} copy bandwidth")
-        q_layer_roof_ms = max(algq["layer_flops"] / (pk["bf16_tflops"] * 1e12),
-                              algq["layer_bytes"] / (pk["hbm_gbs"] * 1e9)) * 1e3
+        q_layer_roof_ms = layer_roofline_ms(algq, pk)
         fp8_obj = {
             "workload": f"{a.fp8_workload} with e4m3 expert weights (per-column fp32 scales)",
             "steps": qsteps, "value": round(q_tokens / (q_ms_max * 1e-3), 1),
@@ -588,6 +601,8 @@ def main():
             "stage_ms": {k: round(v, 4) for k, v in rq["stage_ms"].items()},
             "layer_roofline_ms": round(q_layer_roof_ms, 4),
             "layer_roofline_frac": round(q_layer_roof_ms / (q_ms_max / qsteps), 4),
+            "layer_roofline_frac_nominal": round(
+                layer_roofline_ms(algq, NOMINAL_PEAKS) / (q_ms_max / qsteps), 4),
             "roofline": roof_q, "gpu_launches": launches_per_layer(wq) * qsteps,
         }
         del q
@@ -622,6 +637,8 @@ def main():
             "stage_ms": {k: round(v, 4) for k, v in rp["stage_ms"].items()},
             "layer_roofline_ms": round(layer_roof_ms, 4),
             "layer_roofline_frac": round(layer_roof_ms / (ms_max / a.steps), 4),
+            "layer_roofline_frac_nominal": round(
+                layer_roofline_ms(alg, NOMINAL_PEAKS) / (ms_max / a.steps), 4),
             "roofline": roof_pre,
             "decode": dec_obj,
             "fp8_weights": fp8_obj,

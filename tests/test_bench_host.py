@@ -107,3 +107,12 @@ def test_algorithmic_bytes_with_fp8_weights():
     assert q["up_flops"] == b["up_flops"]
     # one byte per expert weight plus the column scales; router, x and out unchanged
     assert b["layer_bytes"] - q["layer_bytes"] == 8 * (3 * d * f - 4 * (2 * f + d))
+
+
+def test_layer_roofline_takes_the_slower_bound():
+    alg = {"layer_flops": 2.25e12, "layer_bytes": 8e9}   # 1 ms at either nominal peak
+    assert abs(bench.layer_roofline_ms(alg, bench.NOMINAL_PEAKS) - 1.0) < 1e-12
+    alg = {"layer_flops": 4.5e12, "layer_bytes": 8e9}    # flops bound: 2 ms
+    assert abs(bench.layer_roofline_ms(alg, bench.NOMINAL_PEAKS) - 2.0) < 1e-12
+    alg = {"layer_flops": 2.25e12, "layer_bytes": 24e9}  # bytes bound: 3 ms
+    assert abs(bench.layer_roofline_ms(alg, bench.NOMINAL_PEAKS) - 3.0) < 1e-12
