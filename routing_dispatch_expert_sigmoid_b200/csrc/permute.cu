@@ -26,10 +26,12 @@ __device__ __forceinline__ uint4 ldg_nc(const uint4 *p) {
   return v;
 }
 
-// Work items are (row, 2 KB chunk of the row): a batch of a few rows still
-// spreads over the whole GPU, a large one keeps every warp on long streams.
-constexpr int kChunkVecs = 128;  // 16-byte vectors per chunk (4 per lane)
-
+// Work items are (row, chunk of 32 x VPL 16-byte vectors): a lane issues its
+// VPL loads before its stores, and the token index of the warp's next item
+// is loaded before the current item's rows, so each item costs about one
+// memory round trip.  4 KB chunks (VPL = 8), or 2 KB for small batches so
+// that their few rows still spread over the GPU.
+template <int VPL>
 __global__ void __launch_bounds__(256)
     k_dispatch(const uint4 *__restrict__ x, const int32_t *__restrict__ offsets,
                const int32_t *__restrict__ row_src, uint4 *__restrict__ x_perm, int E,
@@ -39,14 +41,17 @@ __global__ void __launch_bounds__(256)
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(err, kErrIndex);
     R = R < 0 ? 0 : rows_cap;
   }
+  constexpr int kChunkVecs = 32 * VPL;
   const int lane = threadIdx.x % 32;
   const int chunks = (row_vecs + kChunkVecs - 1) / kChunkVecs;
   const long long items = (long long)R * chunks;
   const long long warps = (long long)gridDim.x * (blockDim.x / 32);
-  for (long long it = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; it < items;
-       it += warps) {
+  long long it = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  int a_next = it < items ? row_src[it / chunks] : 0;
+  for (; it < items; it += warps) {
     const int row = (int)(it / chunks), ch = (int)(it % chunks);
-    const int a = row_src[row];
+    const int a = a_next;
+    if (it + warps < items) a_next = row_src[(it + warps) / chunks];
     const int t = a / k_max;
     if (a < 0 || t >= T) {
       if (lane == 0) raise_error(err, kErrIndex);
@@ -55,12 +60,12 @@ __global__ void __launch_bounds__(256)
     const uint4 *src = x + (size_t)t * row_vecs;
     uint4 *dst = x_perm + (size_t)row * row_vecs;
     const int v0 = ch * kChunkVecs + lane;
-    uint4 u[4];
+    uint4 u[VPL];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < VPL; ++i)
       if (v0 + 32 * i < row_vecs) u[i] = ldg_nc(src + v0 + 32 * i);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < VPL; ++i)
       if (v0 + 32 * i < row_vecs) dst[v0 + 32 * i] = u[i];
   }
 }
@@ -108,7 +113,9 @@ struct Vec<__nv_bfloat16> {
 // rows are T (row_vecs vectors of Vec<T>::N values).  Work items are (token,
 // 32 consecutive output vectors): lane l of the item's warp owns one output
 // vector and sums the token's kept slots for it in slot order.
-template <typename T>
+// KB: slots whose rows are loaded before they are summed (k_max rounded up
+// to 2, 4 or 8, so that top-2 layers keep their registers few).
+template <typename T, int KB>
 __global__ void __launch_bounds__(256)
     k_combine(const uint4 *__restrict__ y, const int32_t *__restrict__ slot_row,
               const float *__restrict__ topk_w, const uint4 *__restrict__ shared_y,
@@ -123,17 +130,28 @@ __global__ void __launch_bounds__(256)
   const long long items = (long long)Tn * chunks;
   const long long warps = (long long)gridDim.x * (blockDim.x / 32);
   const size_t in_vecs = (size_t)row_vecs * Q;  // fp32 vectors per row
-  for (long long it = (long long)blockIdx.x * (blockDim.x / 32) + wib; it < items; it += warps) {
+  // The token's slots of the warp's next item are loaded while the current
+  // item's rows are summed.
+  long long it = (long long)blockIdx.x * (blockDim.x / 32) + wib;
+  int next_row = -1;
+  float next_w = 0.f;
+  if (it < items && lane < k_max) {
+    const size_t at = (size_t)(it / chunks) * k_max + lane;
+    next_row = slot_row[at];
+    next_w = topk_w ? topk_w[at] : 1.0f;  // fmaf(1, y, acc) = y + acc
+  }
+  for (; it < items; it += warps) {
     const int t = (int)(it / chunks), ch = (int)(it % chunks);
-    int my_row = -1;
-    float my_w = 0.f;
-    if (lane < k_max) {
-      my_row = slot_row[(size_t)t * k_max + lane];
-      my_w = topk_w ? topk_w[(size_t)t * k_max + lane] : 1.0f;  // fmaf(1, y, acc) = y + acc
-      if (my_row >= rows_cap) {
-        raise_error(err, kErrIndex);
-        my_row = -1;
-      }
+    int my_row = next_row;
+    const float my_w = next_w;
+    if (it + warps < items && lane < k_max) {
+      const size_t at = (size_t)((it + warps) / chunks) * k_max + lane;
+      next_row = slot_row[at];
+      next_w = topk_w ? topk_w[at] : 1.0f;
+    }
+    if (my_row >= rows_cap) {
+      raise_error(err, kErrIndex);
+      my_row = -1;
     }
     const unsigned live = __ballot_sync(0xffffffffu, my_row >= 0);
     const int n_live = __popc(live);
@@ -164,17 +182,17 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int i = 0; i < N; ++i) acc[i] = 0.f;
       }
-      for (int j0 = 0; j0 < n_live; j0 += 4) {
-        uint4 u[4][Q];
+      for (int j0 = 0; j0 < n_live; j0 += KB) {
+        uint4 u[KB][Q];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)  // issue the loads before the FMAs
+        for (int j = 0; j < KB; ++j)  // issue the loads before the FMAs
           if (j0 + j < n_live) {
             const uint4 *src = y + (size_t)s_row[wib][j0 + j] * in_vecs + (size_t)v * Q;
 #pragma unroll
             for (int q = 0; q < Q; ++q) u[j][q] = ldg_nc(src + q);
           }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < KB; ++j) {
           if (j0 + j < n_live) {
             const float wj = s_w[wib][j0 + j];
             float f[N];
@@ -209,12 +227,47 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *o
   const int rows_cap = c.T * c.k_max;
   if (rows_cap == 0) return cudaSuccess;
   const int row_vecs = c.d * esz / 16;
-  const long long items = (long long)rows_cap * ((row_vecs + kChunkVecs - 1) / kChunkVecs);
-  k_dispatch<<<grid_for(items), 256, 0, s>>>(
-      static_cast<const uint4 *>(x), offsets, row_src, static_cast<uint4 *>(x_perm), c.E,
-      c.k_max, c.T, rows_cap, row_vecs, err);
+  const auto *xs = static_cast<const uint4 *>(x);
+  auto *xp = static_cast<uint4 *>(x_perm);
+  if ((long long)rows_cap * row_vecs * 16 <= (16ll << 20)) {  // at most 16 MB of rows
+    const long long items = (long long)rows_cap * ((row_vecs + 127) / 128);
+    k_dispatch<4><<<grid_for(items), 256, 0, s>>>(xs, offsets, row_src, xp, c.E, c.k_max, c.T,
+                                                  rows_cap, row_vecs, err);
+  } else {
+    const long long items = (long long)rows_cap * ((row_vecs + 255) / 256);
+    k_dispatch<8><<<grid_for(items), 256, 0, s>>>(xs, offsets, row_src, xp, c.E, c.k_max, c.T,
+                                                  rows_cap, row_vecs, err);
+  }
   return cudaGetLastError();
 }
+
+namespace {
+
+template <typename T, int KB>
+cudaError_t run_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
+                        const float *topk_w, const void *shared_y, void *out, uint32_t *err,
+                        cudaStream_t s, int shared_parts, int grid, int row_vecs) {
+  k_combine<T, KB><<<grid, 256, 0, s>>>(
+      static_cast<const uint4 *>(y_perm), slot_row, topk_w, static_cast<const uint4 *>(shared_y),
+      shared_parts, static_cast<uint4 *>(out), c.T, c.k_max, c.T * c.k_max, row_vecs, err);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t combine_k(const moe_config &c, const void *y_perm, const int32_t *slot_row,
+                      const float *topk_w, const void *shared_y, void *out, uint32_t *err,
+                      cudaStream_t s, int shared_parts, int grid, int row_vecs) {
+  if (c.k_max <= 2)
+    return run_combine<T, 2>(c, y_perm, slot_row, topk_w, shared_y, out, err, s, shared_parts,
+                             grid, row_vecs);
+  if (c.k_max <= 4)
+    return run_combine<T, 4>(c, y_perm, slot_row, topk_w, shared_y, out, err, s, shared_parts,
+                             grid, row_vecs);
+  return run_combine<T, 8>(c, y_perm, slot_row, topk_w, shared_y, out, err, s, shared_parts,
+                           grid, row_vecs);
+}
+
+}  // namespace
 
 cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                            const float *topk_w, const void *shared_y, void *out, uint32_t *err,
@@ -222,19 +275,12 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
   if (c.T == 0) return cudaSuccess;
   const int esz = c.dtype == MOE_F32 ? 4 : 2;
   const int row_vecs = c.d * esz / 16;
-  const int rows_cap = c.T * c.k_max;
   const int grid = grid_for((long long)c.T * ((row_vecs + 31) / 32));
   if (c.dtype == MOE_F32)
-    k_combine<float><<<grid, 256, 0, s>>>(
-        static_cast<const uint4 *>(y_perm), slot_row, topk_w,
-        static_cast<const uint4 *>(shared_y), shared_parts, static_cast<uint4 *>(out), c.T,
-        c.k_max, rows_cap, row_vecs, err);
-  else
-    k_combine<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        static_cast<const uint4 *>(y_perm), slot_row, topk_w,
-        static_cast<const uint4 *>(shared_y), shared_parts, static_cast<uint4 *>(out), c.T,
-        c.k_max, rows_cap, row_vecs, err);
-  return cudaGetLastError();
+    return combine_k<float>(c, y_perm, slot_row, topk_w, shared_y, out, err, s, shared_parts,
+                            grid, row_vecs);
+  return combine_k<__nv_bfloat16>(c, y_perm, slot_row, topk_w, shared_y, out, err, s,
+                                  shared_parts, grid, row_vecs);
 }
 
 }  // namespace moe
