@@ -118,38 +118,62 @@ __device__ __forceinline__ void gate_token(const GatingArgs &g, int t, const flo
   }
 
   if (g.mode == MOE_SIGMOID_GROUPED) {
-    // Group scores: lane g sums, in descending order, the group_score_topk
-    // largest biased scores of group g; then keep the topk_groups best groups.
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E) s_u[e] = key[i];
-    }
-    __syncwarp();
     const int gsz = E / g.n_groups, m = g.group_score_topk;
-    uint32_t gu = 0;  // this lane's group score, ordered (0: no group)
-    if (lane < g.n_groups) {
-      float top[8];
+    uint32_t gu = 0;  // lane g: group g's score, ordered (0: no group)
+    if (gsz == 32) {
+      // Group gi is register gi across the 32 lanes (experts 32*gi + lane):
+      // its m largest biased scores come out of m rounds of warp reductions,
+      // largest first, equal scores in lane (expert) order, and are added in
+      // that order.
 #pragma unroll
-      for (int q = 0; q < 8; ++q) top[q] = -INFINITY;
-      for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) {
-        float v = s_u[e];
-        // insert v into the descending list top[0..m-1]
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (q < m && v > top[q]) {
-            const float tmp = top[q];
-            top[q] = v;
-            v = tmp;
+      for (int gi = 0; gi < NPL; ++gi) {
+        if (gi < g.n_groups) {
+          uint32_t taken = 0;
+          float sc = 0.f;
+          for (int j = 0; j < m; ++j) {
+            const uint32_t u = ((taken >> lane) & 1u) ? 0u : ku[gi];
+            const uint32_t top = __reduce_max_sync(kFull, u);
+            const int w = __reduce_min_sync(kFull, u == top ? lane : 32);
+            taken |= 1u << w;
+            const float v = __shfl_sync(kFull, key[gi], w);
+            sc = j == 0 ? v : __fadd_rn(sc, v);
           }
+          if (lane == gi) gu = order_key(sc);
         }
       }
-      float sc = top[0];
+    } else {
+      // Lane g sums, in descending order, the group_score_topk largest
+      // biased scores of group g (from a copy of the scores in shared memory).
 #pragma unroll
-      for (int q = 1; q < 8; ++q)
-        if (q < m) sc = __fadd_rn(sc, top[q]);
-      gu = order_key(sc);
+      for (int i = 0; i < NPL; ++i) {
+        const int e = i * 32 + lane;
+        if (e < E) s_u[e] = key[i];
+      }
+      __syncwarp();
+      if (lane < g.n_groups) {
+        float top[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) top[q] = -INFINITY;
+        for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) {
+          float v = s_u[e];
+          // insert v into the descending list top[0..m-1]
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (q < m && v > top[q]) {
+              const float tmp = top[q];
+              top[q] = v;
+              v = tmp;
+            }
+          }
+        }
+        float sc = top[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (q < m) sc = __fadd_rn(sc, top[q]);
+        gu = order_key(sc);
+      }
     }
+    // then keep the topk_groups best groups
     uint32_t kept_groups = 0;
     for (int r = 0; r < g.topk_groups; ++r) {
       const int win = warp_best(gu, lane);

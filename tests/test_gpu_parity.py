@@ -264,12 +264,14 @@ def test_small_batch_layer(name, dev):
     _layer_vs_oracle(w, _host_inputs(w, seed=4), dev)
 
 
+@pytest.mark.parametrize("E", [64, 256])
 @pytest.mark.parametrize("T", [512, 128])
-def test_sigmoid_grouped_near_ties_bit_exact(T, dev):
+def test_sigmoid_grouped_near_ties_bit_exact(T, E, dev):
     """Logits on a fine grid with many exact and one-ulp ties in the biased
     scores: selection must follow the specified sigmoid bit for bit (T = 128
-    goes through the fused small-batch routing kernel)."""
-    w = SMALL["dsv3_small"].scaled(T=T)
+    goes through the fused small-batch routing kernel; E = 256 makes groups
+    of 32 experts, whose scores the warp computes by reductions)."""
+    w = SMALL["dsv3_small"].scaled(T=T, E=E)
     hin = _host_inputs(w)
     cfg = ops.config(w)
     g = torch.Generator().manual_seed(5)
