@@ -248,3 +248,44 @@ def test_fp8_widening_bit_formula_gives_every_code():
         val = np.where(sign == 1, -val, val)
         assert (val == ref).all(), pos
         assert (np.signbit(val) == np.signbit(ref)).all(), pos
+
+
+def _shared_split_bytes(w):
+    """The decode-sized shared-expert split's scratch, from its rule: T <= 256
+    (at most two 128-row tiles), d and f_shared multiples of 64, 256-column
+    tiles, splits dividing the 64-deep K steps within one wave of 148 CTAs
+    (at most 16); used when the up projection splits at least twice."""
+    if w.f_shared <= 0 or w.dtype != "bf16":
+        return 0
+    rt = (w.T + 127) // 128
+    if rt > 2 or w.d % 64 or w.f_shared % 64:
+        return 0
+
+    def splits(kb, tiles):
+        return max(s for s in range(1, min(16, kb) + 1) if kb % s == 0 and s * tiles <= 148)
+
+    s_up = splits(w.d // 64, rt * ((w.f_shared + 255) // 256))
+    s_dn = splits(w.f_shared // 64, rt * ((w.d + 255) // 256))
+    if s_up < 2:
+        return 0
+    b = 2 * s_up * w.T * w.f_shared * 4 + (s_dn * w.T * w.d * 4 if s_dn > 1 else 0)
+    return (b + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("w", [
+    WORKLOADS["dsv3_decode"],                                            # 16 up, 4 down splits
+    WORKLOADS["dsv3_decode"].scaled(T=200, d=448, f=64, f_shared=256),   # two row tiles
+    WORKLOADS["dsv3_decode"].scaled(T=300),                              # three tiles: unsplit
+    WORKLOADS["dsv3_decode"].scaled(f_shared=2040),                      # not in 64-steps
+    WORKLOADS["dsv3_prefill"],                                           # prefill: unsplit
+], ids=["dsv3_decode", "t200", "t300", "fsh2040", "prefill"])
+def test_shared_split_workspace_follows_its_rule(w, monkeypatch):
+    """The layer workspace holds the shared expert's split-K partial sums
+    exactly when the split rule (mirrored by bench.py's launch count) applies."""
+    cfg = ops.config(w)
+    with_split = ops.moe_workspace_size(cfg, ops.WS_LAYER)
+    monkeypatch.setenv("MOE_SHARED_SPLIT", "0")
+    without = ops.moe_workspace_size(cfg, ops.WS_LAYER)
+    assert with_split - without == _shared_split_bytes(w)
+    import bench
+    assert bench.shared_split_k(w) == (_shared_split_bytes(w) > 0)
