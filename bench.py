@@ -18,11 +18,16 @@ Extra keys of the JSON line:
   layer_roofline_frac_nominal  the same against nominal B200 peaks (8 TB/s,
                                2.25 PFLOP/s dense bf16);
   roofline     the up-projection + SwiGLU grouped GEMM (the dominant kernel):
-               algorithmic FLOPs (prefill) or bytes (decode) per launch over its
-               mean launch time, from CUDA events recorded on the launching
-               stream at its boundaries inside the timed steps; the bf16 peak
-               is the measured sustained figure when the power cap was active
-               during the timed region, the burst figure otherwise;
+               algorithmic FLOPs or bytes per launch (work_per_launch) over its
+               mean launch time (ms_per_launch), from CUDA events recorded on the
+               launching stream at its boundaries inside the timed steps; bound
+               by whichever of its FLOPs at the measured burst bf16 peak or its
+               bytes at the measured copy bandwidth takes longer (the same peaks
+               as layer_roofline_frac).  Compute-bound kernels also carry
+               frac_at_sampled_clock: achieved over the peak scaled by the
+               median sampled SM clock over the maximum clock;
+  kernels      the same for the dispatch (K4), up projection (K5), down
+               projection (K6) and combine (K7) stages;
   e2e          the same metric through the C ABI with host buffers: per step a
                pinned-host -> device copy of x and a device -> pinned-host copy
                of the layer output are inside the timed region, double-buffered
@@ -34,7 +39,11 @@ Extra keys of the JSON line:
   clocks       nvidia-smi samples taken during the timed region;
   decode       the same layer at decode size (T=64), same keys;
   fp8_weights  the decode-size layer with e4m3 expert weights and per-column
-               scales (quantised before timing), same keys.
+               scales (quantised before timing), same keys;
+  configs      every other workload of the layer definition (tiny fp32,
+               Qwen3-, DeepSeek-V3- (decode and prefill) and GPT-OSS-shaped
+               layers), same keys, each timed on its own inputs after the
+               previous one's memory was freed.
 `--impl reference` times the CPU oracle alone on the same workload (the
 reference arm: there is no other implementation of this layer to run).
 """
@@ -42,6 +51,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import gc
 import hashlib
 import io
 import json
@@ -75,6 +85,7 @@ def layer_roofline_ms(alg: dict, peaks: dict) -> float:
 PROFILES = os.path.join(ROOT, "profiles")
 GEMM_SRC = os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc",
                         "grouped_gemm_sm100.cu")
+PERMUTE_SRC = os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc", "permute.cu")
 METRIC = "MoE-layer tokens/sec on 1 B200 (decode & prefill); % of roofline"
 PREFILL, DECODE = "mixtral_prefill", "mixtral_decode"
 L2_BYTES = 126 * 2 ** 20
@@ -236,28 +247,39 @@ def launches_per_layer(w) -> int:
 
 
 def algorithmic(w, R: int, touched: int, fp8: bool = False) -> dict:
-    """Algorithmic work of the layer and of the up-projection grouped GEMM.
-    With fp8 expert weights each weight is one byte plus its column's fp32
-    scale; the router stays in the layer dtype."""
+    """Algorithmic work of the layer and of its stages.  With fp8 expert
+    weights each weight is one byte plus its column's fp32 scale; the router
+    stays in the layer dtype.  Stage bytes count each tensor a stage must read
+    or write once: K4 reads and writes the R dispatched rows, K5 reads the
+    touched experts' W1 and W3 and the R rows and writes h, K6 reads W2 and h
+    and writes the fp32 expert outputs, K7 -- in the measurement's definition
+    -- reads R expert rows and writes T output rows in the layer dtype."""
     s = w.elem_bytes
     ws = 1 if fp8 else s                              # bytes per expert weight
     sc = 4 if fp8 else 0                              # bytes per column scale
+    hs = s                                            # h: bf16 (or fp32 for fp32 layers)
     return {
         "layer_flops": 2 * w.T * w.d * w.E + 6 * w.d * w.f * R + 6 * w.d * w.f_shared * w.T,
         "layer_bytes": (touched * (3 * w.d * w.f * ws + (2 * w.f + w.d) * sc)
                         + 3 * w.d * w.f_shared * ws + (2 * w.f_shared + w.d) * sc * (w.f_shared > 0)
                         + w.d * w.E * s + 2 * w.T * w.d * s),
-        # K5: gate and up GEMMs over the R kept rows; reads the touched experts'
-        # W1 and W3 and the R dispatched rows, writes h
         "up_flops": 4 * R * w.d * w.f,
-        "up_bytes": touched * 2 * (w.d * w.f * ws + w.f * sc) + R * w.d * s + R * w.f * s,
+        "up_bytes": touched * 2 * (w.d * w.f * ws + w.f * sc) + R * w.d * s + R * w.f * hs,
+        "down_flops": 2 * R * w.f * w.d,
+        "down_bytes": touched * (w.f * w.d * ws + w.d * sc) + R * w.f * hs + R * w.d * 4,
+        "dispatch_bytes": 2 * R * w.d * s,
+        "combine_bytes": (R + w.T) * w.d * s,
+        # what the combine actually moves: fp32 expert rows (y_perm is kept in
+        # fp32 so that the output is rounded once), the output rows, the fp32
+        # shared-expert rows, and each slot's row index and weight
+        "combine_bytes_actual": (R * w.d * 4 + w.T * w.d * s + (w.f_shared > 0) * w.T * w.d * 4
+                                 + w.T * w.k_max * 8),
     }
 
 
-def traffic_from_profile(workload: str):
-    """DRAM bytes per launch of K5 from the committed ncu summary, when that
-    summary was taken on the current source of the kernel; else None."""
-    path = os.path.join(PROFILES, f"k5_up_swiglu_{workload}.md")
+def profile_summary(path: str, src: str):
+    """DRAM bytes per launch from a committed ncu summary, when that summary
+    was taken on the current source of the kernel; else None."""
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -265,8 +287,80 @@ def traffic_from_profile(workload: str):
     m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
     if not (m_hash and m_bytes):
         return None
-    cur = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
+    cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
     return float(m_bytes.group(1)) if cur == m_hash.group(1) else None
+
+
+def traffic_from_profile(workload: str, kernel: str = "k5_up_swiglu"):
+    """DRAM bytes per launch of a stage's kernel from profiles/<kernel>_<workload>.md."""
+    src = PERMUTE_SRC if kernel.startswith(("k4", "k7")) else GEMM_SRC
+    return profile_summary(os.path.join(PROFILES, f"{kernel}_{workload}.md"), src)
+
+
+def alu_peak_tflops(sms: int, sm_max_mhz: float) -> float:
+    """fp32 FMA peak of the CUDA cores: SMs x 128 fp32 lanes x 2 flops x clock."""
+    return sms * 128 * 2 * sm_max_mhz * 1e6 / 1e12
+
+
+def roofline_obj(kind: str, achieved: float, peak: float, unit: str, traffic, peak_src: str,
+                 work: float, ms: float, clocks: dict | None = None) -> dict:
+    o = {"bound": kind, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+         "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
+         "work_per_launch": work, "ms_per_launch": round(ms, 5)}
+    # the tensor and ALU peaks scale with the SM clock; HBM bandwidth does not
+    if kind in ("tensor", "alu") and clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
+        o["sm_mhz"] = clocks["sm_mhz"]
+        o["frac_at_sampled_clock"] = round(
+            achieved / (peak * clocks["sm_mhz"] / clocks["sm_max_mhz"]), 4)
+    return o
+
+
+def kernel_roofline(flops: float, nbytes: float, ms: float, pk: dict, pk_src: str, traffic=None,
+                    clocks: dict | None = None, alu_peak: float | None = None) -> dict:
+    """Roofline of one kernel from its algorithmic work and its mean launch
+    time: bound by whichever of its FLOPs at the compute peak (bf16 tensor
+    cores, measured burst figure; or, for fp32 CUDA-core work, the ALU peak)
+    or its bytes at the measured copy bandwidth takes longer."""
+    peak_tf = alu_peak if alu_peak else pk["bf16_tflops"]
+    t_flops = flops / (peak_tf * 1e12)
+    t_bytes = nbytes / (pk["hbm_gbs"] * 1e9)
+    if flops and t_flops >= t_bytes:
+        kind = "alu" if alu_peak else "tensor"
+        src = ("fp32 FMA peak: SMs x 128 lanes x 2 x max SM clock" if alu_peak
+               else f"{pk_src} bf16 burst (cuBLAS)")
+        return roofline_obj(kind, flops / (ms * 1e-3) / 1e12, round(peak_tf, 1), "TFLOP/s",
+                            traffic, src, flops, ms, clocks)
+    return roofline_obj("hbm", nbytes / (ms * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", traffic,
+                        f"{pk_src} copy bandwidth", nbytes, ms, clocks)
+
+
+def stage_rooflines(w, alg: dict, stage_ms: dict, pk: dict, pk_src: str, clocks: dict,
+                    workload: str, alu_peak: float, profiled: bool = True) -> dict:
+    """Roofline objects of the dispatch (K4), up projection (K5), down
+    projection (K6) and combine (K7) stages, from their event-timed means."""
+    tr = (lambda k: traffic_from_profile(workload, k)) if profiled else (lambda k: None)
+    out = {}
+    if w.dtype == "f32":  # one fp32 CUDA-core FFN kernel runs both projections
+        out["up_swiglu"] = kernel_roofline(
+            alg["up_flops"] + alg["down_flops"], alg["up_bytes"] + alg["down_bytes"],
+            stage_ms["up_swiglu"], pk, pk_src, None, clocks, alu_peak)
+    else:
+        out["up_swiglu"] = kernel_roofline(alg["up_flops"], alg["up_bytes"], stage_ms["up_swiglu"],
+                                           pk, pk_src, tr("k5_up_swiglu"), clocks)
+        out["down"] = kernel_roofline(alg["down_flops"], alg["down_bytes"], stage_ms["down"], pk,
+                                      pk_src, tr("k6_down"), clocks)
+    out["dispatch"] = kernel_roofline(0, alg["dispatch_bytes"], stage_ms["dispatch"], pk, pk_src,
+                                      tr("k4_dispatch"), clocks)
+    comb = kernel_roofline(0, alg["combine_bytes"], stage_ms["combine"], pk, pk_src,
+                           tr("k7_combine"), clocks)
+    act = alg["combine_bytes_actual"] / (stage_ms["combine"] * 1e-3) / 1e9
+    comb["actual_bytes_per_launch"] = alg["combine_bytes_actual"]
+    comb["frac_on_actual_bytes"] = round(act / pk["hbm_gbs"], 4)
+    comb["note"] = ("bytes per the layer definition, (R+T) rows in the layer dtype; the kernel "
+                    "reads fp32 expert rows (the output is rounded once), so its actual "
+                    "traffic is larger: frac_on_actual_bytes")
+    out["combine"] = comb
+    return out
 
 
 class Layer:
@@ -416,24 +510,6 @@ def run_e2e(layer: Layer, steps: int, warmup: int, dist) -> dict:
             "d2h": out_host[0].numel() * out_host[0].element_size()}
 
 
-def kernel_roofline(alg: dict, ms: float, peak_tf: float, peak_gbs: float, traffic, tf_src: str,
-                    bw_src: str) -> dict:
-    """Roofline of K5: bound by whichever of its algorithmic FLOPs at the bf16
-    peak or its algorithmic bytes at the HBM peak takes longer."""
-    t_flops = alg["up_flops"] / (peak_tf * 1e12)
-    t_bytes = alg["up_bytes"] / (peak_gbs * 1e9)
-    if t_flops >= t_bytes:
-        return roofline_obj("tensor", alg["up_flops"] / (ms * 1e-3) / 1e12, peak_tf, "TFLOP/s",
-                            traffic, tf_src)
-    return roofline_obj("hbm", alg["up_bytes"] / (ms * 1e-3) / 1e9, peak_gbs, "GB/s", traffic,
-                        bw_src)
-
-
-def roofline_obj(kind: str, achieved: float, peak: float, unit: str, traffic, peak_src: str):
-    return {"bound": kind, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-            "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src}
-
-
 # ---------------------------------------------------------------------------
 # the CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------
@@ -476,6 +552,64 @@ def cpu_sample_tokens(name: str, budget_s: float) -> int:
 
 
 # ---------------------------------------------------------------------------
+# one measured leg: a workload, timed, with its rooflines
+# ---------------------------------------------------------------------------
+# The workloads of the layer definition besides the Mixtral-shaped legs, each
+# measured by the default run and reported under "configs".
+OTHER_CONFIGS = ("tiny_f32", "qwen3_prefill", "dsv3_decode", "dsv3_prefill", "gptoss_sub")
+
+
+def describe(w) -> str:
+    return (f"{w.name}: T={w.T}, d={w.d}, E={w.E}, top-{w.k_max}"
+            + (f" (k_t in {w.k_min}..{w.k_max})" if w.k_min else "") + f", f={w.f}"
+            + (f", shared f={w.f_shared}" if w.f_shared else "")
+            + f", {w.gating}, capacity factor {w.capacity_factor or 'none'}, {w.dtype}")
+
+
+def measure_leg(name: str, steps: int, warmup: int, dist, local_rank: int, dev, pk: dict,
+                pk_src: str, sms: int, T: int = 0, fp8: bool = False, e2e: bool = False,
+                profiled: bool = True) -> tuple[dict, dict]:
+    """Time one workload; returns (the leg's JSON object, raw numbers)."""
+    layer = Layer(name, dev, seed=int(os.environ.get("RANK", "0")), T=T, fp8=fp8)
+    w = layer.w
+    r = run_device(layer, steps, warmup, dist, local_rank)
+    e2e_r = run_e2e(layer, steps, warmup, dist) if e2e else None
+    ms_max, tokens = aggregate(r["ms"], w.T * steps, dist)
+    alg = algorithmic(w, r["R"], r["touched"], fp8=fp8)
+    clocks = r["clocks"]
+    alu = alu_peak_tflops(sms, clocks.get("sm_max_mhz") or 1965.0)
+    kern = stage_rooflines(w, alg, r["stage_ms"], pk, pk_src, clocks,
+                           w.name + ("_fp8" if fp8 else ""), alu, profiled and T <= 0)
+    roof_ms = layer_roofline_ms(alg, pk)
+    step_ms = ms_max / steps
+    obj = {
+        "workload": describe(w) + (", e4m3 expert weights with per-column fp32 scales"
+                                   if fp8 else ""),
+        "steps": steps, "value": round(tokens / (ms_max * 1e-3), 1), "unit": "tokens/s",
+        "ms_per_step": round(step_ms, 4),
+        "stage_ms": {k: round(v, 4) for k, v in r["stage_ms"].items()},
+        "layer_roofline_ms": round(roof_ms, 4),
+        "layer_roofline_frac": round(roof_ms / step_ms, 4),
+        "layer_roofline_frac_nominal": round(layer_roofline_ms(alg, NOMINAL_PEAKS) / step_ms, 4),
+        # the dominant kernel: the up projection with SwiGLU (K5)
+        "roofline": kern["up_swiglu"],
+        "kernels": kern,
+        "kept_rows": r["R"], "experts_touched": r["touched"],
+        "load_max_over_mean": round(r["load_max_over_mean"], 3), "n_dropped": r["n_dropped"],
+        "gpu_launches": launches_per_layer(w) * steps * (3 if e2e else 1),
+        "clocks": clocks,
+    }
+    raw = {"w": w, "ms_max": ms_max, "tokens": tokens, "e2e": e2e_r}
+    if e2e_r is not None:
+        raw["e2e_ms"] = aggregate(e2e_r["ms"], w.T * steps, dist)[0]
+        raw["e2e_serial_ms"] = aggregate(e2e_r["ms_serial"], w.T * steps, dist)[0]
+    del layer
+    gc.collect()
+    torch.cuda.empty_cache()
+    return obj, raw
+
+
+# ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -492,6 +626,8 @@ def main():
                     choices=sorted(WORKLOADS) + ["none"], help="workload of the decode leg")
     ap.add_argument("--fp8-workload", default=DECODE, choices=sorted(WORKLOADS) + ["none"],
                     help="workload of the leg with fp8 expert weights")
+    ap.add_argument("--configs", default=",".join(OTHER_CONFIGS),
+                    help="comma-separated further workloads to measure ('none': no others)")
     a = ap.parse_args()
     rank, local_rank, world = dist_env()
     warmup = max(a.warmup, 3)
@@ -526,87 +662,22 @@ def main():
     dev = torch.device("cuda", local_rank)
     dist = init_dist(world, "nccl")
     pk, pk_src = peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    leg = dict(dist=dist, local_rank=local_rank, dev=dev, pk=pk, pk_src=pk_src, sms=sms)
 
-    pre = Layer(a.workload, dev, seed=rank, T=a.T)
-    rp = run_device(pre, a.steps, warmup, dist, local_rank)
-    e2e = None if a.no_e2e else run_e2e(pre, a.steps, warmup, dist)
-    w = pre.w
-    ms_max, tokens = aggregate(rp["ms"], w.T * a.steps, dist)
-    e2e_ms = None if e2e is None else aggregate(e2e["ms"], w.T * a.steps, dist)[0]
-    e2e_serial_ms = None if e2e is None else aggregate(e2e["ms_serial"], w.T * a.steps, dist)[0]
-    alg = algorithmic(w, rp["R"], rp["touched"])
-    up_ms = rp["stage_ms"]["up_swiglu"]
-    # The sustained bf16 figure applies when the timed region ran under the
-    # power cap (or for more than a second); the burst figure otherwise.
-    sustained = rp["ms"] > 1000.0 or "sw_power_cap" in rp["clocks"]["reasons"]
-    peak_tf = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
-    roof_pre = kernel_roofline(alg, up_ms, peak_tf, pk["hbm_gbs"],
-                               traffic_from_profile(a.workload) if a.T <= 0 else None,
-                               f"{pk_src} bf16 {'sustained' if sustained else 'burst'}",
-                               f"{pk_src} copy bandwidth")
-    layer_roof_ms = layer_roofline_ms(alg, pk)
-    del pre
-    torch.cuda.empty_cache()
-
+    main_obj, main_raw = measure_leg(a.workload, a.steps, warmup, T=a.T, e2e=not a.no_e2e, **leg)
+    w = main_raw["w"]
     dec_obj = None
     if a.decode_workload != "none":
-        dec = Layer(a.decode_workload, dev, seed=rank)
-        dsteps = max(a.steps, 50)
-        rd = run_device(dec, dsteps, warmup, dist, local_rank)
-        wd = dec.w
-        d_ms_max, d_tokens = aggregate(rd["ms"], wd.T * dsteps, dist)
-        algd = algorithmic(wd, rd["R"], rd["touched"])
-        d_up_ms = rd["stage_ms"]["up_swiglu"]
-        sustained_d = "sw_power_cap" in rd["clocks"]["reasons"]
-        roof_dec = kernel_roofline(
-            algd, d_up_ms, pk["bf16_tflops_sustained"] if sustained_d else pk["bf16_tflops"],
-            pk["hbm_gbs"], traffic_from_profile(a.decode_workload),
-            f"{pk_src} bf16 {'sustained' if sustained_d else 'burst'}", f"{pk_src} copy bandwidth")
-        d_layer_roof_ms = layer_roofline_ms(algd, pk)
-        dec_obj = {
-            "workload": f"{a.decode_workload}: T={wd.T}, d={wd.d}, E={wd.E}, top-{wd.k_max}, "
-                        f"f={wd.f}", "steps": dsteps,
-            "value": round(d_tokens / (d_ms_max * 1e-3), 1), "unit": "tokens/s",
-            "ms_per_step": round(d_ms_max / dsteps, 4),
-            "stage_ms": {k: round(v, 4) for k, v in rd["stage_ms"].items()},
-            "layer_roofline_ms": round(d_layer_roof_ms, 4),
-            "layer_roofline_frac": round(d_layer_roof_ms / (d_ms_max / dsteps), 4),
-            "layer_roofline_frac_nominal": round(
-                layer_roofline_ms(algd, NOMINAL_PEAKS) / (d_ms_max / dsteps), 4),
-            "roofline": roof_dec, "kept_rows": rd["R"], "experts_touched": rd["touched"],
-            "gpu_launches": launches_per_layer(wd) * dsteps,
-        }
-        del dec
-        torch.cuda.empty_cache()
-
+        dec_obj, _ = measure_leg(a.decode_workload, max(a.steps, 50), warmup, **leg)
     fp8_obj = None
     if a.fp8_workload != "none":
-        q = Layer(a.fp8_workload, dev, seed=rank, fp8=True)
-        qsteps = max(a.steps, 50)
-        rq = run_device(q, qsteps, warmup, dist, local_rank)
-        wq = q.w
-        q_ms_max, q_tokens = aggregate(rq["ms"], wq.T * qsteps, dist)
-        algq = algorithmic(wq, rq["R"], rq["touched"], fp8=True)
-        sustained_q = "sw_power_cap" in rq["clocks"]["reasons"]
-        roof_q = kernel_roofline(
-            algq, rq["stage_ms"]["up_swiglu"],
-            pk["bf16_tflops_sustained"] if sustained_q else pk["bf16_tflops"], pk["hbm_gbs"],
-            None, f"{pk_src} bf16 {'sustained' if sustained_q else 'burst'}",
-            f"{pk_src} copy bandwidth")
-        q_layer_roof_ms = layer_roofline_ms(algq, pk)
-        fp8_obj = {
-            "workload": f"{a.fp8_workload} with e4m3 expert weights (per-column fp32 scales)",
-            "steps": qsteps, "value": round(q_tokens / (q_ms_max * 1e-3), 1),
-            "unit": "tokens/s", "ms_per_step": round(q_ms_max / qsteps, 4),
-            "stage_ms": {k: round(v, 4) for k, v in rq["stage_ms"].items()},
-            "layer_roofline_ms": round(q_layer_roof_ms, 4),
-            "layer_roofline_frac": round(q_layer_roof_ms / (q_ms_max / qsteps), 4),
-            "layer_roofline_frac_nominal": round(
-                layer_roofline_ms(algq, NOMINAL_PEAKS) / (q_ms_max / qsteps), 4),
-            "roofline": roof_q, "gpu_launches": launches_per_layer(wq) * qsteps,
-        }
-        del q
-        torch.cuda.empty_cache()
+        fp8_obj, _ = measure_leg(a.fp8_workload, max(a.steps, 50), warmup, fp8=True, **leg)
+    configs = {}
+    for name in [c for c in a.configs.split(",") if c and c != "none"]:
+        wc = WORKLOADS[name]
+        steps = max(a.steps, 50) if wc.T <= 256 else a.steps
+        configs[name], _ = measure_leg(name, steps, warmup, **leg)
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -618,40 +689,41 @@ def main():
                          f"({r['times'][0]:.1f} s)"}
 
     if rank == 0:
-        value = tokens / (ms_max * 1e-3)
+        ms_max, tokens = main_raw["ms_max"], main_raw["tokens"]
+        e2e = main_raw["e2e"]
         line = {
-            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-            "steps": a.steps, "warmup": warmup, "ms_per_step": round(ms_max / a.steps, 4),
+            "metric": METRIC, "value": round(tokens / (ms_max * 1e-3), 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": a.steps, "warmup": warmup,
+            "ms_per_step": round(ms_max / a.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded normal inputs and weights of the stated shapes)",
             "config": {
-                "workload": f"{a.workload}: T={w.T}, d={w.d}, E={w.E}, top-{w.k_max}, f={w.f}"
-                            + (f", shared f={w.f_shared}" if w.f_shared else "")
-                            + f", {w.gating}, capacity factor {w.capacity_factor or 'none'}",
+                "workload": describe(w),
                 "global_batch_tokens": w.T * world, "parallelism": f"replicas x{world}",
                 "l2": "inputs larger than L2 (expert weights > 126 MB L2); no flush",
-                "kept_rows": rp["R"], "experts_touched": rp["touched"],
-                "load_max_over_mean": round(rp["load_max_over_mean"], 3),
-                "n_dropped": rp["n_dropped"],
+                "kept_rows": main_obj["kept_rows"], "experts_touched": main_obj["experts_touched"],
+                "load_max_over_mean": main_obj["load_max_over_mean"],
+                "n_dropped": main_obj["n_dropped"],
             },
-            "stage_ms": {k: round(v, 4) for k, v in rp["stage_ms"].items()},
-            "layer_roofline_ms": round(layer_roof_ms, 4),
-            "layer_roofline_frac": round(layer_roof_ms / (ms_max / a.steps), 4),
-            "layer_roofline_frac_nominal": round(
-                layer_roofline_ms(alg, NOMINAL_PEAKS) / (ms_max / a.steps), 4),
-            "roofline": roof_pre,
+            "stage_ms": main_obj["stage_ms"],
+            "layer_roofline_ms": main_obj["layer_roofline_ms"],
+            "layer_roofline_frac": main_obj["layer_roofline_frac"],
+            "layer_roofline_frac_nominal": main_obj["layer_roofline_frac_nominal"],
+            "roofline": main_obj["roofline"],
+            "kernels": main_obj["kernels"],
             "decode": dec_obj,
             "fp8_weights": fp8_obj,
+            "configs": configs,
             "e2e": None if e2e is None else {
-                "value": round(tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "value": round(tokens / (main_raw["e2e_ms"] * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "copies": "pinned host buffers; each step's input and output copies run on two "
                           "copy streams, overlapping the neighbouring steps' layers",
-                "serial_value": round(tokens / (e2e_serial_ms * 1e-3), 1)},
-            "gpu_launches": (launches_per_layer(w) * a.steps * (1 if e2e is None else 3)
-                             + (dec_obj["gpu_launches"] if dec_obj else 0)
-                             + (fp8_obj["gpu_launches"] if fp8_obj else 0)),
-            "clocks": rp["clocks"],
+                "serial_value": round(tokens / (main_raw["e2e_serial_ms"] * 1e-3), 1)},
+            "gpu_launches": (main_obj["gpu_launches"]
+                             + sum(o["gpu_launches"] for o in (dec_obj, fp8_obj) if o)
+                             + sum(o["gpu_launches"] for o in configs.values())),
+            "clocks": main_obj["clocks"],
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -55,6 +55,12 @@
  *   - Rows: x_perm and y_perm hold at most T*k_max rows (an upper bound known on
  *     the host); the number actually kept, R = offsets[E], stays on the device
  *     and the kernels read it there, so no call needs a device-to-host copy.
+ *   - Per-device state: on its first call on a device the library looks up
+ *     the device addresses of its error word and static scratch and raises
+ *     its kernels' shared-memory limits, and keeps them for the life of the
+ *     process (host threads may make those first calls concurrently).
+ *     cudaDeviceReset destroys this state together with the device's context:
+ *     make no further calls on a device after resetting it.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -289,9 +295,18 @@ MOE_API moe_status moe_layer_fp8(const moe_config *cfg, const void *x, const voi
 
 /* Synchronises `stream`, then reads and clears the device error flags of the
  * current device.  *flags (may be NULL) receives them: bit 0 an index out of
- * range in a gather/scatter, bit 1 a pipeline wait that hit its iteration
- * limit, bit 2 an expert index or k_t out of range.  Returns
- * MOE_ERR_DEVICE_CHECK when any flag was set. */
+ * range in a gather/scatter, bit 1 a pipeline wait that hit its time limit,
+ * bit 2 an expert index or k_t out of range.  Returns MOE_ERR_DEVICE_CHECK
+ * when any flag was set.
+ * Time limit: every wait of the tensor-core GEMMs' pipelines (on data landing
+ * in shared memory, on a free accumulator, ...) gives up after 4 s; the CTA
+ * then sets bit 1, stops its other roles, lets the copies and MMAs it already
+ * issued complete, frees its tensor memory and returns, so a stalled pipeline
+ * ends the kernel instead of hanging the GPU.  The results of that call are
+ * then undefined.  The environment variable MOE_WAIT_LIMIT_NS, read at every
+ * launch, lowers the limit of the single-CTA and swap-AB engines (nanoseconds,
+ * at most 4e9) -- a diagnostic that makes the waits run out on purpose; the
+ * CTA-pair engine always keeps 4 s. */
 MOE_API moe_status moe_check_errors(void *stream, uint32_t *flags);
 
 /* Static description of a status code. */

@@ -55,6 +55,8 @@
 #include <cuda.h>
 #include <stdlib.h>
 
+#include <atomic>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -102,6 +104,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 struct Ctl {
   volatile int *abort;
   uint32_t *err;
+  uint64_t limit_ns;  // how long one pipeline wait may take before the CTA stops
 };
 
 // Wait until the phase of parity `parity` of barrier `bar` has completed.
@@ -112,7 +115,7 @@ __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const Ctl &c
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*c.abort) return false;
-    if (global_timer() - t0 > kWaitLimitNs) {
+    if (global_timer() - t0 > c.limit_ns) {
       *c.abort = 1;
       raise_error(c.err, kErrWait);
       return false;
@@ -120,7 +123,9 @@ __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const Ctl &c
   }
 }
 
-// Wait without honouring the stop flag (used to drain work in flight).
+// Wait without honouring the stop flag (used to drain work in flight); always
+// the long limit, so that every copy and MMA already issued lands before the
+// CTA frees its tensor memory and exits.
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint32_t *err) {
   const uint64_t t0 = global_timer();
   while (!mbar_try_wait(bar, parity)) {
@@ -313,6 +318,8 @@ struct Params {
   // of the slot the row serves), or nothing when row_w is nullptr
   const float *row_w = nullptr;
   const int32_t *w_row_src = nullptr;
+  // Limit of one pipeline wait (the single-CTA and swap-AB engines)
+  uint64_t wait_limit_ns = kWaitLimitNs;
 };
 
 // Gate weights to apply in the down projection's epilogue (both nullptr: none).
@@ -520,7 +527,7 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
   const uint32_t conv0 = smem_addr(bars + 2 * S::kStages + 5);
   const uint32_t qfull0 = smem_addr(bars + 3 * S::kStages + 5);
   const uint32_t qempty0 = smem_addr(bars + 3 * S::kStages + 5 + S::kQStages);
-  const Ctl ctl{abort_flag, p.err};
+  const Ctl ctl{abort_flag, p.err, p.wait_limit_ns};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
@@ -1004,7 +1011,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t accf0 = smem_addr(bars + 2 * S::kStages);
   const uint32_t acce0 = smem_addr(bars + 2 * S::kStages + 2);
   const uint32_t drain = smem_addr(bars + 2 * S::kStages + 4);
-  const Ctl ctl{abort_flag, p.err};
+  // A pair stops only on the long limit: its CTAs complete copies on each
+  // other's barriers, so one CTA stopping early must not outrun its peer.
+  const Ctl ctl{abort_flag, p.err, kWaitLimitNs};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
@@ -1401,7 +1410,7 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
   // FP8W: A slot converted[kASlots], A slot free[kASlots]
   const uint32_t conv0 = smem_addr(bars + 2 * S::kStages + 5);
   const uint32_t cempty0 = smem_addr(bars + 2 * S::kStages + 5 + S::kASlots);
-  const Ctl ctl{abort_flag, p.err};
+  const Ctl ctl{abort_flag, p.err, p.wait_limit_ns};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
@@ -1794,16 +1803,45 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};
+  EncodeTiledFn fn = cached.load(std::memory_order_acquire);
   if (!fn) {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFn>(p);
+      cached.store(fn, std::memory_order_release);
+    }
   }
   return fn;
+}
+
+// Limit of one pipeline wait of the single-CTA and swap-AB engines, read at
+// every launch: MOE_WAIT_LIMIT_NS when it holds a number of nanoseconds up to
+// the default (a diagnostic knob: a tiny limit makes the waits run out, so
+// the stop path can be exercised), else the default 4 s.
+uint64_t pipeline_wait_limit_ns() {
+  const char *env = getenv("MOE_WAIT_LIMIT_NS");
+  if (!env || !*env) return kWaitLimitNs;
+  char *end = nullptr;
+  const unsigned long long v = strtoull(env, &end, 10);
+  return (end && *end == '\0' && v <= kWaitLimitNs) ? (uint64_t)v : kWaitLimitNs;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.  The flags are
+// atomics: host threads that launch on the same device for the first time at
+// once may both set the (same) attribute, without a data race.
+template <typename Kernel>
+cudaError_t set_smem_once(std::atomic<bool> (&done)[64], Kernel kernel, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev].store(true, std::memory_order_release);
+  return e;
 }
 
 // 2-D map over A [rows, K] (K contiguous), box 64 x 128, 128-byte swizzle.
@@ -1874,16 +1912,13 @@ cudaError_t launch_q8(int rows_cap, int K, int N, int G, const int32_t *offsets,
   const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
-  static bool attr_set[64] = {};
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(
-        k_grouped_gemm<SWIGLU, SPANS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm<SWIGLU, SPANS, true>,
+                                    S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+    return e;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
+  p.wait_limit_ns = pipeline_wait_limit_ns();
   p.row_w = rw.w;
   p.w_row_src = rw.row_src;
   p.scale1 = s1;
@@ -1909,16 +1944,13 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
   const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
-  static bool attr_set[64] = {};  // per device
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(
-        k_grouped_gemm<SWIGLU, SPANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm<SWIGLU, SPANS>,
+                                    S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+    return e;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, bias, row_src, k_max, err};
+  p.wait_limit_ns = pipeline_wait_limit_ns();
   p.row_w = rw.w;
   p.w_row_src = rw.row_src;
   // never more CTAs than tiles can exist (a group holds at most rows_cap rows)
@@ -1942,14 +1974,10 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_set[64] = {};
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(
-        k_grouped_gemm_pair<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_pair<SWIGLU>,
+                                    S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+    return e;
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
   p.row_w = rw.w;
   p.w_row_src = rw.row_src;
@@ -1977,15 +2005,12 @@ cudaError_t launch_swap(int rows_cap, int K, int N, int G, const int32_t *offset
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_set[64] = {};
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(
-        k_grouped_gemm_swap<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_swap<SWIGLU>,
+                                    S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+    return e;
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, row_src, k_max, err};
+  p.wait_limit_ns = pipeline_wait_limit_ns();
   p.row_w = rw.w;
   p.w_row_src = rw.row_src;
   const long long max_tiles = (long long)((rows_cap + S::kMaxRows - 1) / S::kMaxRows +
@@ -2012,15 +2037,12 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_set[64] = {};
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(
-        k_grouped_gemm_swap<SWIGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_swap<SWIGLU, true>,
+                                    S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+    return e;
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
+  p.wait_limit_ns = pipeline_wait_limit_ns();
   p.row_w = rw.w;
   p.w_row_src = rw.row_src;
   p.scale1 = s1;
@@ -2171,16 +2193,13 @@ cudaError_t launch_split(int T, int K, int N, int S, int k_split, const void *A,
   const size_t smem = Sh::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(S + 1);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
-  static bool attr_set[64] = {};
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(
-        k_grouped_gemm<false, SPANS, FP8W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(Sh::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm<false, SPANS, FP8W>,
+                                    Sh::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+    return e;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   Params p{nullptr, S, T, S * T, K, N, out, nullptr, nullptr, 1, err, k_split, clear};
+  p.wait_limit_ns = pipeline_wait_limit_ns();
   p.scale1 = scale;
   const long long tiles = (long long)S * ((T + BM - 1) / BM) * ((N + Sh::BN - 1) / Sh::BN);
   const int grid = (int)(tiles < sms ? tiles : sms);

@@ -6,22 +6,33 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "moe_internal.cuh"
 
 namespace moe {
 
 __device__ uint32_t g_moe_error_word;
 
-uint32_t *device_error_word() {
-  static uint32_t *addr[64] = {};
+// Device address of a file-scope __device__ symbol on the current device,
+// looked up with that device current on its first use and cached per device.
+// The slots are atomics: host threads making a device's first call at the
+// same time each look the address up and store the same value, without a
+// data race.
+void *symbol_address_cached(std::atomic<void *> (&cache)[64], const void *symbol) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_moe_error_word) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<uint32_t *>(p);
+  void *p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) return nullptr;
+    cache[dev].store(p, std::memory_order_release);
   }
-  return addr[dev];
+  return p;
+}
+
+uint32_t *device_error_word() {
+  static std::atomic<void *> addr[64];
+  return static_cast<uint32_t *>(symbol_address_cached(addr, &g_moe_error_word));
 }
 
 namespace {
@@ -422,15 +433,8 @@ static constexpr size_t kStaticScratchBytes = 1u << 20;
 static __device__ __align__(256) unsigned char g_route_scratch[kStaticScratchBytes];
 
 static void *route_scratch_address() {
-  static void *addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+  static std::atomic<void *> addr[64];
+  return moe::symbol_address_cached(addr, g_route_scratch);
 }
 
 moe_status moe_route_static_scratch(const moe_config *cfg, const void *x, const void *Wr,

@@ -48,6 +48,11 @@ def half_ulp(ref, storage):
     return np.exp2(e - bits)
 
 
+# (what, max-abs beyond rounding / RMS, raw max-abs / RMS, relative Frobenius,
+# elements) of every output comparison of the session, printed at its end
+MARGINS: list = []
+
+
 def assert_out_close(got, ref, what="output", storage="bf16"):
     got = got if isinstance(got, np.ndarray) else f64(got)
     if ref.size == 0:
@@ -55,10 +60,12 @@ def assert_out_close(got, ref, what="output", storage="bf16"):
     diff = got - ref
     rms = np.sqrt(np.mean(ref ** 2))
     excess = (np.abs(diff) - half_ulp(ref, storage)).max()
+    raw = np.abs(diff).max()
     frob = np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300)
     assert np.isfinite(got).all(), f"{what}: non-finite values"
+    MARGINS.append((what, excess / rms, raw / rms, frob, int(ref.size)))
     msg = (f"{what}: max-abs beyond {storage} rounding / RMS {excess / rms:.3e} (bound "
-           f"{OUT_MAXABS}; raw max-abs/RMS {np.abs(diff).max() / rms:.3e}), "
+           f"{OUT_MAXABS}; raw max-abs/RMS {raw / rms:.3e}), "
            f"relative Frobenius {frob:.3e} (bound {OUT_FROB})")
     assert excess <= OUT_MAXABS * rms and frob <= OUT_FROB, msg
     return excess / rms, frob
@@ -127,26 +134,41 @@ def run_layer(w: Workload, inp, T=None, route_out=True):
     return out, rb
 
 
-def oracle_layer_on_tokens(inp, routing, tokens):
+def oracle_layer_on_tokens(inp, routing, tokens, chunk_bytes=4 << 30):
     """fp64 layer output on the listed tokens, given the oracle's routing.
 
-    Copies to the host only the weights of the experts the listed tokens use."""
+    Copies to the host only the weights of the experts the listed tokens use,
+    at most about chunk_bytes of them at a time: the oracle runs once per
+    chunk of experts with the slots of the other experts masked out (the
+    shared expert in the first chunk only), and the fp64 chunk outputs are
+    added.  That regroups the oracle's fp64 sum over a token's slots, which
+    moves the result by a few fp64 ulps -- nothing next to the tolerances."""
     idx = routing["topk_idx"]
     sr = routing["slot_row"]
+    toks = np.asarray(tokens, np.int32)
     used = sorted({int(e) for t in tokens for j, e in enumerate(idx[t]) if sr[t, j] >= 0})
-    remap = np.full(max(idx.max() + 1, 1), -1, np.int32)
-    remap[used] = np.arange(len(used), dtype=np.int32)
-    n = len(used)
-    W = {}
-    for key in ("W1", "W3", "W2"):
-        src = inp[key]
-        if n == 0:
-            W[key] = to_numpy(src[:1])
-        else:
-            sel = torch.tensor(used, device=src.device, dtype=torch.long)
-            W[key] = to_numpy(src.index_select(0, sel))
-    sub_idx = np.where(idx >= 0, remap[np.maximum(idx, 0)], -1).astype(np.int32)
     x = to_numpy(inp["x"])
     sh = [to_numpy(inp[k]) for k in ("Ws1", "Ws3", "Ws2")]
-    return oracle.layer_tokens(np.asarray(tokens, np.int32), x, W["W1"], W["W3"], W["W2"],
-                               sub_idx, routing["topk_w"], sr, *sh)
+    per_expert = sum(inp[k][0].numel() * inp[k].element_size() for k in ("W1", "W3", "W2"))
+    step = max(1, int(chunk_bytes // max(per_expert, 1)))
+    chunks = [used[i:i + step] for i in range(0, len(used), step)] or [[]]
+    total = None
+    for ci, chunk in enumerate(chunks):
+        remap = np.full(max(int(idx.max()) + 1, 1), -1, np.int32)
+        remap[chunk] = np.arange(len(chunk), dtype=np.int32)
+        W = {}
+        for key in ("W1", "W3", "W2"):
+            src = inp[key]
+            if not chunk:
+                W[key] = to_numpy(src[:1])
+            else:
+                sel = torch.tensor(chunk, device=src.device, dtype=torch.long)
+                W[key] = to_numpy(src.index_select(0, sel))
+        sub_idx = np.where(idx >= 0, remap[np.maximum(idx, 0)], -1).astype(np.int32)
+        # slots of experts outside this chunk take no part in this pass
+        sub_sr = np.where(sub_idx >= 0, sr, -1).astype(np.int32)
+        part = oracle.layer_tokens(toks, x, W["W1"], W["W3"], W["W2"], sub_idx,
+                                   routing["topk_w"], sub_sr, *(sh if ci == 0 else (None,) * 3))
+        total = part if total is None else total + part
+        del W
+    return total

@@ -116,3 +116,60 @@ def test_layer_roofline_takes_the_slower_bound():
     assert abs(bench.layer_roofline_ms(alg, bench.NOMINAL_PEAKS) - 2.0) < 1e-12
     alg = {"layer_flops": 2.25e12, "layer_bytes": 24e9}  # bytes bound: 3 ms
     assert abs(bench.layer_roofline_ms(alg, bench.NOMINAL_PEAKS) - 3.0) < 1e-12
+
+
+PEAKS = {"hbm_gbs": 6548.8, "bf16_tflops": 1661.1, "bf16_tflops_sustained": 1383.9}
+# stage means of a Mixtral-shaped prefill run (T=8192, 16384 kept rows) on B200
+STAGES_MS = {"route": 0.0736, "dispatch": 0.0412, "up_swiglu": 2.7638, "down": 1.385,
+             "shared": 0.0028, "combine": 0.0854}
+
+
+def test_kernel_roofline_uses_the_burst_peak_whatever_the_clock_reasons():
+    """The compute peak is the measured burst figure, the one the layer
+    fraction uses too; a power-cap sample does not switch it.  Up projection:
+    4.R.d.f = 3.848 TFLOP in 2.7638 ms = 1392 TFLOP/s = 0.838 of 1661.1."""
+    w = WORKLOADS["mixtral_prefill"]
+    alg = bench.algorithmic(w, R=16384, touched=8)
+    for reasons in ([], ["sw_power_cap"]):
+        clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": reasons}
+        k = bench.stage_rooflines(w, alg, STAGES_MS, PEAKS, "measured", clocks, "x", 74.5,
+                                  profiled=False)
+        up = k["up_swiglu"]
+        assert up["bound"] == "tensor" and up["peak"] == 1661.1
+        assert up["frac"] == pytest.approx(0.8382, abs=1e-4)
+        assert up["frac"] == pytest.approx(up["work_per_launch"] / (up["ms_per_launch"] * 1e-3)
+                                           / 1e12 / up["peak"], abs=1e-4)
+        # no compute-bound kernel of this run reads above its own peak
+        assert all(o["frac"] <= 1.0 for o in k.values() if o["bound"] != "hbm")
+
+
+def test_frac_at_sampled_clock_scales_the_compute_peak_only():
+    clocks = {"sm_mhz": 1320.0, "sm_max_mhz": 1965.0}
+    t = bench.kernel_roofline(1661.1e9, 1e6, 1.0, PEAKS, "measured", clocks=clocks)
+    assert t["bound"] == "tensor" and t["frac"] == pytest.approx(1.0)
+    assert t["frac_at_sampled_clock"] == pytest.approx(1965.0 / 1320.0, abs=1e-4)
+    h = bench.kernel_roofline(0, 6548.8e6, 1.0, PEAKS, "measured", clocks=clocks)
+    assert h["bound"] == "hbm" and h["frac"] == pytest.approx(1.0)
+    assert "frac_at_sampled_clock" not in h  # HBM bandwidth does not follow the SM clock
+
+
+def test_combine_reports_both_byte_counts():
+    w = WORKLOADS["mixtral_prefill"]
+    alg = bench.algorithmic(w, R=16384, touched=8)
+    assert alg["combine_bytes"] == (16384 + 8192) * 4096 * 2
+    assert alg["combine_bytes_actual"] == 16384 * 4096 * 4 + 8192 * 4096 * 2 + 8192 * 2 * 8
+    k = bench.stage_rooflines(w, alg, STAGES_MS, PEAKS, "measured", {}, "x", 74.5,
+                              profiled=False)
+    c = k["combine"]
+    assert c["frac"] == pytest.approx(alg["combine_bytes"] / 0.0854e-3 / 1e9 / 6548.8, abs=1e-4)
+    assert c["frac_on_actual_bytes"] > c["frac"]
+
+
+def test_tiny_fp32_ffn_is_alu_bound():
+    w = WORKLOADS["tiny_f32"]
+    alg = bench.algorithmic(w, R=369, touched=8)
+    st = dict(STAGES_MS, up_swiglu=0.058)
+    alu = bench.alu_peak_tflops(148, 1965.0)
+    assert alu == pytest.approx(148 * 128 * 2 * 1.965e9 / 1e12)
+    k = bench.stage_rooflines(w, alg, st, PEAKS, "measured", {}, "x", alu, profiled=False)
+    assert k["up_swiglu"]["bound"] == "alu" and "down" not in k

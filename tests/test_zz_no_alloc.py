@@ -26,6 +26,11 @@ CASES = [
     WORKLOADS["gptoss_sub"].scaled(T=2500, d=256, f=64),
     # sigmoid scores, selection bias, group-limited routing
     WORKLOADS["dsv3_decode"].scaled(d=512, f=64, f_shared=64),
+    # decode-sized Mixtral-shaped routing: 8 experts, split-K router partials
+    WORKLOADS["mixtral_decode"].scaled(d=512, f=64),
+    # the split-K partials at their 768 KiB limit: 96 tokens x 1024 experts x
+    # 4 bytes x 2 slices
+    WORKLOADS["qwen3_prefill"].scaled(T=96, d=1024, E=1024, f=64),
 ]
 
 
@@ -75,3 +80,10 @@ def test_static_scratch_rejects_configs_beyond_its_size():
     st = ops.lib().moe_route_static_scratch(ctypes.byref(cfg), fake, fake, None, None, None,
                                             ctypes.byref(out), None)
     assert st == -3 and "workspace" in ops.moe_status_string(st).lower()
+
+
+def test_budget_case_fills_the_partial_logit_budget():
+    """Host-side: the last case's routing scratch is the split-K partial
+    logits at their 768 KiB limit plus the 256-byte ticket word."""
+    cfg = ops.config(CASES[-1])
+    assert ops.moe_workspace_size(cfg, ops.WS_ROUTE) == (768 << 10) + 256
