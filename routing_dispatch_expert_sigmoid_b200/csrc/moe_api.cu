@@ -68,8 +68,18 @@ moe_status check_config(const moe_config *c) {
 // Workspace regions, each 256-byte aligned.
 struct Layout {
   size_t logits, topk_idx, topk_w, counts, kept, offsets, slot_row, row_src, n_dropped;
-  size_t cap_scratch, x_perm, h, y_perm, h_sh, y_sh, sh_part, total;
+  size_t cap_scratch, x_perm, h, y_perm, h_sh, y_sh, sh_part;
+  size_t f8_xplanes, f8_hplanes, f8_scales;  // fp8 weights, decode-sized batches
+  size_t total;
 };
+
+// Decode-sized bf16 layers (at most 32 rows per expert on average) whose
+// rows are whole 16-byte steps of e4m3 codes can run fp8 expert weights on
+// the kind::f8f6f4 engine; their workspace holds the activation planes.
+bool f8_planes_fit(const moe_config &c) {
+  return c.dtype == MOE_BF16 && c.d % 16 == 0 && c.f % 16 == 0 &&
+         (long long)c.T * c.k_max <= 32LL * c.E;
+}
 
 Layout layout(const moe_config &c, int kind) {
   Layout L{};
@@ -102,6 +112,12 @@ Layout layout(const moe_config &c, int kind) {
       const size_t part = shared_split_bytes(c);  // decode-sized batches only
       if (part) L.sh_part = take(part);
     }
+  }
+  if ((kind == MOE_WS_LAYER || kind == MOE_WS_EXPERT_FFN) && f8_planes_fit(c)) {
+    // x's planes: the layer's x_perm region has exactly their size
+    if (kind == MOE_WS_EXPERT_FFN) L.f8_xplanes = take(fp8_planes_bytes((int)slots, c.d));
+    L.f8_hplanes = take(fp8_planes_bytes((int)slots, c.f));
+    L.f8_scales = take(2 * sizeof(float) * slots);
   }
   L.total = o;
   return L;
@@ -293,6 +309,40 @@ bool fuse_dispatch(const moe_config &c, int rows_cap, const int32_t *offsets) {
   return c.dtype == MOE_BF16 && grouped_gemm_can_gather(true, rows_cap, c.E, offsets, 0);
 }
 
+// fp8 weights of decode-sized layers run on the kind::f8f6f4 engine unless
+// MOE_GEMM_ENGINE names one of the widening engines (single, narrow, swap).
+bool use_f8_engine(const moe_config &c) {
+  if (!f8_planes_fit(c)) return false;
+  const char *env = getenv("MOE_GEMM_ENGINE");
+  return !env || !*env || env[0] == 'f';
+}
+
+// The routed experts' FFN on fp8 weights through the kind::f8f6f4 engine:
+// the rows' activation planes (gathered from the token rows A when row_src is
+// given -- the dispatch step of the layer), the up projection with SwiGLU,
+// the planes of h, the down projection.  Events: mark_rows after the first
+// planes, mark_up after the up projection.
+moe_status ffn_f8_impl(const moe_config &c, const int32_t *offsets, const void *A,
+                       const int32_t *row_src, int a_rows, const Weights &w, uint8_t *xplanes,
+                       uint8_t *hplanes, float *scales, void *h, void *y, uint32_t *err,
+                       cudaStream_t s, const Events &ev = Events(), int mark_rows = -1,
+                       int mark_up = -1, const float *gate_w = nullptr,
+                       const int32_t *gate_src = nullptr) {
+  const int rows_cap = c.T * c.k_max;
+  float *xs = scales, *hs = scales + rows_cap;
+  MOE_TRY_CUDA(launch_split_planes(A, offsets + c.E, 0, row_src, c.k_max, a_rows, rows_cap, c.d,
+                                   xplanes, xs, err, s));
+  MOE_TRY_CUDA(ev.mark(mark_rows, s));
+  MOE_TRY_CUDA(launch_grouped_gemm_f8(true, rows_cap, c.d, c.f, c.E, offsets, xplanes, xs, w.W1,
+                                      w.W3, w.s1, w.s3, h, err, s));
+  MOE_TRY_CUDA(ev.mark(mark_up, s));
+  MOE_TRY_CUDA(launch_split_planes(h, offsets + c.E, 0, nullptr, 1, rows_cap, rows_cap, c.f,
+                                   hplanes, hs, err, s));
+  MOE_TRY_CUDA(launch_grouped_gemm_f8(false, rows_cap, c.f, c.d, c.E, offsets, hplanes, hs, w.W2,
+                                      nullptr, w.s2, nullptr, y, err, s, gate_w, gate_src));
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -344,7 +394,12 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   const bool wig = weights_in_gemm(c);
   const float *gate_w = wig ? r.topk_w : nullptr;
   const int32_t *gate_src = wig ? r.row_src : nullptr;
-  if (!we.fp8 && fuse_dispatch(c, rows_cap, r.offsets)) {
+  if (we.fp8 && use_f8_engine(c)) {
+    // dispatch = the planes of the gathered token rows (in the x_perm region)
+    MOE_TRY(ffn_f8_impl(c, r.offsets, x, r.row_src, c.T, we, static_cast<uint8_t *>(x_perm),
+                        at<uint8_t>(ws, L.f8_hplanes), at<float>(ws, L.f8_scales),
+                        at<void>(ws, L.h), y_perm, err, s, ev, 2, 3, gate_w, gate_src));
+  } else if (!we.fp8 && fuse_dispatch(c, rows_cap, r.offsets)) {
     MOE_TRY_CUDA(ev.mark(2, s));
     MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x, we, at<void>(ws, L.h), y_perm, err,
                      s, ev, 3, r.row_src, gate_w, gate_src));
@@ -510,6 +565,11 @@ moe_status moe_expert_ffn_fp8(const moe_config *cfg, const void *x_perm, const i
   uint32_t *err = device_error_word();
   if (!err) return MOE_ERR_CUDA;
   const Layout L = layout(c, MOE_WS_EXPERT_FFN);
+  if (use_f8_engine(c))
+    return ffn_f8_impl(c, offsets, x_perm, nullptr, c.T * c.k_max, we,
+                       at<uint8_t>(ws, L.f8_xplanes), at<uint8_t>(ws, L.f8_hplanes),
+                       at<float>(ws, L.f8_scales), at<void>(ws, L.h), y_perm, err,
+                       static_cast<cudaStream_t>(stream));
   return ffn_impl(c, c.E, offsets, 0, c.T * c.k_max, c.f, x_perm, we, at<void>(ws, L.h), y_perm,
                   err, static_cast<cudaStream_t>(stream));
 }

@@ -110,6 +110,28 @@ cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int
                                     const float *row_w = nullptr,
                                     const int32_t *w_row_src = nullptr);
 
+// K5/K6 with fp8 weights on tcgen05.mma kind::f8f6f4 (grouped_gemm_f8.cu):
+// decode-sized routed groups.  The activations come as two e4m3 planes with a
+// power-of-two scale per row (launch_split_planes): planes [2 * rows_cap, K],
+// plane q's row r at q * rows_cap + r; row_scale [rows_cap].  B1, B3: e4m3
+// codes [G, N, K] with column scales s1, s3 [G, N].  Output types as for
+// launch_grouped_gemm_bf16.
+cudaError_t launch_grouped_gemm_f8(bool swiglu, int rows_cap, int K, int N, int G,
+                                   const int32_t *offsets, const uint8_t *planes,
+                                   const float *row_scale, const void *B1, const void *B3,
+                                   const float *s1, const float *s3, void *out, uint32_t *err,
+                                   cudaStream_t s, const float *row_w = nullptr,
+                                   const int32_t *w_row_src = nullptr);
+// Bytes of the two planes of rows_cap rows of K values.
+size_t fp8_planes_bytes(int rows_cap, int K);
+// Rows r < (*n_rows, or fixed_rows when n_rows is nullptr) of the bf16 rows
+// src [., K] -- with row_src, token row row_src[r] / k_max (< src_rows) of
+// them -- into planes and row scales (K % 16 == 0).
+cudaError_t launch_split_planes(const void *src, const int32_t *n_rows, int fixed_rows,
+                                const int32_t *row_src, int k_max, int src_rows, int rows_cap,
+                                int K, uint8_t *planes, float *row_scale, uint32_t *err,
+                                cudaStream_t s);
+
 // Per-column e4m3 quantisation of bf16 weights W [G, K, N]: scale[g, n] =
 // max_k |W| / 448 (1 for an all-zero column), Wq = e4m3(W / scale), rounded
 // to nearest even with saturation.

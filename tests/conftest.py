@@ -38,7 +38,10 @@ def pytest_terminal_summary(terminalreporter):
     tr.section("output parity margins (largest first)")
     tr.write_line(f"{'comparison':60s} {'beyond-rounding/RMS':>20s} {'raw max-abs/RMS':>16s} "
                   f"{'rel. Frobenius':>15s} {'elements':>10s}")
-    for what, excess, raw, frob, n in sorted(rows, key=lambda r: -r[1])[:60]:
+    # the 40 largest, then every full-size workload
+    shown = sorted(rows, key=lambda r: -r[1])[:40]
+    shown += [r for r in rows if "full size" in r[0] and r not in shown]
+    for what, excess, raw, frob, n in shown:
         tr.write_line(f"{what[:60]:60s} {excess:20.3e} {raw:16.3e} {frob:15.3e} {n:10d}")
     tr.write_line(f"{len(rows)} comparisons; worst beyond-rounding/RMS "
                   f"{max(r[1] for r in rows):.3e}, worst raw max-abs/RMS "

@@ -39,6 +39,14 @@ CASES = {
     # one expert, k = 1: the dense FFN on fp8 weights
     "single_expert": WORKLOADS["mixtral_prefill"].scaled(T=77, d=256, E=1, k_max=1, f=384,
                                                          zipf_s=0.0),
+    # decode-sized layers (the kind::f8f6f4 engine by default): N of both
+    # projections 16 mod 128 and K not a multiple of the 128-deep k-block
+    "f8_decode_ragged": WORKLOADS["mixtral_decode"].scaled(T=40, d=272, f=400),
+    # one hot expert holding several 64-row tiles
+    "f8_decode_hot_expert": WORKLOADS["mixtral_decode"].scaled(T=128, d=256, f=320, zipf_s=3.0),
+    # 256 experts, a row or two each, group-limited sigmoid routing
+    "f8_decode_many_experts": WORKLOADS["dsv3_decode"].scaled(T=64, d=384, E=256, f=144,
+                                                              f_shared=0),
 }
 
 
@@ -158,11 +166,14 @@ def test_fp8_expert_ffn_matches_oracle(name, dev):
     assert_out_close(f64(y[:R]), ref, "fp8 expert FFN", "f32")
 
 
-def test_fp8_every_code_through_the_ffn(fp8_engine, dev):
+@pytest.mark.parametrize("T", [192, 64])
+def test_fp8_every_code_through_the_ffn(T, fp8_engine, dev):
     """Codes drawn uniformly from every finite e4m3 code (subnormals, both
     zeros and the largest magnitude included) with random column scales: the
-    widening to bf16 in shared memory must give each code's exact value."""
-    w = WORKLOADS["mixtral_prefill"].scaled(T=192, d=256, E=3, k_max=1, f=384)
+    widening to bf16 in shared memory, or the tensor cores' own e4m3 inputs
+    (T = 64: 21 rows per expert, the kind::f8f6f4 engine), must give each
+    code's exact value."""
+    w = WORKLOADS["mixtral_prefill"].scaled(T=T, d=256, E=3, k_max=1, f=384)
     cfg = ops.config(w)
     g = np.random.default_rng(41)
     finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
@@ -175,9 +186,9 @@ def test_fp8_every_code_through_the_ffn(fp8_engine, dev):
     for k, (q, sc) in sets.items():  # the library takes the codes K-contiguous
         gpu[k] = torch.from_numpy(np.ascontiguousarray(q.swapaxes(1, 2))).to(dev)
         gpu["s" + k[-1]] = torch.from_numpy(sc).to(dev)
-    offsets = np.array([0, 50, 50, 192], np.int32)  # an empty expert in the middle
-    xb = torch.randn(192, w.d, generator=torch.Generator().manual_seed(42)).to(torch.bfloat16)
-    y = torch.zeros((192, w.d), dtype=torch.float32, device=dev)
+    offsets = np.array([0, T // 4, T // 4, T], np.int32)  # an empty expert in the middle
+    xb = torch.randn(T, w.d, generator=torch.Generator().manual_seed(42)).to(torch.bfloat16)
+    y = torch.zeros((T, w.d), dtype=torch.float32, device=dev)
     ops.moe_expert_ffn_fp8(cfg, xb.to(dev), torch.from_numpy(offsets).to(dev), gpu, y,
                            ops.workspace(cfg, ops.WS_EXPERT_FFN))
     ops.moe_check_errors()
