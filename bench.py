@@ -42,7 +42,8 @@ Extra keys of the JSON line:
                scales (quantised before timing), same keys;
   configs      every other workload of the layer definition (tiny fp32,
                Qwen3-, DeepSeek-V3- (decode and prefill) and GPT-OSS-shaped
-               layers), same keys, each timed on its own inputs after the
+               layers, and the DeepSeek-V3-shaped decode layer with e4m3 expert
+               weights), same keys, each timed on its own inputs after the
                previous one's memory was freed.
 `--impl reference` times the CPU oracle alone on the same workload (the
 reference arm: there is no other implementation of this layer to run).
@@ -556,7 +557,8 @@ def cpu_sample_tokens(name: str, budget_s: float) -> int:
 # ---------------------------------------------------------------------------
 # The workloads of the layer definition besides the Mixtral-shaped legs, each
 # measured by the default run and reported under "configs".
-OTHER_CONFIGS = ("tiny_f32", "qwen3_prefill", "dsv3_decode", "dsv3_prefill", "gptoss_sub")
+OTHER_CONFIGS = ("tiny_f32", "qwen3_prefill", "dsv3_decode", "dsv3_decode:fp8", "dsv3_prefill",
+                 "gptoss_sub")
 
 
 def describe(w) -> str:
@@ -674,10 +676,12 @@ def main():
     if a.fp8_workload != "none":
         fp8_obj, _ = measure_leg(a.fp8_workload, max(a.steps, 50), warmup, fp8=True, **leg)
     configs = {}
-    for name in [c for c in a.configs.split(",") if c and c != "none"]:
+    for entry in [c for c in a.configs.split(",") if c and c != "none"]:
+        name, _, kind = entry.partition(":")  # "<workload>:fp8": e4m3 expert weights
         wc = WORKLOADS[name]
         steps = max(a.steps, 50) if wc.T <= 256 else a.steps
-        configs[name], _ = measure_leg(name, steps, warmup, **leg)
+        configs[name + ("_fp8" if kind == "fp8" else "")], _ = measure_leg(
+            name, steps, warmup, fp8=kind == "fp8", **leg)
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:

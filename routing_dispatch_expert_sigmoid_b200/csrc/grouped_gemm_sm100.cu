@@ -95,6 +95,10 @@ struct Params {
   const int32_t *w_row_src = nullptr;
   // Limit of one pipeline wait (the single-CTA and swap-AB engines)
   uint64_t wait_limit_ns = kWaitLimitNs;
+  // PLAIN, single-CTA and pair engines: when set, out receives the compact
+  // y16 form of the rows, with nblk = ceil(N / 32) block exponents per row
+  int8_t *yexp = nullptr;
+  int nblk = 0;
 };
 
 // Gate weights to apply in the down projection's epilogue (both nullptr: none).
@@ -564,6 +568,14 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
               *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) +
                                          (size_t)grow * p.N + gcol) = val;
           }
+        } else if (p.yexp) {  // y16: fp16 rows, one exponent per 32-column block
+          if (p.row_w && row0 + lane < row_end) {
+            const float wr = p.row_w[p.w_row_src[row0 + lane]];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= wr;
+          }
+          store_y16_lane_rows(v, reinterpret_cast<uint32_t *>(stg), S::kStageRowWords, lane, row0,
+                              row_end, col, p.N, p.out, p.yexp, p.nblk);
         } else {  // fp32 (+ bias), a row is 32 words
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -1032,6 +1044,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) +
                                          (size_t)grow * p.N + gcol) = val;
           }
+        } else if (p.yexp) {  // y16: fp16 rows, one exponent per 32-column block
+          if (p.row_w && row0 + lane < row_end) {
+            const float wr = p.row_w[p.w_row_src[row0 + lane]];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= wr;
+          }
+          store_y16_lane_rows(v, reinterpret_cast<uint32_t *>(stg), S::kStageRowWords, lane, row0,
+                              row_end, col, p.N, p.out, p.yexp, p.nblk);
         } else {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -1662,7 +1682,8 @@ template <bool SWIGLU, int SPANS>
 cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, int fixed_rows,
                    const void *A, const void *B1, const void *B3, void *out, const float *bias,
                    uint32_t *err, cudaStream_t s, const int32_t *row_src = nullptr,
-                   int k_max = 1, int a_rows = 0, RowWeights rw = RowWeights()) {
+                   int k_max = 1, int a_rows = 0, RowWeights rw = RowWeights(),
+                   int8_t *yexp = nullptr) {
   using S = Shape<SWIGLU, SPANS>;
   CUtensorMap ma, mb1, mb3;
   const bool map_ok = row_src ? make_map_rows(&ma, A, a_rows, K, 1) : make_map_a(&ma, A, rows_cap, K);
@@ -1681,6 +1702,8 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
   p.wait_limit_ns = pipeline_wait_limit_ns();
   p.row_w = rw.w;
   p.w_row_src = rw.row_src;
+  p.yexp = yexp;
+  p.nblk = (N + 31) / 32;
   // never more CTAs than tiles can exist (a group holds at most rows_cap rows)
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
@@ -1692,7 +1715,8 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
 template <bool SWIGLU>
 cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offsets,
                         int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
-                        uint32_t *err, cudaStream_t s, RowWeights rw = RowWeights()) {
+                        uint32_t *err, cudaStream_t s, RowWeights rw = RowWeights(),
+                        int8_t *yexp = nullptr) {
   using S = Shape2<SWIGLU>;
   CUtensorMap ma, mb1, mb3;
   if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
@@ -1709,6 +1733,8 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
   p.row_w = rw.w;
   p.w_row_src = rw.row_src;
+  p.yexp = yexp;
+  p.nblk = (N + 31) / 32;
   const long long max_tiles = (long long)((rows_cap + BM2 - 1) / BM2 + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
   long long pairs = sms / 2;
@@ -1785,12 +1811,15 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
 
 }  // namespace tc
 
-// Three engines, all correct for every shape (the tests run each):
+// Engines, all correct for every shape (the tests run each):
 //   single  one CTA per 128-row tile; up projection 128 columns of gate and of
 //           up (N=256 MMA), down projection 256 columns;
 //   narrow  the same with 64-column up-projection tiles (twice the tiles);
 //   pair    CTA pairs on 256-row tiles (tcgen05 cta_group::2);
-//   swap    weights as the M operand, rows in steps of 16 (swap-AB).
+//   swap    weights as the M operand, rows in steps of 16 (swap-AB);
+//   mixed   routed groups only: each group's full 128-row chunks as single
+//           tiles and its remainder as a swap-AB tile, in one launch
+//           (grouped_gemm_mixed.cu).
 // Defaults, from B200 measurements with the engines alternated call by call
 // in one process:
 //   - decode-sized groups (at most 32 rows per group on average): swap-AB for
@@ -1807,11 +1836,10 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
 //     6% on Mixtral prefill.
 //   - except for the up projection of ragged groups of at most 256 rows on
 //     average (routed experts only), where a 256-row pair tile is often
-//     half empty: single-CTA (DeepSeek-V3-shaped prefill, 128 rows per expert
-//     on average: 3.52 vs 3.74 ms; GPT-OSS-shaped sub-experts: 1.27 vs
-//     1.35 ms).
-// MOE_GEMM_ENGINE=single|narrow|pair|swap selects one engine for every GEMM.
-enum class Engine { kSingle, kNarrow, kPair, kSwap };
+//     half empty: mixed tiles.
+// MOE_GEMM_ENGINE=single|narrow|pair|swap|mixed selects one engine for every
+// GEMM (mixed: for routed groups; a single group of rows runs single-CTA).
+enum class Engine { kSingle, kNarrow, kPair, kSwap, kMixed };
 
 static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offsets,
                           int fixed_rows, int N) {
@@ -1820,15 +1848,22 @@ static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offse
   if (env && env[0] == 'n') return Engine::kNarrow;
   if (env && env[0] == 'p') return Engine::kPair;
   if (env && env[0] == 's' && env[1] == 'w') return Engine::kSwap;
+  if (env && env[0] == 'm') return offsets ? Engine::kMixed : Engine::kSingle;
   const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
   if (mean_rows <= 32) return swiglu ? Engine::kSwap : Engine::kSingle;
-  if (swiglu) return (offsets && mean_rows <= 256) ? Engine::kSingle : Engine::kPair;
+  if (swiglu) return (offsets && mean_rows <= 256) ? Engine::kMixed : Engine::kPair;
   return N >= 4096 ? Engine::kPair : Engine::kSingle;
 }
 
 bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *offsets,
                              int fixed_rows) {
-  return swiglu && pick_engine(swiglu, rows_cap, G, offsets, fixed_rows, 0) != Engine::kPair;
+  if (!swiglu) return false;
+  const Engine e = pick_engine(swiglu, rows_cap, G, offsets, fixed_rows, 0);
+  return e == Engine::kSingle || e == Engine::kNarrow || e == Engine::kSwap;
+}
+
+bool grouped_gemm_y16_out(int rows_cap, int G, const int32_t *offsets, int fixed_rows, int N) {
+  return pick_engine(false, rows_cap, G, offsets, fixed_rows, N) != Engine::kSwap;
 }
 
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
@@ -1836,21 +1871,26 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
                                      const void *B1, const void *B3, void *out, uint32_t *err,
                                      cudaStream_t s, const int32_t *row_src, int k_max,
                                      int a_rows, const float *row_w,
-                                     const int32_t *w_row_src) {
+                                     const int32_t *w_row_src, int8_t *yexp) {
   if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if (rows_cap == 0) return cudaSuccess;
   const Engine e = pick_engine(swiglu, rows_cap, G, offsets, fixed_rows, N);
-  if (row_src && (!swiglu || e == Engine::kPair)) return cudaErrorInvalidValue;
+  if (row_src && (!swiglu || e == Engine::kPair || e == Engine::kMixed))
+    return cudaErrorInvalidValue;
+  if (yexp && (swiglu || e == Engine::kSwap)) return cudaErrorInvalidValue;
   if (row_w && swiglu) return cudaErrorInvalidValue;  // gate weights: the down projection only
   tc::RowWeights rw;
   rw.w = row_w;
   rw.row_src = w_row_src;
   switch (e) {
+    case Engine::kMixed:
+      return launch_grouped_gemm_mixed(swiglu, rows_cap, K, N, G, offsets, A, B1, B3, out, err,
+                                       s, row_w, w_row_src, yexp);
     case Engine::kPair:
       return swiglu ? tc::launch_pair<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                             out, err, s)
                     : tc::launch_pair<false>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
-                                             out, err, s, rw);
+                                             out, err, s, rw, yexp);
     case Engine::kSwap:
       return swiglu ? tc::launch_swap<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                             out, err, s, row_src, k_max, a_rows)
@@ -1865,7 +1905,7 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
       return swiglu ? tc::launch<true, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                           out, nullptr, err, s, row_src, k_max, a_rows)
                     : tc::launch<false, 4>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
-                                           out, nullptr, err, s, nullptr, 1, 0, rw);
+                                           out, nullptr, err, s, nullptr, 1, 0, rw, yexp);
   }
 }
 

@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "moe_internal.cuh"
@@ -73,6 +74,11 @@ struct Layout {
   size_t total;
 };
 
+// Bytes of rows of d values in the y16 form: the fp16 values, then (256-byte
+// aligned) one exponent byte per 32-column block of each row.
+size_t y16_exp_offset(size_t rows, int d) { return up(rows * d * 2); }
+size_t y16_bytes(size_t rows, int d) { return y16_exp_offset(rows, d) + rows * ((d + 31) / 32); }
+
 // Decode-sized bf16 layers (at most 32 rows per expert on average) whose
 // rows are whole 16-byte steps of e4m3 codes can run fp8 expert weights on
 // the kind::f8f6f4 engine; their workspace holds the activation planes.
@@ -105,7 +111,9 @@ Layout layout(const moe_config &c, int kind) {
   if (kind == MOE_WS_LAYER) L.x_perm = take(slots * c.d * s);
   if (kind == MOE_WS_LAYER || kind == MOE_WS_EXPERT_FFN) L.h = take(slots * c.f * s);
   if (kind == MOE_WS_LAYER) {
-    L.y_perm = take(slots * c.d * sizeof(float));  // fp32: the combine rounds once
+    // fp32 rows (the combine rounds once), or their compact y16 form (fp16
+    // values, one exponent byte per 32-column block)
+    L.y_perm = take(std::max(slots * c.d * sizeof(float), y16_bytes(slots, c.d)));
     if (c.f_shared > 0) {
       L.h_sh = take((size_t)c.T * c.f_shared * s);
       L.y_sh = take((size_t)c.T * c.d * sizeof(float));
@@ -262,7 +270,7 @@ moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixe
                     int rows_cap, int f, const void *A, const Weights &w, void *h, void *y,
                     uint32_t *err, cudaStream_t s, const Events &ev = Events(), int mid = -1,
                     const int32_t *row_src = nullptr, const float *gate_w = nullptr,
-                    const int32_t *gate_src = nullptr) {
+                    const int32_t *gate_src = nullptr, int8_t *yexp = nullptr) {
   if (w.fp8) {
     MOE_TRY_CUDA(launch_grouped_gemm_fp8(true, rows_cap, c.d, f, G, offsets, fixed_rows, A, w.W1,
                                          w.W3, w.s1, w.s3, h, err, s));
@@ -284,7 +292,8 @@ moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixe
                                         w.W3, h, err, s, row_src, c.k_max, c.T));
   MOE_TRY_CUDA(ev.mark(mid, s));
   MOE_TRY_CUDA(launch_grouped_gemm_bf16(false, rows_cap, f, c.d, G, offsets, fixed_rows, h, w.W2,
-                                        nullptr, y, err, s, nullptr, 1, 0, gate_w, gate_src));
+                                        nullptr, y, err, s, nullptr, 1, 0, gate_w, gate_src,
+                                        yexp));
   return MOE_OK;
 }
 
@@ -295,6 +304,16 @@ moe_status ffn_impl(const moe_config &c, int G, const int32_t *offsets, int fixe
 bool weights_in_gemm(const moe_config &c) {
   const char *env = getenv("MOE_WEIGHTS_IN_GEMM");
   return c.dtype == MOE_BF16 && env && env[0] == '1';
+}
+
+// The routed experts' outputs of bf16 layers travel from the down projection
+// to the combine in the compact y16 form (half the bytes of fp32 rows, a
+// relative error of at most 2^-11 per value) when the down projection's
+// engine writes it; MOE_Y16=0 keeps fp32 rows.
+bool use_y16(const moe_config &c, int rows_cap, const int32_t *offsets) {
+  const char *env = getenv("MOE_Y16");
+  if (env && env[0] == '0') return false;
+  return c.dtype == MOE_BF16 && grouped_gemm_y16_out(rows_cap, c.E, offsets, 0, c.d);
 }
 
 // The dispatch copy can be fused into the up projection (bf16 layers, engines
@@ -392,6 +411,9 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   const int rows_cap = c.T * c.k_max;
   void *x_perm = at<void>(ws, L.x_perm), *y_perm = at<void>(ws, L.y_perm);
   const bool wig = weights_in_gemm(c);
+  int8_t *yexp = (!we.fp8 && use_y16(c, rows_cap, r.offsets))
+                     ? at<int8_t>(ws, L.y_perm + y16_exp_offset((size_t)rows_cap, c.d))
+                     : nullptr;
   const float *gate_w = wig ? r.topk_w : nullptr;
   const int32_t *gate_src = wig ? r.row_src : nullptr;
   if (we.fp8 && use_f8_engine(c)) {
@@ -402,12 +424,12 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   } else if (!we.fp8 && fuse_dispatch(c, rows_cap, r.offsets)) {
     MOE_TRY_CUDA(ev.mark(2, s));
     MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x, we, at<void>(ws, L.h), y_perm, err,
-                     s, ev, 3, r.row_src, gate_w, gate_src));
+                     s, ev, 3, r.row_src, gate_w, gate_src, yexp));
   } else {
     MOE_TRY_CUDA(launch_dispatch(c, x, r.offsets, r.row_src, x_perm, err, s));
     MOE_TRY_CUDA(ev.mark(2, s));
     MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x_perm, we, at<void>(ws, L.h), y_perm,
-                     err, s, ev, 3, nullptr, gate_w, gate_src));
+                     err, s, ev, 3, nullptr, gate_w, gate_src, yexp));
   }
   MOE_TRY_CUDA(ev.mark(4, s));
   const void *shared_y = nullptr;
@@ -428,7 +450,7 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
   }
   MOE_TRY_CUDA(ev.mark(5, s));
   MOE_TRY_CUDA(launch_combine(c, y_perm, r.slot_row, wig ? nullptr : r.topk_w, shared_y, out,
-                               err, s, shared_parts));
+                               err, s, shared_parts, yexp));
   MOE_TRY_CUDA(ev.mark(6, s));
   return MOE_OK;
 }

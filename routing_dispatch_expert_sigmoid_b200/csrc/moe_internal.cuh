@@ -68,10 +68,11 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *o
 // shared are fp32, out is in the layer dtype.  topk_w == nullptr: the rows
 // already carry their gate weights (applied by the down projection).
 // shared_y: shared_parts fp32 blocks [T, d] (partial sums of the shared
-// expert, added in order), or nullptr.
+// expert, added in order), or nullptr.  yexp (bf16 layers): y_perm holds
+// y16 rows with these block exponents [rows, ceil(d / 32)] instead of fp32.
 cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                            const float *topk_w, const void *shared_y, void *out, uint32_t *err,
-                           cudaStream_t s, int shared_parts = 1);
+                           cudaStream_t s, int shared_parts = 1, const int8_t *yexp = nullptr);
 
 // K9: fp32 SIMT grouped SwiGLU FFN (fp32 layers).  h: [rows_cap, f] fp32.
 cudaError_t launch_ffn_simt_f32(int rows_cap, int d, int f, int G, const int32_t *offsets,
@@ -91,13 +92,18 @@ bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *of
                              int fixed_rows);
 // row_w (plain only): output row r is multiplied by row_w[w_row_src[r]], the
 // gate weight of the slot it serves (the combine then only sums).
+// yexp (plain only, engines other than swap-AB: grouped_gemm_y16_out):
+// out receives the compact y16 form of the rows, see launch_grouped_gemm_mixed.
 cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, int G,
                                      const int32_t *offsets, int fixed_rows, const void *A,
                                      const void *B1, const void *B3, void *out, uint32_t *err,
                                      cudaStream_t s, const int32_t *row_src = nullptr,
                                      int k_max = 1, int a_rows = 0,
                                      const float *row_w = nullptr,
-                                     const int32_t *w_row_src = nullptr);
+                                     const int32_t *w_row_src = nullptr,
+                                     int8_t *yexp = nullptr);
+// Whether the down projection of this shape can write y16 rows.
+bool grouped_gemm_y16_out(int rows_cap, int G, const int32_t *offsets, int fixed_rows, int N);
 
 // K5/K6 with fp8 weights: B1, B3 are e4m3 codes [G, K, N] (N % 16 == 0) with
 // per-column fp32 scales s1, s3 [G, N] (16-byte aligned); the codes are
@@ -109,6 +115,19 @@ cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int
                                     const float *s3, void *out, uint32_t *err, cudaStream_t s,
                                     const float *row_w = nullptr,
                                     const int32_t *w_row_src = nullptr);
+
+// K5/K6 for ragged routed groups (grouped_gemm_mixed.cu): each group's full
+// 128-row chunks on ordinary tiles and its remainder on a swap-AB tile, in
+// one launch.  Operands and outputs as for launch_grouped_gemm_bf16.
+// yexp (plain only): when given, out receives the compact y16 form of the
+// fp32 rows (fp16 values, one power-of-two exponent per 32-column block in
+// yexp [rows_cap, ceil(N / 32)]; see tcgen05_common.cuh).
+cudaError_t launch_grouped_gemm_mixed(bool swiglu, int rows_cap, int K, int N, int G,
+                                      const int32_t *offsets, const void *A, const void *B1,
+                                      const void *B3, void *out, uint32_t *err, cudaStream_t s,
+                                      const float *row_w = nullptr,
+                                      const int32_t *w_row_src = nullptr,
+                                      int8_t *yexp = nullptr);
 
 // K5/K6 with fp8 weights on tcgen05.mma kind::f8f6f4 (grouped_gemm_f8.cu):
 // decode-sized routed groups.  The activations come as two e4m3 planes with a

@@ -13,6 +13,8 @@
 // (rows of d*s bytes, d*s a multiple of 16); a warp takes a chunk of one row
 // (dispatch) or of one token's output (combine) at a time.  The number of rows R lives on the device
 // (offsets[E]); a fixed grid strides over the row space and stops at R.
+#include <cuda_fp16.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -209,6 +211,106 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The same combine on y16 rows (fp16 values, one power-of-two exponent per
+// 32-column block, written by the down projection): value = y16 * 2^e.  The
+// bf16 output vector of lane l spans 8 columns of one block, so each slot
+// costs one 16-byte load and one exponent byte; the exponent is folded into
+// the slot's weight (w * 2^e is exact).
+template <int KB>
+__global__ void __launch_bounds__(256)
+    k_combine_y16(const uint4 *__restrict__ y, const int8_t *__restrict__ yexp, int nblk,
+                  const int32_t *__restrict__ slot_row, const float *__restrict__ topk_w,
+                  const uint4 *__restrict__ shared_y, int shared_parts, uint4 *__restrict__ out,
+                  int Tn, int k_max, int rows_cap, int row_vecs, uint32_t *err) {
+  __shared__ int32_t s_row[8][32];
+  __shared__ float s_w[8][32];
+  const int lane = threadIdx.x % 32, wib = threadIdx.x / 32;
+  const int chunks = (row_vecs + 31) / 32;
+  const long long items = (long long)Tn * chunks;
+  const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+  const size_t sh_vecs = (size_t)row_vecs * 2;  // fp32 vectors per shared row
+  long long it = (long long)blockIdx.x * (blockDim.x / 32) + wib;
+  int next_row = -1;
+  float next_w = 0.f;
+  if (it < items && lane < k_max) {
+    const size_t at = (size_t)(it / chunks) * k_max + lane;
+    next_row = slot_row[at];
+    next_w = topk_w ? topk_w[at] : 1.0f;
+  }
+  for (; it < items; it += warps) {
+    const int t = (int)(it / chunks), ch = (int)(it % chunks);
+    int my_row = next_row;
+    const float my_w = next_w;
+    if (it + warps < items && lane < k_max) {
+      const size_t at = (size_t)((it + warps) / chunks) * k_max + lane;
+      next_row = slot_row[at];
+      next_w = topk_w ? topk_w[at] : 1.0f;
+    }
+    if (my_row >= rows_cap) {
+      raise_error(err, kErrIndex);
+      my_row = -1;
+    }
+    const unsigned live = __ballot_sync(0xffffffffu, my_row >= 0);
+    const int n_live = __popc(live);
+    if (my_row >= 0) {  // compact the kept slots, in slot order
+      const int pos = __popc(live & ((1u << lane) - 1u));
+      s_row[wib][pos] = my_row;
+      s_w[wib][pos] = my_w;
+    }
+    __syncwarp();
+    const int v = ch * 32 + lane;
+    if (v < row_vecs) {
+      float acc[8];
+      if (shared_y) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          Vec<float>::load(ldg_nc(shared_y + (size_t)t * sh_vecs + (size_t)v * 2 + q),
+                           acc + 4 * q);
+        for (int sp = 1; sp < shared_parts; ++sp) {  // further partial sums, in order
+          const uint4 *part = shared_y + (size_t)sp * Tn * sh_vecs + (size_t)t * sh_vecs;
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            float f[4];
+            Vec<float>::load(ldg_nc(part + (size_t)v * 2 + q), f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[4 * q + i] += f[i];
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      }
+      const int blk = v >> 2;  // 8 columns per vector, 32 per exponent
+      for (int j0 = 0; j0 < n_live; j0 += KB) {
+        uint4 u[KB];
+        int e[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j)  // issue the loads before the FMAs
+          if (j0 + j < n_live) {
+            const int r = s_row[wib][j0 + j];
+            u[j] = ldg_nc(y + (size_t)r * row_vecs + v);
+            e[j] = __ldg(yexp + (size_t)r * nblk + blk);
+          }
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+          if (j0 + j < n_live) {
+            const float wj = s_w[wib][j0 + j] * __int_as_float((e[j] + 127) << 23);
+            const uint32_t hw[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[i]));
+              acc[2 * i] = fmaf(wj, f.x, acc[2 * i]);
+              acc[2 * i + 1] = fmaf(wj, f.y, acc[2 * i + 1]);
+            }
+          }
+        }
+      }
+      out[(size_t)t * row_vecs + v] = Vec<__nv_bfloat16>::store(acc);
+    }
+    __syncwarp();
+  }
+}
+
 int grid_for(long long warps_needed) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -271,11 +373,28 @@ cudaError_t combine_k(const moe_config &c, const void *y_perm, const int32_t *sl
 
 cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                            const float *topk_w, const void *shared_y, void *out, uint32_t *err,
-                           cudaStream_t s, int shared_parts) {
+                           cudaStream_t s, int shared_parts, const int8_t *yexp) {
   if (c.T == 0) return cudaSuccess;
   const int esz = c.dtype == MOE_F32 ? 4 : 2;
   const int row_vecs = c.d * esz / 16;
   const int grid = grid_for((long long)c.T * ((row_vecs + 31) / 32));
+  if (yexp) {  // y16 rows (bf16 layers only)
+    if (c.dtype != MOE_BF16) return cudaErrorInvalidValue;
+    const auto *y = static_cast<const uint4 *>(y_perm);
+    const auto *sh = static_cast<const uint4 *>(shared_y);
+    auto *o = static_cast<uint4 *>(out);
+    const int nblk = (c.d + 31) / 32, rows_cap = c.T * c.k_max;
+    if (c.k_max <= 2)
+      k_combine_y16<2><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o,
+                                            c.T, c.k_max, rows_cap, row_vecs, err);
+    else if (c.k_max <= 4)
+      k_combine_y16<4><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o,
+                                            c.T, c.k_max, rows_cap, row_vecs, err);
+    else
+      k_combine_y16<8><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o,
+                                            c.T, c.k_max, rows_cap, row_vecs, err);
+    return cudaGetLastError();
+  }
   if (c.dtype == MOE_F32)
     return combine_k<float>(c, y_perm, slot_row, topk_w, shared_y, out, err, s, shared_parts,
                             grid, row_vecs);

@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <stdlib.h>
 
 #include <atomic>
@@ -238,6 +239,98 @@ constexpr uint32_t instr_desc(int M, int N) {
 __host__ __device__ constexpr uint32_t instr_desc_kk(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Compact expert outputs ("y16"): the down projection's fp32 rows stored as
+// fp16 values with one power-of-two scale per 32-column block of a row,
+// value = y16 * 2^e.  For a block whose largest magnitude is M * 2^E (M in
+// [1, 2)), e = E - 14, so the scaled block lies within 2^15 and fp16 keeps a
+// relative error of at most 2^-11 on every value down to 2^-29 of the
+// block's largest (below that, an absolute error under 2^-40 of it).  Half
+// the bytes of fp32 rows; the combine undoes the scale.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int y16_exponent(float m) {
+  if (!(m > 0.0f) || !(m <= 3.4028234e38f)) return 0;  // zero or non-finite block
+  int e2;
+  frexpf(m, &e2);  // m = f * 2^e2 with f in [0.5, 1): E = e2 - 1
+  const int e = (e2 - 1) - 14;
+  return e < -120 ? -120 : (e > 120 ? 120 : e);
+}
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
+
+// One warp, lane = row: its row's 32 values v (columns col .. col+31 of rows
+// row0 + lane) into y16 rows of N columns and their block exponents
+// (nblk = ceil(N / 32) per row), through the warp's staging buffer st (32
+// rows of row_words words); rows from row_end on are not written.
+__device__ __forceinline__ void store_y16_lane_rows(const float (&v)[32], uint32_t *st,
+                                                    int row_words, int lane, int row0,
+                                                    int row_end, int col, int N, void *out,
+                                                    int8_t *yexp, int nblk) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+  const int e = y16_exponent(m);
+  const float inv = pow2f(-e);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h2 = __floats2half2_rn(v[q * 8 + 2 * i] * inv, v[q * 8 + 2 * i + 1] * inv);
+      w[i] = *reinterpret_cast<uint32_t *>(&h2);
+    }
+    *reinterpret_cast<uint4 *>(st + lane * row_words + 4 * q) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (row0 + lane < row_end && col < N) yexp[(size_t)(row0 + lane) * nblk + col / 32] = (int8_t)e;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // 8 rows x 64 bytes per instruction
+    const int r = i * 8 + (lane >> 2), q = lane & 3;
+    const int grow = row0 + r, gcol = col + q * 8;
+    const uint4 val = *reinterpret_cast<const uint4 *>(st + r * row_words + 4 * q);
+    if (grow < row_end && gcol < N)
+      *reinterpret_cast<uint4 *>(static_cast<__half *>(out) + (size_t)grow * N + gcol) = val;
+  }
+}
+
+// One warp, rows staged transposed (stg[j * row_words + c] = value of row j,
+// column col0 + c): rows j < nr of rows row0 .. into y16 rows and their block
+// exponents; 8 lanes per row, 4 columns each.  wr: per-row factor source
+// (row_w[w_row_src[row]]) or nullptr.
+__device__ __forceinline__ void store_y16_staged(const float *stg, int row_words, int lane,
+                                                 int row0, int nr, int col0, int N, void *out,
+                                                 int8_t *yexp, int nblk, const float *row_w,
+                                                 const int32_t *w_row_src) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {  // 4 rows per step
+    const int j = i * 4 + (lane >> 3), q = lane & 7;
+    const int grow = row0 + j, gcol = col0 + q * 4;
+    const bool live = j < nr;
+    float4 f = *reinterpret_cast<const float4 *>(stg + j * row_words + 4 * q);
+    if (live && row_w) {
+      const float wr = row_w[w_row_src[grow]];
+      f.x *= wr;
+      f.y *= wr;
+      f.z *= wr;
+      f.w *= wr;
+    }
+    float m = fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w)));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    const int e = y16_exponent(m);
+    const float inv = pow2f(-e);
+    if (live && gcol < N) {
+      __half2 lo = __floats2half2_rn(f.x * inv, f.y * inv);
+      __half2 hi = __floats2half2_rn(f.z * inv, f.w * inv);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t *>(&lo);
+      w.y = *reinterpret_cast<uint32_t *>(&hi);
+      *reinterpret_cast<uint2 *>(static_cast<__half *>(out) + (size_t)grow * N + gcol) = w;
+      if (q == 0) yexp[(size_t)grow * nblk + col0 / 32] = (int8_t)e;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -302,7 +302,7 @@ def test_sigmoid_grouped_near_ties_bit_exact(T, E, dev):
 # ---------------------------------------------------------------------------
 # Every grouped-GEMM engine (single-CTA, CTA-pair and swap-AB tiles) on every shape
 # ---------------------------------------------------------------------------
-@pytest.fixture(params=["single", "narrow", "pair", "swap"])
+@pytest.fixture(params=["single", "narrow", "pair", "swap", "mixed"])
 def gemm_engine(request):
     import os
     old = os.environ.get("MOE_GEMM_ENGINE")
@@ -331,6 +331,50 @@ def test_layer_each_engine(name, gemm_engine, dev):
 def test_tile_row_edges(T, gemm_engine, dev):
     w = SMALL["mixtral_small"].scaled(T=T)
     _layer_vs_oracle(w, _host_inputs(w, seed=T), dev)
+
+
+# group sizes around every tile edge: empty, a few rows, the 16-row steps of a
+# swap-AB tile, the 32-row boxes, full 128-row chunks with and without a
+# remainder
+GROUP_SIZES = [0, 1, 15, 16, 17, 31, 33, 127, 128, 129, 0, 255, 256, 300, 5]
+
+
+def test_expert_ffn_group_size_edges(gemm_engine, dev):
+    """moe_expert_ffn on hand-made expert groups (ragged K and N), every engine."""
+    E, d, f = len(GROUP_SIZES), 200, 200
+    offsets = np.concatenate([[0], np.cumsum(GROUP_SIZES)]).astype(np.int32)
+    R = int(offsets[-1])
+    w = WORKLOADS["qwen3_prefill"].scaled(T=R, d=d, E=E, k_max=1, f=f)
+    cfg = ops.config(w)
+    hin = _host_inputs(w, seed=5)
+    xp = torch.randn(R, d, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    y = torch.zeros((R, d), dtype=torch.float32, device=dev)
+    ops.moe_expert_ffn(cfg, xp.to(dev), torch.from_numpy(offsets).to(dev), hin["W1"].to(dev),
+                       hin["W3"].to(dev), hin["W2"].to(dev), y,
+                       ops.workspace(cfg, ops.WS_EXPERT_FFN))
+    ops.moe_check_errors()
+    ref = oracle.grouped_ffn(to_numpy(xp), offsets, to_numpy(hin["W1"]), to_numpy(hin["W3"]),
+                             to_numpy(hin["W2"]))
+    assert_out_close(f64(y), ref, "y_perm, group sizes across tile edges", "f32")
+
+
+@pytest.fixture
+def fp32_expert_rows():
+    """MOE_Y16=0: the down projection writes fp32 rows instead of the compact
+    y16 form (fp16 values with a power-of-two exponent per 32-column block)."""
+    import os
+    old = os.environ.get("MOE_Y16")
+    os.environ["MOE_Y16"] = "0"
+    yield
+    if old is None:
+        os.environ.pop("MOE_Y16", None)
+    else:
+        os.environ["MOE_Y16"] = old
+
+
+@pytest.mark.parametrize("name", BF16_SMALL)
+def test_layer_with_fp32_expert_rows(name, fp32_expert_rows, dev):
+    test_layer_matches_oracle(name, dev)
 
 
 @pytest.fixture
