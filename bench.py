@@ -259,6 +259,10 @@ def algorithmic(w, R: int, touched: int, fp8: bool = False) -> dict:
     ws = 1 if fp8 else s                              # bytes per expert weight
     sc = 4 if fp8 else 0                              # bytes per column scale
     hs = s                                            # h: bf16 (or fp32 for fp32 layers)
+    # expert output rows between the down projection and the combine: fp32,
+    # or (bf16 layers, bf16 weights) the compact y16 form -- fp16 values and
+    # one exponent byte per 32-column block
+    ys = w.d * 2 + (w.d + 31) // 32 if y16_rows(w, fp8) else w.d * 4
     return {
         "layer_flops": 2 * w.T * w.d * w.E + 6 * w.d * w.f * R + 6 * w.d * w.f_shared * w.T,
         "layer_bytes": (touched * (3 * w.d * w.f * ws + (2 * w.f + w.d) * sc)
@@ -267,15 +271,24 @@ def algorithmic(w, R: int, touched: int, fp8: bool = False) -> dict:
         "up_flops": 4 * R * w.d * w.f,
         "up_bytes": touched * 2 * (w.d * w.f * ws + w.f * sc) + R * w.d * s + R * w.f * hs,
         "down_flops": 2 * R * w.f * w.d,
-        "down_bytes": touched * (w.f * w.d * ws + w.d * sc) + R * w.f * hs + R * w.d * 4,
+        "down_bytes": touched * (w.f * w.d * ws + w.d * sc) + R * w.f * hs + R * ys,
         "dispatch_bytes": 2 * R * w.d * s,
         "combine_bytes": (R + w.T) * w.d * s,
-        # what the combine actually moves: fp32 expert rows (y_perm is kept in
-        # fp32 so that the output is rounded once), the output rows, the fp32
-        # shared-expert rows, and each slot's row index and weight
-        "combine_bytes_actual": (R * w.d * 4 + w.T * w.d * s + (w.f_shared > 0) * w.T * w.d * 4
+        # what the combine actually moves: the expert rows (fp32 or y16), the
+        # output rows, the fp32 shared-expert rows, and each slot's row index
+        # and weight
+        "combine_bytes_actual": (R * ys + w.T * w.d * s + (w.f_shared > 0) * w.T * w.d * 4
                                  + w.T * w.k_max * 8),
     }
+
+
+def y16_rows(w, fp8: bool = False) -> bool:
+    """Whether moe_layer passes the routed experts' outputs to the combine in
+    the compact y16 form: bf16 layers with bf16 expert weights, unless
+    MOE_Y16=0 or the down projection is forced onto the swap-AB engine."""
+    eng = os.environ.get("MOE_GEMM_ENGINE", "")
+    return (w.dtype == "bf16" and not fp8 and not os.environ.get("MOE_Y16", "1").startswith("0")
+            and not eng.startswith("sw"))
 
 
 def profile_summary(path: str, src: str):
@@ -357,9 +370,10 @@ def stage_rooflines(w, alg: dict, stage_ms: dict, pk: dict, pk_src: str, clocks:
     act = alg["combine_bytes_actual"] / (stage_ms["combine"] * 1e-3) / 1e9
     comb["actual_bytes_per_launch"] = alg["combine_bytes_actual"]
     comb["frac_on_actual_bytes"] = round(act / pk["hbm_gbs"], 4)
-    comb["note"] = ("bytes per the layer definition, (R+T) rows in the layer dtype; the kernel "
-                    "reads fp32 expert rows (the output is rounded once), so its actual "
-                    "traffic is larger: frac_on_actual_bytes")
+    comb["note"] = ("bytes per the layer definition, (R+T) rows in the layer dtype; "
+                    "frac_on_actual_bytes counts what the kernel moves: the expert rows "
+                    + ("in y16 form (fp16 + a block exponent)" if y16_rows(w) else "in fp32")
+                    + ", the output rows, the slots' rows and weights")
     out["combine"] = comb
     return out
 

@@ -72,6 +72,11 @@ struct ParamsMixed {
   uint64_t wait_limit_ns;
   int8_t *yexp;            // PLAIN: non-null -> out is y16 rows with these block exponents
   int nblk;                // exponents per row: ceil(N / 32)
+  // GATHER: row r of A is row row_src[r] / k_max (< a_count) of a_rows [a_count, K]
+  const void *a_rows;
+  const int32_t *row_src;
+  int k_max, a_count;
+  int l2_hints;  // L2 eviction hints on the TMA loads (rows kept, weights streamed)
 };
 
 // A tile of the list: group g, column tile n, and either a full chunk (rows
@@ -81,13 +86,39 @@ struct TileRef {
   bool full;
 };
 
-template <bool SWIGLU>
-__global__ void __launch_bounds__(kThreads, 1)
+// GATHER (up projection): the rows of A are token rows of x, row r being
+// x[row_src[r] / k_max] -- the dispatch copy fused into the GEMM.  Four more
+// warps (6-9) fetch them with cp.async (16 bytes per thread, 8 threads per
+// 128-byte row segment) into the 128-byte-swizzled layout the MMA reads, wait
+// for their copies, make them visible to the tensor cores (proxy fence) and
+// arrive on the stage's "full" barrier, which also counts the weights' TMA
+// bytes.  x is read from L2: it is T rows, each needed by its k_t experts.
+constexpr int kGatherLag = 2;  // stages a gather warp keeps in flight before it signals
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <bool SWIGLU, bool GATHER>
+__global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
     k_grouped_gemm_mixed(const __grid_constant__ CUtensorMap tmA,   // rows, 128-row box
                          const __grid_constant__ CUtensorMap tmX,   // rows, 32-row box
                          const __grid_constant__ CUtensorMap tmW1,  // [G, K, N]
                          const __grid_constant__ CUtensorMap tmW3, const ParamsMixed p) {
   using S = ShapeMixed<SWIGLU>;
+  constexpr int kCta = GATHER ? kThreads + 128 : kThreads;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -109,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
+      // the weights' arrive.expect_tx, plus one arrival per gather warp
+      mbar_init(full0 + 8 * s, GATHER ? 5 : 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -126,71 +158,98 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmW1);
     if (SWIGLU) prefetch_tmap(&tmW3);
   }
-  // Group table: row offsets and tile starts (chunks = ceil(rows / 128) per
-  // column tile), checked against the buffer size.
+  // Group table: row offsets, then two tile lists, each an exclusive scan of
+  // per-group tile counts:
+  //   heavy: groups of at least 128 rows -- their full chunks and remainder,
+  //          chunks fastest within a column tile (CTAs running together share
+  //          the weight tile, L2 serves all but the first read);
+  //   light: groups of 1..127 rows -- one remainder tile per column tile.
+  // The deal merges the two lists evenly (tile t is light when the count of
+  // light tiles among the first t+1 tiles, round-down of (t+1) L / total,
+  // steps up), so every wave mixes compute-bound heavy tiles with light tiles
+  // that mostly stream their group's weights, instead of running those
+  // phases one after the other.
   bool bad = false;
-  for (int g = threadIdx.x; g <= p.G; g += kThreads) {
+  for (int g = threadIdx.x; g <= p.G; g += kCta) {
     const int v = p.offsets[g];
     s_off[g] = v;
     if (v < 0 || v > p.rows_cap) bad = true;
   }
   if (warp == 1) tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
   __syncthreads();
+  int32_t *s_lstart = s_tstart + (p.G + 1);
   const int n_tiles = (p.N + S::BN - 1) / S::BN;
-  for (int g = threadIdx.x; g < p.G; g += kThreads) {
+  for (int g = threadIdx.x; g < p.G; g += kCta) {
     const int rows = s_off[g + 1] - s_off[g];
     if (rows < 0) bad = true;
-    s_tstart[g] = rows > 0 ? ((rows + BM - 1) / BM) * n_tiles : 0;
+    s_tstart[g] = rows >= BM ? ((rows + BM - 1) / BM) * n_tiles : 0;
+    s_lstart[g] = (rows > 0 && rows < BM) ? n_tiles : 0;
   }
   if (bad) {
     *abort_flag = 1;
     raise_error(p.err, kErrIndex);
   }
   __syncthreads();
-  if (warp == 0) {  // in-place exclusive scan, 32 groups per step
+  if (warp == 0 || warp == 1) {  // in-place exclusive scans, 32 groups per step
+    int32_t *sc = warp == 0 ? s_tstart : s_lstart;
     int carry = 0;
     for (int base = 0; base < p.G; base += 32) {
       const int g = base + lane;
-      const int v = g < p.G ? s_tstart[g] : 0;
+      const int v = g < p.G ? sc[g] : 0;
       int incl = v;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
       }
-      if (g < p.G) s_tstart[g] = carry + incl - v;
+      if (g < p.G) sc[g] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) s_tstart[p.G] = carry;
+    if (lane == 0) sc[p.G] = carry;
   }
   if (warp == 1) tmem_relinquish();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = *abort_flag ? 0 : s_tstart[p.G];
+  const int n_heavy = s_tstart[p.G], n_light = s_lstart[p.G];
+  const int total = *abort_flag ? 0 : n_heavy + n_light;
   const int num_kb = (p.K + BK - 1) / BK;
 
-  // tile -> (group, column tile, chunk), chunks fastest: CTAs running at the
-  // same time share a weight tile
-  auto tile_ref = [&](int tile) {
+  // largest g with start[g] <= idx (a group with tiles: an empty group shares
+  // its start with the next one)
+  auto find_group = [&](const int32_t *start, int idx) {
     int lo = 0, hi = p.G - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (s_tstart[mid] <= tile)
+      if (start[mid] <= idx)
         lo = mid;
       else
         hi = mid - 1;
     }
+    return lo;
+  };
+  auto tile_ref = [&](int tile) {
     TileRef t;
-    t.g = lo;
-    const int rows = s_off[lo + 1] - s_off[lo];
-    const int chunks = (rows + BM - 1) / BM;
-    const int local = tile - s_tstart[lo];
-    t.n = local / chunks;
-    const int m = local - t.n * chunks;
-    t.row0 = s_off[lo] + m * BM;
-    t.nr = min(BM, rows - m * BM);
+    const long long l0 = (long long)tile * n_light / total;
+    const long long l1 = (long long)(tile + 1) * n_light / total;
+    if (l1 > l0) {  // light: the whole group, column tile n
+      const int li = (int)l0;
+      t.g = find_group(s_lstart, li);
+      t.n = li - s_lstart[t.g];
+      t.row0 = s_off[t.g];
+      t.nr = s_off[t.g + 1] - s_off[t.g];
+    } else {  // heavy: chunk m of column tile n
+      const int hi = tile - (int)l0;
+      t.g = find_group(s_tstart, hi);
+      const int rows = s_off[t.g + 1] - s_off[t.g];
+      const int chunks = (rows + BM - 1) / BM;
+      const int local = hi - s_tstart[t.g];
+      t.n = local / chunks;
+      const int m = local - t.n * chunks;
+      t.row0 = s_off[t.g] + m * BM;
+      t.nr = min(BM, rows - m * BM);
+    }
     t.full = t.nr == BM;
     return t;
   };
@@ -198,13 +257,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      const uint64_t pol_keep = l2_policy_evict_last(), pol_stream = l2_policy_evict_first();
       int s = 0;
       uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileRef t = tile_ref(tile);
         const int nq = t.full ? 0 : (t.nr + 31) / 32;  // remainder: 32-row boxes
-        const uint32_t bytes = (t.full ? S::kABytes : nq * S::kRowBoxBytes) + S::kBBytes;
+        const uint32_t bytes =
+            (GATHER ? 0u : (t.full ? S::kABytes : nq * S::kRowBoxBytes)) + S::kBBytes;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
             ok = false;
@@ -213,18 +274,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = smem_addr(ring + s * S::kStageBytes);
           const uint32_t fb = full0 + 8 * s;
           mbar_expect_tx(fb, bytes);
-          if (t.full) {
-            tma_load_2d(st, &tmA, fb, kb * BK, t.row0);
+          if (GATHER) {
+            // the rows come from the gather warps
+          } else if (t.full) {
+            if (p.l2_hints)
+              tma_load_2d_hint(st, &tmA, fb, kb * BK, t.row0, pol_keep);
+            else
+              tma_load_2d(st, &tmA, fb, kb * BK, t.row0);
           } else {
-            for (int q = 0; q < nq; ++q)
-              tma_load_2d(st + q * S::kRowBoxBytes, &tmX, fb, kb * BK, t.row0 + 32 * q);
+            for (int q = 0; q < nq; ++q) {
+              if (p.l2_hints)
+                tma_load_2d_hint(st + q * S::kRowBoxBytes, &tmX, fb, kb * BK, t.row0 + 32 * q,
+                                 pol_keep);
+              else
+                tma_load_2d(st + q * S::kRowBoxBytes, &tmX, fb, kb * BK, t.row0 + 32 * q);
+            }
           }
           // weights: four 64-column spans (gate 0-1 and up 2-3, or 256 columns)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const CUtensorMap *m = (SWIGLU && j >= 2) ? &tmW3 : &tmW1;
             const int col = SWIGLU ? t.n * S::BN + (j & 1) * 64 : t.n * S::BN + j * 64;
-            tma_load_3d(st + S::kABytes + j * S::kSpanBytes, m, fb, col, kb * BK, t.g);
+            if (p.l2_hints)
+              tma_load_3d_hint(st + S::kABytes + j * S::kSpanBytes, m, fb, col, kb * BK, t.g,
+                               pol_stream);
+            else
+              tma_load_3d(st + S::kABytes + j * S::kSpanBytes, m, fb, col, kb * BK, t.g);
           }
           issued_mask |= 1u << s;
           issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
@@ -298,6 +373,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (GATHER && warp >= 6) {
+    // ------------------------------------------------------------ row gather
+    // Warp gw fetches rows 32*gw .. 32*gw+31 of the tile: instruction k moves
+    // rows 32*gw + 4k + lane/8, 16-byte chunk lane%8 of the k-block's 128-byte
+    // row segment, into slot chunk ^ (row % 8) (the 128-byte swizzle).  A
+    // stage is signalled kGatherLag stages later, once its copies have landed.
+    const int gw = warp - 6, c = lane & 7;
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(p.a_rows);
+    int s = 0, n_issued = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileRef t = tile_ref(tile);
+      int tok[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = gw * 32 + 4 * k + (lane >> 3);
+        tok[k] = -1;
+        if (i < t.nr) {
+          const int a = p.row_src[t.row0 + i];
+          const int tk = a / p.k_max;
+          if (a >= 0 && tk < p.a_count)
+            tok[k] = tk;
+          else if (c == 0)
+            raise_error(p.err, kErrIndex);
+        }
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
+        int okw = 1;
+        if (lane == 0) okw = wait(empty0 + 8 * s, ph ^ 1, ctl) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) {
+          ok = false;
+          break;
+        }
+        const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+        const int kcol = kb * BK + c * 8;  // first K element of this lane's chunk
+        const uint32_t nbytes = kcol < p.K ? 16u : 0u;  // past K: zeros
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (tok[k] < 0) continue;
+          const int i = gw * 32 + 4 * k + (lane >> 3);
+          const __nv_bfloat16 *src = x + (size_t)tok[k] * p.K + (nbytes ? kcol : 0);
+          cp_async_16(st + i * 128 + ((c ^ (i & 7)) << 4), src, nbytes);
+        }
+        cp_async_commit();
+        if (++n_issued > kGatherLag) {  // the stage issued kGatherLag stages ago
+          cp_async_wait<kGatherLag>();
+          fence_proxy_async_shared();
+          __syncwarp();
+          const int sd = (s - kGatherLag + S::kStages) % S::kStages;
+          if (lane == 0) mbar_arrive(full0 + 8 * sd);
+        }
+        if (++s == S::kStages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+    cp_async_wait<0>();  // every copy has landed before the CTA moves on
+    if (ok) {  // signal the stages still pending
+      fence_proxy_async_shared();
+      __syncwarp();
+      for (int q = (n_issued < kGatherLag ? n_issued : kGatherLag); q >= 1; --q) {
+        const int sd = (s - q + S::kStages) % S::kStages;
+        if (lane == 0) mbar_arrive(full0 + 8 * sd);
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
@@ -490,30 +633,36 @@ bool make_map_w_m(CUtensorMap *m, const void *B, int G, int K, int N) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool GATHER>
 cudaError_t launch_mixed(int rows_cap, int K, int N, int G, const int32_t *offsets,
                          const void *A, const void *B1, const void *B3, void *out,
                          const float *row_w, const int32_t *w_row_src, uint32_t *err,
-                         cudaStream_t s, int8_t *yexp) {
+                         cudaStream_t s, int8_t *yexp, const int32_t *row_src, int k_max,
+                         int a_count) {
   using S = ShapeMixed<SWIGLU>;
+  constexpr int kCta = GATHER ? kThreads + 128 : kThreads;
   CUtensorMap ma, mx, mw1, mw3;
-  if (!make_map_rows_m(&ma, A, rows_cap, K, BM) || !make_map_rows_m(&mx, A, rows_cap, K, 32) ||
+  // with GATHER the row maps are not read; they describe the token rows
+  const int map_rows = GATHER ? a_count : rows_cap;
+  if (!make_map_rows_m(&ma, A, map_rows, K, BM) || !make_map_rows_m(&mx, A, map_rows, K, 32) ||
       !make_map_w_m(&mw1, B1, G, K, N) || !make_map_w_m(&mw3, SWIGLU ? B3 : B1, G, K, N))
     return cudaErrorInvalidValue;
-  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
+  // group tables: row offsets, heavy and light tile starts
+  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 3 * (size_t)(G + 1);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static std::atomic<bool> attr_set[64];
-  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_mixed<SWIGLU>,
-                                    S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_mixed<SWIGLU, GATHER>,
+                                    S::kSmemFixed + sizeof(int32_t) * 3 * (kMaxGroups + 1)))
     return e;
   ParamsMixed p{offsets, G,   rows_cap, K, N, out, row_w, w_row_src, err,
-                pipeline_wait_limit_ns(), yexp, (N + 31) / 32};
+                pipeline_wait_limit_ns(), yexp, (N + 31) / 32, A, row_src, k_max, a_count,
+                l2_hints_enabled()};
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + G) *
                               ((N + S::BN - 1) / S::BN);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
-  k_grouped_gemm_mixed<SWIGLU><<<grid, kThreads, smem, s>>>(ma, mx, mw1, mw3, p);
+  k_grouped_gemm_mixed<SWIGLU, GATHER><<<grid, kCta, smem, s>>>(ma, mx, mw1, mw3, p);
   return cudaGetLastError();
 }
 
@@ -524,14 +673,19 @@ cudaError_t launch_grouped_gemm_mixed(bool swiglu, int rows_cap, int K, int N, i
                                       const int32_t *offsets, const void *A, const void *B1,
                                       const void *B3, void *out, uint32_t *err, cudaStream_t s,
                                       const float *row_w, const int32_t *w_row_src,
-                                      int8_t *yexp) {
+                                      int8_t *yexp, const int32_t *row_src, int k_max,
+                                      int a_rows) {
   if (rows_cap <= 0) return cudaSuccess;
   if (!offsets || G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if ((row_w || yexp) && swiglu) return cudaErrorInvalidValue;  // down projection only
-  return swiglu ? tc::launch_mixed<true>(rows_cap, K, N, G, offsets, A, B1, B3, out, nullptr,
-                                         nullptr, err, s, nullptr)
-                : tc::launch_mixed<false>(rows_cap, K, N, G, offsets, A, B1, B1, out, row_w,
-                                          w_row_src, err, s, yexp);
+  if (row_src && (!swiglu || k_max < 1 || a_rows < 1)) return cudaErrorInvalidValue;
+  if (row_src)
+    return tc::launch_mixed<true, true>(rows_cap, K, N, G, offsets, A, B1, B3, out, nullptr,
+                                        nullptr, err, s, nullptr, row_src, k_max, a_rows);
+  return swiglu ? tc::launch_mixed<true, false>(rows_cap, K, N, G, offsets, A, B1, B3, out,
+                                                nullptr, nullptr, err, s, nullptr, nullptr, 1, 0)
+                : tc::launch_mixed<false, false>(rows_cap, K, N, G, offsets, A, B1, B1, out, row_w,
+                                                 w_row_src, err, s, yexp, nullptr, 1, 0);
 }
 
 }  // namespace moe

@@ -99,6 +99,8 @@ struct Params {
   // y16 form of the rows, with nblk = ceil(N / 32) block exponents per row
   int8_t *yexp = nullptr;
   int nblk = 0;
+  // L2 eviction hints on the TMA loads (bf16 single-CTA and pair engines)
+  int l2_hints = 0;
 };
 
 // Gate weights to apply in the down projection's epilogue (both nullptr: none).
@@ -390,6 +392,7 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
     const bool codes = FP8W && warp == 0;
     const bool load_a = !FP8W || warp == 10;
     const bool gather = p.row_src != nullptr;
+    const uint64_t pol_keep = l2_policy_evict_last(), pol_stream = l2_policy_evict_first();
     const int nst = codes ? S::kQStages : S::kStages;
     const uint32_t fullb = codes ? qfull0 : full0, emptyb = codes ? qempty0 : empty0;
     int s = 0;
@@ -432,17 +435,22 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
           if (gather)
             tma_gather4(st + lane * 4 * 128, &tmA, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
           if (lane == 0) {
-            if (!gather && load_a) tma_load_2d(st, &tmA, fb, k0 + kb * BK, row);
+            if (!gather && load_a) {
+              if (p.l2_hints)
+                tma_load_2d_hint(st, &tmA, fb, k0 + kb * BK, row, pol_keep);
+              else
+                tma_load_2d(st, &tmA, fb, k0 + kb * BK, row);
+            }
             if (!FP8W) {
 #pragma unroll
-              for (int j = 0; j < S::kSpans; ++j)
-                tma_load_3d(st + S::kABytes + j * S::kSpanBytes, &tmB1, fb, n * S::BN + j * 64,
-                            k0 + kb * BK, gb);
-              if (SWIGLU) {
-#pragma unroll
-                for (int j = 0; j < S::kSpans; ++j)
-                  tma_load_3d(st + S::kABytes + (S::kSpans + j) * S::kSpanBytes, &tmB3, fb,
-                              n * S::BN + j * 64, k0 + kb * BK, gb);
+              for (int j = 0; j < S::kSpans * S::kBOps; ++j) {
+                const CUtensorMap *mb = (SWIGLU && j >= S::kSpans) ? &tmB3 : &tmB1;
+                const int col = n * S::BN + (j % S::kSpans) * 64;
+                if (p.l2_hints)
+                  tma_load_3d_hint(st + S::kABytes + j * S::kSpanBytes, mb, fb, col,
+                                   k0 + kb * BK, gb, pol_stream);
+                else
+                  tma_load_3d(st + S::kABytes + j * S::kSpanBytes, mb, fb, col, k0 + kb * BK, gb);
               }
             }
           }
@@ -715,6 +723,24 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(leader_bar)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap *map,
+                                                      uint32_t leader_bar, int c0, int c1,
+                                                      uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(leader_bar), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair_hint(uint32_t dst, const CUtensorMap *map,
+                                                      uint32_t leader_bar, int c0, int c1, int c2,
+                                                      uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(leader_bar), "l"(pol)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    slot_smem),
@@ -871,6 +897,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producers (both CTAs)
     if (lane == 0) {
+      const uint64_t pol_keep = l2_policy_evict_last(), pol_stream = l2_policy_evict_first();
       int s = 0;
       uint32_t ph = 0;
       int issued = 0;
@@ -898,18 +925,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t st = smem_addr(ring + s * S::kStageBytes);
           const uint32_t lfb = leader_full0 + 8 * s;
           if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * S::kStageBytes);
-          tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
-          if (SWIGLU) {
-            const CUtensorMap *mb = rank == 0 ? &tmB1 : &tmB3;
+          const CUtensorMap *mb = (SWIGLU && rank == 1) ? &tmB3 : &tmB1;
+          const int bcol = SWIGLU ? n * S::BN : n * S::BN + (int)rank * 128;
+          if (p.l2_hints) {
+            tma_load_2d_pair_hint(st, &tmA, lfb, kb * BK, row, pol_keep);
 #pragma unroll
             for (int j = 0; j < 2; ++j)
-              tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb,
-                               n * S::BN + j * 64, kb * BK, g);
+              tma_load_3d_pair_hint(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
+                                    kb * BK, g, pol_stream);
           } else {
+            tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
 #pragma unroll
             for (int j = 0; j < 2; ++j)
-              tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, &tmB1, lfb,
-                               n * S::BN + (int)rank * 128 + j * 64, kb * BK, g);
+              tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
+                               kb * BK, g);
           }
           ++issued;
           if (++s == S::kStages) {
@@ -1704,6 +1733,7 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
   p.w_row_src = rw.row_src;
   p.yexp = yexp;
   p.nblk = (N + 31) / 32;
+  p.l2_hints = l2_hints_enabled();
   // never more CTAs than tiles can exist (a group holds at most rows_cap rows)
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
@@ -1735,6 +1765,7 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   p.w_row_src = rw.row_src;
   p.yexp = yexp;
   p.nblk = (N + 31) / 32;
+  p.l2_hints = l2_hints_enabled();
   const long long max_tiles = (long long)((rows_cap + BM2 - 1) / BM2 + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
   long long pairs = sms / 2;
@@ -1859,7 +1890,8 @@ bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *of
                              int fixed_rows) {
   if (!swiglu) return false;
   const Engine e = pick_engine(swiglu, rows_cap, G, offsets, fixed_rows, 0);
-  return e == Engine::kSingle || e == Engine::kNarrow || e == Engine::kSwap;
+  return e == Engine::kSingle || e == Engine::kNarrow || e == Engine::kSwap ||
+         e == Engine::kMixed;
 }
 
 bool grouped_gemm_y16_out(int rows_cap, int G, const int32_t *offsets, int fixed_rows, int N) {
@@ -1875,8 +1907,7 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
   if (G <= 0 || G > tc::kMaxGroups) return cudaErrorInvalidValue;
   if (rows_cap == 0) return cudaSuccess;
   const Engine e = pick_engine(swiglu, rows_cap, G, offsets, fixed_rows, N);
-  if (row_src && (!swiglu || e == Engine::kPair || e == Engine::kMixed))
-    return cudaErrorInvalidValue;
+  if (row_src && (!swiglu || e == Engine::kPair)) return cudaErrorInvalidValue;
   if (yexp && (swiglu || e == Engine::kSwap)) return cudaErrorInvalidValue;
   if (row_w && swiglu) return cudaErrorInvalidValue;  // gate weights: the down projection only
   tc::RowWeights rw;
@@ -1885,7 +1916,7 @@ cudaError_t launch_grouped_gemm_bf16(bool swiglu, int rows_cap, int K, int N, in
   switch (e) {
     case Engine::kMixed:
       return launch_grouped_gemm_mixed(swiglu, rows_cap, K, N, G, offsets, A, B1, B3, out, err,
-                                       s, row_w, w_row_src, yexp);
+                                       s, row_w, w_row_src, yexp, row_src, k_max, a_rows);
     case Engine::kPair:
       return swiglu ? tc::launch_pair<true>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3,
                                             out, err, s)

@@ -122,12 +122,16 @@ cudaError_t launch_grouped_gemm_fp8(bool swiglu, int rows_cap, int K, int N, int
 // yexp (plain only): when given, out receives the compact y16 form of the
 // fp32 rows (fp16 values, one power-of-two exponent per 32-column block in
 // yexp [rows_cap, ceil(N / 32)]; see tcgen05_common.cuh).
+// row_src (swiglu only): row r of A is row row_src[r] / k_max of A itself
+// ([a_rows, K], the token rows), fetched with cp.async by the kernel -- the
+// dispatch copy fused into the up projection.
 cudaError_t launch_grouped_gemm_mixed(bool swiglu, int rows_cap, int K, int N, int G,
                                       const int32_t *offsets, const void *A, const void *B1,
                                       const void *B3, void *out, uint32_t *err, cudaStream_t s,
                                       const float *row_w = nullptr,
                                       const int32_t *w_row_src = nullptr,
-                                      int8_t *yexp = nullptr);
+                                      int8_t *yexp = nullptr, const int32_t *row_src = nullptr,
+                                      int k_max = 1, int a_rows = 0);
 
 // K5/K6 with fp8 weights on tcgen05.mma kind::f8f6f4 (grouped_gemm_f8.cu):
 // decode-sized routed groups.  The activations come as two e4m3 planes with a

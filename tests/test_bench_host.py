@@ -153,11 +153,18 @@ def test_frac_at_sampled_clock_scales_the_compute_peak_only():
     assert "frac_at_sampled_clock" not in h  # HBM bandwidth does not follow the SM clock
 
 
-def test_combine_reports_both_byte_counts():
+def test_combine_reports_both_byte_counts(monkeypatch):
     w = WORKLOADS["mixtral_prefill"]
     alg = bench.algorithmic(w, R=16384, touched=8)
     assert alg["combine_bytes"] == (16384 + 8192) * 4096 * 2
-    assert alg["combine_bytes_actual"] == 16384 * 4096 * 4 + 8192 * 4096 * 2 + 8192 * 2 * 8
+    # y16 rows: fp16 values plus one exponent byte per 32 columns
+    assert alg["combine_bytes_actual"] == (16384 * (4096 * 2 + 128) + 8192 * 4096 * 2
+                                           + 8192 * 2 * 8)
+    monkeypatch.setenv("MOE_Y16", "0")  # fp32 rows
+    a32 = bench.algorithmic(w, R=16384, touched=8)
+    assert a32["combine_bytes_actual"] == 16384 * 4096 * 4 + 8192 * 4096 * 2 + 8192 * 2 * 8
+    assert a32["down_bytes"] - alg["down_bytes"] == 16384 * (4096 * 2 - 128)
+    monkeypatch.delenv("MOE_Y16")
     k = bench.stage_rooflines(w, alg, STAGES_MS, PEAKS, "measured", {}, "x", 74.5,
                               profiled=False)
     c = k["combine"]
