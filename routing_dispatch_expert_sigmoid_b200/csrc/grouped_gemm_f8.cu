@@ -85,6 +85,17 @@ __host__ __device__ constexpr uint32_t instr_desc_f8(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Bring a tile of the codes into L2 ahead of its TMA load (no shared memory,
+// no completion to wait for): a decode-sized layer streams every weight once,
+// and with only a few stages of shared memory per SM the HBM latency, not
+// its bandwidth, would set the pace.
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem], e4m3 inputs, fp32 accumulation.
 __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                         uint32_t idesc, uint32_t accumulate) {
@@ -107,6 +118,7 @@ struct ParamsF8 {
   const int32_t *w_row_src;
   uint32_t *err;
   uint64_t wait_limit_ns;
+  int prefetch;  // k-blocks of codes prefetched into L2 ahead of their loads (0: none)
 };
 
 template <bool SWIGLU>
@@ -235,6 +247,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t st = smem_addr(ring + s * S::kStageBytes);
           const uint32_t fb = full0 + 8 * s;
+          if (p.prefetch > 0) {  // the k-block p.prefetch ahead (the first ones too)
+            for (int q = kb == 0 ? 0 : p.prefetch; q <= p.prefetch; ++q) {
+              const int kq = kb + q;
+              if (kq >= num_kb) break;
+              tma_prefetch_3d(&tmW1, kq * kQK, col_a, g);
+              tma_prefetch_3d(SWIGLU ? &tmW3 : &tmW1, kq * kQK, col_b, g);
+            }
+          }
           mbar_expect_tx(fb, bytes);
           // codes [G, N, K]: coordinates (k, n, group)
           tma_load_3d(st, &tmW1, fb, kb * kQK, col_a, g);
@@ -558,8 +578,9 @@ cudaError_t launch_f8(int rows_cap, int K, int N, int G, const int32_t *offsets,
   if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_f8<SWIGLU>,
                                     S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
     return e;
+  const char *pf = getenv("MOE_F8_PREFETCH");
   ParamsF8 p{offsets, G, rows_cap, K, N, out, s1, SWIGLU ? s3 : nullptr, row_scale,
-             row_w, w_row_src, err, pipeline_wait_limit_ns()};
+             row_w, w_row_src, err, pipeline_wait_limit_ns(), pf ? atoi(pf) : 0};
   const long long max_tiles = (long long)((rows_cap + kQRows - 1) / kQRows + G) *
                               ((N + S::kTileCols - 1) / S::kTileCols);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);

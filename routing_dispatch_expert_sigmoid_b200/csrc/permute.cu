@@ -213,10 +213,12 @@ __global__ void __launch_bounds__(256)
 
 // The same combine on y16 rows (fp16 values, one power-of-two exponent per
 // 32-column block, written by the down projection): value = y16 * 2^e.  The
-// bf16 output vector of lane l spans 8 columns of one block, so each slot
+// bf16 output vector of a lane spans 8 columns of one block, so each slot
 // costs one 16-byte load and one exponent byte; the exponent is folded into
-// the slot's weight (w * 2^e is exact).
-template <int KB>
+// the slot's weight (w * 2^e is exact).  A lane owns VPL output vectors
+// (work items of 32 VPL vectors), so that a top-2 layer still has a few
+// loads in flight per lane.
+template <int KB, int VPL>
 __global__ void __launch_bounds__(256)
     k_combine_y16(const uint4 *__restrict__ y, const int8_t *__restrict__ yexp, int nblk,
                   const int32_t *__restrict__ slot_row, const float *__restrict__ topk_w,
@@ -225,7 +227,8 @@ __global__ void __launch_bounds__(256)
   __shared__ int32_t s_row[8][32];
   __shared__ float s_w[8][32];
   const int lane = threadIdx.x % 32, wib = threadIdx.x / 32;
-  const int chunks = (row_vecs + 31) / 32;
+  constexpr int kItemVecs = 32 * VPL;
+  const int chunks = (row_vecs + kItemVecs - 1) / kItemVecs;
   const long long items = (long long)Tn * chunks;
   const long long warps = (long long)gridDim.x * (blockDim.x / 32);
   const size_t sh_vecs = (size_t)row_vecs * 2;  // fp32 vectors per shared row
@@ -258,54 +261,65 @@ __global__ void __launch_bounds__(256)
       s_w[wib][pos] = my_w;
     }
     __syncwarp();
-    const int v = ch * 32 + lane;
-    if (v < row_vecs) {
-      float acc[8];
-      if (shared_y) {
+    const int v0 = ch * kItemVecs + lane;  // this lane's vectors: v0 + 32 i
+    float acc[VPL][8];
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-          Vec<float>::load(ldg_nc(shared_y + (size_t)t * sh_vecs + (size_t)v * 2 + q),
-                           acc + 4 * q);
-        for (int sp = 1; sp < shared_parts; ++sp) {  // further partial sums, in order
+    for (int i = 0; i < VPL; ++i) {
+      const int v = v0 + 32 * i;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[i][q] = 0.f;
+      if (shared_y && v < row_vecs) {
+        for (int sp = 0; sp < shared_parts; ++sp) {  // partial sums, in order
           const uint4 *part = shared_y + (size_t)sp * Tn * sh_vecs + (size_t)t * sh_vecs;
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             float f[4];
             Vec<float>::load(ldg_nc(part + (size_t)v * 2 + q), f);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[4 * q + i] += f[i];
+            for (int c = 0; c < 4; ++c) acc[i][4 * q + c] += f[c];
           }
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
       }
-      const int blk = v >> 2;  // 8 columns per vector, 32 per exponent
-      for (int j0 = 0; j0 < n_live; j0 += KB) {
-        uint4 u[KB];
-        int e[KB];
+    }
+    for (int j0 = 0; j0 < n_live; j0 += KB) {
+      uint4 u[KB][VPL];
+      int e[KB][VPL];
 #pragma unroll
-        for (int j = 0; j < KB; ++j)  // issue the loads before the FMAs
-          if (j0 + j < n_live) {
-            const int r = s_row[wib][j0 + j];
-            u[j] = ldg_nc(y + (size_t)r * row_vecs + v);
-            e[j] = __ldg(yexp + (size_t)r * nblk + blk);
+      for (int j = 0; j < KB; ++j)  // issue the loads before the FMAs
+        if (j0 + j < n_live) {
+          const int r = s_row[wib][j0 + j];
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) {
+            const int v = v0 + 32 * i;
+            if (v < row_vecs) {
+              u[j][i] = ldg_nc(y + (size_t)r * row_vecs + v);
+              e[j][i] = __ldg(yexp + (size_t)r * nblk + (v >> 2));  // 8 columns per vector
+            }
           }
+        }
 #pragma unroll
-        for (int j = 0; j < KB; ++j) {
-          if (j0 + j < n_live) {
-            const float wj = s_w[wib][j0 + j] * __int_as_float((e[j] + 127) << 23);
-            const uint32_t hw[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+      for (int j = 0; j < KB; ++j) {
+        if (j0 + j < n_live) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[i]));
-              acc[2 * i] = fmaf(wj, f.x, acc[2 * i]);
-              acc[2 * i + 1] = fmaf(wj, f.y, acc[2 * i + 1]);
+          for (int i = 0; i < VPL; ++i) {
+            if (v0 + 32 * i < row_vecs) {
+              const float wj = s_w[wib][j0 + j] * __int_as_float((e[j][i] + 127) << 23);
+              const uint32_t hw[4] = {u[j][i].x, u[j][i].y, u[j][i].z, u[j][i].w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[q]));
+                acc[i][2 * q] = fmaf(wj, f.x, acc[i][2 * q]);
+                acc[i][2 * q + 1] = fmaf(wj, f.y, acc[i][2 * q + 1]);
+              }
             }
           }
         }
       }
-      out[(size_t)t * row_vecs + v] = Vec<__nv_bfloat16>::store(acc);
+    }
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int v = v0 + 32 * i;
+      if (v < row_vecs) out[(size_t)t * row_vecs + v] = Vec<__nv_bfloat16>::store(acc[i]);
     }
     __syncwarp();
   }
@@ -384,15 +398,17 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
     const auto *sh = static_cast<const uint4 *>(shared_y);
     auto *o = static_cast<uint4 *>(out);
     const int nblk = (c.d + 31) / 32, rows_cap = c.T * c.k_max;
-    if (c.k_max <= 2)
-      k_combine_y16<2><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o,
-                                            c.T, c.k_max, rows_cap, row_vecs, err);
-    else if (c.k_max <= 4)
-      k_combine_y16<4><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o,
-                                            c.T, c.k_max, rows_cap, row_vecs, err);
-    else
-      k_combine_y16<8><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o,
-                                            c.T, c.k_max, rows_cap, row_vecs, err);
+    if (c.k_max <= 2) {  // two vectors per lane: items of 64 vectors
+      const int g2 = grid_for((long long)c.T * ((row_vecs + 63) / 64));
+      k_combine_y16<2, 2><<<g2, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o,
+                                             c.T, c.k_max, rows_cap, row_vecs, err);
+    } else if (c.k_max <= 4) {
+      k_combine_y16<4, 1><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts,
+                                               o, c.T, c.k_max, rows_cap, row_vecs, err);
+    } else {
+      k_combine_y16<8, 1><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts,
+                                               o, c.T, c.k_max, rows_cap, row_vecs, err);
+    }
     return cudaGetLastError();
   }
   if (c.dtype == MOE_F32)
