@@ -379,10 +379,12 @@ def stage_rooflines(w, alg: dict, stage_ms: dict, pk: dict, pk_src: str, clocks:
 
 
 class Layer:
-    def __init__(self, name: str, dev, seed: int, T: int = 0, fp8: bool = False):
+    def __init__(self, name: str, dev, seed: int, T: int = 0, fp8: bool = False, E: int = 0):
         from routing_dispatch_expert_sigmoid_b200 import ops
         self.ops = ops
         self.w = WORKLOADS[name] if T <= 0 else WORKLOADS[name].scaled(T=T)
+        if E > 0:
+            self.w = self.w.scaled(E=E)
         self.inp = make_inputs(self.w, seed, device=dev)
         self.cfg = ops.config(self.w)
         self.ws = ops.workspace(self.cfg, ops.WS_LAYER, device=dev)
@@ -584,9 +586,9 @@ def describe(w) -> str:
 
 def measure_leg(name: str, steps: int, warmup: int, dist, local_rank: int, dev, pk: dict,
                 pk_src: str, sms: int, T: int = 0, fp8: bool = False, e2e: bool = False,
-                profiled: bool = True) -> tuple[dict, dict]:
+                profiled: bool = True, E: int = 0) -> tuple[dict, dict]:
     """Time one workload; returns (the leg's JSON object, raw numbers)."""
-    layer = Layer(name, dev, seed=int(os.environ.get("RANK", "0")), T=T, fp8=fp8)
+    layer = Layer(name, dev, seed=int(os.environ.get("RANK", "0")), T=T, fp8=fp8, E=E)
     w = layer.w
     r = run_device(layer, steps, warmup, dist, local_rank)
     e2e_r = run_e2e(layer, steps, warmup, dist) if e2e else None
@@ -595,7 +597,7 @@ def measure_leg(name: str, steps: int, warmup: int, dist, local_rank: int, dev, 
     clocks = r["clocks"]
     alu = alu_peak_tflops(sms, clocks.get("sm_max_mhz") or 1965.0)
     kern = stage_rooflines(w, alg, r["stage_ms"], pk, pk_src, clocks,
-                           w.name + ("_fp8" if fp8 else ""), alu, profiled and T <= 0)
+                           w.name + ("_fp8" if fp8 else ""), alu, profiled and T <= 0 and E <= 0)
     roof_ms = layer_roofline_ms(alg, pk)
     step_ms = ms_max / steps
     obj = {
@@ -638,6 +640,8 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=sorted(WORKLOADS),
                     help="workload of the main (prefill) leg")
     ap.add_argument("--T", type=int, default=0, help="override the main leg's token count")
+    ap.add_argument("--E", type=int, default=0,
+                    help="override the main leg's expert count (a smaller case for profiling)")
     ap.add_argument("--decode-workload", default=DECODE,
                     choices=sorted(WORKLOADS) + ["none"], help="workload of the decode leg")
     ap.add_argument("--fp8-workload", default=DECODE, choices=sorted(WORKLOADS) + ["none"],
@@ -681,7 +685,8 @@ def main():
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     leg = dict(dist=dist, local_rank=local_rank, dev=dev, pk=pk, pk_src=pk_src, sms=sms)
 
-    main_obj, main_raw = measure_leg(a.workload, a.steps, warmup, T=a.T, e2e=not a.no_e2e, **leg)
+    main_obj, main_raw = measure_leg(a.workload, a.steps, warmup, T=a.T, E=a.E,
+                                     e2e=not a.no_e2e, **leg)
     w = main_raw["w"]
     dec_obj = None
     if a.decode_workload != "none":

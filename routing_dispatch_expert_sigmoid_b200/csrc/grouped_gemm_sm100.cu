@@ -1852,22 +1852,21 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
 //           tiles and its remainder as a swap-AB tile, in one launch
 //           (grouped_gemm_mixed.cu).
 // Defaults, from B200 measurements with the engines alternated call by call
-// in one process:
+// in one process (whole layers, the same box):
 //   - decode-sized groups (at most 32 rows per group on average): swap-AB for
 //     the up projection, which loads only the valid rows (Mixtral-shaped
 //     decode: 0.298 vs 0.320 ms single-CTA), single-CTA for the down
 //     projection (CTA pairs: 0.171 vs 0.146 ms);
-//   - larger groups: CTA pairs for the up projection, and for the down
-//     projection when it is at least 4096 columns wide.  Sharing each B tile
-//     between two SMs cuts the shared-memory and L2 traffic per FLOP by a
-//     third, which under the 1 kW power cap keeps the clock up: Mixtral
-//     prefill 4.22 vs 6.31 ms, DeepSeek-V3 prefill 5.89 vs 6.36, Qwen3 up
-//     0.54 vs 0.67 ms (down, 2048 wide: 0.43 vs 0.40, single kept).  On
-//     boxes that did not reach the cap the single-CTA engine was ahead by
-//     6% on Mixtral prefill.
-//   - except for the up projection of ragged groups of at most 256 rows on
-//     average (routed experts only), where a 256-row pair tile is often
-//     half empty: mixed tiles.
+//   - every larger shape, both projections: CTA pairs.  Sharing each weight
+//     tile between two SMs halves the weight bytes each SM streams and cuts
+//     the shared-memory and L2 traffic per FLOP by a third, which under the
+//     1 kW power cap keeps the clock up.  Layer times, pair vs single vs
+//     mixed: Mixtral-shaped prefill 4.36 vs 7.47 (single) ms; Qwen3-shaped
+//     1.35 vs 1.64 vs 1.72 ms (down projection 0.39 vs 0.46 ms);
+//     DeepSeek-V3-shaped prefill 5.91 vs 6.51 vs 6.95 ms; GPT-OSS-shaped
+//     sub-experts 2.58 vs 2.85 vs 2.78 ms -- even the ragged layers, whose
+//     small groups leave a 256-row pair tile mostly empty, gain more from the
+//     halved per-SM weight stream than they lose in padding.
 // MOE_GEMM_ENGINE=single|narrow|pair|swap|mixed selects one engine for every
 // GEMM (mixed: for routed groups; a single group of rows runs single-CTA).
 enum class Engine { kSingle, kNarrow, kPair, kSwap, kMixed };
@@ -1882,8 +1881,7 @@ static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offse
   if (env && env[0] == 'm') return offsets ? Engine::kMixed : Engine::kSingle;
   const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
   if (mean_rows <= 32) return swiglu ? Engine::kSwap : Engine::kSingle;
-  if (swiglu) return (offsets && mean_rows <= 256) ? Engine::kMixed : Engine::kPair;
-  return N >= 4096 ? Engine::kPair : Engine::kSingle;
+  return Engine::kPair;
 }
 
 bool grouped_gemm_can_gather(bool swiglu, int rows_cap, int G, const int32_t *offsets,

@@ -137,11 +137,15 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(pol)
       : "memory");
 }
-// Whether the GEMMs give their TMA loads L2 eviction hints: MOE_L2_HINTS=0
-// turns them off (read at every launch).
+// Whether the GEMMs give their TMA loads L2 eviction hints: MOE_L2_HINTS=1
+// turns them on (read at every launch).  Off by default: on B200, alternated
+// call by call, the hints made the Mixtral-shaped prefill layer 6% slower
+// (4.63 vs 4.36 ms) and the Qwen3- and GPT-OSS-shaped layers 2-3% slower;
+// streamed weights marked evict-first leave L2 before the other CTAs of the
+// same row tiles read them.
 inline int l2_hints_enabled() {
   const char *env = getenv("MOE_L2_HINTS");
-  return (env && env[0] == '0') ? 0 : 1;
+  return (env && env[0] == '1') ? 1 : 0;
 }
 
 // Four rows (r0..r3) of 64 columns starting at column c0 into 4 consecutive
