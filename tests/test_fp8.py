@@ -222,3 +222,19 @@ def test_fp8_layer_with_weights_in_gemm(name, fp8_engine, dev):
             os.environ.pop("MOE_WEIGHTS_IN_GEMM", None)
         else:
             os.environ["MOE_WEIGHTS_IN_GEMM"] = old
+
+
+@pytest.mark.parametrize("name", ["mixtral_decode_small", "f8_decode_ragged",
+                                  "f8_decode_many_experts"])
+def test_fp8_layer_with_code_prefetch(name, dev):
+    """MOE_F8_PREFETCH=3: the kind::f8f6f4 engine prefetches code tiles into L2."""
+    import os
+    old = os.environ.get("MOE_F8_PREFETCH")
+    os.environ["MOE_F8_PREFETCH"] = "3"
+    try:
+        test_fp8_layer_matches_oracle(name, "default", dev)
+    finally:
+        if old is None:
+            os.environ.pop("MOE_F8_PREFETCH", None)
+        else:
+            os.environ["MOE_F8_PREFETCH"] = old

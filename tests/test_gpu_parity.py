@@ -378,6 +378,24 @@ def test_layer_with_fp32_expert_rows(name, fp32_expert_rows, dev):
 
 
 @pytest.fixture
+def l2_hints():
+    """MOE_L2_HINTS=1: the GEMMs' TMA loads carry L2 eviction hints."""
+    import os
+    old = os.environ.get("MOE_L2_HINTS")
+    os.environ["MOE_L2_HINTS"] = "1"
+    yield
+    if old is None:
+        os.environ.pop("MOE_L2_HINTS", None)
+    else:
+        os.environ["MOE_L2_HINTS"] = old
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "qwen3_medium", "dsv3_medium", "gptoss_small"])
+def test_layer_with_l2_hints(name, l2_hints, gemm_engine, dev):
+    test_layer_matches_oracle(name, dev)
+
+
+@pytest.fixture
 def fused_dispatch():
     import os
     old = os.environ.get("MOE_FUSED_DISPATCH")
