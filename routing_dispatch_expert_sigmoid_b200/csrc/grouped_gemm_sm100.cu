@@ -101,6 +101,8 @@ struct Params {
   int nblk = 0;
   // L2 eviction hints on the TMA loads (bf16 single-CTA and pair engines)
   int l2_hints = 0;
+  // pair engine: a group's last, partial 256-row chunk runs swap-AB
+  int pair_swap = 0;
 };
 
 // Gate weights to apply in the down projection's epilogue (both nullptr: none).
@@ -779,6 +781,17 @@ __device__ __forceinline__ void umma_commit_pair_self(uint32_t bar) {
       : "memory");
 }
 
+// kind::f16 descriptor of a swap-AB pair tile: M = 256 weight columns (128
+// per CTA, MN-major), N = the chunk's rows rounded up to 16 (K-major, N/2 of
+// them in each CTA's shared memory).
+__device__ __forceinline__ uint32_t instr_desc_pair_swap(int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(BM2 >> 4) << 24);
+}
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 template <bool SWIGLU>
 struct Shape2 {
   static constexpr int BN = SWIGLU ? 128 : 256;       // output columns per tile
@@ -802,7 +815,9 @@ template <bool SWIGLU>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB1,
-                        const __grid_constant__ CUtensorMap tmB3, const Params p) {
+                        const __grid_constant__ CUtensorMap tmB3,
+                        const __grid_constant__ CUtensorMap tmX32,
+                        const __grid_constant__ CUtensorMap tmX8, const Params p) {
   using S = Shape2<SWIGLU>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -812,6 +827,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // bars: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain[1]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S::kStages + 5);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+  // per tile parity and epilogue warp: whether its accumulator became ready
+  volatile int *s_ready = reinterpret_cast<volatile int *>(abort_flag + 1);
   float *s_epi = reinterpret_cast<float *>(ring + S::kStages * S::kStageBytes + 256);
   int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kStages * S::kStageBytes + 256 +
                                                S::kEpiBytes);
@@ -845,6 +862,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB1);
     if (SWIGLU) prefetch_tmap(&tmB3);
+    if (p.pair_swap) {
+      prefetch_tmap(&tmX32);
+      prefetch_tmap(&tmX8);
+    }
   }
   bool bad = false;
   for (int g = threadIdx.x; g <= p.G; g += kThreads) {
@@ -894,6 +915,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t leader_full0 = mapa_shared(full0, 0);
   const uint32_t leader_acce0 = mapa_shared(acce0, 0);
 
+  // tile -> group g, column tile n, 256-row chunk from row0 with nr rows;
+  // chunks fastest.  A group's last, partial chunk runs swap-AB (p.pair_swap):
+  // the weights are the MMA's M (256 columns, 128 per CTA), the chunk's rows
+  // its N, rounded up to 16, so a chunk of a few rows costs a 16-row MMA, not
+  // a 256-row one, while each CTA still streams only half of the weights.
+  struct PairTile {
+    int g, n, row0, nr;
+    bool swap;
+  };
+  auto pair_tile = [&](int tile) {
+    int lo = 0, hi = p.G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_tstart[mid] <= tile)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    PairTile t;
+    t.g = lo;
+    const int rows = s_off[lo + 1] - s_off[lo];
+    const int mt = (rows + BM2 - 1) / BM2;
+    const int local = tile - s_tstart[lo];
+    t.n = local / mt;
+    const int m = local - t.n * mt;
+    t.row0 = s_off[lo] + m * BM2;
+    t.nr = min(BM2, rows - m * BM2);
+    t.swap = p.pair_swap && t.nr < BM2;
+    return t;
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producers (both CTAs)
     if (lane == 0) {
@@ -903,20 +955,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int issued = 0;
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += npairs) {
-        int g, m, n;
-        {
-          int lo = 0, hi = p.G - 1;
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
-          }
-          g = lo;
-          const int mt = (s_off[g + 1] - s_off[g] + BM2 - 1) / BM2;
-          const int local = tile - s_tstart[g];
-          n = local / mt;
-          m = local - n * mt;
-        }
-        const int row = s_off[g] + m * BM2 + (int)rank * 128;
+        const PairTile t = pair_tile(tile);
+        const int h = t.swap ? ((t.nr + 15) & ~15) / 2 : 0;  // swap: rows of B per CTA
+        const uint32_t cta_bytes = t.swap ? (uint32_t)h * 128u + S::kBBytes : S::kStageBytes;
+        const int row = t.row0 + (int)rank * 128;  // full tile: this CTA's 128 rows of A
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
             ok = false;
@@ -924,21 +966,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           const uint32_t st = smem_addr(ring + s * S::kStageBytes);
           const uint32_t lfb = leader_full0 + 8 * s;
-          if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * S::kStageBytes);
-          const CUtensorMap *mb = (SWIGLU && rank == 1) ? &tmB3 : &tmB1;
-          const int bcol = SWIGLU ? n * S::BN : n * S::BN + (int)rank * 128;
-          if (p.l2_hints) {
-            tma_load_2d_pair_hint(st, &tmA, lfb, kb * BK, row, pol_keep);
+          if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * cta_bytes);
+          if (t.swap) {
+            // B: this CTA's h rows (32-row, then 8-row boxes); A: its 128
+            // weight columns, two 64-column spans (the up projection: gate
+            // and up of the same 64 columns, so each CTA's accumulator holds
+            // both halves of its columns' SwiGLU)
+            const int xrow = t.row0 + (int)rank * h;
+            int q = 0;
+            for (; q + 32 <= h; q += 32)
+              tma_load_2d_pair(st + q * 128, &tmX32, lfb, kb * BK, xrow + q);
+            for (; q < h; q += 8) tma_load_2d_pair(st + q * 128, &tmX8, lfb, kb * BK, xrow + q);
+            if (SWIGLU) {
+              const int col = t.n * S::BN + (int)rank * 64;
+              tma_load_3d_pair(st + S::kABytes, &tmB1, lfb, col, kb * BK, t.g);
+              tma_load_3d_pair(st + S::kABytes + S::kSpanBytes, &tmB3, lfb, col, kb * BK, t.g);
+            } else {
+              const int col = t.n * S::BN + (int)rank * 128;
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-              tma_load_3d_pair_hint(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
-                                    kb * BK, g, pol_stream);
+              for (int j = 0; j < 2; ++j)
+                tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, &tmB1, lfb, col + j * 64,
+                                 kb * BK, t.g);
+            }
           } else {
-            tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
+            const CUtensorMap *mb = (SWIGLU && rank == 1) ? &tmB3 : &tmB1;
+            const int bcol = SWIGLU ? t.n * S::BN : t.n * S::BN + (int)rank * 128;
+            if (p.l2_hints) {
+              tma_load_2d_pair_hint(st, &tmA, lfb, kb * BK, row, pol_keep);
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-              tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
-                               kb * BK, g);
+              for (int j = 0; j < 2; ++j)
+                tma_load_3d_pair_hint(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
+                                      kb * BK, t.g, pol_stream);
+            } else {
+              tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
+                                 kb * BK, t.g);
+            }
           }
           ++issued;
           if (++s == S::kStages) {
@@ -974,6 +1039,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t ph = 0, acc_ph = 0;
       bool ok = true, any = false;
       for (int tile = pair; tile < total && ok; tile += npairs) {
+        const PairTile t = pair_tile(tile);
+        const uint32_t idesc_swap = instr_desc_pair_swap((t.nr + 15) & ~15);
         if (!wait(acce0 + 8 * buf, acc_ph ^ 1, ctl)) {
           ok = false;
           break;
@@ -989,9 +1056,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t st = smem_addr(ring + s * S::kStageBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc(st + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc(st + S::kABytes + kk * 2048, S::kSpanBytes, 1024);
-            umma_pair(d_tmem, ad, bd, S::kIdesc, (kb | kk) != 0);
+            // rows: K-major; weights: MN-major 64-column spans (LBO = span stride)
+            const uint64_t rd = smem_desc(st + kk * 32, 16, 1024);
+            const uint64_t wd = smem_desc(st + S::kABytes + kk * 2048, S::kSpanBytes, 1024);
+            if (t.swap)
+              umma_pair(d_tmem, wd, rd, idesc_swap, (kb | kk) != 0);
+            else
+              umma_pair(d_tmem, rd, wd, S::kIdesc, (kb | kk) != 0);
           }
           any = true;
           umma_commit_pair_both(empty0 + 8 * s);
@@ -1013,32 +1084,117 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Warp w reads TMEM lanes 32*quarter ..  The warps of quarters q and
+    // q ^ 2 form a pair: on an up-projection swap tile one holds the gate and
+    // the other the up values of the same 32 columns, and they meet through
+    // shared memory (named barrier 1 + (q & 1)).  So that neither ever waits
+    // there for a partner that has stopped, the pair decides together, tile
+    // by tile, whether to go on.
     const int quarter = warp & 3;
-    int buf = 0;
+    const int partner = ((quarter ^ 2) < 2 ? (quarter ^ 2) + 4 : (quarter ^ 2));  // its warp
+    const int bar_id = 1 + (quarter & 1);
+    int buf = 0, it = 0;
     uint32_t acc_ph = 0;
-    for (int tile = pair; tile < total; tile += npairs) {
-      int g, m, n;
-      {
-        int lo = 0, hi = p.G - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
-        }
-        g = lo;
-        const int mt = (s_off[g + 1] - s_off[g] + BM2 - 1) / BM2;
-        const int local = tile - s_tstart[g];
-        n = local / mt;
-        m = local - n * mt;
-      }
+    float *stg = s_epi + (warp - 2) * 32 * S::kStageRowWords;
+    const float *pstg = s_epi + (partner - 2) * 32 * S::kStageRowWords;
+    for (int tile = pair; tile < total; tile += npairs, ++it) {
+      const PairTile t = pair_tile(tile);
+      const int g = t.g, n = t.n;
       int ready = 0;
       if (lane == 0) ready = wait(accf0 + 8 * buf, acc_ph, ctl) ? 1 : 0;
       ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (lane == 0) s_ready[(it & 1) * 4 + (warp - 2)] = ready;
+      named_bar_sync(bar_id, 64);
+      ready = ready && s_ready[(it & 1) * 4 + (partner - 2)];
       if (!ready) break;
       tc_fence_after();
-      const int row0 = s_off[g] + m * BM2 + (int)rank * 128 + quarter * 32;
-      const int row_end = s_off[g + 1];
       const uint32_t tb = tmem_base + buf * S::kAccCols + ((uint32_t)(quarter * 32) << 16);
-      float *stg = s_epi + (warp - 2) * 32 * S::kStageRowWords;
+      if (t.swap) {
+        // lane = weight column of this CTA's half, TMEM column = row of the chunk
+        if (SWIGLU) {
+          // lanes 0-63: gate of columns n*128 + rank*64 .. +63; lanes 64-127: up
+          const bool gate = quarter < 2;
+          const float *g_stg = gate ? stg : pstg;
+          const float *u_stg = gate ? pstg : stg;
+          const int col0 = n * S::BN + (int)rank * 64 + (quarter & 1) * 32;
+          const int jb = gate ? 0 : 16;  // the 16 rows of each chunk this warp writes
+#pragma unroll 1
+          for (int j0 = 0; j0 < t.nr; j0 += 32) {
+            float v[32];
+            tmem_ld32(tb + j0, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stg[j * S::kStageRowWords + lane] = v[j];
+            named_bar_sync(bar_id, 64);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int j = jb + i * 4 + (lane >> 3), q = lane & 7;
+              const int grow = t.row0 + j0 + j, gcol = col0 + q * 4;
+              const float4 gv =
+                  *reinterpret_cast<const float4 *>(g_stg + j * S::kStageRowWords + 4 * q);
+              const float4 uv =
+                  *reinterpret_cast<const float4 *>(u_stg + j * S::kStageRowWords + 4 * q);
+              if (j0 + j < t.nr && gcol < p.N) {
+                __nv_bfloat162 lo = __floats2bfloat162_rn((gv.x / (1.0f + __expf(-gv.x))) * uv.x,
+                                                          (gv.y / (1.0f + __expf(-gv.y))) * uv.y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn((gv.z / (1.0f + __expf(-gv.z))) * uv.z,
+                                                          (gv.w / (1.0f + __expf(-gv.w))) * uv.w);
+                uint2 w;
+                w.x = *reinterpret_cast<uint32_t *>(&lo);
+                w.y = *reinterpret_cast<uint32_t *>(&hi);
+                *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) +
+                                           (size_t)grow * p.N + gcol) = w;
+              }
+            }
+            named_bar_sync(bar_id, 64);  // both read before the next chunk is staged
+          }
+        } else {
+          const int col0 = n * S::BN + (int)rank * 128 + quarter * 32;
+#pragma unroll 1
+          for (int j0 = 0; j0 < t.nr; j0 += 32) {
+            float v[32];
+            tmem_ld32(tb + j0, v);  // v[j] = y[row j0 + j][col0 + lane]
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stg[j * S::kStageRowWords + lane] = v[j];
+            __syncwarp();
+            if (p.yexp) {
+              store_y16_staged(stg, S::kStageRowWords, lane, t.row0 + j0, t.nr - j0, col0, p.N,
+                               p.out, p.yexp, p.nblk, p.row_w, p.w_row_src);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {  // fp32 rows: 8 lanes x 16 bytes, 4 rows per step
+                const int j = i * 4 + (lane >> 3), q = lane & 7;
+                const int grow = t.row0 + j0 + j, gcol = col0 + q * 4;
+                float4 o = *reinterpret_cast<const float4 *>(stg + j * S::kStageRowWords + 4 * q);
+                if (j0 + j < t.nr && gcol < p.N) {
+                  if (p.row_w) {
+                    const float wr = p.row_w[p.w_row_src[grow]];
+                    o.x *= wr;
+                    o.y *= wr;
+                    o.z *= wr;
+                    o.w *= wr;
+                  }
+                  *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)grow * p.N +
+                                              gcol) = o;
+                }
+              }
+            }
+            __syncwarp();
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(acce0 + 8 * buf);
+          else
+            mbar_arrive_cluster(leader_acce0 + 8 * buf);
+        }
+        buf ^= 1;
+        if (buf == 0) acc_ph ^= 1;
+        continue;
+      }
+      const int row0 = t.row0 + (int)rank * 128 + quarter * 32;
+      const int row_end = s_off[g + 1];
 #pragma unroll 1
       for (int c = 0; c < S::BN; c += 32) {
         float v[32];
@@ -1766,11 +1922,17 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   p.yexp = yexp;
   p.nblk = (N + 31) / 32;
   p.l2_hints = l2_hints_enabled();
+  const char *ps = getenv("MOE_PAIR_SWAP");  // 0: partial chunks as ordinary pair tiles
+  p.pair_swap = (ps && ps[0] == '0') ? 0 : 1;
+  CUtensorMap mx32, mx8;
+  if (!make_map_rows(&mx32, A, rows_cap, K, 32) || !make_map_rows(&mx8, A, rows_cap, K, 8))
+    return cudaErrorInvalidValue;
   const long long max_tiles = (long long)((rows_cap + BM2 - 1) / BM2 + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
   long long pairs = sms / 2;
   if (max_tiles < pairs) pairs = max_tiles < 1 ? 1 : max_tiles;
-  k_grouped_gemm_pair<SWIGLU><<<(int)(2 * pairs), kThreads, smem, s>>>(ma, mb1, mb3, p);
+  k_grouped_gemm_pair<SWIGLU><<<(int)(2 * pairs), kThreads, smem, s>>>(ma, mb1, mb3, mx32, mx8,
+                                                                       p);
   return cudaGetLastError();
 }
 

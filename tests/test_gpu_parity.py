@@ -378,6 +378,31 @@ def test_layer_with_fp32_expert_rows(name, fp32_expert_rows, dev):
 
 
 @pytest.fixture
+def pair_no_swap():
+    """MOE_GEMM_ENGINE=pair with MOE_PAIR_SWAP=0: every 256-row chunk, the
+    partial last one of each group included, as an ordinary CTA-pair tile."""
+    import os
+    old = {k: os.environ.get(k) for k in ("MOE_GEMM_ENGINE", "MOE_PAIR_SWAP")}
+    os.environ["MOE_GEMM_ENGINE"] = "pair"
+    os.environ["MOE_PAIR_SWAP"] = "0"
+    yield
+    for k, v in old.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "qwen3_medium", "dsv3_medium", "gptoss_small"])
+def test_layer_pair_without_swap_tiles(name, pair_no_swap, dev):
+    test_layer_matches_oracle(name, dev)
+
+
+def test_expert_ffn_group_size_edges_pair_without_swap(pair_no_swap, dev):
+    test_expert_ffn_group_size_edges("pair", dev)
+
+
+@pytest.fixture
 def l2_hints():
     """MOE_L2_HINTS=1: the GEMMs' TMA loads carry L2 eviction hints."""
     import os
