@@ -293,6 +293,78 @@ MOE_API moe_status moe_layer_fp8(const moe_config *cfg, const void *x, const voi
                                  const moe_route_out *route_out, void *ws, size_t ws_bytes,
                                  void *stream, void *const *events, int32_t n_events);
 
+/* ---- Expert parallelism ----------------------------------------------------
+ * "Expert Parallelism: MoE 模型的并行切分" (SGLang learning notes), sections
+ * 3 and 8, and "LLM MoE Expert Parallel 生产实战", steps 2 and 4: the E
+ * experts are split over n_ranks ranks (rank r owns experts
+ * [r*E/n_ranks, (r+1)*E/n_ranks)); every rank routes its own T tokens, sends
+ * each kept row to the rank that owns its expert (dispatch), runs its own
+ * experts on the rows it received, and sends every result back to the rank
+ * and row it came from (combine), where the weighted combine runs as usual.
+ *
+ * The exchange is done by stores straight into the destination rank's
+ * buffers (peer pointers: another GPU's memory mapped into this one over
+ * NVLink, or -- when the ranks are emulated on one GPU -- plain pointers into
+ * that GPU's memory); no rows are staged and the host never reads a count.
+ * Every rank needs the kept-row counts of all ranks first, counts_all
+ * [n_ranks][E] int32 on its device (rank s's row = its moe_route `kept`,
+ * gathered by the caller, e.g. an all-gather), and the caller orders the
+ * steps across ranks (the destination buffers must be free before a
+ * dispatch, and a rank may read what it received only after every sender
+ * finished: a barrier after each exchange).
+ *
+ * Receive layout on rank r: its experts' rows grouped by expert (ascending),
+ * inside an expert by source rank (ascending), inside a source in the
+ * source's own row order.  recv_offsets [E/n_ranks + 1] (from
+ * moe_ep_plan) delimits the experts, so the received rows feed
+ * moe_expert_ffn with E/n_ranks experts directly.  The returned rows land in
+ * the source rank's y_back [T*k_max, d] fp32 at the rows of its own
+ * dispatch layout, which moe_combine reads through slot_row.
+ * n_ranks divides E; 1 <= n_ranks <= 8. */
+#define MOE_EP_MAX_RANKS 8
+typedef struct {
+  int32_t rank;
+  int32_t n_ranks;
+  const int32_t *counts_all;              /* device [n_ranks][E] */
+  void *recv_rows[MOE_EP_MAX_RANKS];      /* per rank: its received rows [n_ranks*T*k_max, d], cfg->dtype */
+  float *y_back[MOE_EP_MAX_RANKS];        /* per rank: its returned rows [T*k_max, d] fp32 */
+} moe_ep_ranks;
+
+/* This rank's part of the exchange plan, from counts_all (device work, on
+ * `stream`): recv_offsets [E/n_ranks + 1] int32 (rows received per local
+ * expert, prefix summed), and send_base [E] int32 (for each expert e, the
+ * row of the owner's receive buffer where this rank's rows of e start).
+ * Both are device buffers owned by the caller. */
+MOE_API moe_status moe_ep_plan(const moe_config *cfg, const moe_ep_ranks *ep,
+                               int32_t *recv_offsets, int32_t *send_base, void *stream);
+
+/* Dispatch: every kept row of this rank (offsets, row_src, topk_idx of its
+ * moe_route) goes from the token rows x [T, d] to row
+ * send_base[e] + (its index among this rank's rows of e) of the owner's
+ * recv_rows. */
+MOE_API moe_status moe_ep_dispatch(const moe_config *cfg, const moe_ep_ranks *ep,
+                                   const void *x, const int32_t *offsets, const int32_t *row_src,
+                                   const int32_t *topk_idx, const int32_t *send_base,
+                                   void *stream);
+
+/* Combine exchange: every received row's expert output (y_recv [n_ranks*T*
+ * k_max, d] fp32, from moe_expert_ffn over this rank's experts) goes back to
+ * its source rank's y_back, at the row the source's own dispatch layout
+ * gave it. */
+MOE_API moe_status moe_ep_return(const moe_config *cfg, const moe_ep_ranks *ep,
+                                 const float *y_recv, const int32_t *recv_offsets, void *stream);
+
+/* Host-only mirror of the plan (touches no device): from counts_all
+ * [n_ranks][E] in host memory, rank `rank`'s recv_offsets [E/n_ranks + 1] and
+ * send_base [E], and for every row p it receives (p < recv_offsets[E/n_ranks]
+ * <= max_recv) the source rank recv_src[p] and the row recv_src_row[p] of the
+ * source's own layout that it returns to.  For schedulers and tests that
+ * check the exchange layout on the host. */
+MOE_API moe_status moe_ep_plan_host(int32_t n_ranks, int32_t E, int32_t rank,
+                                    const int32_t *counts_all, int32_t *recv_offsets,
+                                    int32_t *send_base, int32_t *recv_src, int32_t *recv_src_row,
+                                    int32_t max_recv);
+
 /* Synchronises `stream`, then reads and clears the device error flags of the
  * current device.  *flags (may be NULL) receives them: bit 0 an index out of
  * range in a gather/scatter, bit 1 a pipeline wait that hit its time limit,

@@ -665,6 +665,96 @@ moe_status moe_layer_fp8(const moe_config *cfg, const void *x, const void *Wr,
                     out, route_out, ws, ws_bytes, stream, ev);
 }
 
+// ---------------------------------------------------------------------------
+// Expert parallelism
+static moe_status check_ep(const moe_config *cfg, const moe_ep_ranks *ep) {
+  MOE_TRY(check_config(cfg));
+  if (!ep) return MOE_ERR_INVALID_ARG;
+  if (ep->n_ranks < 1 || ep->n_ranks > MOE_EP_MAX_RANKS || cfg->E % ep->n_ranks) return MOE_ERR_INVALID_ARG;
+  if (ep->rank < 0 || ep->rank >= ep->n_ranks) return MOE_ERR_INVALID_ARG;
+  if ((long long)cfg->T * cfg->k_max * ep->n_ranks > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  return need4(ep->counts_all);
+}
+
+moe_status moe_ep_plan(const moe_config *cfg, const moe_ep_ranks *ep, int32_t *recv_offsets,
+                       int32_t *send_base, void *stream) {
+  MOE_TRY(check_ep(cfg, ep));
+  MOE_TRY(need4(recv_offsets));
+  MOE_TRY(need4(send_base));
+  return cuda_status(launch_ep_plan(ep->counts_all, ep->n_ranks, cfg->E, ep->rank, recv_offsets,
+                                    send_base, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_dispatch(const moe_config *cfg, const moe_ep_ranks *ep, const void *x,
+                           const int32_t *offsets, const int32_t *row_src,
+                           const int32_t *topk_idx, const int32_t *send_base, void *stream) {
+  MOE_TRY(check_ep(cfg, ep));
+  if (cfg->T == 0) return MOE_OK;  // empty batch: nothing to send
+  MOE_TRY(need(x));
+  MOE_TRY(need4(offsets));
+  MOE_TRY(need4(row_src));
+  MOE_TRY(need4(topk_idx));
+  MOE_TRY(need4(send_base));
+  for (int r = 0; r < ep->n_ranks; ++r) MOE_TRY(need(ep->recv_rows[r]));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  return cuda_status(launch_ep_dispatch(*cfg, ep->n_ranks, ep->recv_rows, x, offsets, row_src,
+                                        topk_idx, send_base, err,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_return(const moe_config *cfg, const moe_ep_ranks *ep, const float *y_recv,
+                         const int32_t *recv_offsets, void *stream) {
+  MOE_TRY(check_ep(cfg, ep));
+  MOE_TRY(need(y_recv));
+  MOE_TRY(need4(recv_offsets));
+  for (int r = 0; r < ep->n_ranks; ++r) MOE_TRY(need(ep->y_back[r]));
+  uint32_t *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  return cuda_status(launch_ep_return(*cfg, ep->n_ranks, ep->rank, ep->counts_all, ep->y_back,
+                                      y_recv, recv_offsets, err,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_plan_host(int32_t n_ranks, int32_t E, int32_t rank, const int32_t *C,
+                            int32_t *recv_offsets, int32_t *send_base, int32_t *recv_src,
+                            int32_t *recv_src_row, int32_t max_recv) {
+  if (n_ranks < 1 || n_ranks > MOE_EP_MAX_RANKS || E < 1 || E > 1024 || E % n_ranks)
+    return MOE_ERR_INVALID_ARG;
+  if (rank < 0 || rank >= n_ranks || !C || !recv_offsets || !send_base || max_recv < 0)
+    return MOE_ERR_INVALID_ARG;
+  const int e_loc = E / n_ranks;
+  // send bases: rows of the owner's experts before e, then of e's earlier sources
+  for (int r = 0; r < n_ranks; ++r) {
+    long long run = 0;
+    for (int j = 0; j < e_loc; ++j) {
+      const int e = r * e_loc + j;
+      long long before = 0;
+      for (int s = 0; s < rank; ++s) before += C[(size_t)s * E + e];
+      send_base[e] = (int32_t)(run + before);
+      if (r == rank) recv_offsets[j] = (int32_t)run;
+      for (int s = 0; s < n_ranks; ++s) run += C[(size_t)s * E + e];
+    }
+    if (r == rank) recv_offsets[e_loc] = (int32_t)run;
+  }
+  const int R = recv_offsets[e_loc];
+  if (!recv_src && !recv_src_row) return MOE_OK;
+  if (!recv_src || !recv_src_row || R > max_recv) return MOE_ERR_INVALID_ARG;
+  // every received row: its source and the row of the source's own layout
+  for (int j = 0, p = recv_offsets[0]; j < e_loc; ++j) {
+    const int e = rank * e_loc + j;
+    for (int s = 0; s < n_ranks; ++s) {
+      long long first = 0;  // rows of s's experts before e
+      for (int e2 = 0; e2 < e; ++e2) first += C[(size_t)s * E + e2];
+      for (int i = 0; i < C[(size_t)s * E + e]; ++i, ++p) {
+        recv_src[p] = s;
+        recv_src_row[p] = (int32_t)(first + i);
+      }
+    }
+  }
+  return MOE_OK;
+}
+
 moe_status moe_check_errors(void *stream, uint32_t *flags) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
   uint32_t *err = device_error_word();

@@ -155,6 +155,20 @@ cudaError_t launch_split_planes(const void *src, const int32_t *n_rows, int fixe
                                 int K, uint8_t *planes, float *row_scale, uint32_t *err,
                                 cudaStream_t s);
 
+// Expert parallelism (expert_parallel.cu): the exchange plan of one rank
+// from the counts of all ranks C [n_ranks][E], the dispatch of its kept rows
+// into the owners' receive buffers, and the return of its experts' outputs to
+// the sources' y_back buffers (fp32 rows).
+cudaError_t launch_ep_plan(const int32_t *C, int n_ranks, int E, int rank, int32_t *recv_offsets,
+                           int32_t *send_base, cudaStream_t s);
+cudaError_t launch_ep_dispatch(const moe_config &c, int n_ranks, void *const *recv_rows,
+                               const void *x, const int32_t *offsets, const int32_t *row_src,
+                               const int32_t *topk_idx, const int32_t *send_base, uint32_t *err,
+                               cudaStream_t s);
+cudaError_t launch_ep_return(const moe_config &c, int n_ranks, int rank, const int32_t *C,
+                             float *const *y_back, const float *y_recv,
+                             const int32_t *recv_offsets, uint32_t *err, cudaStream_t s);
+
 // Per-column e4m3 quantisation of bf16 weights W [G, K, N]: scale[g, n] =
 // max_k |W| / 448 (1 for an all-zero column), Wq = e4m3(W / scale), rounded
 // to nearest even with saturation.

@@ -43,6 +43,16 @@ class MoeRouteOut(ctypes.Structure):
                  "row_src", "n_dropped")]
 
 
+EP_MAX_RANKS = 8
+
+
+class MoeEpRanks(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_int32), ("n_ranks", ctypes.c_int32),
+                ("counts_all", ctypes.c_void_p),
+                ("recv_rows", ctypes.c_void_p * EP_MAX_RANKS),
+                ("y_back", ctypes.c_void_p * EP_MAX_RANKS)]
+
+
 class MoeFp8Weights(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in ("W1", "W3", "W2", "s1", "s3", "s2")]
 
@@ -74,13 +84,19 @@ def lib() -> ctypes.CDLL:
         L.moe_expert_ffn_fp8.argtypes = [cfgp, P, P, fp8p, P, P, S, P]
         L.moe_layer_fp8.argtypes = [cfgp, P, P, P, P, P, fp8p, fp8p, P, outp, P, S, P,
                                     ctypes.POINTER(ctypes.c_void_p), I]
+        epp = ctypes.POINTER(MoeEpRanks)
+        L.moe_ep_plan.argtypes = [cfgp, epp, P, P, P]
+        L.moe_ep_dispatch.argtypes = [cfgp, epp, P, P, P, P, P, P]
+        L.moe_ep_return.argtypes = [cfgp, epp, P, P, P]
+        L.moe_ep_plan_host.argtypes = [I, I, I, P, P, P, P, P, I]
         L.moe_check_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         for fn in ("moe_workspace_size", "moe_route", "moe_route_static_scratch", "moe_dispatch",
                    "moe_expert_ffn",
                    "moe_combine", "moe_layer", "moe_layer_timed", "moe_check_errors",
-                   "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_layer_fp8"):
+                   "moe_quantize_fp8", "moe_expert_ffn_fp8", "moe_layer_fp8", "moe_ep_plan",
+                   "moe_ep_dispatch", "moe_ep_return", "moe_ep_plan_host"):
             getattr(L, fn).restype = I
         _lib = L
     return _lib
@@ -261,3 +277,49 @@ def moe_layer_fp8(cfg, x, Wr, logit_bias, sel_bias, k_per_token, experts: dict,
                                None if wsh is None else ctypes.byref(wsh), _p(out), r, _p(ws),
                                0 if ws is None else ws.numel(), _stream(stream), handles, n),
            "moe_layer_fp8")
+
+
+# ---- expert parallelism -----------------------------------------------------
+def ep_ranks(rank: int, n_ranks: int, counts_all, recv_rows, y_back) -> MoeEpRanks:
+    """The moe_ep_ranks of one rank: counts_all [n_ranks, E] int32 on its
+    device, and every rank's receive and return buffers (device tensors)."""
+    ep = MoeEpRanks()
+    ep.rank, ep.n_ranks = rank, n_ranks
+    ep.counts_all = counts_all.data_ptr()
+    for r in range(n_ranks):
+        ep.recv_rows[r] = recv_rows[r].data_ptr()
+        ep.y_back[r] = y_back[r].data_ptr()
+    return ep
+
+
+def moe_ep_plan(cfg, ep: MoeEpRanks, recv_offsets, send_base, stream=None):
+    _check(lib().moe_ep_plan(ctypes.byref(cfg), ctypes.byref(ep), _p(recv_offsets),
+                             _p(send_base), _stream(stream)), "moe_ep_plan")
+
+
+def moe_ep_dispatch(cfg, ep: MoeEpRanks, x, offsets, row_src, topk_idx, send_base, stream=None):
+    _check(lib().moe_ep_dispatch(ctypes.byref(cfg), ctypes.byref(ep), _p(x), _p(offsets),
+                                 _p(row_src), _p(topk_idx), _p(send_base), _stream(stream)),
+           "moe_ep_dispatch")
+
+
+def moe_ep_return(cfg, ep: MoeEpRanks, y_recv, recv_offsets, stream=None):
+    _check(lib().moe_ep_return(ctypes.byref(cfg), ctypes.byref(ep), _p(y_recv),
+                               _p(recv_offsets), _stream(stream)), "moe_ep_return")
+
+
+def moe_ep_plan_host(n_ranks: int, E: int, rank: int, counts_all, max_recv: int):
+    """Host mirror of the plan: (recv_offsets, send_base, recv_src, recv_src_row)
+    as int32 numpy arrays, from counts_all [n_ranks, E] (numpy)."""
+    import numpy as np
+    C = np.ascontiguousarray(counts_all, dtype=np.int32)
+    e_loc = E // max(n_ranks, 1)
+    ro = np.zeros(e_loc + 1, np.int32)
+    sb = np.zeros(E, np.int32)
+    rs = np.zeros(max(max_recv, 1), np.int32)
+    rr = np.zeros(max(max_recv, 1), np.int32)
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(lib().moe_ep_plan_host(n_ranks, E, rank, ptr(C), ptr(ro), ptr(sb), ptr(rs), ptr(rr),
+                                  max_recv), "moe_ep_plan_host")
+    R = int(ro[-1])
+    return ro, sb, rs[:R], rr[:R]
