@@ -875,32 +875,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   if (warp == 1) tmem_alloc_pair(smem_addr(tmem_slot), S::kTmemCols);
   __syncthreads();
+  // Two tile lists, each an exclusive scan of per-group tile counts: heavy
+  // (groups of at least 256 rows: their chunks, the partial last one
+  // included, chunks fastest within a column tile) and -- when partial chunks
+  // run swap-AB -- light (smaller groups: one swap-AB tile per column tile).
+  // The deal merges them evenly (tile t is light when the count of light
+  // tiles among the first t+1, round-down of (t+1) L / total, steps up), so
+  // every wave mixes compute-bound heavy tiles with light tiles that mostly
+  // stream their group's weights.
+  int32_t *s_lstart = s_tstart + (p.G + 1);
   const int n_tiles = (p.N + S::BN - 1) / S::BN;
   for (int g = threadIdx.x; g < p.G; g += kThreads) {
     const int rows = s_off[g + 1] - s_off[g];
     if (rows < 0) bad = true;
-    s_tstart[g] = rows > 0 ? ((rows + BM2 - 1) / BM2) * n_tiles : 0;
+    const bool light = p.pair_swap && rows > 0 && rows < BM2;
+    s_tstart[g] = (rows > 0 && !light) ? ((rows + BM2 - 1) / BM2) * n_tiles : 0;
+    s_lstart[g] = light ? n_tiles : 0;
   }
   if (bad) {
     *abort_flag = 1;
     raise_error(p.err, kErrIndex);
   }
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 0 || warp == 1) {  // in-place exclusive scans, 32 groups per step
+    int32_t *sc = warp == 0 ? s_tstart : s_lstart;
     int carry = 0;
     for (int base = 0; base < p.G; base += 32) {
       const int g = base + lane;
-      const int v = g < p.G ? s_tstart[g] : 0;
+      const int v = g < p.G ? sc[g] : 0;
       int incl = v;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
       }
-      if (g < p.G) s_tstart[g] = carry + incl - v;
+      if (g < p.G) sc[g] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) s_tstart[p.G] = carry;
+    if (lane == 0) sc[p.G] = carry;
   }
   if (warp == 1) tmem_relinquish_pair();
   tc_fence_before();
@@ -910,7 +922,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   // Both CTAs see the same offsets, so they agree on the tile list; a CTA
   // that found bad offsets stops, and its peer's waits time out.
-  const int total = *abort_flag ? 0 : s_tstart[p.G];
+  const int n_heavy = s_tstart[p.G], n_light = s_lstart[p.G];
+  const int total = *abort_flag ? 0 : n_heavy + n_light;
   const int num_kb = (p.K + BK - 1) / BK;
   const uint32_t leader_full0 = mapa_shared(full0, 0);
   const uint32_t leader_acce0 = mapa_shared(acce0, 0);
@@ -924,24 +937,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int g, n, row0, nr;
     bool swap;
   };
-  auto pair_tile = [&](int tile) {
-    int lo = 0, hi = p.G - 1;
+  auto find_group = [&](const int32_t *start, int idx) {
+    int lo = 0, hi = p.G - 1;  // largest g with start[g] <= idx
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (s_tstart[mid] <= tile)
+      if (start[mid] <= idx)
         lo = mid;
       else
         hi = mid - 1;
     }
+    return lo;
+  };
+  auto pair_tile = [&](int tile) {
     PairTile t;
-    t.g = lo;
-    const int rows = s_off[lo + 1] - s_off[lo];
-    const int mt = (rows + BM2 - 1) / BM2;
-    const int local = tile - s_tstart[lo];
-    t.n = local / mt;
-    const int m = local - t.n * mt;
-    t.row0 = s_off[lo] + m * BM2;
-    t.nr = min(BM2, rows - m * BM2);
+    const long long l0 = (long long)tile * n_light / total;
+    const long long l1 = (long long)(tile + 1) * n_light / total;
+    if (l1 > l0) {  // light: the whole group, column tile n
+      const int li = (int)l0;
+      t.g = find_group(s_lstart, li);
+      t.n = li - s_lstart[t.g];
+      t.row0 = s_off[t.g];
+      t.nr = s_off[t.g + 1] - s_off[t.g];
+    } else {  // heavy: chunk m of column tile n
+      const int hi = tile - (int)l0;
+      t.g = find_group(s_tstart, hi);
+      const int rows = s_off[t.g + 1] - s_off[t.g];
+      const int mt = (rows + BM2 - 1) / BM2;
+      const int local = hi - s_tstart[t.g];
+      t.n = local / mt;
+      const int m = local - t.n * mt;
+      t.row0 = s_off[t.g] + m * BM2;
+      t.nr = min(BM2, rows - m * BM2);
+    }
     t.swap = p.pair_swap && t.nr < BM2;
     return t;
   };
@@ -1908,13 +1935,14 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
       !make_map_b(&mb3, SWIGLU ? B3 : B1, G, K, N))
     return cudaErrorInvalidValue;
-  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
+  // group tables: row offsets, heavy and light tile starts
+  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 3 * (size_t)(G + 1);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static std::atomic<bool> attr_set[64];
   if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_pair<SWIGLU>,
-                                    S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+                                    S::kSmemFixed + sizeof(int32_t) * 3 * (kMaxGroups + 1)))
     return e;
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
   p.row_w = rw.w;
