@@ -53,7 +53,7 @@ namespace tc {
 namespace {
 
 constexpr int kQK = 128;    // K per stage: one 128-byte swizzle span of e4m3
-constexpr int kQRows = 64;  // rows per tile (the MMA's N, at most)
+constexpr int kQRows = 32;  // rows per tile (the MMA's N, at most)
 constexpr int kPlanes = 2;
 constexpr int kRowBoxQ = 16;  // rows per TMA box of a plane
 
@@ -62,12 +62,14 @@ struct ShapeF8 {
   static constexpr int kCols = 128;                       // columns per code tile (MMA M)
   static constexpr int kTileCols = SWIGLU ? 128 : 256;    // output columns per tile
   static constexpr uint32_t kCodeBytes = kCols * kQK;     // 16 KB
-  static constexpr uint32_t kPlaneBytes = kQRows * kQK;   // 8 KB: the tile's rows of one plane
-  static constexpr uint32_t kStageBytes = 2 * kCodeBytes + kPlanes * kPlaneBytes;  // 48 KB
-  static constexpr int kStages = 4;
+  static constexpr uint32_t kPlaneBytes = kQRows * kQK;   // 4 KB: the tile's rows of one plane
+  static constexpr uint32_t kStageBytes = 2 * kCodeBytes + kPlanes * kPlaneBytes;  // 40 KB
+  // A decode-sized layer streams every weight once, so the pace is set by the
+  // bytes each SM keeps in flight: five stages hold 160 KB of codes.
+  static constexpr int kStages = 5;
   static constexpr uint32_t kRingBytes = kStages * kStageBytes;
   static constexpr uint32_t kAccCols = 2 * kQRows;        // two accumulators
-  static constexpr uint32_t kTmemCols = 2 * kAccCols;     // double-buffered: 256
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;     // double-buffered: 128
   static constexpr uint32_t kStageRowWords = 36;
   static constexpr uint32_t kEpiBytes = 4 * 32 * kStageRowWords * 4;  // 18 KB
   static constexpr int kBars = 2 * kStages + 5;
@@ -76,6 +78,7 @@ struct ShapeF8 {
                 "swizzled tiles start on 1024-byte boundaries");
   static_assert(kBars * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit 256 bytes");
   static_assert(kQRows % 32 == 0 && kQRows <= 256, "MMA N");
+  static_assert(kSmemFixed + 4 * 1025 <= 232448, "shared memory of a CTA");
 };
 
 // kind::f8f6f4 instruction descriptor: fp32 accumulator (bits 4-5 = 1), A and
@@ -135,8 +138,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + S::kBars);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   float *s_epi = reinterpret_cast<float *>(ring + S::kRingBytes + 256);
-  int32_t *s_off = reinterpret_cast<int32_t *>(ring + S::kRingBytes + 256 + S::kEpiBytes);
-  int32_t *s_tstart = s_off + (p.G + 1);
+  // the tile starts live in shared memory; the row offsets are read from
+  // global memory (L1-cached): five stages leave no room for both tables
+  int32_t *s_tstart = reinterpret_cast<int32_t *>(ring + S::kRingBytes + 256 + S::kEpiBytes);
+  const int32_t *s_off = p.offsets;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + S::kStages);
@@ -163,11 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmW1);
     if (SWIGLU) prefetch_tmap(&tmW3);
   }
-  // Group table: row offsets and tile starts, checked against the buffer size.
+  // Tile starts, from the row offsets checked against the buffer size.
   bool bad = false;
   for (int g = threadIdx.x; g <= p.G; g += kThreads) {
     const int v = p.offsets[g];
-    s_off[g] = v;
     if (v < 0 || v > p.rows_cap) bad = true;
   }
   if (warp == 1) tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
@@ -570,13 +574,13 @@ cudaError_t launch_f8(int rows_cap, int K, int N, int G, const int32_t *offsets,
   if (!make_map_planes(&mp, planes, rows_cap, K) || !make_map_codes_k128(&mw1, B1, G, N, K) ||
       !make_map_codes_k128(&mw3, SWIGLU ? B3 : B1, G, N, K))
     return cudaErrorInvalidValue;
-  const size_t smem = S::kSmemFixed + sizeof(int32_t) * 2 * (size_t)(G + 1);
+  const size_t smem = S::kSmemFixed + sizeof(int32_t) * (size_t)(G + 1);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static std::atomic<bool> attr_set[64];
   if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_f8<SWIGLU>,
-                                    S::kSmemFixed + sizeof(int32_t) * 2 * (kMaxGroups + 1)))
+                                    S::kSmemFixed + sizeof(int32_t) * (kMaxGroups + 1)))
     return e;
   const char *pf = getenv("MOE_F8_PREFETCH");
   ParamsF8 p{offsets, G, rows_cap, K, N, out, s1, SWIGLU ? s3 : nullptr, row_scale,

@@ -2047,16 +2047,23 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
 //     the up projection, which loads only the valid rows (Mixtral-shaped
 //     decode: 0.298 vs 0.320 ms single-CTA), single-CTA for the down
 //     projection (CTA pairs: 0.171 vs 0.146 ms);
-//   - every larger shape, both projections: CTA pairs.  Sharing each weight
+//   - routed groups of at most 256 rows on average (ragged layers: many
+//     small experts next to a few large ones), both projections: mixed tiles
+//     (each group's full 128-row chunks single-CTA, its remainder swap-AB,
+//     heavy and light tiles interleaved in the deal).  Alternated call by
+//     call on two boxes: GPT-OSS-shaped sub-experts 2.41 vs 2.73 ms (pairs),
+//     DeepSeek-V3-shaped prefill 7.34 vs 8.06 ms; a light tile mostly streams
+//     its group's weights, and a single CTA keeps 128 KB of them in flight
+//     where a CTA of a pair keeps 96 KB;
+//   - every other shape, both projections: CTA pairs.  Sharing each weight
 //     tile between two SMs halves the weight bytes each SM streams and cuts
 //     the shared-memory and L2 traffic per FLOP by a third, which under the
-//     1 kW power cap keeps the clock up.  Layer times, pair vs single vs
-//     mixed: Mixtral-shaped prefill 4.36 vs 7.47 (single) ms; Qwen3-shaped
-//     1.35 vs 1.64 vs 1.72 ms (down projection 0.39 vs 0.46 ms);
-//     DeepSeek-V3-shaped prefill 5.91 vs 6.51 vs 6.95 ms; GPT-OSS-shaped
-//     sub-experts 2.58 vs 2.85 vs 2.78 ms -- even the ragged layers, whose
-//     small groups leave a 256-row pair tile mostly empty, gain more from the
-//     halved per-SM weight stream than they lose in padding.
+//     1 kW power cap keeps the clock up: Mixtral-shaped prefill 4.36 vs 7.47
+//     ms (single CTA), Qwen3-shaped 1.35 vs 1.64 ms (mixed 1.72; its 2048-wide
+//     down projection 0.39 vs 0.46 ms single).  A pair's partial last
+//     256-row chunk runs swap-AB (weights as M, the chunk's rows as N): the
+//     tensor pipe then idles less on padding (ncu, GPT-OSS-shaped up
+//     projection: 74% → 28% tensor-active), though no layer measured faster.
 // MOE_GEMM_ENGINE=single|narrow|pair|swap|mixed selects one engine for every
 // GEMM (mixed: for routed groups; a single group of rows runs single-CTA).
 enum class Engine { kSingle, kNarrow, kPair, kSwap, kMixed };
@@ -2071,6 +2078,7 @@ static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offse
   if (env && env[0] == 'm') return offsets ? Engine::kMixed : Engine::kSingle;
   const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
   if (mean_rows <= 32) return swiglu ? Engine::kSwap : Engine::kSingle;
+  if (offsets && mean_rows <= 256) return Engine::kMixed;
   return Engine::kPair;
 }
 
