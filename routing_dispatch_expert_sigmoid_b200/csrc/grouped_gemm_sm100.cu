@@ -1950,8 +1950,11 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   p.yexp = yexp;
   p.nblk = (N + 31) / 32;
   p.l2_hints = l2_hints_enabled();
-  const char *ps = getenv("MOE_PAIR_SWAP");  // 0: partial chunks as ordinary pair tiles
-  p.pair_swap = (ps && ps[0] == '0') ? 0 : 1;
+  // MOE_PAIR_SWAP=1: partial chunks as swap-AB pair tiles (off by default:
+  // alternated call by call, the Qwen3-shaped layer ran 1.52 vs 1.46 ms with
+  // them, the others within noise)
+  const char *ps = getenv("MOE_PAIR_SWAP");
+  p.pair_swap = (ps && ps[0] == '1') ? 1 : 0;
   CUtensorMap mx32, mx8;
   if (!make_map_rows(&mx32, A, rows_cap, K, 32) || !make_map_rows(&mx8, A, rows_cap, K, 8))
     return cudaErrorInvalidValue;
@@ -2061,9 +2064,10 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
 //     1 kW power cap keeps the clock up: Mixtral-shaped prefill 4.36 vs 7.47
 //     ms (single CTA), Qwen3-shaped 1.35 vs 1.64 ms (mixed 1.72; its 2048-wide
 //     down projection 0.39 vs 0.46 ms single).  A pair's partial last
-//     256-row chunk runs swap-AB (weights as M, the chunk's rows as N): the
-//     tensor pipe then idles less on padding (ncu, GPT-OSS-shaped up
-//     projection: 74% → 28% tensor-active), though no layer measured faster.
+//     256-row chunk can run swap-AB (MOE_PAIR_SWAP=1: weights as M, the
+//     chunk's rows as N): the tensor pipe then does far less padding work
+//     (ncu, GPT-OSS-shaped up projection: 74% → 28% tensor-active), but no
+//     layer measured faster (Qwen3-shaped: 1.52 vs 1.46 ms), so it is off.
 // MOE_GEMM_ENGINE=single|narrow|pair|swap|mixed selects one engine for every
 // GEMM (mixed: for routed groups; a single group of rows runs single-CTA).
 enum class Engine { kSingle, kNarrow, kPair, kSwap, kMixed };

@@ -378,13 +378,14 @@ def test_layer_with_fp32_expert_rows(name, fp32_expert_rows, dev):
 
 
 @pytest.fixture
-def pair_no_swap():
-    """MOE_GEMM_ENGINE=pair with MOE_PAIR_SWAP=0: every 256-row chunk, the
-    partial last one of each group included, as an ordinary CTA-pair tile."""
+def pair_swap():
+    """MOE_GEMM_ENGINE=pair with MOE_PAIR_SWAP=1: each group's partial last
+    256-row chunk as a swap-AB pair tile, groups below 256 rows dealt as a
+    light list among the others."""
     import os
     old = {k: os.environ.get(k) for k in ("MOE_GEMM_ENGINE", "MOE_PAIR_SWAP")}
     os.environ["MOE_GEMM_ENGINE"] = "pair"
-    os.environ["MOE_PAIR_SWAP"] = "0"
+    os.environ["MOE_PAIR_SWAP"] = "1"
     yield
     for k, v in old.items():
         if v is None:
@@ -393,13 +394,18 @@ def pair_no_swap():
             os.environ[k] = v
 
 
-@pytest.mark.parametrize("name", ["mixtral_small", "qwen3_medium", "dsv3_medium", "gptoss_small"])
-def test_layer_pair_without_swap_tiles(name, pair_no_swap, dev):
+@pytest.mark.parametrize("name", BF16_SMALL)
+def test_layer_pair_with_swap_tiles(name, pair_swap, dev):
     test_layer_matches_oracle(name, dev)
 
 
-def test_expert_ffn_group_size_edges_pair_without_swap(pair_no_swap, dev):
+def test_expert_ffn_group_size_edges_pair_with_swap(pair_swap, dev):
     test_expert_ffn_group_size_edges("pair", dev)
+
+
+@pytest.mark.parametrize("name", BF16_SMALL)
+def test_expert_ffn_pair_with_swap_tiles(name, pair_swap, dev):
+    test_expert_ffn_matches_oracle(name, dev)
 
 
 @pytest.fixture
