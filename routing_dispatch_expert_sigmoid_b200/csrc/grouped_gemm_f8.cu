@@ -122,6 +122,7 @@ struct ParamsF8 {
   uint32_t *err;
   uint64_t wait_limit_ns;
   int prefetch;  // k-blocks of codes prefetched into L2 ahead of their loads (0: none)
+  int kstagger;  // rotate each CTA's k-block order (MOE_F8_KSTAGGER=1)
 };
 
 template <bool SWIGLU>
@@ -210,6 +211,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = *abort_flag ? 0 : s_tstart[p.G];
   const int num_kb = (p.K + kQK - 1) / kQK;
+  // p.kstagger: each CTA walks the k-blocks of its tiles from its own
+  // starting block (the MMAs accumulate the same products in a rotated
+  // order), so that the CTAs streaming at the same time read codes at
+  // different offsets of their rows instead of all at the same one
+  const int kstart = p.kstagger ? (int)((blockIdx.x * 37u) % (unsigned)num_kb) : 0;
 
   // tile -> (group g, column tile c, row tile r); rows fastest, so CTAs running
   // at the same time share a weight tile
@@ -253,21 +259,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = full0 + 8 * s;
           if (p.prefetch > 0) {  // the k-block p.prefetch ahead (the first ones too)
             for (int q = kb == 0 ? 0 : p.prefetch; q <= p.prefetch; ++q) {
-              const int kq = kb + q;
-              if (kq >= num_kb) break;
-              tma_prefetch_3d(&tmW1, kq * kQK, col_a, g);
-              tma_prefetch_3d(SWIGLU ? &tmW3 : &tmW1, kq * kQK, col_b, g);
+              if (kb + q >= num_kb) break;
+              const int kp = (kb + q + kstart) % num_kb;
+              tma_prefetch_3d(&tmW1, kp * kQK, col_a, g);
+              tma_prefetch_3d(SWIGLU ? &tmW3 : &tmW1, kp * kQK, col_b, g);
             }
           }
           mbar_expect_tx(fb, bytes);
+          // the k-blocks of a tile in a rotated order (kq), see p.kstagger
+          const int kq = kb + kstart < num_kb ? kb + kstart : kb + kstart - num_kb;
           // codes [G, N, K]: coordinates (k, n, group)
-          tma_load_3d(st, &tmW1, fb, kb * kQK, col_a, g);
-          tma_load_3d(st + S::kCodeBytes, SWIGLU ? &tmW3 : &tmW1, fb, kb * kQK, col_b, g);
+          tma_load_3d(st, &tmW1, fb, kq * kQK, col_a, g);
+          tma_load_3d(st + S::kCodeBytes, SWIGLU ? &tmW3 : &tmW1, fb, kq * kQK, col_b, g);
           // planes [2*rows_cap, K]: plane q's row r at q*rows_cap + r
           for (int q = 0; q < kPlanes; ++q)
             for (int b = 0; b < nq; ++b)
               tma_load_2d(st + 2 * S::kCodeBytes + q * S::kPlaneBytes + b * kRowBoxQ * kQK, &tmP,
-                          fb, kb * kQK, q * p.rows_cap + row0 + b * kRowBoxQ);
+                          fb, kq * kQK, q * p.rows_cap + row0 + b * kRowBoxQ);
           issued_mask |= 1u << s;
           issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
           if (++s == S::kStages) {
@@ -583,8 +591,10 @@ cudaError_t launch_f8(int rows_cap, int K, int N, int G, const int32_t *offsets,
                                     S::kSmemFixed + sizeof(int32_t) * (kMaxGroups + 1)))
     return e;
   const char *pf = getenv("MOE_F8_PREFETCH");
+  const char *ks = getenv("MOE_F8_KSTAGGER");
   ParamsF8 p{offsets, G, rows_cap, K, N, out, s1, SWIGLU ? s3 : nullptr, row_scale,
-             row_w, w_row_src, err, pipeline_wait_limit_ns(), pf ? atoi(pf) : 0};
+             row_w, w_row_src, err, pipeline_wait_limit_ns(), pf ? atoi(pf) : 0,
+             (ks && ks[0] == '1') ? 1 : 0};
   const long long max_tiles = (long long)((rows_cap + kQRows - 1) / kQRows + G) *
                               ((N + S::kTileCols - 1) / S::kTileCols);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);

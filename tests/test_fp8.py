@@ -238,3 +238,20 @@ def test_fp8_layer_with_code_prefetch(name, dev):
             os.environ.pop("MOE_F8_PREFETCH", None)
         else:
             os.environ["MOE_F8_PREFETCH"] = old
+
+
+@pytest.mark.parametrize("name", ["mixtral_decode_small", "f8_decode_ragged",
+                                  "f8_decode_hot_expert", "f8_decode_many_experts"])
+def test_fp8_layer_with_rotated_k_order(name, dev):
+    """MOE_F8_KSTAGGER=1: each CTA of the kind::f8f6f4 engine walks the
+    k-blocks of its tiles from its own starting block."""
+    import os
+    old = os.environ.get("MOE_F8_KSTAGGER")
+    os.environ["MOE_F8_KSTAGGER"] = "1"
+    try:
+        test_fp8_layer_matches_oracle(name, "default", dev)
+    finally:
+        if old is None:
+            os.environ.pop("MOE_F8_KSTAGGER", None)
+        else:
+            os.environ["MOE_F8_KSTAGGER"] = old
