@@ -88,16 +88,6 @@ __host__ __device__ constexpr uint32_t instr_desc_f8(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// Bring a tile of the codes into L2 ahead of its TMA load (no shared memory,
-// no completion to wait for): a decode-sized layer streams every weight once,
-// and with only a few stages of shared memory per SM the HBM latency, not
-// its bandwidth, would set the pace.
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
-}
 
 // D[tmem] (+)= A[smem] * B[smem], e4m3 inputs, fp32 accumulation.
 __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,

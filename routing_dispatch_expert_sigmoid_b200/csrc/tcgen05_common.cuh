@@ -159,6 +159,15 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map
       "r"(bar)
       : "memory");
 }
+// Bring a box of a 3-D tensor into L2 ahead of its TMA load: no shared
+// memory, no completion to wait for.  A stream of weights that each SM reads
+// once is paced by the bytes it keeps in flight; prefetches add to them.
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
