@@ -77,7 +77,6 @@ struct ParamsMixed {
   const int32_t *row_src;
   int k_max, a_count;
   int l2_hints;  // L2 eviction hints on the TMA loads (rows kept, weights streamed)
-  int prefetch;  // light tiles: k-blocks of weights prefetched into L2 ahead of the loads
 };
 
 // A tile of the list: group g, column tile n, and either a full chunk (rows
@@ -110,15 +109,6 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// MOE_MIXED_PREFETCH=n: light tiles keep n k-blocks of weights (32 KB each)
-// on their way to L2 ahead of their loads.
-int mixed_prefetch_kblocks() {
-  const char *env = getenv("MOE_MIXED_PREFETCH");
-  if (!env || !env[0]) return 0;
-  const int v = atoi(env);
-  return v < 0 ? 0 : (v > 16 ? 16 : v);
 }
 
 template <bool SWIGLU, bool GATHER>
@@ -271,42 +261,12 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
       int s = 0;
       uint32_t ph = 0, issued_parity = 0, issued_mask = 0;
       bool ok = true;
-      // weights of k-block kb of a light tile into L2 (the four spans its load reads)
-      auto prefetch_w = [&](const TileRef &u, int kb) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const CUtensorMap *m = (SWIGLU && j >= 2) ? &tmW3 : &tmW1;
-          const int col = SWIGLU ? u.n * S::BN + (j & 1) * 64 : u.n * S::BN + j * 64;
-          tma_prefetch_3d(m, col, kb * BK, u.g);
-        }
-      };
-      const int pf = p.prefetch < num_kb ? p.prefetch : num_kb;
-      bool head_fetched = false;  // the light tile's first pf k-blocks already prefetched
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileRef t = tile_ref(tile);
         const int nq = t.full ? 0 : (t.nr + 31) / 32;  // remainder: 32-row boxes
         const uint32_t bytes =
             (GATHER ? 0u : (t.full ? S::kABytes : nq * S::kRowBoxBytes)) + S::kBBytes;
-        // a light tile streams weights no other tile reads: keep pf k-blocks of
-        // them on their way to L2 beyond the stages in shared memory, and start
-        // on the next light tile's first ones while this tile ends
-        const bool light = !t.full && s_off[t.g + 1] - s_off[t.g] < BM;
-        const int next = tile + (int)gridDim.x;
-        TileRef tn{};
-        bool next_light = false;
-        if (pf > 0 && next < total) {
-          tn = tile_ref(next);
-          next_light = !tn.full && s_off[tn.g + 1] - s_off[tn.g] < BM;
-        }
-        if (pf > 0 && light && !head_fetched)
-          for (int q = 0; q < pf; ++q) prefetch_w(t, q);
-        head_fetched = false;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (pf > 0 && light && kb + pf < num_kb) prefetch_w(t, kb + pf);
-          if (next_light && kb == num_kb - pf) {
-            for (int q = 0; q < pf; ++q) prefetch_w(tn, q);
-            head_fetched = true;
-          }
           if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
             ok = false;
             break;
@@ -698,7 +658,7 @@ cudaError_t launch_mixed(int rows_cap, int K, int N, int G, const int32_t *offse
     return e;
   ParamsMixed p{offsets, G,   rows_cap, K, N, out, row_w, w_row_src, err,
                 pipeline_wait_limit_ns(), yexp, (N + 31) / 32, A, row_src, k_max, a_count,
-                l2_hints_enabled(), mixed_prefetch_kblocks()};
+                l2_hints_enabled()};
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + G) *
                               ((N + S::BN - 1) / S::BN);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);

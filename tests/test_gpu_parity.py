@@ -426,32 +426,6 @@ def test_layer_with_l2_hints(name, l2_hints, gemm_engine, dev):
     test_layer_matches_oracle(name, dev)
 
 
-@pytest.fixture(params=[1, 3, 8])
-def mixed_prefetch(request):
-    """MOE_MIXED_PREFETCH=n on the mixed engine: light tiles prefetch n
-    k-blocks of weights into L2 ahead of their loads (and the next light
-    tile's first n while a tile ends)."""
-    import os
-    old = {k: os.environ.get(k) for k in ("MOE_MIXED_PREFETCH", "MOE_GEMM_ENGINE")}
-    os.environ["MOE_MIXED_PREFETCH"] = str(request.param)
-    os.environ["MOE_GEMM_ENGINE"] = "mixed"
-    yield request.param
-    for k, v in old.items():
-        if v is None:
-            os.environ.pop(k, None)
-        else:
-            os.environ[k] = v
-
-
-@pytest.mark.parametrize("name", ["mixtral_small", "qwen3_medium", "dsv3_medium", "gptoss_small"])
-def test_layer_mixed_with_light_prefetch(name, mixed_prefetch, dev):
-    test_layer_matches_oracle(name, dev)
-
-
-def test_expert_ffn_group_size_edges_mixed_with_light_prefetch(mixed_prefetch, dev):
-    test_expert_ffn_group_size_edges("mixed", dev)
-
-
 @pytest.fixture
 def fused_dispatch():
     import os
