@@ -77,6 +77,9 @@ struct ParamsMixed {
   const int32_t *row_src;
   int k_max, a_count;
   int l2_hints;  // L2 eviction hints on the TMA loads (rows kept, weights streamed)
+  int lists;     // bit 0: the heavy list, bit 1: the light list
+  int phased;    // 1: every heavy tile before the first light one
+  int light_evict_first;  // evict-first hint on the light tiles' weights only
 };
 
 // A tile of the list: group g, column tile n, and either a full chunk (rows
@@ -109,6 +112,21 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Deal variants of the tile lists, from the environment: MOE_MIXED_SPLIT=1
+// runs the heavy and the light list as two launches, MOE_MIXED_PHASED=1 deals
+// every heavy tile before the light ones, MOE_MIXED_LIGHT_EVICT=1 marks the
+// light tiles' weights evict-first in L2.
+struct MixedOptions {
+  int split, phased, light_evict_first;
+};
+inline MixedOptions mixed_options() {
+  auto on = [](const char *name) {
+    const char *v = getenv(name);
+    return (v && v[0] == '1') ? 1 : 0;
+  };
+  return {on("MOE_MIXED_SPLIT"), on("MOE_MIXED_PHASED"), on("MOE_MIXED_LIGHT_EVICT")};
 }
 
 template <bool SWIGLU, bool GATHER>
@@ -182,8 +200,8 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
   for (int g = threadIdx.x; g < p.G; g += kCta) {
     const int rows = s_off[g + 1] - s_off[g];
     if (rows < 0) bad = true;
-    s_tstart[g] = rows >= BM ? ((rows + BM - 1) / BM) * n_tiles : 0;
-    s_lstart[g] = (rows > 0 && rows < BM) ? n_tiles : 0;
+    s_tstart[g] = ((p.lists & 1) && rows >= BM) ? ((rows + BM - 1) / BM) * n_tiles : 0;
+    s_lstart[g] = ((p.lists & 2) && rows > 0 && rows < BM) ? n_tiles : 0;
   }
   if (bad) {
     *abort_flag = 1;
@@ -231,8 +249,14 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
   };
   auto tile_ref = [&](int tile) {
     TileRef t;
-    const long long l0 = (long long)tile * n_light / total;
-    const long long l1 = (long long)(tile + 1) * n_light / total;
+    long long l0, l1;
+    if (p.phased) {  // heavy tiles 0 .. n_heavy-1, then the light ones
+      l0 = tile < n_heavy ? 0 : tile - n_heavy;
+      l1 = tile < n_heavy ? 0 : l0 + 1;
+    } else {
+      l0 = (long long)tile * n_light / total;
+      l1 = (long long)(tile + 1) * n_light / total;
+    }
     if (l1 > l0) {  // light: the whole group, column tile n
       const int li = (int)l0;
       t.g = find_group(s_lstart, li);
@@ -263,6 +287,8 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileRef t = tile_ref(tile);
+        const bool light = !t.full && s_off[t.g + 1] - s_off[t.g] < BM;
+        const bool hint_w = p.l2_hints || (p.light_evict_first && light);
         const int nq = t.full ? 0 : (t.nr + 31) / 32;  // remainder: 32-row boxes
         const uint32_t bytes =
             (GATHER ? 0u : (t.full ? S::kABytes : nq * S::kRowBoxBytes)) + S::kBBytes;
@@ -295,7 +321,7 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
           for (int j = 0; j < 4; ++j) {
             const CUtensorMap *m = (SWIGLU && j >= 2) ? &tmW3 : &tmW1;
             const int col = SWIGLU ? t.n * S::BN + (j & 1) * 64 : t.n * S::BN + j * 64;
-            if (p.l2_hints)
+            if (hint_w)
               tma_load_3d_hint(st + S::kABytes + j * S::kSpanBytes, m, fb, col, kb * BK, t.g,
                                pol_stream);
             else
@@ -320,6 +346,18 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
       int s = 0, buf = 0;
       uint32_t ph = 0, acc_ph = 0;
       bool ok = true, any = false;
+      // Shared-memory descriptors of stage 0; the address field counts 16-byte
+      // units in bits 0-13 and every stage lies below 256 KB, so stage s, K
+      // step kk and weight span j are plain additions to it.  A remainder
+      // tile issues eight small MMAs per k-block, so the issuing thread's own
+      // instruction count per MMA sets its pace.
+      //   rows: K-major 128-byte rows, 8-row groups 1024 B apart, K step 32 B
+      //   weights: MN-major 64-column spans kSpanBytes apart (LBO), 8-row K
+      //   groups 1024 B apart (SBO), K step 16 rows = 2048 B
+      const uint64_t rows_d0 = smem_desc(smem_addr(ring), 16, 1024);
+      const uint64_t w_d0 = smem_desc(smem_addr(ring) + S::kABytes, S::kSpanBytes, 1024);
+      constexpr uint32_t kStageStep = S::kStageBytes >> 4, kRowK = 32 >> 4, kWK = 2048 >> 4;
+      constexpr uint32_t kW3 = (2 * S::kSpanBytes) >> 4;  // spans 2-3: the second 128 columns
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileRef t = tile_ref(tile);
         const uint32_t idesc_rem = instr_desc_rem((t.nr + 15) & ~15);
@@ -335,24 +373,18 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
-          const uint32_t wt = st + S::kABytes;
+          const uint64_t rd = rows_d0 + s * kStageStep, wd = w_d0 + s * kStageStep;
+          const uint32_t acc0 = kb != 0;
+          if (t.full) {  // rows as A (M = 128), weights as B (N = 256)
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint32_t acc = (kb | kk) != 0;
-            // rows: K-major 128-byte rows, 8-row groups 1024 B apart, K step 32 B
-            const uint64_t rd = smem_desc(st + kk * 32, 16, 1024);
-            if (t.full) {
-              // weights as B: MN-major, 64-column spans kSpanBytes apart (LBO),
-              // 8-row K groups 1024 B apart (SBO); K step 16 rows = 2048 B
-              const uint64_t bd = smem_desc(wt + kk * 2048, S::kSpanBytes, 1024);
-              umma(d_tmem, rd, bd, S::kIdescFull, acc);
-            } else {
-              // weights as A (128 columns = spans 0-1, and spans 2-3), rows as B
-              const uint64_t w0 = smem_desc(wt + kk * 2048, S::kSpanBytes, 1024);
-              const uint64_t w1 = smem_desc(wt + 2 * S::kSpanBytes + kk * 2048, S::kSpanBytes, 1024);
-              umma(d_tmem, w0, rd, idesc_rem, acc);
-              umma(d_tmem + S::kHalf, w1, rd, idesc_rem, acc);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma(d_tmem, rd + kk * kRowK, wd + kk * kWK, S::kIdescFull, kk ? 1u : acc0);
+          } else {  // weights as A (two MMAs of 128 columns), rows as B
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint32_t acc = kk ? 1u : acc0;
+              umma(d_tmem, wd + kk * kWK, rd + kk * kRowK, idesc_rem, acc);
+              umma(d_tmem + S::kHalf, wd + kW3 + kk * kWK, rd + kk * kRowK, idesc_rem, acc);
             }
           }
           any = true;
@@ -656,14 +688,23 @@ cudaError_t launch_mixed(int rows_cap, int K, int N, int G, const int32_t *offse
   if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_mixed<SWIGLU, GATHER>,
                                     S::kSmemFixed + sizeof(int32_t) * 3 * (kMaxGroups + 1)))
     return e;
+  const MixedOptions o = mixed_options();
   ParamsMixed p{offsets, G,   rows_cap, K, N, out, row_w, w_row_src, err,
                 pipeline_wait_limit_ns(), yexp, (N + 31) / 32, A, row_src, k_max, a_count,
-                l2_hints_enabled()};
+                l2_hints_enabled(), 3, o.phased, o.light_evict_first};
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + G) *
                               ((N + S::BN - 1) / S::BN);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
-  k_grouped_gemm_mixed<SWIGLU, GATHER><<<grid, kCta, smem, s>>>(ma, mx, mw1, mw3, p);
-  return cudaGetLastError();
+  if (!o.split) {
+    k_grouped_gemm_mixed<SWIGLU, GATHER><<<grid, kCta, smem, s>>>(ma, mx, mw1, mw3, p);
+    return cudaGetLastError();
+  }
+  for (int lists = 1; lists <= 2; ++lists) {  // heavy groups, then light ones
+    p.lists = lists;
+    k_grouped_gemm_mixed<SWIGLU, GATHER><<<grid, kCta, smem, s>>>(ma, mx, mw1, mw3, p);
+    if (cudaError_t e = cudaGetLastError()) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace

@@ -426,6 +426,32 @@ def test_layer_with_l2_hints(name, l2_hints, gemm_engine, dev):
     test_layer_matches_oracle(name, dev)
 
 
+@pytest.fixture(params=["MOE_MIXED_SPLIT", "MOE_MIXED_PHASED", "MOE_MIXED_LIGHT_EVICT"])
+def mixed_deal(request):
+    """Deal variants of the mixed engine: heavy and light lists as two
+    launches, heavy tiles before light ones, evict-first light weights."""
+    import os
+    keys = (request.param, "MOE_GEMM_ENGINE")
+    old = {k: os.environ.get(k) for k in keys}
+    os.environ[request.param] = "1"
+    os.environ["MOE_GEMM_ENGINE"] = "mixed"
+    yield request.param
+    for k, v in old.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "qwen3_medium", "dsv3_medium", "gptoss_small"])
+def test_layer_mixed_deal_variants(name, mixed_deal, dev):
+    test_layer_matches_oracle(name, dev)
+
+
+def test_expert_ffn_group_size_edges_mixed_deal_variants(mixed_deal, dev):
+    test_expert_ffn_group_size_edges("mixed", dev)
+
+
 @pytest.fixture
 def fused_dispatch():
     import os
