@@ -68,8 +68,11 @@ struct ShapeF8 {
   // bytes each SM keeps in flight: five stages hold 160 KB of codes.
   static constexpr int kStages = 5;
   static constexpr uint32_t kRingBytes = kStages * kStageBytes;
-  static constexpr uint32_t kAccCols = 2 * kQRows;        // two accumulators
-  static constexpr uint32_t kTmemCols = 2 * kAccCols;     // double-buffered: 128
+  // an accumulator per code span, each 2 * kQRows columns: the hi plane's
+  // rows in the first kQRows, the lo plane's in the next (one MMA covers both
+  // planes, which lie one after the other in shared memory)
+  static constexpr uint32_t kAccCols = 4 * kQRows;
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;     // double-buffered: 256
   static constexpr uint32_t kStageRowWords = 36;
   static constexpr uint32_t kEpiBytes = 4 * 32 * kStageRowWords * 4;  // 18 KB
   static constexpr int kBars = 2 * kStages + 5;
@@ -285,10 +288,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0, buf = 0;
       uint32_t ph = 0, acc_ph = 0;
       bool ok = true, any = false;
+      // Every operand K-major, 128-byte rows, 8-row groups 1024 B apart; a K
+      // step of 32 e4m3 values is 32 bytes.  The descriptor of stage 0's
+      // first code span plus offsets (16-byte units, all below 256 KB) gives
+      // every operand, so the issuing thread spends about one instruction per
+      // address.
+      const uint64_t st_d0 = smem_desc(smem_addr(ring), 16, 1024);
+      constexpr uint32_t kStageStep = S::kStageBytes >> 4, kK = 32 >> 4;
+      constexpr uint32_t kSpan1 = S::kCodeBytes >> 4, kPlanesAt = (2 * S::kCodeBytes) >> 4;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int g, c, row0, nr;
         tile_coords(tile, g, c, row0, nr);
-        const uint32_t idesc = instr_desc_f8(S::kCols, (nr + 15) & ~15);
+        // N: the hi plane's kQRows rows, then the lo plane's rows (nr rounded
+        // up to 16); hi-plane rows beyond nr only touch accumulator columns
+        // the epilogue never reads
+        const uint32_t idesc = instr_desc_f8(S::kCols, kQRows + ((nr + 15) & ~15));
         if (!wait(acce0 + 8 * buf, acc_ph ^ 1, ctl)) {
           ok = false;
           break;
@@ -301,21 +315,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
-          const uint32_t pl = st + 2 * S::kCodeBytes;
+          const uint64_t sd = st_d0 + s * kStageStep;
+          const uint32_t acc0 = kb != 0;
 #pragma unroll
           for (int kk = 0; kk < kQK / 32; ++kk) {
-            // every operand K-major, 128-byte rows, 8-row groups 1024 B apart;
-            // a K step of 32 e4m3 values is 32 bytes
-            const uint64_t a0 = smem_desc(st + kk * 32, 16, 1024);
-            const uint64_t a1 = smem_desc(st + S::kCodeBytes + kk * 32, 16, 1024);
-#pragma unroll
-            for (int q = 0; q < kPlanes; ++q) {
-              const uint64_t bd = smem_desc(pl + q * S::kPlaneBytes + kk * 32, 16, 1024);
-              const uint32_t acc = (kb | kk | q) != 0;
-              umma_f8(d_tmem, a0, bd, idesc, acc);
-              umma_f8(d_tmem + kQRows, a1, bd, idesc, acc);
-            }
+            const uint32_t acc = kk ? 1u : acc0;
+            umma_f8(d_tmem, sd + kk * kK, sd + kPlanesAt + kk * kK, idesc, acc);
+            umma_f8(d_tmem + 2 * kQRows, sd + kSpan1 + kk * kK, sd + kPlanesAt + kk * kK, idesc,
+                    acc);
           }
           any = true;
           umma_commit(empty0 + 8 * s);
@@ -366,11 +373,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j0 = 0; j0 < nr; j0 += 32) {
           // the row scales of rows j0 .. j0+31 of the tile, one per lane
           const float rs = (j0 + lane < nr) ? p.row_scale[row0 + j0 + lane] : 0.f;
+          // v[j] = out[row j0 + j][col]: the hi plane's and the lo plane's sums
           float v[32];
-          tmem_ld32(tb + h * kQRows + j0, v);  // v[j] = out[row j0 + j][col]
+          tmem_ld32_sum2(tb + h * 2 * kQRows + j0, kQRows, v);
           if (SWIGLU) {
             float u[32];
-            tmem_ld32(tb + kQRows + j0, u);
+            tmem_ld32_sum2(tb + 2 * kQRows + j0, kQRows, u);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float r = __shfl_sync(0xffffffffu, rs, j);

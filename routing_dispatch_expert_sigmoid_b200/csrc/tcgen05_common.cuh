@@ -267,6 +267,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+// Sum of two 32-column loads `off` columns apart (partial sums of one output
+// kept in two accumulators).
+__device__ __forceinline__ void tmem_ld32_sum2(uint32_t taddr, uint32_t off, float *v) {
+  float w[32];
+  tmem_ld32(taddr, v);
+  tmem_ld32(taddr + off, w);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] += w[i];
+}
 
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and
 // stride byte offsets (all >> 4), descriptor version 1, 128-byte swizzle.
