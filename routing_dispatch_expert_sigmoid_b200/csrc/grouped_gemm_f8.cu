@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) {
               const float r = __shfl_sync(0xffffffffu, rs, j);
               const float gt = v[j] * (sc1 * r), up = u[j] * (sc3 * r);
-              v[j] = (gt / (1.0f + __expf(-gt))) * up;
+              v[j] = silu_times(gt, up);
             }
           } else {
 #pragma unroll

@@ -490,16 +490,8 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
       if (t.full) {
         // lane = row: rows row0 + 32*quarter .. of the chunk, 32 columns at a time
         const int row0 = t.row0 + quarter * 32;
-#pragma unroll 1
-        for (int c = 0; c < S::BN; c += 32) {
-          float v[32];
-          tmem_ld32(tb + c, v);
-          if (SWIGLU) {
-            float u[32];
-            tmem_ld32(tb + S::BN + c, u);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
-          }
+        // one 32-column chunk of this warp's 32 rows, from registers to memory
+        auto store_chunk = [&](float(&v)[32], int c) {
           const int col = t.n * S::BN + c;
           if (SWIGLU) {  // h: bf16, a staged row is 16 words
             uint32_t *st = reinterpret_cast<uint32_t *>(stg);
@@ -558,6 +550,22 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
             }
           }
           __syncwarp();  // the next chunk overwrites the staging buffer
+        };
+        // two chunks per wait for tensor memory: gate and up of the same
+        // columns, or two neighbouring column chunks of the plain product
+#pragma unroll 1
+        for (int c = 0; c < S::BN; c += SWIGLU ? 32 : 64) {
+          float v[32], u[32];
+          if (SWIGLU) {
+            tmem_ld32x2(tb + c, tb + S::BN + c, v, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = silu_times(v[i], u[i]);
+            store_chunk(v, c);
+          } else {
+            tmem_ld32x2(tb + c, tb + c + 32, v, u);
+            store_chunk(v, c);
+            store_chunk(u, c + 32);
+          }
         }
       } else {
         // lane = output column (32*quarter .. of each 128-column half), TMEM
@@ -566,13 +574,14 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
           const int col0 = t.n * S::BN + h * 128 + quarter * 32;
 #pragma unroll 1
           for (int j0 = 0; j0 < t.nr; j0 += 32) {
-            float v[32];
-            tmem_ld32(tb + h * S::kHalf + j0, v);  // v[j] = out[row j0 + j][col0 + lane]
+            float v[32], u[32];  // v[j] = out[row j0 + j][col0 + lane]
+            if (SWIGLU)
+              tmem_ld32x2(tb + h * S::kHalf + j0, tb + S::kHalf + j0, v, u);
+            else
+              tmem_ld32(tb + h * S::kHalf + j0, v);
             if (SWIGLU) {
-              float u[32];
-              tmem_ld32(tb + S::kHalf + j0, u);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
+              for (int i = 0; i < 32; ++i) v[i] = silu_times(v[i], u[i]);
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j) stg[j * S::kStageRowWords + lane] = v[j];

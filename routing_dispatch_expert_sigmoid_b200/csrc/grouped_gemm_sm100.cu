@@ -541,17 +541,18 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < S::BN; c += 32) {
         // lane = row: 32 consecutive columns of its row from tensor memory
-        float v[32];
-        tmem_ld32(tb + c, v);
+        float v[32], u[32];
+        if (SWIGLU)
+          tmem_ld32x2(tb + c, tb + S::BN + c, v, u);
+        else
+          tmem_ld32(tb + c, v);
         const int col = n * S::BN + c;
         // split K: every split is the same weight group 0
         if (FP8W) scale_cols(v, p.scale1 + (size_t)(p.k_split ? 0 : g) * p.N, col, p.N);
         if (SWIGLU) {
-          float u[32];
-          tmem_ld32(tb + S::BN + c, u);
           if (FP8W) scale_cols(u, p.scale3 + (size_t)(p.k_split ? 0 : g) * p.N, col, p.N);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
+          for (int i = 0; i < 32; ++i) v[i] = silu_times(v[i], u[i]);
         }
         // Stage the 32 x 32 chunk in shared memory, then write it back row by
         // row so that each warp store covers whole 64/128-byte row segments.
@@ -1065,6 +1066,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int s = 0, buf = 0;
       uint32_t ph = 0, acc_ph = 0;
       bool ok = true, any = false;
+      // descriptors of stage 0 (rows: K-major; weights: MN-major 64-column
+      // spans, LBO = span stride); stage s and K step kk are additions to the
+      // 16-byte address field (every stage lies below 256 KB)
+      const uint64_t rows_d0 = smem_desc(smem_addr(ring), 16, 1024);
+      const uint64_t w_d0 = smem_desc(smem_addr(ring) + S::kABytes, S::kSpanBytes, 1024);
+      constexpr uint32_t kStageStep = S::kStageBytes >> 4, kRowK = 32 >> 4, kWK = 2048 >> 4;
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const PairTile t = pair_tile(tile);
         const uint32_t idesc_swap = instr_desc_pair_swap((t.nr + 15) & ~15);
@@ -1080,16 +1087,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+          const uint64_t rd = rows_d0 + s * kStageStep, wd = w_d0 + s * kStageStep;
+          const uint32_t acc0 = kb != 0;
+          if (t.swap) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            // rows: K-major; weights: MN-major 64-column spans (LBO = span stride)
-            const uint64_t rd = smem_desc(st + kk * 32, 16, 1024);
-            const uint64_t wd = smem_desc(st + S::kABytes + kk * 2048, S::kSpanBytes, 1024);
-            if (t.swap)
-              umma_pair(d_tmem, wd, rd, idesc_swap, (kb | kk) != 0);
-            else
-              umma_pair(d_tmem, rd, wd, S::kIdesc, (kb | kk) != 0);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_pair(d_tmem, wd + kk * kWK, rd + kk * kRowK, idesc_swap, kk ? 1u : acc0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_pair(d_tmem, rd + kk * kRowK, wd + kk * kWK, S::kIdesc, kk ? 1u : acc0);
           }
           any = true;
           umma_commit_pair_both(empty0 + 8 * s);
@@ -1161,10 +1168,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               const float4 uv =
                   *reinterpret_cast<const float4 *>(u_stg + j * S::kStageRowWords + 4 * q);
               if (j0 + j < t.nr && gcol < p.N) {
-                __nv_bfloat162 lo = __floats2bfloat162_rn((gv.x / (1.0f + __expf(-gv.x))) * uv.x,
-                                                          (gv.y / (1.0f + __expf(-gv.y))) * uv.y);
-                __nv_bfloat162 hi = __floats2bfloat162_rn((gv.z / (1.0f + __expf(-gv.z))) * uv.z,
-                                                          (gv.w / (1.0f + __expf(-gv.w))) * uv.w);
+                __nv_bfloat162 lo = __floats2bfloat162_rn(silu_times(gv.x, uv.x),
+                                                          silu_times(gv.y, uv.y));
+                __nv_bfloat162 hi = __floats2bfloat162_rn(silu_times(gv.z, uv.z),
+                                                          silu_times(gv.w, uv.w));
                 uint2 w;
                 w.x = *reinterpret_cast<uint32_t *>(&lo);
                 w.y = *reinterpret_cast<uint32_t *>(&hi);
@@ -1222,16 +1229,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       const int row0 = t.row0 + (int)rank * 128 + quarter * 32;
       const int row_end = s_off[g + 1];
-#pragma unroll 1
-      for (int c = 0; c < S::BN; c += 32) {
-        float v[32];
-        tmem_ld32(tb + c, v);
-        if (SWIGLU) {
-          float u[32];
-          tmem_ld32(tb + S::BN + c, u);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
-        }
+      // one 32-column chunk of this warp's 32 rows, from registers to memory
+      auto store_chunk = [&](float(&v)[32], int c) {
         const int col = n * S::BN + c;
         if (SWIGLU) {
           uint32_t *st = reinterpret_cast<uint32_t *>(stg);
@@ -1296,6 +1295,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         __syncwarp();
+      };
+      // two chunks per wait for tensor memory: gate and up of the same
+      // columns, or two neighbouring column chunks of the plain product
+#pragma unroll 1
+      for (int c = 0; c < S::BN; c += SWIGLU ? 32 : 64) {
+        float v[32], u[32];
+        if (SWIGLU) {
+          tmem_ld32x2(tb + c, tb + S::BN + c, v, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = silu_times(v[i], u[i]);
+          store_chunk(v, c);
+        } else {
+          tmem_ld32x2(tb + c, tb + c + 32, v, u);
+          store_chunk(v, c);
+          store_chunk(u, c + 32);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -1671,21 +1686,22 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
       }
 #pragma unroll 1
       for (int j0 = 0; j0 < nr; j0 += 32) {
-        float v[32];
-        tmem_ld32(tb + j0, v);  // v[j] = out[row j0 + j][col0 + lane]
+        float v[32], u[32];  // v[j] = out[row j0 + j][col0 + lane]
+        if (SWIGLU)
+          tmem_ld32x2(tb + j0, tb + S::kW3Off + j0, v, u);
+        else
+          tmem_ld32(tb + j0, v);
         if (FP8W) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] *= sc1;
         }
         if (SWIGLU) {
-          float u[32];
-          tmem_ld32(tb + S::kW3Off + j0, u);
           if (FP8W) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) u[i] *= sc3;
           }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = (v[i] / (1.0f + __expf(-v[i]))) * u[i];
+          for (int i = 0; i < 32; ++i) v[i] = silu_times(v[i], u[i]);
         }
         // transpose through shared memory: stage[row j][column lane]
 #pragma unroll

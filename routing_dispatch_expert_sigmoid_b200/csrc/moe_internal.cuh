@@ -21,6 +21,14 @@ enum : uint32_t {
 // moe_api.cu), looked up once per device.
 uint32_t *device_error_word();
 
+// SwiGLU's elementwise step, silu(g) * u = g / (1 + e^-g) * u, with the fast
+// reciprocal division (at most 2 ulp; h is rounded to bf16 right after).  For
+// g below about -87 the denominator exceeds 2^126 and the quotient is 0, the
+// limit of silu there.
+__device__ __forceinline__ float silu_times(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
 __device__ __forceinline__ void raise_error(uint32_t *err, uint32_t bit) {
   if (err) atomicOr(err, bit);
 }

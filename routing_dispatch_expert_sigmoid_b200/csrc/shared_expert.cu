@@ -54,10 +54,10 @@ __global__ void __launch_bounds__(256)
       b.w += ub.w;
     }
     // the same SiLU as the grouped GEMM's SwiGLU epilogue
-    const float v0 = (a.x / (1.0f + __expf(-a.x))) * b.x;
-    const float v1 = (a.y / (1.0f + __expf(-a.y))) * b.y;
-    const float v2 = (a.z / (1.0f + __expf(-a.z))) * b.z;
-    const float v3 = (a.w / (1.0f + __expf(-a.w))) * b.w;
+    const float v0 = silu_times(a.x, b.x);
+    const float v1 = silu_times(a.y, b.y);
+    const float v2 = silu_times(a.z, b.z);
+    const float v3 = silu_times(a.w, b.w);
     __nv_bfloat162 p01 = __floats2bfloat162_rn(v0, v1), p23 = __floats2bfloat162_rn(v2, v3);
     h[i] = make_uint2(*reinterpret_cast<uint32_t *>(&p01), *reinterpret_cast<uint32_t *>(&p23));
   }
