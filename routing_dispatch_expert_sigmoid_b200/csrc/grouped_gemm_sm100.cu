@@ -101,8 +101,11 @@ struct Params {
   int nblk = 0;
   // L2 eviction hints on the TMA loads (bf16 single-CTA and pair engines)
   int l2_hints = 0;
-  // pair engine: a group's last, partial 256-row chunk runs swap-AB
+  // pair engine swap-AB tiles: 0 none; 1 groups under 256 rows (a light
+  // list dealt evenly among the others); 2 those and every group's last,
+  // partial 256-row chunk
   int pair_swap = 0;
+  int swap_rows = 0;  // the light list: groups of 1 .. swap_rows rows (< 256)
 };
 
 // Gate weights to apply in the down projection's epilogue (both nullptr: none).
@@ -691,6 +694,12 @@ __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
 // "accumulator empty" barrier.
 // ---------------------------------------------------------------------------
 constexpr int BM2 = 256;  // rows per pair tile
+// Groups of at most this many rows run as swap-AB pair tiles (the light
+// list); larger ones as 256-row pair tiles, padded.  Alternated call by call,
+// swap tiles paid off for groups of a few dozen rows (GPT-OSS-shaped
+// sub-experts) and lost for groups of about 128 (DeepSeek-V3-shaped prefill),
+// whose plain-output swap epilogue is slower than a padded tile's.
+constexpr int kPairSwapRows = 32;
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -889,7 +898,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   for (int g = threadIdx.x; g < p.G; g += kThreads) {
     const int rows = s_off[g + 1] - s_off[g];
     if (rows < 0) bad = true;
-    const bool light = p.pair_swap && rows > 0 && rows < BM2;
+    const bool light = p.pair_swap && rows > 0 && rows <= p.swap_rows;
     s_tstart[g] = (rows > 0 && !light) ? ((rows + BM2 - 1) / BM2) * n_tiles : 0;
     s_lstart[g] = light ? n_tiles : 0;
   }
@@ -930,10 +939,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t leader_acce0 = mapa_shared(acce0, 0);
 
   // tile -> group g, column tile n, 256-row chunk from row0 with nr rows;
-  // chunks fastest.  A group's last, partial chunk runs swap-AB (p.pair_swap):
-  // the weights are the MMA's M (256 columns, 128 per CTA), the chunk's rows
-  // its N, rounded up to 16, so a chunk of a few rows costs a 16-row MMA, not
-  // a 256-row one, while each CTA still streams only half of the weights.
+  // chunks fastest.  A light tile (and, with p.pair_swap == 2, a group's last,
+  // partial chunk) runs swap-AB: the weights are the MMA's M (256 columns,
+  // 128 per CTA), the rows its N, rounded up to 16, so a group of a few rows
+  // costs a 16-row MMA, not a 256-row one, while each CTA still streams only
+  // half of the weights.
   struct PairTile {
     int g, n, row0, nr;
     bool swap;
@@ -970,7 +980,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       t.row0 = s_off[t.g] + m * BM2;
       t.nr = min(BM2, rows - m * BM2);
     }
-    t.swap = p.pair_swap && t.nr < BM2;
+    t.swap = l1 > l0 || (p.pair_swap == 2 && t.nr < BM2);
     return t;
   };
 
@@ -1966,11 +1976,18 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   p.yexp = yexp;
   p.nblk = (N + 31) / 32;
   p.l2_hints = l2_hints_enabled();
-  // MOE_PAIR_SWAP=1: partial chunks as swap-AB pair tiles (off by default:
-  // alternated call by call, the Qwen3-shaped layer ran 1.52 vs 1.46 ms with
-  // them, the others within noise)
+  // Swap-AB pair tiles for groups under 256 rows by default (MOE_PAIR_SWAP=0:
+  // none; =2: every group's partial last chunk too).  Alternated call by
+  // call, the light list made the GPT-OSS- and DeepSeek-V3-shaped layers
+  // faster, while swapping the large remainders of big groups made the
+  // Qwen3- and Mixtral-shaped ones slower (their plain-output swap epilogue
+  // takes twice as long as a row-major one).
   const char *ps = getenv("MOE_PAIR_SWAP");
-  p.pair_swap = (ps && ps[0] == '1') ? 1 : 0;
+  p.pair_swap = (ps && ps[0] == '0') ? 0 : ((ps && ps[0] == '2') ? 2 : 1);
+  // the light list's largest group (MOE_PAIR_SWAP_ROWS, 1..255)
+  const char *sr = getenv("MOE_PAIR_SWAP_ROWS");
+  const int swap_rows = sr ? atoi(sr) : kPairSwapRows;
+  p.swap_rows = swap_rows < 1 ? 1 : (swap_rows > BM2 - 1 ? BM2 - 1 : swap_rows);
   CUtensorMap mx32, mx8;
   if (!make_map_rows(&mx32, A, rows_cap, K, 32) || !make_map_rows(&mx8, A, rows_cap, K, 8))
     return cudaErrorInvalidValue;
@@ -2098,7 +2115,6 @@ static Engine pick_engine(bool swiglu, int rows_cap, int G, const int32_t *offse
   if (env && env[0] == 'm') return offsets ? Engine::kMixed : Engine::kSingle;
   const long long mean_rows = offsets ? (long long)rows_cap / G : fixed_rows;
   if (mean_rows <= 32) return swiglu ? Engine::kSwap : Engine::kSingle;
-  if (offsets && mean_rows <= 256) return Engine::kMixed;
   return Engine::kPair;
 }
 

@@ -377,16 +377,24 @@ def test_layer_with_fp32_expert_rows(name, fp32_expert_rows, dev):
     test_layer_matches_oracle(name, dev)
 
 
-@pytest.fixture
-def pair_swap():
-    """MOE_GEMM_ENGINE=pair with MOE_PAIR_SWAP=1: each group's partial last
-    256-row chunk as a swap-AB pair tile, groups below 256 rows dealt as a
-    light list among the others."""
+@pytest.fixture(params=[("0", None), ("2", None), ("1", "255"), ("1", "1")],
+                ids=["no-swap", "swap-remainders", "light-below-256", "light-1-row"])
+def pair_swap(request):
+    """MOE_GEMM_ENGINE=pair with MOE_PAIR_SWAP=0 (no swap-AB tiles: small
+    groups padded to 256-row pair tiles), 2 (every group's partial last
+    256-row chunk as a swap-AB pair tile too), or the default mode with the
+    light list's row limit (MOE_PAIR_SWAP_ROWS) at its extremes; the default
+    limit runs in every other pair test."""
     import os
-    old = {k: os.environ.get(k) for k in ("MOE_GEMM_ENGINE", "MOE_PAIR_SWAP")}
+    keys = ("MOE_GEMM_ENGINE", "MOE_PAIR_SWAP", "MOE_PAIR_SWAP_ROWS")
+    old = {k: os.environ.get(k) for k in keys}
     os.environ["MOE_GEMM_ENGINE"] = "pair"
-    os.environ["MOE_PAIR_SWAP"] = "1"
-    yield
+    os.environ["MOE_PAIR_SWAP"] = request.param[0]
+    if request.param[1] is None:
+        os.environ.pop("MOE_PAIR_SWAP_ROWS", None)
+    else:
+        os.environ["MOE_PAIR_SWAP_ROWS"] = request.param[1]
+    yield request.param
     for k, v in old.items():
         if v is None:
             os.environ.pop(k, None)
