@@ -563,8 +563,22 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
             store_chunk(v, c);
           } else {
             tmem_ld32x2(tb + c, tb + c + 32, v, u);
-            store_chunk(v, c);
-            store_chunk(u, c + 32);
+            if (p.yexp) {  // y16: both blocks of a row in one 128-byte segment
+              if (p.row_w) {
+                const float wr = p.row_w[p.w_row_src[row0 + lane]];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  v[i] *= wr;
+                  u[i] *= wr;
+                }
+              }
+              store_y16_lane_rows2(v, u, reinterpret_cast<uint32_t *>(stg), S::kStageRowWords,
+                                   lane, row0, row0 + 32, t.n * S::BN + c, p.N, p.out, p.yexp,
+                                   p.nblk);
+            } else {
+              store_chunk(v, c);
+              store_chunk(u, c + 32);
+            }
           }
         }
       } else {

@@ -1318,8 +1318,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           store_chunk(v, c);
         } else {
           tmem_ld32x2(tb + c, tb + c + 32, v, u);
-          store_chunk(v, c);
-          store_chunk(u, c + 32);
+          if (p.yexp) {  // y16: both blocks of a row in one 128-byte segment
+            if (p.row_w && row0 + lane < row_end) {
+              const float wr = p.row_w[p.w_row_src[row0 + lane]];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                v[i] *= wr;
+                u[i] *= wr;
+              }
+            }
+            store_y16_lane_rows2(v, u, reinterpret_cast<uint32_t *>(stg), S::kStageRowWords, lane,
+                                 row0, row_end, n * S::BN + c, p.N, p.out, p.yexp, p.nblk);
+          } else {
+            store_chunk(v, c);
+            store_chunk(u, c + 32);
+          }
         }
       }
       tc_fence_before();

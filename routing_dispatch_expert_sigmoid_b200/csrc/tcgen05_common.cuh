@@ -331,9 +331,9 @@ __host__ __device__ constexpr uint32_t instr_desc_kk(int M, int N) {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int y16_exponent(float m) {
   if (!(m > 0.0f) || !(m <= 3.4028234e38f)) return 0;  // zero or non-finite block
-  int e2;
-  frexpf(m, &e2);  // m = f * 2^e2 with f in [0.5, 1): E = e2 - 1
-  const int e = (e2 - 1) - 14;
+  // E from the exponent field: exact for normal m; a subnormal m reads as
+  // E = -127 and, like its true exponent, ends at the clamp below
+  const int e = (((__float_as_int(m) >> 23) & 0xFF) - 127) - 14;
   return e < -120 ? -120 : (e > 120 ? 120 : e);
 }
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
@@ -371,6 +371,53 @@ __device__ __forceinline__ void store_y16_lane_rows(const float (&v)[32], uint32
     if (grow < row_end && gcol < N)
       *reinterpret_cast<uint4 *>(static_cast<__half *>(out) + (size_t)grow * N + gcol) = val;
   }
+}
+
+// The same for two neighbouring 32-column blocks (v: columns col .., u:
+// col + 32 ..; col a multiple of 64): both blocks of a row are staged as one
+// 128-byte fp16 row, written by 8 lanes with 16-byte stores, 4 rows per
+// instruction.
+__device__ __forceinline__ void store_y16_lane_rows2(const float (&v)[32], const float (&u)[32],
+                                                     uint32_t *st, int row_words, int lane,
+                                                     int row0, int row_end, int col, int N,
+                                                     void *out, int8_t *yexp, int nblk) {
+  float mv = 0.0f, mu = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    mv = fmaxf(mv, fabsf(v[i]));
+    mu = fmaxf(mu, fabsf(u[i]));
+  }
+  const int ev = y16_exponent(mv), eu = y16_exponent(mu);
+  const float iv = pow2f(-ev), iu = pow2f(-eu);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t a[4], b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = __floats2half2_rn(v[q * 8 + 2 * i] * iv, v[q * 8 + 2 * i + 1] * iv);
+      a[i] = *reinterpret_cast<uint32_t *>(&h);
+      h = __floats2half2_rn(u[q * 8 + 2 * i] * iu, u[q * 8 + 2 * i + 1] * iu);
+      b[i] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    *reinterpret_cast<uint4 *>(st + lane * row_words + 4 * q) = make_uint4(a[0], a[1], a[2], a[3]);
+    *reinterpret_cast<uint4 *>(st + lane * row_words + 16 + 4 * q) =
+        make_uint4(b[0], b[1], b[2], b[3]);
+  }
+  if (row0 + lane < row_end) {
+    int8_t *ye = yexp + (size_t)(row0 + lane) * nblk + col / 32;
+    if (col < N) ye[0] = (int8_t)ev;
+    if (col + 32 < N) ye[1] = (int8_t)eu;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {  // 4 rows x 128 bytes per instruction
+    const int r = i * 4 + (lane >> 3), q = lane & 7;
+    const int grow = row0 + r, gcol = col + q * 8;
+    const uint4 val = *reinterpret_cast<const uint4 *>(st + r * row_words + 4 * q);
+    if (grow < row_end && gcol < N)
+      *reinterpret_cast<uint4 *>(static_cast<__half *>(out) + (size_t)grow * N + gcol) = val;
+  }
+  __syncwarp();
 }
 
 // One warp, rows staged transposed (stg[j * row_words + c] = value of row j,
