@@ -338,6 +338,19 @@ __device__ __forceinline__ int y16_exponent(float m) {
 }
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
 
+// Largest magnitude of 32 values as a tree of maxima (depth 5 instead of a
+// chain of 32 dependent steps).  A NaN is skipped, like fmaxf does.
+__device__ __forceinline__ float absmax32(const float (&v)[32]) {
+  float m[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m[i] = fmaxf(fabsf(v[i]), fabsf(v[i + 16]));
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  return m[0];
+}
+
 // One warp, lane = row: its row's 32 values v (columns col .. col+31 of rows
 // row0 + lane) into y16 rows of N columns and their block exponents
 // (nblk = ceil(N / 32) per row), through the warp's staging buffer st (32
@@ -346,10 +359,7 @@ __device__ __forceinline__ void store_y16_lane_rows(const float (&v)[32], uint32
                                                     int row_words, int lane, int row0,
                                                     int row_end, int col, int N, void *out,
                                                     int8_t *yexp, int nblk) {
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
-  const int e = y16_exponent(m);
+  const int e = y16_exponent(absmax32(v));
   const float inv = pow2f(-e);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -381,13 +391,7 @@ __device__ __forceinline__ void store_y16_lane_rows2(const float (&v)[32], const
                                                      uint32_t *st, int row_words, int lane,
                                                      int row0, int row_end, int col, int N,
                                                      void *out, int8_t *yexp, int nblk) {
-  float mv = 0.0f, mu = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    mv = fmaxf(mv, fabsf(v[i]));
-    mu = fmaxf(mu, fabsf(u[i]));
-  }
-  const int ev = y16_exponent(mv), eu = y16_exponent(mu);
+  const int ev = y16_exponent(absmax32(v)), eu = y16_exponent(absmax32(u));
   const float iv = pow2f(-ev), iu = pow2f(-eu);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
