@@ -1197,13 +1197,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int j0 = 0; j0 < t.nr; j0 += 32) {
             float v[32];
             tmem_ld32(tb + j0, v);  // v[j] = y[row j0 + j][col0 + lane]
+            if (p.yexp) {
+              store_y16_lane_cols(v, reinterpret_cast<uint32_t *>(stg), S::kStageRowWords, lane,
+                                  t.row0 + j0, t.nr - j0, col0, p.N, p.out, p.yexp, p.nblk,
+                                  p.row_w, p.w_row_src);
+              continue;
+            }
 #pragma unroll
             for (int j = 0; j < 32; ++j) stg[j * S::kStageRowWords + lane] = v[j];
             __syncwarp();
-            if (p.yexp) {
-              store_y16_staged(stg, S::kStageRowWords, lane, t.row0 + j0, t.nr - j0, col0, p.N,
-                               p.out, p.yexp, p.nblk, p.row_w, p.w_row_src);
-            } else {
+            {
 #pragma unroll
               for (int i = 0; i < 8; ++i) {  // fp32 rows: 8 lanes x 16 bytes, 4 rows per step
                 const int j = i * 4 + (lane >> 3), q = lane & 7;

@@ -424,6 +424,48 @@ __device__ __forceinline__ void store_y16_lane_rows2(const float (&v)[32], const
   __syncwarp();
 }
 
+// One warp, lane = column: v[j] is row row0 + j, column col0 + lane (col0 a
+// multiple of 32, so the warp holds exactly one exponent block of each row).
+// Rows j < nr into y16 rows and their block exponents: each row's largest
+// magnitude is one warp reduction on the magnitudes' bit patterns (their
+// order as unsigned integers is the order of the values; a NaN counts as 0,
+// as fmaxf skips it); the fp16 values go through the staging buffer st (32
+// rows of row_words words) and leave as whole 64-byte row segments.  wr:
+// per-row factor source (row_w[w_row_src[row]]) or nullptr.
+__device__ __forceinline__ void store_y16_lane_cols(float (&v)[32], uint32_t *st, int row_words,
+                                                    int lane, int row0, int nr, int col0, int N,
+                                                    void *out, int8_t *yexp, int nblk,
+                                                    const float *row_w,
+                                                    const int32_t *w_row_src) {
+  if (row_w) {
+    const float wl = lane < nr ? row_w[w_row_src[row0 + lane]] : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
+  }
+  __half *sh = reinterpret_cast<__half *>(st);
+  const int rh = 2 * row_words;  // halves per staged row
+  int my_e = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float a = fabsf(v[j]);
+    const uint32_t key = a != a ? 0u : __float_as_uint(a);
+    const int e = y16_exponent(__uint_as_float(__reduce_max_sync(0xffffffffu, key)));
+    if (lane == j) my_e = e;
+    sh[j * rh + lane] = __float2half_rn(v[j] * pow2f(-e));
+  }
+  if (lane < nr && col0 < N) yexp[(size_t)(row0 + lane) * nblk + col0 / 32] = (int8_t)my_e;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // 8 rows x 64 bytes per instruction
+    const int r = i * 8 + (lane >> 2), q = lane & 3;
+    const int gcol = col0 + q * 8;
+    const uint4 val = *reinterpret_cast<const uint4 *>(sh + r * rh + q * 8);
+    if (r < nr && gcol < N)
+      *reinterpret_cast<uint4 *>(static_cast<__half *>(out) + (size_t)(row0 + r) * N + gcol) = val;
+  }
+  __syncwarp();
+}
+
 // One warp, rows staged transposed (stg[j * row_words + c] = value of row j,
 // column col0 + c): rows j < nr of rows row0 .. into y16 rows and their block
 // exponents; 8 lanes per row, 4 columns each.  wr: per-row factor source
