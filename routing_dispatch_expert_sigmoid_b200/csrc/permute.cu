@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(256)
 // the slot's weight (w * 2^e is exact).  A lane owns VPL output vectors
 // (work items of 32 VPL vectors), so that a top-2 layer still has a few
 // loads in flight per lane.
-template <int KB, int VPL>
+template <int KB, int VPL, typename Idx>
 __global__ void __launch_bounds__(256)
     k_combine_y16(const uint4 *__restrict__ y, const int8_t *__restrict__ yexp, int nblk,
                   const int32_t *__restrict__ slot_row, const float *__restrict__ topk_w,
@@ -229,10 +229,11 @@ __global__ void __launch_bounds__(256)
   const int lane = threadIdx.x % 32, wib = threadIdx.x / 32;
   constexpr int kItemVecs = 32 * VPL;
   const int chunks = (row_vecs + kItemVecs - 1) / kItemVecs;
-  const long long items = (long long)Tn * chunks;
-  const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+  // Idx: int when the work items fit (no 64-bit divisions in the loop)
+  const Idx items = (Idx)Tn * chunks;
+  const Idx warps = (Idx)gridDim.x * (blockDim.x / 32);
   const size_t sh_vecs = (size_t)row_vecs * 2;  // fp32 vectors per shared row
-  long long it = (long long)blockIdx.x * (blockDim.x / 32) + wib;
+  Idx it = (Idx)blockIdx.x * (blockDim.x / 32) + wib;
   int next_row = -1;
   float next_w = 0.f;
   if (it < items && lane < k_max) {
@@ -398,16 +399,29 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
     const auto *sh = static_cast<const uint4 *>(shared_y);
     auto *o = static_cast<uint4 *>(out);
     const int nblk = (c.d + 31) / 32, rows_cap = c.T * c.k_max;
+    // 32-bit item indices unless T x chunks (plus a grid's worth of warps)
+    // could pass 2^31
+    const bool narrow = (long long)c.T * ((row_vecs + 31) / 32) + 148LL * 64 < (1LL << 31);
+    auto launch = [&](auto kernel, int g) {
+      kernel<<<g, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o, c.T, c.k_max,
+                               rows_cap, row_vecs, err);
+    };
     if (c.k_max <= 2) {  // two vectors per lane: items of 64 vectors
       const int g2 = grid_for((long long)c.T * ((row_vecs + 63) / 64));
-      k_combine_y16<2, 2><<<g2, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o,
-                                             c.T, c.k_max, rows_cap, row_vecs, err);
+      if (narrow)
+        launch(k_combine_y16<2, 2, int>, g2);
+      else
+        launch(k_combine_y16<2, 2, long long>, g2);
     } else if (c.k_max <= 4) {
-      k_combine_y16<4, 1><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts,
-                                               o, c.T, c.k_max, rows_cap, row_vecs, err);
+      if (narrow)
+        launch(k_combine_y16<4, 1, int>, grid);
+      else
+        launch(k_combine_y16<4, 1, long long>, grid);
     } else {
-      k_combine_y16<8, 1><<<grid, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts,
-                                               o, c.T, c.k_max, rows_cap, row_vecs, err);
+      if (narrow)
+        launch(k_combine_y16<8, 1, int>, grid);
+      else
+        launch(k_combine_y16<8, 1, long long>, grid);
     }
     return cudaGetLastError();
   }
