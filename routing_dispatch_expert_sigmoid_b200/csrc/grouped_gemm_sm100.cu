@@ -1971,7 +1971,7 @@ template <bool SWIGLU>
 cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offsets,
                         int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
                         uint32_t *err, cudaStream_t s, RowWeights rw = RowWeights(),
-                        int8_t *yexp = nullptr) {
+                        int8_t *yexp = nullptr, const float *bias = nullptr) {
   using S = Shape2<SWIGLU>;
   CUtensorMap ma, mb1, mb3;
   if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
@@ -1986,7 +1986,7 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_pair<SWIGLU>,
                                     S::kSmemFixed + sizeof(int32_t) * 3 * (kMaxGroups + 1)))
     return e;
-  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, nullptr, nullptr, 1, err};
+  Params p{offsets, G, fixed_rows, rows_cap, K, N, out, bias, nullptr, 1, err};
   p.row_w = rw.w;
   p.w_row_src = rw.row_src;
   p.yexp = yexp;
@@ -2283,6 +2283,14 @@ cudaError_t launch_router_tc(int T, int d, int E, const void *x, const void *Wr,
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Many experts and a long batch: CTA pairs (256 x 256 tiles, half the
+  // operand bytes per SM of a single-CTA tile), as for the expert GEMMs.
+  // MOE_ROUTER_PAIR=0/1 forces the choice.
+  const char *rp = getenv("MOE_ROUTER_PAIR");
+  const bool pair = rp ? rp[0] == '1' : (E >= 512 && T >= 2048);
+  if (pair)
+    return tc::launch_pair<false>(T, d, E, 1, nullptr, T, x, Wr, Wr, logits, err, s,
+                                  tc::RowWeights(), nullptr, bias);
   const long long row_tiles = (T + tc::BM - 1) / tc::BM;
   int spans = 1;
   long long best = -1;

@@ -61,6 +61,38 @@ def test_route_bit_exact_and_logits(name, dev):
     check_routing_bit_exact(w, hin, out)
 
 
+# The router GEMM on CTA pairs (default for E >= 512 and T >= 2048; forced on
+# here): ragged T and E across the 256-row and 256-column tile edges, every
+# gating mode, with and without the logit bias.
+PAIR_ROUTER = {
+    "gptoss_like": WORKLOADS["gptoss_sub"].scaled(T=600, d=200, E=512, k_max=16, k_min=8, f=64),
+    "qwen3_like_ragged": WORKLOADS["qwen3_prefill"].scaled(T=257, d=136, E=136, k_max=8, f=64),
+    "dsv3_like": WORKLOADS["dsv3_prefill"].scaled(T=300, d=256, E=256, f=64, f_shared=64),
+    "mixtral_like_e8": WORKLOADS["mixtral_prefill"].scaled(T=513, d=128, f=64),
+}
+
+
+@pytest.mark.parametrize("name", list(PAIR_ROUTER))
+def test_pair_router_bit_exact_and_logits(name, dev):
+    import os
+    old = os.environ.get("MOE_ROUTER_PAIR")
+    os.environ["MOE_ROUTER_PAIR"] = "1"
+    try:
+        w = PAIR_ROUTER[name]
+        hin = _host_inputs(w, seed=7)
+        inp = gpu_inputs(w, 7, dev, hin)
+        cfg, out = run_route(w, inp)
+        ref = oracle.router_logits(to_numpy(hin["x"]), to_numpy(hin["Wr"]),
+                                   to_numpy(hin["logit_bias"]))
+        assert_logits_close(out["logits"], ref)
+        check_routing_bit_exact(w, hin, out)
+    finally:
+        if old is None:
+            os.environ.pop("MOE_ROUTER_PAIR", None)
+        else:
+            os.environ["MOE_ROUTER_PAIR"] = old
+
+
 # The CUDA-core router (fp32 layers, and bf16 layers whose E is not a multiple
 # of 8): one warp per token for short batches with at most 16 experts, the
 # tiled kernel beyond 2048 tokens or 16 experts.
