@@ -1030,11 +1030,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const CUtensorMap *mb = (SWIGLU && rank == 1) ? &tmB3 : &tmB1;
             const int bcol = SWIGLU ? t.n * S::BN : t.n * S::BN + (int)rank * 128;
             if (p.l2_hints) {
-              tma_load_2d_pair_hint(st, &tmA, lfb, kb * BK, row, pol_keep);
+              // 1: rows evict-last, weights evict-first; 2: rows evict-last,
+              // weights unhinted; 3: rows unhinted, weights evict-last
+              if (p.l2_hints == 3)
+                tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
+              else
+                tma_load_2d_pair_hint(st, &tmA, lfb, kb * BK, row, pol_keep);
 #pragma unroll
-              for (int j = 0; j < 2; ++j)
-                tma_load_3d_pair_hint(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
-                                      kb * BK, t.g, pol_stream);
+              for (int j = 0; j < 2; ++j) {
+                if (p.l2_hints == 2)
+                  tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
+                                   kb * BK, t.g);
+                else
+                  tma_load_3d_pair_hint(st + S::kABytes + j * S::kSpanBytes, mb, lfb,
+                                        bcol + j * 64, kb * BK, t.g,
+                                        p.l2_hints == 3 ? pol_keep : pol_stream);
+              }
             } else {
               tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
 #pragma unroll

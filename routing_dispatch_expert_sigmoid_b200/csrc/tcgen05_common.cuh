@@ -143,9 +143,12 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap
 // (4.63 vs 4.36 ms) and the Qwen3- and GPT-OSS-shaped layers 2-3% slower;
 // streamed weights marked evict-first leave L2 before the other CTAs of the
 // same row tiles read them.
+// MOE_L2_HINTS: 0 none (default); 1 rows evict-last and weights
+// evict-first; the CTA-pair engine also takes 2 (rows evict-last only) and 3
+// (weights evict-last only).
 inline int l2_hints_enabled() {
   const char *env = getenv("MOE_L2_HINTS");
-  return (env && env[0] == '1') ? 1 : 0;
+  return (env && env[0] >= '1' && env[0] <= '3') ? env[0] - '0' : 0;
 }
 
 // Four rows (r0..r3) of 64 columns starting at column c0 into 4 consecutive

@@ -448,12 +448,13 @@ def test_expert_ffn_pair_with_swap_tiles(name, pair_swap, dev):
     test_expert_ffn_matches_oracle(name, dev)
 
 
-@pytest.fixture
-def l2_hints():
-    """MOE_L2_HINTS=1: the GEMMs' TMA loads carry L2 eviction hints."""
+@pytest.fixture(params=["1", "2", "3"])
+def l2_hints(request):
+    """MOE_L2_HINTS=1|2|3: the GEMMs' TMA loads carry L2 eviction hints (the
+    CTA-pair engine's three policies)."""
     import os
     old = os.environ.get("MOE_L2_HINTS")
-    os.environ["MOE_L2_HINTS"] = "1"
+    os.environ["MOE_L2_HINTS"] = request.param
     yield
     if old is None:
         os.environ.pop("MOE_L2_HINTS", None)
