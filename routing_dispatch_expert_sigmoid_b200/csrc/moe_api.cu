@@ -426,7 +426,13 @@ static moe_status layer_impl(const moe_config *cfg, const void *x, const void *W
     MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x, we, at<void>(ws, L.h), y_perm, err,
                      s, ev, 3, r.row_src, gate_w, gate_src, yexp));
   } else {
-    MOE_TRY_CUDA(launch_dispatch(c, x, r.offsets, r.row_src, x_perm, err, s));
+    // long batches: walked by token, so that each row of x leaves HBM once
+    // (MOE_DISPATCH_BY_ROW=1 keeps the walk by destination row)
+    const char *byrow = getenv("MOE_DISPATCH_BY_ROW");
+    if (c.T >= 1024 && !(byrow && byrow[0] == '1'))
+      MOE_TRY_CUDA(launch_dispatch_by_token(c, x, r.slot_row, x_perm, err, s));
+    else
+      MOE_TRY_CUDA(launch_dispatch(c, x, r.offsets, r.row_src, x_perm, err, s));
     MOE_TRY_CUDA(ev.mark(2, s));
     MOE_TRY(ffn_impl(c, c.E, r.offsets, 0, rows_cap, c.f, x_perm, we, at<void>(ws, L.h), y_perm,
                      err, s, ev, 3, nullptr, gate_w, gate_src, yexp));

@@ -69,6 +69,10 @@ cudaError_t launch_capacity(const moe_config &c, const int32_t *topk_idx, int32_
                             cudaStream_t s);
 
 // K4: x_perm[r] = x[row_src[r] / k_max] for r < offsets[E].
+// The dispatch walked by token (x rows read once; moe_layer, long batches).
+cudaError_t launch_dispatch_by_token(const moe_config &c, const void *x,
+                                     const int32_t *slot_row, void *x_perm, uint32_t *err,
+                                     cudaStream_t s);
 cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *offsets,
                             const int32_t *row_src, void *x_perm, uint32_t *err, cudaStream_t s);
 

@@ -72,6 +72,48 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The same copy walked by token: a warp reads a token's row once and stores
+// it to each of the token's kept rows (slot_row[t, j] >= 0).  For long
+// batches the rows of x are then read from HBM once: walked by destination
+// row, each token row is fetched k_t times, and the x_perm stores push it
+// out of L2 between the fetches.
+template <int VPL>
+__global__ void __launch_bounds__(256)
+    k_dispatch_tok(const uint4 *__restrict__ x, const int32_t *__restrict__ slot_row,
+                   uint4 *__restrict__ x_perm, int T, int k_max, int rows_cap, int row_vecs,
+                   uint32_t *err) {
+  constexpr int kChunkVecs = 32 * VPL;
+  const int lane = threadIdx.x % 32;
+  const int warps = gridDim.x * (blockDim.x / 32);
+  for (int t = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; t < T; t += warps) {
+    int my_row = -1;  // lane j: the destination of slot j
+    if (lane < k_max) my_row = slot_row[(size_t)t * k_max + lane];
+    if (my_row >= rows_cap || my_row < -1) {
+      raise_error(err, kErrIndex);
+      my_row = -1;
+    }
+    const unsigned live = __ballot_sync(0xffffffffu, my_row >= 0);
+    const uint4 *src = x + (size_t)t * row_vecs;
+    for (int c0 = 0; c0 < row_vecs; c0 += kChunkVecs) {
+      uint4 u[VPL];
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int v = c0 + lane + 32 * i;
+        if (v < row_vecs) u[i] = ldg_nc(src + v);
+      }
+      for (unsigned m = live; m; m &= m - 1) {
+        const int j = __ffs(m) - 1;
+        uint4 *dst = x_perm + (size_t)__shfl_sync(0xffffffffu, my_row, j) * row_vecs;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          const int v = c0 + lane + 32 * i;
+          if (v < row_vecs) dst[v] = u[i];
+        }
+      }
+    }
+  }
+}
+
 // 16 bytes of T as fp32 values.
 template <typename T>
 struct Vec;
@@ -336,6 +378,19 @@ int grid_for(long long warps_needed) {
 }
 
 }  // namespace
+
+cudaError_t launch_dispatch_by_token(const moe_config &c, const void *x,
+                                     const int32_t *slot_row, void *x_perm, uint32_t *err,
+                                     cudaStream_t s) {
+  const int esz = c.dtype == MOE_F32 ? 4 : 2;
+  const int rows_cap = c.T * c.k_max;
+  if (rows_cap == 0) return cudaSuccess;
+  const int row_vecs = c.d * esz / 16;
+  k_dispatch_tok<8><<<grid_for(c.T), 256, 0, s>>>(static_cast<const uint4 *>(x), slot_row,
+                                                  static_cast<uint4 *>(x_perm), c.T, c.k_max,
+                                                  rows_cap, row_vecs, err);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *offsets,
                             const int32_t *row_src, void *x_perm, uint32_t *err,

@@ -493,6 +493,34 @@ def test_expert_ffn_group_size_edges_mixed_deal_variants(mixed_deal, dev):
     test_expert_ffn_group_size_edges("mixed", dev)
 
 
+# moe_layer dispatches long batches (T >= 1024) walking tokens: each row of x
+# is read once and stored to every kept row of the token.  Ragged d (rows not
+# a whole number of 4 KB chunks), capacity drops, variable k.
+TOKEN_DISPATCH = {
+    "qwen3_drops_ragged_d": WORKLOADS["qwen3_prefill"].scaled(T=1100, d=200, E=16, k_max=4,
+                                                              f=64),
+    "gptoss_variable_k": WORKLOADS["gptoss_sub"].scaled(T=1500, d=136, E=64, k_max=8, k_min=2,
+                                                        f=64),
+    "mixtral_wide_rows": WORKLOADS["mixtral_prefill"].scaled(T=1024, d=2056, f=64),
+}
+
+
+@pytest.mark.parametrize("by_row", ["0", "1"], ids=["by-token", "by-row"])
+@pytest.mark.parametrize("name", list(TOKEN_DISPATCH))
+def test_layer_dispatch_walks(name, by_row, dev):
+    import os
+    old = os.environ.get("MOE_DISPATCH_BY_ROW")
+    os.environ["MOE_DISPATCH_BY_ROW"] = by_row
+    try:
+        w = TOKEN_DISPATCH[name]
+        _layer_vs_oracle(w, _host_inputs(w, seed=11), dev)
+    finally:
+        if old is None:
+            os.environ.pop("MOE_DISPATCH_BY_ROW", None)
+        else:
+            os.environ["MOE_DISPATCH_BY_ROW"] = old
+
+
 @pytest.fixture
 def fused_dispatch():
     import os
