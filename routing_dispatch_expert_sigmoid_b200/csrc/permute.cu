@@ -260,8 +260,11 @@ __global__ void __launch_bounds__(256)
 // the slot's weight (w * 2^e is exact).  A lane owns VPL output vectors
 // (work items of 32 VPL vectors), so that a top-2 layer still has a few
 // loads in flight per lane.
+// At least two CTAs (16 warps) per SM: left alone the compiler gives the
+// kernel over 160 registers, one CTA per SM, and the y16 reads half the
+// loads in flight they need (Qwen3-shaped combine 0.20 vs 0.13 ms).
 template <int KB, int VPL, typename Idx>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
     k_combine_y16(const uint4 *__restrict__ y, const int8_t *__restrict__ yexp, int nblk,
                   const int32_t *__restrict__ slot_row, const float *__restrict__ topk_w,
                   const uint4 *__restrict__ shared_y, int shared_parts, uint4 *__restrict__ out,
