@@ -87,6 +87,12 @@ PROFILES = os.path.join(ROOT, "profiles")
 GEMM_SRC = os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc",
                         "grouped_gemm_sm100.cu")
 PERMUTE_SRC = os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc", "permute.cu")
+F8_SRC = os.path.join(ROOT, "routing_dispatch_expert_sigmoid_b200", "csrc", "grouped_gemm_f8.cu")
+
+
+def w_is_decode(workload: str) -> bool:
+    """Decode-sized legs with fp8 weights run on the kind::f8f6f4 engine."""
+    return "decode" in workload
 METRIC = "MoE-layer tokens/sec on 1 B200 (decode & prefill); % of roofline"
 PREFILL, DECODE = "mixtral_prefill", "mixtral_decode"
 L2_BYTES = 126 * 2 ** 20
@@ -306,8 +312,14 @@ def profile_summary(path: str, src: str):
 
 
 def traffic_from_profile(workload: str, kernel: str = "k5_up_swiglu"):
-    """DRAM bytes per launch of a stage's kernel from profiles/<kernel>_<workload>.md."""
-    src = PERMUTE_SRC if kernel.startswith(("k4", "k7")) else GEMM_SRC
+    """DRAM bytes per launch of a stage's kernel from profiles/<kernel>_<workload>.md
+    (workload names ending in _fp8: the legs with e4m3 expert weights)."""
+    if kernel.startswith(("k4", "k7")):
+        src = PERMUTE_SRC
+    elif workload.endswith("_fp8") and w_is_decode(workload):
+        src = F8_SRC
+    else:
+        src = GEMM_SRC
     return profile_summary(os.path.join(PROFILES, f"{kernel}_{workload}.md"), src)
 
 
