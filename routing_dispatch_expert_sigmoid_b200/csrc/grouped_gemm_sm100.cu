@@ -1359,7 +1359,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
       };
       // two chunks per wait for tensor memory: gate and up of the same
-      // columns, or two neighbouring column chunks of the plain product
+      // columns, or two neighbouring column chunks of the plain product;
+      // y16: the row's eight block exponents of the tile gathered in exps
+      uint64_t exps = 0;
 #pragma unroll 1
       for (int c = 0; c < S::BN; c += SWIGLU ? 32 : 64) {
         float v[32], u[32];
@@ -1379,12 +1381,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 u[i] *= wr;
               }
             }
+            uint32_t e2;
             store_y16_lane_rows2(v, u, reinterpret_cast<uint32_t *>(stg), S::kStageRowWords, lane,
-                                 row0, row_end, n * S::BN + c, p.N, p.out, p.yexp, p.nblk);
+                                 row0, row_end, n * S::BN + c, p.N, p.out, nullptr, p.nblk, &e2);
+            exps |= (uint64_t)e2 << (2 * c / 8);  // blocks c/32 and c/32 + 1 of the tile
           } else {
             store_chunk(v, c);
             store_chunk(u, c + 32);
           }
+        }
+      }
+      if (!SWIGLU && p.yexp && row0 + lane < row_end) {
+        // one 8-byte store per row when the tile's 8 blocks are whole and
+        // aligned, else the valid ones a byte each
+        const int b0 = n * (S::BN / 32), nb = min(S::BN / 32, p.nblk - b0);
+        int8_t *ye = p.yexp + (size_t)(row0 + lane) * p.nblk + b0;
+        if (nb == 8 && (reinterpret_cast<uintptr_t>(ye) & 7) == 0) {
+          *reinterpret_cast<uint64_t *>(ye) = exps;
+        } else {
+          for (int b = 0; b < nb; ++b) ye[b] = (int8_t)(exps >> (8 * b));
         }
       }
       tc_fence_before();

@@ -389,11 +389,13 @@ __device__ __forceinline__ void store_y16_lane_rows(const float (&v)[32], uint32
 // The same for two neighbouring 32-column blocks (v: columns col .., u:
 // col + 32 ..; col a multiple of 64): both blocks of a row are staged as one
 // 128-byte fp16 row, written by 8 lanes with 16-byte stores, 4 rows per
-// instruction.
+// instruction.  With yexp == nullptr the two exponents are returned in
+// *e2 (block col/32 in the low byte) for the caller to store with others.
 __device__ __forceinline__ void store_y16_lane_rows2(const float (&v)[32], const float (&u)[32],
                                                      uint32_t *st, int row_words, int lane,
                                                      int row0, int row_end, int col, int N,
-                                                     void *out, int8_t *yexp, int nblk) {
+                                                     void *out, int8_t *yexp, int nblk,
+                                                     uint32_t *e2 = nullptr) {
   const int ev = y16_exponent(absmax32(v)), eu = y16_exponent(absmax32(u));
   const float iv = pow2f(-ev), iu = pow2f(-eu);
 #pragma unroll
@@ -410,7 +412,9 @@ __device__ __forceinline__ void store_y16_lane_rows2(const float (&v)[32], const
     *reinterpret_cast<uint4 *>(st + lane * row_words + 16 + 4 * q) =
         make_uint4(b[0], b[1], b[2], b[3]);
   }
-  if (row0 + lane < row_end) {
+  if (!yexp) {
+    *e2 = (uint32_t)(uint8_t)ev | ((uint32_t)(uint8_t)eu << 8);
+  } else if (row0 + lane < row_end) {
     int8_t *ye = yexp + (size_t)(row0 + lane) * nblk + col / 32;
     if (col < N) ye[0] = (int8_t)ev;
     if (col + 32 < N) ye[1] = (int8_t)eu;
