@@ -1396,8 +1396,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // aligned, else the valid ones a byte each
         const int b0 = n * (S::BN / 32), nb = min(S::BN / 32, p.nblk - b0);
         int8_t *ye = p.yexp + (size_t)(row0 + lane) * p.nblk + b0;
-        if (nb == 8 && (reinterpret_cast<uintptr_t>(ye) & 7) == 0) {
+        const uintptr_t al = reinterpret_cast<uintptr_t>(ye);
+        if (nb == 8 && (al & 7) == 0) {
           *reinterpret_cast<uint64_t *>(ye) = exps;
+        } else if (nb == 8 && (al & 1) == 0) {  // e.g. 90 blocks a row: 2-byte aligned
+#pragma unroll
+          for (int b = 0; b < 8; b += 2)
+            *reinterpret_cast<uint16_t *>(ye + b) = (uint16_t)(exps >> (8 * b));
         } else {
           for (int b = 0; b < nb; ++b) ye[b] = (int8_t)(exps >> (8 * b));
         }
