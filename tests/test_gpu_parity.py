@@ -521,6 +521,22 @@ def test_layer_dispatch_walks(name, by_row, dev):
             os.environ["MOE_DISPATCH_BY_ROW"] = old
 
 
+@pytest.mark.parametrize("name", ["qwen3_medium", "dsv3_medium", "gptoss_small"])
+def test_layer_combine_one_vector_per_lane(name, dev):
+    """MOE_COMBINE_VPL=1: the top-8 y16 combine with one 16-byte vector per
+    lane per row (the default takes two)."""
+    import os
+    old = os.environ.get("MOE_COMBINE_VPL")
+    os.environ["MOE_COMBINE_VPL"] = "1"
+    try:
+        test_layer_matches_oracle(name, dev)
+    finally:
+        if old is None:
+            os.environ.pop("MOE_COMBINE_VPL", None)
+        else:
+            os.environ["MOE_COMBINE_VPL"] = old
+
+
 @pytest.fixture
 def fused_dispatch():
     import os
