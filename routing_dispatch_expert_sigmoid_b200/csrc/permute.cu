@@ -354,8 +354,11 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[q]));
-                acc[i][2 * q] = fmaf(wj, f.x, acc[i][2 * q]);
-                acc[i][2 * q + 1] = fmaf(wj, f.y, acc[i][2 * q + 1]);
+                // one packed fp32 FMA for the pair (each half rounded as fmaf)
+                const float2 s2 = __ffma2_rn(make_float2(wj, wj), f,
+                                             make_float2(acc[i][2 * q], acc[i][2 * q + 1]));
+                acc[i][2 * q] = s2.x;
+                acc[i][2 * q + 1] = s2.y;
               }
             }
           }

@@ -402,10 +402,12 @@ __device__ __forceinline__ void store_y16_lane_rows2(const float (&v)[32], const
   for (int q = 0; q < 4; ++q) {
     uint32_t a[4], b[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __half2 h = __floats2half2_rn(v[q * 8 + 2 * i] * iv, v[q * 8 + 2 * i + 1] * iv);
+    for (int i = 0; i < 4; ++i) {  // packed scaling by the powers of two (exact)
+      __half2 h = __float22half2_rn(
+          __fmul2_rn(make_float2(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]), make_float2(iv, iv)));
       a[i] = *reinterpret_cast<uint32_t *>(&h);
-      h = __floats2half2_rn(u[q * 8 + 2 * i] * iu, u[q * 8 + 2 * i + 1] * iu);
+      h = __float22half2_rn(
+          __fmul2_rn(make_float2(u[q * 8 + 2 * i], u[q * 8 + 2 * i + 1]), make_float2(iu, iu)));
       b[i] = *reinterpret_cast<uint32_t *>(&h);
     }
     *reinterpret_cast<uint4 *>(st + lane * row_words + 4 * q) = make_uint4(a[0], a[1], a[2], a[3]);
