@@ -25,7 +25,9 @@ Extra keys of the JSON line:
                bytes at the measured copy bandwidth takes longer (the same peaks
                as layer_roofline_frac).  Compute-bound kernels also carry
                frac_at_sampled_clock: achieved over the peak scaled by the
-               median sampled SM clock over the maximum clock;
+               median sampled SM clock over the maximum clock (null, with
+               sampled_clock_note, under 8 samples or when it would exceed 1:
+               the snapshots then missed the clock the kernel ran at);
   kernels      the same for the dispatch (K4), up projection (K5), down
                projection (K6) and combine (K7) stages;
   e2e          the same metric through the C ABI with host buffers: per step a
@@ -152,6 +154,9 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
                 "enforced.power.limit")
 
 
+MIN_CLOCK_SAMPLES = 8  # before a clock-scaled fraction is reported
+
+
 class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
@@ -163,7 +168,7 @@ class ClockSampler:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.file,
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.file,
                 stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -333,11 +338,23 @@ def roofline_obj(kind: str, achieved: float, peak: float, unit: str, traffic, pe
     o = {"bound": kind, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
          "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
          "work_per_launch": work, "ms_per_launch": round(ms, 5)}
-    # the tensor and ALU peaks scale with the SM clock; HBM bandwidth does not
+    # the tensor and ALU peaks scale with the SM clock; HBM bandwidth does not.
+    # nvidia-smi gives clock snapshots, which swing by hundreds of MHz under
+    # the power cap: the scaled fraction needs enough of them, and one above
+    # 1 says the snapshots missed the clock the kernel ran at
     if kind in ("tensor", "alu") and clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
         o["sm_mhz"] = clocks["sm_mhz"]
-        o["frac_at_sampled_clock"] = round(
-            achieved / (peak * clocks["sm_mhz"] / clocks["sm_max_mhz"]), 4)
+        n = clocks.get("samples", 0)
+        v = achieved / (peak * clocks["sm_mhz"] / clocks["sm_max_mhz"])
+        if n < MIN_CLOCK_SAMPLES:
+            o["frac_at_sampled_clock"] = None
+            o["sampled_clock_note"] = f"{n} clock samples in the timed region: too few"
+        elif v > 1.0:
+            o["frac_at_sampled_clock"] = None
+            o["sampled_clock_note"] = ("the median sampled clock is below the clock the kernel "
+                                       "ran at (snapshots under the power cap): not reported")
+        else:
+            o["frac_at_sampled_clock"] = round(v, 4)
     return o
 
 

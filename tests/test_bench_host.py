@@ -144,13 +144,24 @@ def test_kernel_roofline_uses_the_burst_peak_whatever_the_clock_reasons():
 
 
 def test_frac_at_sampled_clock_scales_the_compute_peak_only():
-    clocks = {"sm_mhz": 1320.0, "sm_max_mhz": 1965.0}
-    t = bench.kernel_roofline(1661.1e9, 1e6, 1.0, PEAKS, "measured", clocks=clocks)
-    assert t["bound"] == "tensor" and t["frac"] == pytest.approx(1.0)
-    assert t["frac_at_sampled_clock"] == pytest.approx(1965.0 / 1320.0, abs=1e-4)
+    clocks = {"sm_mhz": 1320.0, "sm_max_mhz": 1965.0, "samples": 20}
+    t = bench.kernel_roofline(0.6 * 1661.1e9, 1e6, 1.0, PEAKS, "measured", clocks=clocks)
+    assert t["bound"] == "tensor" and t["frac"] == pytest.approx(0.6)
+    assert t["frac_at_sampled_clock"] == pytest.approx(0.6 * 1965.0 / 1320.0, abs=1e-4)
     h = bench.kernel_roofline(0, 6548.8e6, 1.0, PEAKS, "measured", clocks=clocks)
     assert h["bound"] == "hbm" and h["frac"] == pytest.approx(1.0)
     assert "frac_at_sampled_clock" not in h  # HBM bandwidth does not follow the SM clock
+
+
+def test_frac_at_sampled_clock_needs_enough_samples_and_stays_below_one():
+    few = {"sm_mhz": 1320.0, "sm_max_mhz": 1965.0, "samples": 4}
+    t = bench.kernel_roofline(0.6 * 1661.1e9, 1e6, 1.0, PEAKS, "measured", clocks=few)
+    assert t["frac_at_sampled_clock"] is None and "too few" in t["sampled_clock_note"]
+    many = dict(few, samples=20)
+    t = bench.kernel_roofline(0.9 * 1661.1e9, 1e6, 1.0, PEAKS, "measured", clocks=many)
+    assert t["frac"] == pytest.approx(0.9)
+    assert t["frac_at_sampled_clock"] is None  # 0.9 x 1965 / 1320 > 1: a missed clock
+    assert "not reported" in t["sampled_clock_note"]
 
 
 def test_combine_reports_both_byte_counts(monkeypatch):
