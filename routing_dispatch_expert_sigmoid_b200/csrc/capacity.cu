@@ -16,10 +16,11 @@
 //        chunk's first rank; each expert's chunks split into ranges summed
 //        by separate threads), totals, C = ceil(cf * sum k_t / E) in double,
 //        kept = min(count, C), offsets = exclusive scan of kept, drops;
-//   K3c  one warp per chunk loads the chunk's expert ids, then walks them
-//        32 at a time in order; lanes with the same expert find each other
-//        with __match_any_sync and rank themselves by lane order on top of
-//        the chunk's running count.
+//   K3c  one CTA per chunk, eight warps of 128 slots each: a warp counts its
+//        slots per expert, the counts give each warp's first rank per
+//        expert, then each warp walks its slots 32 at a time in order; lanes
+//        with the same expert find each other with __match_any_sync and rank
+//        themselves by lane order on top of the warp's running count.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -161,32 +162,49 @@ __global__ void __launch_bounds__(kScanThreads)
   }
 }
 
-__global__ void __launch_bounds__(32)
+// kRankWarps warps per chunk, warp w walking slots [w 128, (w+1) 128) of it:
+// each warp first counts its own slots per expert, the counts become each
+// warp's first rank per expert (the chunk's base plus the earlier warps'
+// counts), then every warp walks its 128 slots in order.  The ranks are the
+// same as one warp walking the whole chunk; the walk is 4 steps instead of 32.
+constexpr int kRankWarps = kChunk / 128;
+
+__global__ void __launch_bounds__(32 * kRankWarps)
     k_rank(const int32_t *__restrict__ idx, long long n_slots, int E,
            const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ offsets,
            const int32_t *__restrict__ cap, int32_t *__restrict__ slot_row,
            int32_t *__restrict__ row_src) {
-  extern __shared__ int32_t s_rank[];  // run[E] (running count), off[E] (first row)
-  int32_t *run = s_rank, *off = s_rank + E;
-  const int lane = threadIdx.x;
-  const long long a0 = (long long)blockIdx.x * kChunk;
-  const long long a1 = min(a0 + kChunk, n_slots);
-  // Every load is issued before the ordered walk, which then only touches
-  // registers and shared memory.
-  int ev[kChunk / 32];
+  extern __shared__ int32_t s_rank[];  // run[kRankWarps][E] (running ranks), off[E] (first row)
+  int32_t *off = s_rank + kRankWarps * E;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  int32_t *run = s_rank + warp * E;
+  const long long a0 = (long long)blockIdx.x * kChunk + warp * 128;
+  const long long a1 = min((long long)blockIdx.x * kChunk + kChunk, n_slots);
+  int ev[4];
 #pragma unroll
-  for (int i = 0; i < kChunk / 32; ++i) {
+  for (int i = 0; i < 4; ++i) {
     const long long a = a0 + 32 * i + lane;
     ev[i] = a < a1 ? idx[a] : -1;
   }
-  for (int e = lane; e < E; e += 32) {
-    run[e] = chunk_base[(size_t)blockIdx.x * E + e];
+  for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) s_rank[i] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (ev[i] >= 0 && ev[i] < E) atomicAdd(&run[ev[i]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int base = chunk_base[(size_t)blockIdx.x * E + e];
+    for (int w = 0; w < kRankWarps; ++w) {
+      const int c = s_rank[w * E + e];
+      s_rank[w * E + e] = base;
+      base += c;
+    }
     off[e] = offsets[e];
   }
   const int C = cap[0];
-  __syncwarp();
+  __syncthreads();
 #pragma unroll
-  for (int i = 0; i < kChunk / 32; ++i) {
+  for (int i = 0; i < 4; ++i) {
     const long long a = a0 + 32 * i + lane;
     const bool valid = a < a1;
     const int e = ev[i];
@@ -236,8 +254,8 @@ cudaError_t launch_capacity(const moe_config &c, const int32_t *topk_idx, int32_
   k_scan<<<1, kScanThreads, 0, s>>>(chunk_counts, nch, c.E, (double)c.capacity_factor, chunk_base,
                                     counts, kept, offsets, n_dropped, cap);
   if (nch > 0)
-    k_rank<<<nch, 32, 2 * eb, s>>>(topk_idx, slots, c.E, chunk_base, offsets, cap, slot_row,
-                                   row_src);
+    k_rank<<<nch, 32 * kRankWarps, (kRankWarps + 1) * eb, s>>>(topk_idx, slots, c.E, chunk_base,
+                                                                offsets, cap, slot_row, row_src);
   return cudaGetLastError();
 }
 

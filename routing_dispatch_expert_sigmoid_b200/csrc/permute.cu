@@ -262,8 +262,12 @@ __global__ void __launch_bounds__(256)
 // loads in flight per lane.
 // At least two CTAs (16 warps) per SM: left alone the compiler gives the
 // kernel over 160 registers, one CTA per SM, and the y16 reads half the
-// loads in flight they need (Qwen3-shaped combine 0.20 vs 0.13 ms).
-template <int KB, int VPL, typename Idx>
+// loads in flight they need (Qwen3-shaped combine 0.20 vs 0.13 ms).  SH =
+// false leaves out the shared expert's partial sums: the registers that
+// frees hold more row loads in flight (top-2 with four vectors per lane:
+// Mixtral-shaped combine 0.065 -> 0.050 ms; top-8 with two vectors, no
+// spills: Qwen3-shaped 0.123 -> 0.107 ms).
+template <int KB, int VPL, typename Idx, bool SH = true>
 __global__ void __launch_bounds__(256, 2)
     k_combine_y16(const uint4 *__restrict__ y, const int8_t *__restrict__ yexp, int nblk,
                   const int32_t *__restrict__ slot_row, const float *__restrict__ topk_w,
@@ -314,7 +318,7 @@ __global__ void __launch_bounds__(256, 2)
       const int v = v0 + 32 * i;
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[i][q] = 0.f;
-      if (shared_y && v < row_vecs) {
+      if (SH && shared_y && v < row_vecs) {
         for (int sp = 0; sp < shared_parts; ++sp) {  // partial sums, in order
           const uint4 *part = shared_y + (size_t)sp * Tn * sh_vecs + (size_t)t * sh_vecs;
 #pragma unroll
@@ -467,28 +471,35 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
       kernel<<<g, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o, c.T, c.k_max,
                                rows_cap, row_vecs, err);
     };
-    if (c.k_max <= 2) {  // two vectors per lane: items of 64 vectors
-      const int g2 = grid_for((long long)c.T * ((row_vecs + 63) / 64));
-      if (narrow)
-        launch(k_combine_y16<2, 2, int>, g2);
+    // MOE_COMBINE_VPL=1: one 16-byte vector per lane per row (two for top-2)
+    const char *cv = getenv("MOE_COMBINE_VPL");
+    const bool one = cv && cv[0] == '1';
+    if (c.k_max <= 2) {
+      if (narrow && !sh && !one)  // four vectors per lane: items of 128 vectors
+        launch(k_combine_y16<2, 4, int, false>,
+               grid_for((long long)c.T * ((row_vecs + 127) / 128)));
+      else if (narrow)  // two vectors per lane: items of 64 vectors
+        launch(k_combine_y16<2, 2, int>, grid_for((long long)c.T * ((row_vecs + 63) / 64)));
       else
-        launch(k_combine_y16<2, 2, long long>, g2);
+        launch(k_combine_y16<2, 2, long long>,
+               grid_for((long long)c.T * ((row_vecs + 63) / 64)));
     } else if (c.k_max <= 4) {
       if (narrow)
         launch(k_combine_y16<4, 1, int>, grid);
       else
         launch(k_combine_y16<4, 1, long long>, grid);
-    } else {
+    } else if (narrow && !one) {
       // two vectors per lane (twice the loads in flight per warp): 6% faster
-      // on the Qwen3- and GPT-OSS-shaped layers; MOE_COMBINE_VPL=1 for one
-      const char *cv = getenv("MOE_COMBINE_VPL");
-      if (narrow && !(cv && cv[0] == '1')) {
-        const int g2 = grid_for((long long)c.T * ((row_vecs + 63) / 64));
+      // on the Qwen3- and GPT-OSS-shaped layers than one
+      const int g2 = grid_for((long long)c.T * ((row_vecs + 63) / 64));
+      if (sh)
         launch(k_combine_y16<8, 2, int>, g2);
-      } else if (narrow)
-        launch(k_combine_y16<8, 1, int>, grid);
       else
-        launch(k_combine_y16<8, 1, long long>, grid);
+        launch(k_combine_y16<8, 2, int, false>, g2);
+    } else if (narrow) {
+      launch(k_combine_y16<8, 1, int>, grid);
+    } else {
+      launch(k_combine_y16<8, 1, long long>, grid);
     }
     return cudaGetLastError();
   }
