@@ -12,10 +12,12 @@
 // expert:
 //   K3a  one CTA per chunk of kChunk slots: per-chunk expert histogram
 //        (shared-memory atomics; counts do not depend on order);
-//   K3b  one CTA: per expert, exclusive scan of the chunk histograms (the
-//        chunk's first rank; each expert's chunks split into ranges summed
-//        by separate threads), totals, C = ceil(cf * sum k_t / E) in double,
-//        kept = min(count, C), offsets = exclusive scan of kept, drops;
+//   K3b  one CTA per 32 experts: per expert, exclusive scan of the chunk
+//        histograms (the chunk's first rank; each expert's chunks split into
+//        ranges summed by separate warps) and its total; the last CTA to
+//        finish (an atomic ticket only picks which one) computes
+//        C = ceil(cf * sum k_t / E) in double, kept = min(count, C),
+//        offsets = exclusive scan of kept, drops;
 //   K3c  one CTA per chunk, eight warps of 128 slots each: a warp counts its
 //        slots per expert, the counts give each warp's first rank per
 //        expert, then each warp walks its slots 32 at a time in order; lanes
@@ -35,8 +37,9 @@ int num_chunks(const moe_config &c) {
 
 __global__ void __launch_bounds__(256) k_hist(const int32_t *__restrict__ idx, long long n_slots,
                                               int E, int32_t *__restrict__ chunk_counts,
-                                              uint32_t *err) {
+                                              int32_t *__restrict__ ticket, uint32_t *err) {
   extern __shared__ int32_t cnt[];
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;  // the scan's ticket
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   const long long a0 = (long long)blockIdx.x * kChunk;
@@ -56,64 +59,70 @@ __global__ void __launch_bounds__(256) k_hist(const int32_t *__restrict__ idx, l
 }
 
 constexpr int kScanThreads = 1024;
-constexpr int kScanBatch = 16;  // chunk histograms loaded before they are summed
+constexpr int kScanBatch = 16;    // chunk histograms loaded before they are summed
+constexpr int kScanExperts = 32;  // experts per CTA: lane = expert, warp = chunk range
 
+// One CTA per 32 experts.  Expert e's chunks are split into 32 contiguous
+// ranges, one warp each (lane = expert, so a warp's loads are one 128-byte
+// row of a chunk histogram): the ranges are summed, each thread takes the sum
+// of the earlier ranges as its base and writes its chunks' bases; the last
+// range's end is the expert's count.  The CTA that finishes last (a ticket,
+// zeroed by the histogram kernel) then computes, for all experts, the
+// capacity, kept counts, offsets and drops.
 __global__ void __launch_bounds__(kScanThreads)
     k_scan(const int32_t *__restrict__ chunk_counts, int n_chunks, int E, double cf,
            int32_t *__restrict__ chunk_base, int32_t *__restrict__ counts,
            int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
-           int32_t *__restrict__ n_dropped, int32_t *__restrict__ cap_out) {
+           int32_t *__restrict__ n_dropped, int32_t *__restrict__ cap_out,
+           int32_t *__restrict__ ticket) {
   __shared__ long long s_part[kScanThreads / 32];
   __shared__ long long s_total;
-  __shared__ int32_t s_cnt[1024];
-  __shared__ int32_t s_sum[kScanThreads];  // [part][expert] chunk-range sums
+  __shared__ int32_t s_sum[32][kScanExperts + 1];  // [range][expert] range sums
+  __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
-  // E <= 1024 = blockDim.  Expert e's chunks are split into P contiguous
-  // ranges, one thread (part, e) each: the ranges are summed, each thread
-  // takes the sum of the earlier ranges as its base and writes its chunks'
-  // bases.
-  int P = kScanThreads / E;
-  if (P > n_chunks) P = n_chunks;
-  if (P < 1) P = 1;
-  const int per = (n_chunks + P - 1) / P;
-  const int e = tid % E, part = tid / E;
-  const bool active = part < P;
-  const int c0 = active ? min(part * per, n_chunks) : 0;
-  const int c1 = active ? min(c0 + per, n_chunks) : 0;
-  int sum = 0;
-  for (int c = c0; c < c1; c += kScanBatch) {
-    int v[kScanBatch];
-#pragma unroll
-    for (int i = 0; i < kScanBatch; ++i)
-      v[i] = c + i < c1 ? chunk_counts[(size_t)(c + i) * E + e] : 0;
-#pragma unroll
-    for (int i = 0; i < kScanBatch; ++i) sum += v[i];
-  }
-  if (active) s_sum[tid] = sum;
-  __syncthreads();
-  if (active) {
-    int run = 0;
-    for (int q = 0; q < part; ++q) run += s_sum[q * E + e];
+  {
+    const int e = blockIdx.x * kScanExperts + lane;
+    const bool ev = e < E;
+    const int per = (n_chunks + 31) / 32;
+    const int c0 = min(warp * per, n_chunks), c1 = min(c0 + per, n_chunks);
+    int sum = 0;
     for (int c = c0; c < c1; c += kScanBatch) {
       int v[kScanBatch];
 #pragma unroll
       for (int i = 0; i < kScanBatch; ++i)
-        v[i] = c + i < c1 ? chunk_counts[(size_t)(c + i) * E + e] : 0;
+        v[i] = ev && c + i < c1 ? chunk_counts[(size_t)(c + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) sum += v[i];
+    }
+    s_sum[warp][lane] = sum;
+    __syncthreads();
+    int run = 0;
+    for (int q = 0; q < warp; ++q) run += s_sum[q][lane];
+    for (int c = c0; c < c1; c += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+        v[i] = ev && c + i < c1 ? chunk_counts[(size_t)(c + i) * E + e] : 0;
 #pragma unroll
       for (int i = 0; i < kScanBatch; ++i)
         if (c + i < c1) {
-          chunk_base[(size_t)(c + i) * E + e] = run;
+          if (ev) chunk_base[(size_t)(c + i) * E + e] = run;
           run += v[i];
         }
     }
-    if (part == P - 1) s_cnt[e] = run;
+    if (warp == 31 && ev) counts[e] = run;
+  }
+  if (gridDim.x > 1) {
+    __threadfence();  // this CTA's counts before its ticket
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();  // every other CTA's counts are visible past its ticket
   }
   __syncthreads();
   long long my = 0;
-  if (tid < E) {
-    my = s_cnt[tid];
-    counts[tid] = (int32_t)my;
-  }
+  if (tid < E) my = __ldcg(counts + tid);
   // block sum of counts = sum over tokens of k_t
   long long v = my;
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -130,7 +139,7 @@ __global__ void __launch_bounds__(kScanThreads)
   if (cf > 0.0) C = (long long)ceil(cf * (double)sum_k / (double)E);
   int k = 0;
   if (tid < E) {
-    k = s_cnt[tid];
+    k = (int)my;
     if (C >= 0 && k > C) k = (int)C;
     kept[tid] = k;
   }
@@ -250,9 +259,13 @@ cudaError_t launch_capacity(const moe_config &c, const int32_t *topk_idx, int32_
   int32_t *cap = reinterpret_cast<int32_t *>(static_cast<char *>(scratch) +
                                              ((2 * n * sizeof(int32_t) + 255) / 256) * 256);
   const size_t eb = sizeof(int32_t) * (size_t)c.E;
-  if (nch > 0) k_hist<<<nch, 256, eb, s>>>(topk_idx, slots, c.E, chunk_counts, err);
-  k_scan<<<1, kScanThreads, 0, s>>>(chunk_counts, nch, c.E, (double)c.capacity_factor, chunk_base,
-                                    counts, kept, offsets, n_dropped, cap);
+  int32_t *ticket = cap + 1;  // in the scratch's last 256 bytes, with the capacity word
+  if (nch > 0) k_hist<<<nch, 256, eb, s>>>(topk_idx, slots, c.E, chunk_counts, ticket, err);
+  // one CTA when there is no histogram kernel to zero the ticket
+  const int scan_ctas = nch > 0 ? (c.E + kScanExperts - 1) / kScanExperts : 1;
+  k_scan<<<scan_ctas, kScanThreads, 0, s>>>(chunk_counts, nch, c.E, (double)c.capacity_factor,
+                                            chunk_base, counts, kept, offsets, n_dropped, cap,
+                                            ticket);
   if (nch > 0)
     k_rank<<<nch, 32 * kRankWarps, (kRankWarps + 1) * eb, s>>>(topk_idx, slots, c.E, chunk_base,
                                                                 offsets, cap, slot_row, row_src);

@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(256)
 // false leaves out the shared expert's partial sums: the registers that
 // frees hold more row loads in flight (top-2 with four vectors per lane:
 // Mixtral-shaped combine 0.065 -> 0.050 ms; top-8 with two vectors, no
-// spills: Qwen3-shaped 0.123 -> 0.107 ms).
+// spills: Qwen3-shaped 0.123 -> 0.107 ms).  With a shared expert its partial
+// sums are read after the first batch of rows is issued (one vector per lane).
 template <int KB, int VPL, typename Idx, bool SH = true>
 __global__ void __launch_bounds__(256, 2)
     k_combine_y16(const uint4 *__restrict__ y, const int8_t *__restrict__ yexp, int nblk,
@@ -314,24 +315,14 @@ __global__ void __launch_bounds__(256, 2)
     const int v0 = ch * kItemVecs + lane;  // this lane's vectors: v0 + 32 i
     float acc[VPL][8];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int v = v0 + 32 * i;
+    for (int i = 0; i < VPL; ++i)
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[i][q] = 0.f;
-      if (SH && shared_y && v < row_vecs) {
-        for (int sp = 0; sp < shared_parts; ++sp) {  // partial sums, in order
-          const uint4 *part = shared_y + (size_t)sp * Tn * sh_vecs + (size_t)t * sh_vecs;
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            float f[4];
-            Vec<float>::load(ldg_nc(part + (size_t)v * 2 + q), f);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[i][4 * q + c] += f[c];
-          }
-        }
-      }
-    }
-    for (int j0 = 0; j0 < n_live; j0 += KB) {
+    // The shared expert's partial sums go into acc first, but they are read
+    // after the first batch of rows has been issued, so the two sets of
+    // loads are in flight together.
+    bool sh_pending = SH && shared_y != nullptr;
+    for (int j0 = 0; j0 < n_live || sh_pending; j0 += KB) {
       uint4 u[KB][VPL];
       int e[KB][VPL];
 #pragma unroll
@@ -347,6 +338,25 @@ __global__ void __launch_bounds__(256, 2)
             }
           }
         }
+      if (SH && sh_pending) {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          const int v = v0 + 32 * i;
+          if (v < row_vecs) {
+            for (int sp = 0; sp < shared_parts; ++sp) {  // partial sums, in order
+              const uint4 *part = shared_y + (size_t)sp * Tn * sh_vecs + (size_t)t * sh_vecs;
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                float f[4];
+                Vec<float>::load(ldg_nc(part + (size_t)v * 2 + q), f);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[i][4 * q + c] += f[c];
+              }
+            }
+          }
+        }
+        sh_pending = false;
+      }
 #pragma unroll
       for (int j = 0; j < KB; ++j) {
         if (j0 + j < n_live) {
@@ -488,15 +498,14 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
         launch(k_combine_y16<4, 1, int>, grid);
       else
         launch(k_combine_y16<4, 1, long long>, grid);
-    } else if (narrow && !one) {
+    } else if (narrow && !one && !sh) {
       // two vectors per lane (twice the loads in flight per warp): 6% faster
       // on the Qwen3- and GPT-OSS-shaped layers than one
-      const int g2 = grid_for((long long)c.T * ((row_vecs + 63) / 64));
-      if (sh)
-        launch(k_combine_y16<8, 2, int>, g2);
-      else
-        launch(k_combine_y16<8, 2, int, false>, g2);
+      launch(k_combine_y16<8, 2, int, false>, grid_for((long long)c.T * ((row_vecs + 63) / 64)));
     } else if (narrow) {
+      // with a shared expert one vector per lane: the partial sums' registers
+      // leave no room for two without spills (DeepSeek-V3-shaped prefill
+      // combine 0.136 -> 0.122 ms with the shared loads overlapped)
       launch(k_combine_y16<8, 1, int>, grid);
     } else {
       launch(k_combine_y16<8, 1, long long>, grid);

@@ -524,8 +524,8 @@ def test_layer_dispatch_walks(name, by_row, dev):
 @pytest.mark.parametrize("name", ["mixtral_small", "qwen3_medium", "dsv3_medium", "gptoss_small"])
 def test_layer_combine_one_vector_per_lane(name, dev):
     """MOE_COMBINE_VPL=1: the y16 combine with one 16-byte vector per lane
-    per row (two for top-2; the defaults without a shared expert take four
-    for top-2 and two for top-8)."""
+    per row (two for top-2; without a shared expert the defaults take four
+    for top-2 and two for top-8, with one the same one)."""
     import os
     old = os.environ.get("MOE_COMBINE_VPL")
     os.environ["MOE_COMBINE_VPL"] = "1"
