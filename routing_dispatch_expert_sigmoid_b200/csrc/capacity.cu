@@ -38,6 +38,7 @@ int num_chunks(const moe_config &c) {
 __global__ void __launch_bounds__(256) k_hist(const int32_t *__restrict__ idx, long long n_slots,
                                               int E, int32_t *__restrict__ chunk_counts,
                                               int32_t *__restrict__ ticket, uint32_t *err) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   extern __shared__ int32_t cnt[];
   if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;  // the scan's ticket
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(kScanThreads)
            int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
            int32_t *__restrict__ n_dropped, int32_t *__restrict__ cap_out,
            int32_t *__restrict__ ticket) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   __shared__ long long s_part[kScanThreads / 32];
   __shared__ long long s_total;
   __shared__ int32_t s_sum[32][kScanExperts + 1];  // [range][expert] range sums
@@ -183,6 +185,7 @@ __global__ void __launch_bounds__(32 * kRankWarps)
            const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ offsets,
            const int32_t *__restrict__ cap, int32_t *__restrict__ slot_row,
            int32_t *__restrict__ row_src) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   extern __shared__ int32_t s_rank[];  // run[kRankWarps][E] (running ranks), off[E] (first row)
   int32_t *off = s_rank + kRankWarps * E;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
@@ -260,14 +263,14 @@ cudaError_t launch_capacity(const moe_config &c, const int32_t *topk_idx, int32_
                                              ((2 * n * sizeof(int32_t) + 255) / 256) * 256);
   const size_t eb = sizeof(int32_t) * (size_t)c.E;
   int32_t *ticket = cap + 1;  // in the scratch's last 256 bytes, with the capacity word
-  if (nch > 0) k_hist<<<nch, 256, eb, s>>>(topk_idx, slots, c.E, chunk_counts, ticket, err);
+  if (nch > 0) launch_k(k_hist, nch, 256, eb, s, topk_idx, slots, c.E, chunk_counts, ticket, err);
   // one CTA when there is no histogram kernel to zero the ticket
   const int scan_ctas = nch > 0 ? (c.E + kScanExperts - 1) / kScanExperts : 1;
-  k_scan<<<scan_ctas, kScanThreads, 0, s>>>(chunk_counts, nch, c.E, (double)c.capacity_factor,
+  launch_k(k_scan, scan_ctas, kScanThreads, 0, s, chunk_counts, nch, c.E, (double)c.capacity_factor,
                                             chunk_base, counts, kept, offsets, n_dropped, cap,
                                             ticket);
   if (nch > 0)
-    k_rank<<<nch, 32 * kRankWarps, (kRankWarps + 1) * eb, s>>>(topk_idx, slots, c.E, chunk_base,
+    launch_k(k_rank, nch, 32 * kRankWarps, (kRankWarps + 1) * eb, s, topk_idx, slots, c.E, chunk_base,
                                                                 offsets, cap, slot_row, row_src);
   return cudaGetLastError();
 }

@@ -38,6 +38,7 @@ __device__ __forceinline__ uint4 ldg_nc16(const uint4 *p) {
 __global__ void __launch_bounds__(kPlanThreads)
     k_ep_plan(const int32_t *__restrict__ C, int n_ranks, int E, int rank,
               int32_t *__restrict__ recv_offsets, int32_t *__restrict__ send_base) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   __shared__ int32_t s_tot[1024];  // rows of expert e over all sources
   const int e_loc = E / n_ranks;
   for (int e = threadIdx.x; e < E; e += kPlanThreads) {
@@ -76,6 +77,7 @@ __global__ void __launch_bounds__(256)
                   const int32_t *__restrict__ row_src, const int32_t *__restrict__ topk_idx,
                   const int32_t *__restrict__ send_base, PeerRows dst, int n_ranks, int E,
                   int k_max, int T, int rows_cap, int recv_cap, int row_vecs, uint32_t *err) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   int R = offsets[E];
   if (R > rows_cap || R < 0) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(err, kErrIndex);
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(256)
     k_ep_return(const uint4 *__restrict__ y, const int32_t *__restrict__ recv_offsets,
                 const int32_t *__restrict__ C, PeerY dst, int n_ranks, int E, int rank,
                 int src_cap, int recv_cap, int row_vecs, uint32_t *err) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   extern __shared__ int32_t s_tab[];
   const int e_loc = E / n_ranks, e0 = rank * e_loc;
   int32_t *s_in = s_tab;                         // [e_loc][n_ranks + 1]: source starts in e's block

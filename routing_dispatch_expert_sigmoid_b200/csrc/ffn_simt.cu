@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(256)
     k_ffn_f32(const float *__restrict__ A, const float *__restrict__ B1,
               const float *__restrict__ B3, float *__restrict__ C, const int32_t *offsets,
               int fixed_rows, int K, int N) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   __shared__ float as[BK][BM + 1];
   __shared__ float b1s[BK][BN];
   __shared__ float b3s[SWIGLU ? BK : 1][BN];
@@ -104,9 +105,9 @@ cudaError_t launch_ffn_simt_f32(int rows_cap, int d, int f, int G, const int32_t
   const int max_rows = offsets ? rows_cap : fixed_rows;
   if (max_rows == 0 || G == 0) return cudaSuccess;
   dim3 g1((f + BN - 1) / BN, (max_rows + BM - 1) / BM, G);
-  k_ffn_f32<true><<<g1, 256, 0, s>>>(x_perm, W1, W3, h, offsets, fixed_rows, d, f);
+  launch_k(k_ffn_f32<true>, g1, 256, 0, s, x_perm, W1, W3, h, offsets, fixed_rows, d, f);
   dim3 g2((d + BN - 1) / BN, (max_rows + BM - 1) / BM, G);
-  k_ffn_f32<false><<<g2, 256, 0, s>>>(h, W2, nullptr, y, offsets, fixed_rows, f, d);
+  launch_k(k_ffn_f32<false>, g2, 256, 0, s, h, W2, nullptr, y, offsets, fixed_rows, f, d);
   return cudaGetLastError();
 }
 

@@ -35,6 +35,7 @@ constexpr int kWarpsPerBlock = 4;
 
 template <int NPL>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_gating(GatingArgs g) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   extern __shared__ float s_u_all[];  // [kWarpsPerBlock][E], sigmoid mode only
   const int warp = threadIdx.x / 32;
   const int t = blockIdx.x * kWarpsPerBlock + warp;
@@ -47,7 +48,7 @@ cudaError_t run(const GatingArgs &a, cudaStream_t s) {
   const int blocks = (a.T + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const size_t smem =
       a.mode == MOE_SIGMOID_GROUPED ? sizeof(float) * kWarpsPerBlock * (size_t)a.E : 0;
-  k_gating<NPL><<<blocks, kWarpsPerBlock * 32, smem, s>>>(a);
+  launch_k(k_gating<NPL>, blocks, kWarpsPerBlock * 32, smem, s, a);
   return cudaGetLastError();
 }
 

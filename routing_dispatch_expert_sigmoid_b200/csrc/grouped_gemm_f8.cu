@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_f8(const __grid_constant__ CUtensorMap tmP,   // planes [2*rows_cap, K]
                       const __grid_constant__ CUtensorMap tmW1,  // codes [G, N, K]
                       const __grid_constant__ CUtensorMap tmW3, const ParamsF8 p) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   using S = ShapeF8<SWIGLU>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -469,6 +470,7 @@ __global__ void __launch_bounds__(kSplitThreads)
                    int fixed_rows, const int32_t *__restrict__ row_src, int k_max, int src_rows,
                    int rows_cap, int K, uint8_t *__restrict__ planes,
                    float *__restrict__ row_scale, uint32_t *err) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   __shared__ float s_red[kSplitThreads / 32];
   int R = n_rows ? *n_rows : fixed_rows;
   if (R < 0 || R > rows_cap) {
@@ -596,7 +598,7 @@ cudaError_t launch_f8(int rows_cap, int K, int N, int G, const int32_t *offsets,
   const long long max_tiles = (long long)((rows_cap + kQRows - 1) / kQRows + G) *
                               ((N + S::kTileCols - 1) / S::kTileCols);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
-  k_grouped_gemm_f8<SWIGLU><<<grid, kThreads, smem, s>>>(mp, mw1, mw3, p);
+  launch_k(k_grouped_gemm_f8<SWIGLU>, grid, kThreads, smem, s, mp, mw1, mw3, p);
   return cudaGetLastError();
 }
 
@@ -615,7 +617,7 @@ cudaError_t launch_split_planes(const void *src, const int32_t *n_rows, int fixe
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = rows_cap < 8 * sms ? rows_cap : 8 * sms;
-  tc::k_split_planes<<<grid, tc::kSplitThreads, 0, s>>>(
+  launch_k(tc::k_split_planes, grid, tc::kSplitThreads, 0, s, 
       static_cast<const __nv_bfloat16 *>(src), n_rows, fixed_rows, row_src, k_max, src_rows,
       rows_cap, K, planes, row_scale, err);
   return cudaGetLastError();

@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 128 : kThreads, 1)
                          const __grid_constant__ CUtensorMap tmX,   // rows, 32-row box
                          const __grid_constant__ CUtensorMap tmW1,  // [G, K, N]
                          const __grid_constant__ CUtensorMap tmW3, const ParamsMixed p) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   using S = ShapeMixed<SWIGLU>;
   constexpr int kCta = GATHER ? kThreads + 128 : kThreads;
   extern __shared__ uint8_t smem_raw[];
@@ -719,12 +720,12 @@ cudaError_t launch_mixed(int rows_cap, int K, int N, int G, const int32_t *offse
                               ((N + S::BN - 1) / S::BN);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
   if (!o.split) {
-    k_grouped_gemm_mixed<SWIGLU, GATHER><<<grid, kCta, smem, s>>>(ma, mx, mw1, mw3, p);
+    launch_k(k_grouped_gemm_mixed<SWIGLU, GATHER>, grid, kCta, smem, s, ma, mx, mw1, mw3, p);
     return cudaGetLastError();
   }
   for (int lists = 1; lists <= 2; ++lists) {  // heavy groups, then light ones
     p.lists = lists;
-    k_grouped_gemm_mixed<SWIGLU, GATHER><<<grid, kCta, smem, s>>>(ma, mx, mw1, mw3, p);
+    launch_k(k_grouped_gemm_mixed<SWIGLU, GATHER>, grid, kCta, smem, s, ma, mx, mw1, mw3, p);
     if (cudaError_t e = cudaGetLastError()) return e;
   }
   return cudaSuccess;

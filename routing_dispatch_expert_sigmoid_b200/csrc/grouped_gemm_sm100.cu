@@ -290,6 +290,7 @@ template <bool SWIGLU, int SPANS, bool FP8W = false>
 __global__ void __launch_bounds__(Shape<SWIGLU, SPANS, FP8W>::kCtaThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
                    const __grid_constant__ CUtensorMap tmB3, const Params p) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   using S = Shape<SWIGLU, SPANS, FP8W>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -828,6 +829,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmB3,
                         const __grid_constant__ CUtensorMap tmX32,
                         const __grid_constant__ CUtensorMap tmX8, const Params p) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   using S = Shape2<SWIGLU>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -1506,6 +1508,7 @@ __global__ void __launch_bounds__(ShapeSwap<SWIGLU, FP8W>::kCtaThreads, 1)
     k_grouped_gemm_swap(const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmW1,
                         const __grid_constant__ CUtensorMap tmW3, const Params p) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   using S = ShapeSwap<SWIGLU, FP8W>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -1997,7 +2000,7 @@ cudaError_t launch_q8(int rows_cap, int K, int N, int G, const int32_t *offsets,
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
-  k_grouped_gemm<SWIGLU, SPANS, true><<<grid, S::kCtaThreads, smem, s>>>(ma, mb1, mb3, p);
+  launch_k(k_grouped_gemm<SWIGLU, SPANS, true>, grid, S::kCtaThreads, smem, s, ma, mb1, mb3, p);
   return cudaGetLastError();
 }
 
@@ -2032,7 +2035,7 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
   const long long max_tiles = (long long)((rows_cap + BM - 1) / BM + (offsets ? G : 0)) *
                               ((N + S::BN - 1) / S::BN);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
-  k_grouped_gemm<SWIGLU, SPANS><<<grid, kThreads, smem, s>>>(ma, mb1, mb3, p);
+  launch_k(k_grouped_gemm<SWIGLU, SPANS>, grid, kThreads, smem, s, ma, mb1, mb3, p);
   return cudaGetLastError();
 }
 
@@ -2080,7 +2083,7 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
                               ((N + S::BN - 1) / S::BN);
   long long pairs = sms / 2;
   if (max_tiles < pairs) pairs = max_tiles < 1 ? 1 : max_tiles;
-  k_grouped_gemm_pair<SWIGLU><<<(int)(2 * pairs), kThreads, smem, s>>>(ma, mb1, mb3, mx32, mx8,
+  launch_k(k_grouped_gemm_pair<SWIGLU>, (int)(2 * pairs), kThreads, smem, s, ma, mb1, mb3, mx32, mx8,
                                                                        p);
   return cudaGetLastError();
 }
@@ -2113,7 +2116,7 @@ cudaError_t launch_swap(int rows_cap, int K, int N, int G, const int32_t *offset
                                           (offsets ? G : 0)) *
                               ((N + S::kCols - 1) / S::kCols);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
-  k_grouped_gemm_swap<SWIGLU><<<grid, kThreads, smem, s>>>(mx, mw1, mw3, p);
+  launch_k(k_grouped_gemm_swap<SWIGLU>, grid, kThreads, smem, s, mx, mw1, mw3, p);
   return cudaGetLastError();
 }
 
@@ -2147,7 +2150,7 @@ cudaError_t launch_swap_q8(int rows_cap, int K, int N, int G, const int32_t *off
                                           (offsets ? G : 0)) *
                               ((N + S::kTileCols - 1) / S::kTileCols);
   const int grid = (int)(max_tiles < sms ? (max_tiles < 1 ? 1 : max_tiles) : sms);
-  k_grouped_gemm_swap<SWIGLU, true><<<grid, S::kCtaThreads, smem, s>>>(mx, mw1, mw3, p);
+  launch_k(k_grouped_gemm_swap<SWIGLU, true>, grid, S::kCtaThreads, smem, s, mx, mw1, mw3, p);
   return cudaGetLastError();
 }
 
@@ -2319,7 +2322,7 @@ cudaError_t launch_split(int T, int K, int N, int S, int k_split, const void *A,
   p.scale1 = scale;
   const long long tiles = (long long)S * ((T + BM - 1) / BM) * ((N + Sh::BN - 1) / Sh::BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
-  k_grouped_gemm<false, SPANS, FP8W><<<grid, Sh::kCtaThreads, smem, s>>>(ma, mb, mb, p);
+  launch_k(k_grouped_gemm<false, SPANS, FP8W>, grid, Sh::kCtaThreads, smem, s, ma, mb, mb, p);
   return cudaGetLastError();
 }
 

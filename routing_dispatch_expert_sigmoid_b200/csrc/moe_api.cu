@@ -36,6 +36,11 @@ uint32_t *device_error_word() {
   return static_cast<uint32_t *>(symbol_address_cached(addr, &g_moe_error_word));
 }
 
+bool pdl_enabled() {
+  const char *v = getenv("MOE_PDL");  // read per launch, like the other switches
+  return !(v && v[0] == '0');
+}
+
 namespace {
 
 constexpr size_t kAlign = 256;

@@ -33,6 +33,41 @@ __device__ __forceinline__ void raise_error(uint32_t *err, uint32_t bit) {
   if (err) atomicOr(err, bit);
 }
 
+// ---- programmatic dependent launch ----------------------------------------
+// Every kernel of the library starts with grid_dependency(): it waits until
+// the grid launched before it on the stream has finished and its memory is
+// visible (an immediate return when the kernel was launched without the
+// programmatic-serialization attribute), then allows the grid launched after
+// it to start its launch and prologue.  So a kernel never reads or writes
+// memory before its predecessor is complete, whichever way it was launched,
+// and launch_k can overlap one kernel's launch with the previous one's tail.
+__device__ __forceinline__ void grid_dependency() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Whether launch_k sets the programmatic-serialization attribute
+// (MOE_PDL=0: plain stream order).
+bool pdl_enabled();
+
+// kernel<<<grid, block, smem, s>>>(args...), with programmatic stream
+// serialization when pdl_enabled().  Returns the launch's status.
+template <typename... Params, typename... Args>
+cudaError_t launch_k(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t s, Args &&...args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
 // ---- element access -------------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(256)
     k_dispatch(const uint4 *__restrict__ x, const int32_t *__restrict__ offsets,
                const int32_t *__restrict__ row_src, uint4 *__restrict__ x_perm, int E,
                int k_max, int T, int rows_cap, int row_vecs, uint32_t *err) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   int R = offsets[E];
   if (R > rows_cap || R < 0) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(err, kErrIndex);
@@ -82,6 +83,7 @@ __global__ void __launch_bounds__(256)
     k_dispatch_tok(const uint4 *__restrict__ x, const int32_t *__restrict__ slot_row,
                    uint4 *__restrict__ x_perm, int T, int k_max, int rows_cap, int row_vecs,
                    uint32_t *err) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   constexpr int kChunkVecs = 32 * VPL;
   const int lane = threadIdx.x % 32;
   const int warps = gridDim.x * (blockDim.x / 32);
@@ -165,6 +167,7 @@ __global__ void __launch_bounds__(256)
               const float *__restrict__ topk_w, const uint4 *__restrict__ shared_y,
               int shared_parts, uint4 *__restrict__ out, int Tn, int k_max, int rows_cap,
               int row_vecs, uint32_t *err) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   constexpr int N = Vec<T>::N;  // output values per 16-byte vector
   constexpr int Q = N / 4;      // fp32 input vectors per output vector
   __shared__ int32_t s_row[8][32];
@@ -274,6 +277,7 @@ __global__ void __launch_bounds__(256, 2)
                   const int32_t *__restrict__ slot_row, const float *__restrict__ topk_w,
                   const uint4 *__restrict__ shared_y, int shared_parts, uint4 *__restrict__ out,
                   int Tn, int k_max, int rows_cap, int row_vecs, uint32_t *err) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   __shared__ int32_t s_row[8][32];
   __shared__ float s_w[8][32];
   const int lane = threadIdx.x % 32, wib = threadIdx.x / 32;
@@ -406,7 +410,7 @@ cudaError_t launch_dispatch_by_token(const moe_config &c, const void *x,
   const int rows_cap = c.T * c.k_max;
   if (rows_cap == 0) return cudaSuccess;
   const int row_vecs = c.d * esz / 16;
-  k_dispatch_tok<8><<<grid_for(c.T), 256, 0, s>>>(static_cast<const uint4 *>(x), slot_row,
+  launch_k(k_dispatch_tok<8>, grid_for(c.T), 256, 0, s, static_cast<const uint4 *>(x), slot_row,
                                                   static_cast<uint4 *>(x_perm), c.T, c.k_max,
                                                   rows_cap, row_vecs, err);
   return cudaGetLastError();
@@ -423,11 +427,11 @@ cudaError_t launch_dispatch(const moe_config &c, const void *x, const int32_t *o
   auto *xp = static_cast<uint4 *>(x_perm);
   if ((long long)rows_cap * row_vecs * 16 <= (16ll << 20)) {  // at most 16 MB of rows
     const long long items = (long long)rows_cap * ((row_vecs + 127) / 128);
-    k_dispatch<4><<<grid_for(items), 256, 0, s>>>(xs, offsets, row_src, xp, c.E, c.k_max, c.T,
+    launch_k(k_dispatch<4>, grid_for(items), 256, 0, s, xs, offsets, row_src, xp, c.E, c.k_max, c.T,
                                                   rows_cap, row_vecs, err);
   } else {
     const long long items = (long long)rows_cap * ((row_vecs + 255) / 256);
-    k_dispatch<8><<<grid_for(items), 256, 0, s>>>(xs, offsets, row_src, xp, c.E, c.k_max, c.T,
+    launch_k(k_dispatch<8>, grid_for(items), 256, 0, s, xs, offsets, row_src, xp, c.E, c.k_max, c.T,
                                                   rows_cap, row_vecs, err);
   }
   return cudaGetLastError();
@@ -439,7 +443,7 @@ template <typename T, int KB>
 cudaError_t run_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                         const float *topk_w, const void *shared_y, void *out, uint32_t *err,
                         cudaStream_t s, int shared_parts, int grid, int row_vecs) {
-  k_combine<T, KB><<<grid, 256, 0, s>>>(
+  launch_k(k_combine<T, KB>, grid, 256, 0, s, 
       static_cast<const uint4 *>(y_perm), slot_row, topk_w, static_cast<const uint4 *>(shared_y),
       shared_parts, static_cast<uint4 *>(out), c.T, c.k_max, c.T * c.k_max, row_vecs, err);
   return cudaGetLastError();
@@ -478,7 +482,7 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
     // could pass 2^31
     const bool narrow = (long long)c.T * ((row_vecs + 31) / 32) + 148LL * 64 < (1LL << 31);
     auto launch = [&](auto kernel, int g) {
-      kernel<<<g, 256, 0, s>>>(y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o, c.T, c.k_max,
+      launch_k(kernel, g, 256, 0, s, y, yexp, nblk, slot_row, topk_w, sh, shared_parts, o, c.T, c.k_max,
                                rows_cap, row_vecs, err);
     };
     // MOE_COMBINE_VPL=1: one 16-byte vector per lane per row (two for top-2)

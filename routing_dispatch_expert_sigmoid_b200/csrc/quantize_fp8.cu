@@ -29,6 +29,7 @@ constexpr int kCols = 32;
 __global__ void __launch_bounds__(256)
     k_quantize_fp8(const __nv_bfloat16 *__restrict__ W, int K, int N, uint8_t *__restrict__ Wq,
                    float *__restrict__ scale) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   __shared__ float s_max[8][kCols];
   __shared__ float s_scale[kCols];
   __shared__ uint8_t s_tile[kCols][kCols + 4];  // [n][k]
@@ -80,7 +81,7 @@ cudaError_t launch_quantize_fp8(int G, int K, int N, const void *W, uint8_t *Wq,
                                 cudaStream_t s) {
   if ((long long)G * K * N == 0) return cudaSuccess;
   const dim3 grid((N + kCols - 1) / kCols, G);
-  k_quantize_fp8<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(W), K, N, Wq, scale);
+  launch_k(k_quantize_fp8, grid, 256, 0, s, static_cast<const __nv_bfloat16 *>(W), K, N, Wq, scale);
   return cudaGetLastError();
 }
 

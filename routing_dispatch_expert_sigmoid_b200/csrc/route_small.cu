@@ -164,6 +164,7 @@ __device__ void rank_slots(const SmallArgs &a, int32_t *smem) {
 
 template <int NPL>
 __global__ void __launch_bounds__(kWarps * 32) k_route_small(SmallArgs a) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   extern __shared__ int32_t s_dyn[];
   __shared__ int s_last;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -232,7 +233,7 @@ __global__ void __launch_bounds__(kWarps * 32) k_route_small(SmallArgs a) {
 template <int NPL>
 cudaError_t run(const SmallArgs &a, size_t smem, cudaStream_t s) {
   const int blocks = (a.g.T + kWarps - 1) / kWarps;
-  k_route_small<NPL><<<blocks, kWarps * 32, smem, s>>>(a);
+  launch_k(k_route_small<NPL>, blocks, kWarps * 32, smem, s, a);
   return cudaGetLastError();
 }
 

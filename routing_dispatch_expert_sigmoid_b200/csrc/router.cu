@@ -20,6 +20,7 @@ template <typename T, int BM, int BN, int BK, int TM, int TN>
 __global__ void __launch_bounds__(256) k_router(const T *__restrict__ x, const T *__restrict__ Wr,
                                                 const float *__restrict__ bias,
                                                 float *__restrict__ logits, int Tn, int d, int E) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   static_assert((BM / TM) * (BN / TN) == 256, "256 threads");
   __shared__ float xs[BK][BM + 4];
   __shared__ float ws[BK][BN];
@@ -78,6 +79,7 @@ template <typename T, int EMAX>
 __global__ void __launch_bounds__(256)
     k_router_warp(const T *__restrict__ x, const T *__restrict__ Wr, const float *__restrict__ bias,
                   float *__restrict__ logits, int Tn, int d, int E) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   const int t = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
   if (t >= Tn) return;  // whole warp leaves together
   float acc[EMAX];
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(256)
 template <typename T, int EMAX>
 cudaError_t run_warp(const moe_config &c, const void *x, const void *Wr, const float *bias,
                      float *logits, cudaStream_t s) {
-  k_router_warp<T, EMAX><<<(c.T + 7) / 8, 256, 0, s>>>(
+  launch_k(k_router_warp<T, EMAX>, (c.T + 7) / 8, 256, 0, s, 
       static_cast<const T *>(x), static_cast<const T *>(Wr), bias, logits, c.T, c.d, c.E);
   return cudaGetLastError();
 }
@@ -115,7 +117,7 @@ template <typename T, int BM, int BN, int BK, int TM, int TN>
 cudaError_t run(const moe_config &c, const void *x, const void *Wr, const float *bias,
                 float *logits, cudaStream_t s) {
   dim3 grid((c.T + BM - 1) / BM, (c.E + BN - 1) / BN);
-  k_router<T, BM, BN, BK, TM, TN><<<grid, 256, 0, s>>>(
+  launch_k(k_router<T, BM, BN, BK, TM, TN>, grid, 256, 0, s, 
       static_cast<const T *>(x), static_cast<const T *>(Wr), bias, logits, c.T, c.d, c.E);
   return cudaGetLastError();
 }

@@ -39,6 +39,7 @@ int pick_splits(int kb, long long tiles) {
 __global__ void __launch_bounds__(256)
     k_swiglu_parts(const float4 *__restrict__ gate, const float4 *__restrict__ up, int parts,
                    long long n4, uint2 *__restrict__ h) {
+  grid_dependency();  // the previous grid is complete; the next may launch
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (long long)gridDim.x * blockDim.x) {
     float4 a = gate[i], b = up[i];
@@ -105,7 +106,7 @@ cudaError_t launch_shared_split(const moe_config &c, const SharedSplitPlan &p, b
   const long long n4 = (long long)c.T * c.f_shared / 4;
   long long blocks = (n4 + 255) / 256;
   if (blocks > 4 * kTargetCtas) blocks = 4 * kTargetCtas;
-  k_swiglu_parts<<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(pg),
+  launch_k(k_swiglu_parts, (int)blocks, 256, 0, s, reinterpret_cast<const float4 *>(pg),
                                               reinterpret_cast<const float4 *>(pu), p.s_up, n4,
                                               static_cast<uint2 *>(h));
   e = cudaGetLastError();
