@@ -538,6 +538,35 @@ def test_layer_combine_one_vector_per_lane(name, dev):
             os.environ["MOE_COMBINE_VPL"] = old
 
 
+@pytest.mark.parametrize("name", ["mixtral_small", "qwen3_medium", "dsv3_medium", "gptoss_small",
+                                  "mixtral_decode_small"])
+def test_layer_same_with_and_without_dependent_launch(name, dev):
+    """MOE_PDL=0 launches every kernel in plain stream order; by default each
+    launch overlaps the previous kernel's tail, and every kernel waits for
+    its predecessor before it touches memory.  The outputs and routing must
+    be the same bit for bit."""
+    import os
+    w = SMALL[name]
+    hin = _host_inputs(w, seed=5)
+    inp = gpu_inputs(w, 0, dev, hin)
+    old = os.environ.get("MOE_PDL")
+    try:
+        os.environ["MOE_PDL"] = "0"
+        plain, rb0 = run_layer(w, inp)
+        os.environ.pop("MOE_PDL", None)
+        pdl, rb1 = run_layer(w, inp)
+    finally:
+        if old is None:
+            os.environ.pop("MOE_PDL", None)
+        else:
+            os.environ["MOE_PDL"] = old
+    assert torch.equal(plain, pdl)
+    for k in ("logits", "topk_idx", "topk_w", "slot_row", "offsets"):
+        assert torch.equal(rb0[k], rb1[k]), k
+    R = int(rb0["offsets"][-1])  # row_src holds the kept rows only
+    assert torch.equal(rb0["row_src"][:R], rb1["row_src"][:R])
+
+
 @pytest.fixture
 def fused_dispatch():
     import os
