@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(256)
 template <typename T, int EMAX>
 cudaError_t run_warp(const moe_config &c, const void *x, const void *Wr, const float *bias,
                      float *logits, cudaStream_t s) {
-  launch_k(k_router_warp<T, EMAX>, (c.T + 7) / 8, 256, 0, s, 
+  launch_k(k_router_warp<T, EMAX>, (c.T + 7) / 8, 256, 0, s,
       static_cast<const T *>(x), static_cast<const T *>(Wr), bias, logits, c.T, c.d, c.E);
   return cudaGetLastError();
 }
@@ -117,7 +117,7 @@ template <typename T, int BM, int BN, int BK, int TM, int TN>
 cudaError_t run(const moe_config &c, const void *x, const void *Wr, const float *bias,
                 float *logits, cudaStream_t s) {
   dim3 grid((c.T + BM - 1) / BM, (c.E + BN - 1) / BN);
-  launch_k(k_router<T, BM, BN, BK, TM, TN>, grid, 256, 0, s, 
+  launch_k(k_router<T, BM, BN, BK, TM, TN>, grid, 256, 0, s,
       static_cast<const T *>(x), static_cast<const T *>(Wr), bias, logits, c.T, c.d, c.E);
   return cudaGetLastError();
 }
