@@ -191,26 +191,83 @@ __device__ __forceinline__ void gate_token(const GatingArgs &g, int t, const flo
   // k_t rounds of warp argmax; lane j keeps slot j.
   int my_idx = -1;
   float my_val = 0.f;
-  for (int j = 0; j < kt; ++j) {
-    uint32_t bu = 0;  // this lane's best alive candidate (the lowest i among equals)
-    int bi = 0x7fffffff;
-    float bv = 0.f;
+  if constexpr (NPL >= 8) {
+    // Wide rows: each lane keeps its kCache best alive candidates in order
+    // (larger key first, lower index among equals).  A round compares the
+    // lanes' heads; the winning lane drops its head, and a lane whose cache
+    // runs dry while candidates remain refills it from the rest.  The heads
+    // are always the lanes' best remaining candidates, so the winners and
+    // their order are those of scanning every candidate each round, for
+    // a quarter of the scans.
+    constexpr int kCache = 4;
+    uint32_t cu[kCache];
+    int ci[kCache];
+    float cv[kCache];
+    uint32_t pool = alive;  // alive candidates not yet in the cache
+    auto fill = [&]() {
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      if (((alive >> i) & 1u) && ku[i] > bu) {
-        bu = ku[i];
-        bi = i * 32 + lane;
-        bv = val[i];
+      for (int q = 0; q < kCache; ++q) {
+        uint32_t bu = 0;
+        int bi = 0;
+        float bv = 0.f;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+          if (((pool >> i) & 1u) && ku[i] > bu) {
+            bu = ku[i];
+            bi = i;
+            bv = val[i];
+          }
+        }
+        cu[q] = bu;
+        ci[q] = bi;
+        cv[q] = bv;
+        if (bu) pool &= ~(1u << bi);
       }
+    };
+    fill();
+    for (int j = 0; j < kt; ++j) {
+      const int win = warp_best(cu[0], cu[0] ? ci[0] * 32 + lane : 0x7fffffff);
+      if (win < 0) break;  // fewer candidates than k_t (rejected on the host)
+      const int owner = win & 31;
+      const float v = __shfl_sync(kFull, cv[0], owner);
+      if (lane == owner) {
+#pragma unroll
+        for (int q = 0; q + 1 < kCache; ++q) {
+          cu[q] = cu[q + 1];
+          ci[q] = ci[q + 1];
+          cv[q] = cv[q + 1];
+        }
+        cu[kCache - 1] = 0;
+      }
+      if (lane == j) {
+        my_idx = win;
+        my_val = v;
+      }
+      const bool dry = cu[0] == 0 && pool != 0;
+      if (__any_sync(kFull, dry) && dry) fill();
     }
-    const int win = warp_best(bu, bi);
-    if (win < 0) break;  // fewer candidates than k_t (rejected on the host)
-    const int owner = win & 31;
-    const float v = __shfl_sync(kFull, bv, owner);
-    if (lane == owner) alive &= ~(1u << (win >> 5));
-    if (lane == j) {
-      my_idx = win;
-      my_val = v;
+  } else {
+    for (int j = 0; j < kt; ++j) {
+      uint32_t bu = 0;  // this lane's best alive candidate (the lowest i among equals)
+      int bi = 0x7fffffff;
+      float bv = 0.f;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        if (((alive >> i) & 1u) && ku[i] > bu) {
+          bu = ku[i];
+          bi = i * 32 + lane;
+          bv = val[i];
+        }
+      }
+      const int win = warp_best(bu, bi);
+      if (win < 0) break;  // fewer candidates than k_t (rejected on the host)
+      const int owner = win & 31;
+      const float v = __shfl_sync(kFull, bv, owner);
+      if (lane == owner) alive &= ~(1u << (win >> 5));
+      if (lane == j) {
+        my_idx = win;
+        my_val = v;
+      }
     }
   }
 
