@@ -803,15 +803,21 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, int KPS>
 struct Shape2 {
+  static_assert(KPS == 1 || KPS == 2, "k-blocks per ring stage");
   static constexpr int BN = SWIGLU ? 128 : 256;       // output columns per tile
   static constexpr int kSpansPerCta = 2;              // 64-column B spans each CTA loads
   static constexpr uint32_t kABytes = 128 * BK * 2;   // 16 KB: this CTA's 128 rows
   static constexpr uint32_t kSpanBytes = BK * 128;    // 8 KB
   static constexpr uint32_t kBBytes = kSpansPerCta * kSpanBytes;  // 16 KB
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes;      // 32 KB per CTA
-  static constexpr int kStages = 6;
+  static constexpr uint32_t kKbBytes = kABytes + kBBytes;         // one k-block: 32 KB per CTA
+  // k-blocks per ring stage: the loads of a stage complete on one barrier
+  // and the MMAs of a stage release it with one commit, so two k-blocks a
+  // stage halve the barrier round trips per byte (same bytes in flight)
+  static constexpr int kKbPerStage = KPS;
+  static constexpr uint32_t kStageBytes = kKbPerStage * kKbBytes;
+  static constexpr int kStages = 6 / kKbPerStage;
   static constexpr int kMmaN = 256;                   // N of the pair instruction
   static constexpr uint32_t kAccCols = 256;
   static constexpr uint32_t kTmemCols = 512;
@@ -822,7 +828,7 @@ struct Shape2 {
       1024 + kStages * kStageBytes + 256 + kEpiBytes;
 };
 
-template <bool SWIGLU>
+template <bool SWIGLU, int KPS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB1,
@@ -830,7 +836,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmX32,
                         const __grid_constant__ CUtensorMap tmX8, const Params p) {
   grid_dependency();  // the previous grid is complete; the next may launch
-  using S = Shape2<SWIGLU>;
+  using S = Shape2<SWIGLU, KPS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -1033,63 +1039,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int tile = pair; tile < total && ok; tile += npairs, walk_next(w)) {
         const PairTile t = pair_tile(tile, w);
         const int h = t.swap ? ((t.nr + 15) & ~15) / 2 : 0;  // swap: rows of B per CTA
-        const uint32_t cta_bytes = t.swap ? (uint32_t)h * 128u + S::kBBytes : S::kStageBytes;
+        // bytes this CTA loads per k-block
+        const uint32_t cta_bytes = t.swap ? (uint32_t)h * 128u + S::kBBytes : S::kKbBytes;
         const int row = t.row0 + (int)rank * 128;  // full tile: this CTA's 128 rows of A
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb0 = 0; kb0 < num_kb; kb0 += S::kKbPerStage) {
           if (!wait(empty0 + 8 * s, ph ^ 1, ctl)) {
             ok = false;
             break;
           }
-          const uint32_t st = smem_addr(ring + s * S::kStageBytes);
+          const int nk = min(S::kKbPerStage, num_kb - kb0);
           const uint32_t lfb = leader_full0 + 8 * s;
-          if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * cta_bytes);
-          if (t.swap) {
-            // B: this CTA's h rows (32-row, then 8-row boxes); A: its 128
-            // weight columns, two 64-column spans (the up projection: gate
-            // and up of the same 64 columns, so each CTA's accumulator holds
-            // both halves of its columns' SwiGLU)
-            const int xrow = t.row0 + (int)rank * h;
-            int q = 0;
-            for (; q + 32 <= h; q += 32)
-              tma_load_2d_pair(st + q * 128, &tmX32, lfb, kb * BK, xrow + q);
-            for (; q < h; q += 8) tma_load_2d_pair(st + q * 128, &tmX8, lfb, kb * BK, xrow + q);
-            if (SWIGLU) {
-              const int col = t.n * S::BN + (int)rank * 64;
-              tma_load_3d_pair(st + S::kABytes, &tmB1, lfb, col, kb * BK, t.g);
-              tma_load_3d_pair(st + S::kABytes + S::kSpanBytes, &tmB3, lfb, col, kb * BK, t.g);
-            } else {
-              const int col = t.n * S::BN + (int)rank * 128;
+          if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * cta_bytes * (uint32_t)nk);
+          for (int hk = 0; hk < nk; ++hk) {
+            const int kb = kb0 + hk;
+            const uint32_t st = smem_addr(ring + s * S::kStageBytes + hk * S::kKbBytes);
+            if (t.swap) {
+              // B: this CTA's h rows (32-row, then 8-row boxes); A: its 128
+              // weight columns, two 64-column spans (the up projection: gate
+              // and up of the same 64 columns, so each CTA's accumulator holds
+              // both halves of its columns' SwiGLU)
+              const int xrow = t.row0 + (int)rank * h;
+              int q = 0;
+              for (; q + 32 <= h; q += 32)
+                tma_load_2d_pair(st + q * 128, &tmX32, lfb, kb * BK, xrow + q);
+              for (; q < h; q += 8) tma_load_2d_pair(st + q * 128, &tmX8, lfb, kb * BK, xrow + q);
+              if (SWIGLU) {
+                const int col = t.n * S::BN + (int)rank * 64;
+                tma_load_3d_pair(st + S::kABytes, &tmB1, lfb, col, kb * BK, t.g);
+                tma_load_3d_pair(st + S::kABytes + S::kSpanBytes, &tmB3, lfb, col, kb * BK, t.g);
+              } else {
+                const int col = t.n * S::BN + (int)rank * 128;
 #pragma unroll
-              for (int j = 0; j < 2; ++j)
-                tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, &tmB1, lfb, col + j * 64,
-                                 kb * BK, t.g);
-            }
-          } else {
-            const CUtensorMap *mb = (SWIGLU && rank == 1) ? &tmB3 : &tmB1;
-            const int bcol = SWIGLU ? t.n * S::BN : t.n * S::BN + (int)rank * 128;
-            if (p.l2_hints) {
-              // 1: rows evict-last, weights evict-first; 2: rows evict-last,
-              // weights unhinted; 3: rows unhinted, weights evict-last
-              if (p.l2_hints == 3)
-                tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
-              else
-                tma_load_2d_pair_hint(st, &tmA, lfb, kb * BK, row, pol_keep);
-#pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                if (p.l2_hints == 2)
-                  tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
+                for (int j = 0; j < 2; ++j)
+                  tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, &tmB1, lfb, col + j * 64,
                                    kb * BK, t.g);
-                else
-                  tma_load_3d_pair_hint(st + S::kABytes + j * S::kSpanBytes, mb, lfb,
-                                        bcol + j * 64, kb * BK, t.g,
-                                        p.l2_hints == 3 ? pol_keep : pol_stream);
               }
             } else {
-              tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
+              const CUtensorMap *mb = (SWIGLU && rank == 1) ? &tmB3 : &tmB1;
+              const int bcol = SWIGLU ? t.n * S::BN : t.n * S::BN + (int)rank * 128;
+              if (p.l2_hints) {
+                // 1: rows evict-last, weights evict-first; 2: rows evict-last,
+                // weights unhinted; 3: rows unhinted, weights evict-last
+                if (p.l2_hints == 3)
+                  tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
+                else
+                  tma_load_2d_pair_hint(st, &tmA, lfb, kb * BK, row, pol_keep);
 #pragma unroll
-              for (int j = 0; j < 2; ++j)
-                tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
-                                 kb * BK, t.g);
+                for (int j = 0; j < 2; ++j) {
+                  if (p.l2_hints == 2)
+                    tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
+                                     kb * BK, t.g);
+                  else
+                    tma_load_3d_pair_hint(st + S::kABytes + j * S::kSpanBytes, mb, lfb,
+                                          bcol + j * 64, kb * BK, t.g,
+                                          p.l2_hints == 3 ? pol_keep : pol_stream);
+                }
+              } else {
+                tma_load_2d_pair(st, &tmA, lfb, kb * BK, row);
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+                  tma_load_3d_pair(st + S::kABytes + j * S::kSpanBytes, mb, lfb, bcol + j * 64,
+                                   kb * BK, t.g);
+              }
             }
           }
           ++issued;
@@ -1130,7 +1141,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // 16-byte address field (every stage lies below 256 KB)
       const uint64_t rows_d0 = smem_desc(smem_addr(ring), 16, 1024);
       const uint64_t w_d0 = smem_desc(smem_addr(ring) + S::kABytes, S::kSpanBytes, 1024);
-      constexpr uint32_t kStageStep = S::kStageBytes >> 4, kRowK = 32 >> 4, kWK = 2048 >> 4;
+      constexpr uint32_t kStageStep = S::kStageBytes >> 4, kKbStep = S::kKbBytes >> 4;
+      constexpr uint32_t kRowK = 32 >> 4, kWK = 2048 >> 4;
       Walk w = walk_start();
       for (int tile = pair; tile < total && ok; tile += npairs, walk_next(w)) {
         const PairTile t = pair_tile(tile, w);
@@ -1141,22 +1153,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * S::kAccCols;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb0 = 0; kb0 < num_kb; kb0 += S::kKbPerStage) {
           if (!wait(full0 + 8 * s, ph, ctl)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t rd = rows_d0 + s * kStageStep, wd = w_d0 + s * kStageStep;
-          const uint32_t acc0 = kb != 0;
-          if (t.swap) {
+          const int nk = min(S::kKbPerStage, num_kb - kb0);
+          for (int hk = 0; hk < nk; ++hk) {
+            const uint64_t rd = rows_d0 + s * kStageStep + hk * kKbStep;
+            const uint64_t wd = w_d0 + s * kStageStep + hk * kKbStep;
+            const uint32_t acc0 = (kb0 + hk) != 0;
+            if (t.swap) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma_pair(d_tmem, wd + kk * kWK, rd + kk * kRowK, idesc_swap, kk ? 1u : acc0);
-          } else {
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma_pair(d_tmem, wd + kk * kWK, rd + kk * kRowK, idesc_swap, kk ? 1u : acc0);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma_pair(d_tmem, rd + kk * kRowK, wd + kk * kWK, S::kIdesc, kk ? 1u : acc0);
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma_pair(d_tmem, rd + kk * kRowK, wd + kk * kWK, S::kIdesc, kk ? 1u : acc0);
+            }
           }
           any = true;
           umma_commit_pair_both(empty0 + 8 * s);
@@ -2039,12 +2055,12 @@ cudaError_t launch(int rows_cap, int K, int N, int G, const int32_t *offsets, in
   return cudaGetLastError();
 }
 
-template <bool SWIGLU>
-cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offsets,
-                        int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
-                        uint32_t *err, cudaStream_t s, RowWeights rw = RowWeights(),
-                        int8_t *yexp = nullptr, const float *bias = nullptr) {
-  using S = Shape2<SWIGLU>;
+template <bool SWIGLU, int KPS>
+cudaError_t launch_pair_kps(int rows_cap, int K, int N, int G, const int32_t *offsets,
+                            int fixed_rows, const void *A, const void *B1, const void *B3,
+                            void *out, uint32_t *err, cudaStream_t s, RowWeights rw,
+                            int8_t *yexp, const float *bias) {
+  using S = Shape2<SWIGLU, KPS>;
   CUtensorMap ma, mb1, mb3;
   if (!make_map_a(&ma, A, rows_cap, K) || !make_map_b(&mb1, B1, G, K, N) ||
       !make_map_b(&mb3, SWIGLU ? B3 : B1, G, K, N))
@@ -2055,7 +2071,7 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static std::atomic<bool> attr_set[64];
-  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_pair<SWIGLU>,
+  if (cudaError_t e = set_smem_once(attr_set, k_grouped_gemm_pair<SWIGLU, KPS>,
                                     S::kSmemFixed + sizeof(int32_t) * 3 * (kMaxGroups + 1)))
     return e;
   Params p{offsets, G, fixed_rows, rows_cap, K, N, out, bias, nullptr, 1, err};
@@ -2083,9 +2099,30 @@ cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offset
                               ((N + S::BN - 1) / S::BN);
   long long pairs = sms / 2;
   if (max_tiles < pairs) pairs = max_tiles < 1 ? 1 : max_tiles;
-  launch_k(k_grouped_gemm_pair<SWIGLU>, (int)(2 * pairs), kThreads, smem, s, ma, mb1, mb3, mx32, mx8,
-                                                                       p);
+  launch_k(k_grouped_gemm_pair<SWIGLU, KPS>, (int)(2 * pairs), kThreads, smem, s, ma, mb1, mb3,
+           mx32, mx8, p);
   return cudaGetLastError();
+}
+
+// Two k-blocks per ring stage for long K (at least 32 k-blocks), one for
+// short K.  Alternated call by call on one B200, two per stage made the
+// Mixtral-shaped layer 3% faster (up and down), the DeepSeek-V3-shaped
+// prefill 3-5% and the Qwen3-shaped up projection (K = 2048) 2.6%, while the
+// short-K down projections (K = 720-768, 12 k-blocks) lost 3.6% with half
+// as many stages.  MOE_PAIR_KPS=1|2 forces the choice.
+template <bool SWIGLU>
+cudaError_t launch_pair(int rows_cap, int K, int N, int G, const int32_t *offsets,
+                        int fixed_rows, const void *A, const void *B1, const void *B3, void *out,
+                        uint32_t *err, cudaStream_t s, RowWeights rw = RowWeights(),
+                        int8_t *yexp = nullptr, const float *bias = nullptr) {
+  const char *ks = getenv("MOE_PAIR_KPS");
+  const int num_kb = (K + BK - 1) / BK;
+  const int kps = ks && (ks[0] == '1' || ks[0] == '2') ? ks[0] - '0' : (num_kb >= 32 ? 2 : 1);
+  if (kps == 2)
+    return launch_pair_kps<SWIGLU, 2>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out, err,
+                                      s, rw, yexp, bias);
+  return launch_pair_kps<SWIGLU, 1>(rows_cap, K, N, G, offsets, fixed_rows, A, B1, B3, out, err, s,
+                                    rw, yexp, bias);
 }
 
 template <bool SWIGLU>

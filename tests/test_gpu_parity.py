@@ -448,6 +448,34 @@ def test_expert_ffn_pair_with_swap_tiles(name, pair_swap, dev):
     test_expert_ffn_matches_oracle(name, dev)
 
 
+@pytest.fixture(params=["1", "2"])
+def pair_kps(request):
+    """k-blocks per ring stage of the CTA-pair engine (the default picks 2
+    only for K of 32 k-blocks or more, so small shapes would test 1 alone)."""
+    import os
+    keys = ("MOE_GEMM_ENGINE", "MOE_PAIR_KPS")
+    old = {k: os.environ.get(k) for k in keys}
+    os.environ["MOE_GEMM_ENGINE"] = "pair"
+    os.environ["MOE_PAIR_KPS"] = request.param
+    yield request.param
+    for k, v in old.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
+
+
+# qwen3_small has d = 192: three k-blocks, so two per stage leaves a ragged last stage
+@pytest.mark.parametrize("name", ["mixtral_small", "qwen3_small", "dsv3_small", "gptoss_small",
+                                  "qwen3_medium"])
+def test_layer_pair_kblocks_per_stage(name, pair_kps, dev):
+    test_layer_matches_oracle(name, dev)
+
+
+def test_expert_ffn_group_size_edges_pair_kblocks_per_stage(pair_kps, dev):
+    test_expert_ffn_group_size_edges("pair", dev)
+
+
 @pytest.fixture(params=["1", "2", "3"])
 def l2_hints(request):
     """MOE_L2_HINTS=1|2|3: the GEMMs' TMA loads carry L2 eviction hints (the
